@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Paged-decode benchmark: KV-read GB/s (and % of HBM peak), attention tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--partition P] [--no-cpu-baseline]
+
+One step is one pass of the hot path over one batch: copy_blocks (when the
+batch has copy-on-write pairs), reshape_and_cache of the step's new tokens,
+and paged_attn_decode of every sequence.  Inputs are seeded synthetic data
+(paged_kv_cache_394_b200.workloads); the default workload is the
+LLaMA-7B-shaped decode layer (64 sequences, 32 heads, head_dim 128, block 16,
+fp16, context lengths uniform in [128, 2048]).
+
+`value` is the step's algorithmic bytes (K+V read by decode, q read, out
+written, plus the bytes the cache write and block copy move) over the
+device-timed step, summed over ranks.  Under torchrun each rank runs its own
+replica batch (weak scaling, no collective on the data path); the step time is
+the max over ranks.  `e2e` times the same step through the host-buffer entry
+point, with the step's inputs copied from pinned host memory and the output
+read back inside the timed region.
+
+`--impl reference` times the CPU oracle on the host cores instead (rank 0
+only), each step a bounded sample of the same workload.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; barrier and max-reduce only)
+# ---------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(backend, timeout_s=120):
+    import datetime
+
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x, device=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, device=None):
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def replica_seed(base_seed, rank):
+    """Each rank draws its own replica batch of the same shape."""
+    return base_seed + 7919 * rank
+
+
+# ---------------------------------------------------------------------------
+# bytes
+# ---------------------------------------------------------------------------
+def decode_bytes(w):
+    """Algorithmic bytes of one decode call: K and V of every cached token of
+    every kv head, q read, out written."""
+    e = 2
+    kv = 2 * int(w.context_lens.astype("int64").sum()) * w.num_kv_heads * w.head_dim * e
+    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * e
+    return kv + qo
+
+
+def write_bytes(w):
+    """reshape_and_cache: read key and value, write them, read the slots."""
+    t = len(w.slot_mapping)
+    return 2 * 2 * t * w.num_kv_heads * w.head_dim * 2 + 8 * t
+
+
+def copy_bytes(w):
+    """copy_blocks: read and write K and V of every copied block, read the pairs."""
+    blk = w.num_kv_heads * w.block_size * w.head_dim * 2
+    return len(w.cow_pairs) * (2 * 2 * blk + 16)
+
+
+def step_bytes(w):
+    return decode_bytes(w) + write_bytes(w) + copy_bytes(w)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# peaks and the committed ncu traffic summary
+# ---------------------------------------------------------------------------
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    csrc = os.path.join(ROOT, "paged_kv_cache_394_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload):
+    """DRAM bytes per decode launch from profiles/, if taken on the current kernels."""
+    path = os.path.join(ROOT, "profiles", "paged_decode_%s_traffic.md" % workload)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_src = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", text)
+    if not (m_src and m_b) or m_src.group(1) != kernel_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    from paged_kv_cache_394_b200 import workloads as W
+
+    rank, world = init_dist("nccl") if dist_env()[1] > 1 else (0, 1)
+    local = dist_env()[2]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = W.SEED_BASE + W.NAMES.index(args.workload)
+    w = W.make(args.workload, seed=replica_seed(base, rank))
+    tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(tdt)
+
+    q, kc, vc, key, val = up(w.q), up(w.k_cache), up(w.v_cache), up(w.key), up(w.value)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    pairs = torch.from_numpy(np.ascontiguousarray(w.cow_pairs)).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    lens = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    part_req = w.partition_size if args.partition is None else args.partition
+    part = pk.partition_size(w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len, part_req)
+    split = part < w.max_context_len
+    ws = pk.alloc_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                            w.max_context_len, part_req, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    has_pairs = len(w.cow_pairs) > 0
+    launches_per_step = 1 + 1 + (1 if split else 0) + (1 if has_pairs else 0)
+
+    def step(ev_a=None, ev_b=None):
+        if has_pairs:
+            pk.copy_blocks(kc, vc, pairs, dev_err=err, stream=stream)
+        pk.reshape_and_cache(key, val, kc, vc, slots, dev_err=err, stream=stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        pk.paged_attn_decode(out, q, kc, vc, tables, lens, w.scale, w.num_kv_heads, w.block_size,
+                             w.max_context_len, partition_size=part_req, workspace=ws,
+                             dev_err=err, stream=stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError("device error word %d during warm-up" % int(err.item()))
+
+    # ---- timed region: K steps, device events, barrier + sync both sides ----
+    clocks = ClockSampler(local)
+    clocks.start()
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(*dec_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+    total_ms_max = max_over_ranks(total_ms, dev)
+    ms_per_step = total_ms_max / args.steps
+    sbytes = step_bytes(w)
+    all_bytes = sum_over_ranks(sbytes, dev)
+    value = all_bytes / (ms_per_step * 1e-3) / 1e9
+    dec_avg_ms = statistics.mean(dec_ms)
+    dbytes = decode_bytes(w)
+    achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    # ---- end to end through the host-buffer entry point ----------------------
+    def pinned(a, view=None):
+        return torch.from_numpy(np.ascontiguousarray(a if view is None else a.view(view))).pin_memory()
+    h_q = pinned(w.q, np.int16).view(tdt)
+    h_key = pinned(w.key, np.int16).view(tdt)
+    h_val = pinned(w.value, np.int16).view(tdt)
+    h_slots, h_pairs = pinned(w.slot_mapping), pinned(w.cow_pairs)
+    h_tables, h_lens = pinned(w.block_tables), pinned(w.context_lens)
+    h_out = torch.empty(w.q.shape, dtype=tdt).pin_memory()
+    staging = torch.empty(pk.staging_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim,
+                                           w.max_blocks_per_seq, len(w.slot_mapping),
+                                           len(w.cow_pairs)), dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_val, h_slots, h_pairs,
+                                                     h_tables, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        pk.decode_step_host(h_out, h_q, h_key, h_val, h_slots, h_pairs, h_tables, h_lens, kc, vc,
+                            w.scale, w.max_context_len, staging, workspace=ws,
+                            partition_size=part_req, dev_err=err, stream=stream)
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    e2e_value = all_bytes / (e2e_ms * 1e-3) / 1e9
+    if int(err.item()) != 0:
+        raise RuntimeError("device error word %d" % int(err.item()))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        tokens = w.num_seqs * world
+        line = {
+            "metric": "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": dict(W.describe(w), parallelism="replicas%d" % world,
+                           partition_used=part, split_k=split,
+                           l2="no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
+                              % (dbytes / 1e9)),
+            "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+            "pct_of_8tbs_nominal": round(100.0 * value / world / 8000.0, 2),
+            "tokens_per_s": round(tokens / (ms_per_step * 1e-3), 1),
+            "context_tokens_per_s": round(world * int(w.context_lens.sum()) / (ms_per_step * 1e-3), 1),
+            "step_bytes": sbytes,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": committed_traffic(args.workload),
+                         "kernel": "paged_decode_kernel" + (" + reduce" if split else ""),
+                         "algorithmic_bytes_per_launch": dbytes,
+                         "avg_launch_ms": round(dec_avg_ms, 5),
+                         "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                         if peak_kind == "measured" else "fallback 6.65 TB/s"},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "pkv_decode_step_host"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    del ws, staging
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(w, seconds):
+    """Times the oracle's step (cache write, then decode of whole sequences in
+    order, all heads) until `seconds` have passed or the batch is done."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attention as OA
+    from oracle import cache_ops as OC
+    cores = len(os.sched_getaffinity(0))
+    done_seqs = 0
+    nbytes = 0
+    with threadpool_limits(limits=cores):
+        t0 = time.perf_counter()
+        kc, vc, _ = OC.copy_blocks(w.k_cache, w.v_cache, w.cow_pairs, inplace=True)
+        kc, vc, _ = OC.reshape_and_cache(w.key, w.value, kc, vc, w.slot_mapping, w.block_size,
+                                         inplace=True)
+        nbytes += write_bytes(w) + copy_bytes(w)
+        for s in range(w.num_seqs):
+            pairs = [(s, h) for h in range(w.num_heads)]
+            OA.paged_attention_decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale,
+                                      w.num_kv_heads, w.block_size, w.dtype, pairs=pairs)
+            done_seqs += 1
+            nbytes += (2 * int(w.context_lens[s]) * w.num_kv_heads * w.head_dim * 2
+                       + 2 * w.num_heads * w.head_dim * 2)
+            if time.perf_counter() - t0 > seconds:
+                break
+        dt = time.perf_counter() - t0
+    _ = np
+    return nbytes, dt, done_seqs, cores
+
+
+def cpu_baseline(w, seconds):
+    nbytes, dt, n, cores = oracle_sample(w, seconds)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": "cache write + float64 decode of the first %d of %d sequences (all %d "
+                      "heads), %.1f s on the host cores" % (n, w.num_seqs, w.num_heads, dt)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from paged_kv_cache_394_b200 import workloads as W
+    w0 = W.make(args.workload)
+    for _ in range(args.warmup):
+        oracle_sample(W.make(args.workload), 0.5)
+    times, total_bytes, n_last, cores = [], 0, 0, 1
+    for _ in range(args.steps):
+        w = W.make(args.workload)
+        nbytes, dt, n_last, cores = oracle_sample(w, args.cpu_seconds)
+        times.append(dt)
+        total_bytes += nbytes
+    value = total_bytes / sum(times) / 1e9
+    line = {
+        "impl": "reference",
+        "metric": "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1000 * statistics.mean(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(W.describe(w0), parallelism="host cores"),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": "per step: cache write + float64 decode of the first %d of "
+                                   "%d sequences (all heads), bounded to %.0f s"
+                                   % (n_last, w0.num_seqs, args.cpu_seconds)},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="llama7b")
+    ap.add_argument("--partition", type=int, default=None,
+                    help="partition size in tokens (0 = let the library choose)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    # at least three untimed warm-up steps, whatever was asked
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

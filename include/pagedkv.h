@@ -1,0 +1,251 @@
+/*
+ * pagedkv.h — C ABI of libpagedkv.so: PagedAttention decode on NVIDIA B200
+ * (sm_100a), the cache-write scatter, the copy-on-write block copy, and a
+ * host-side block allocator.
+ *
+ * Sources cited by page title and section:
+ *   [csdn]       devpress.csdn.net, "vLLM镜像深度优化：PagedAttention助力大模型推理效率飞跃"
+ *   [cortexgrid] aidocs.cortexgrid.cn/docs/0a2c4066ef83, vLLM explainer with an FAQ
+ *   [betteryeah] betteryeah.com, "vLLM是什么？完整解析高性能LLM推理引擎的技术原理与部署实践"
+ *
+ * The KV cache is cut into fixed-size blocks (pages) of block_size tokens that
+ * sit anywhere in a physical pool; a per-sequence block table maps logical
+ * block j of sequence i to a physical block ([csdn] "分页式KV缓存"; [betteryeah]
+ * §2.2; [cortexgrid] FAQ on block tables).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layouts are row-major.  The caches are
+ *        k_cache, v_cache : [num_blocks, num_kv_heads, block_size, head_dim]
+ *    so one (block, kv head) is one contiguous run of block_size*head_dim
+ *    elements.  Elements are 16-bit (PKV_FP16 or PKV_BF16).
+ *  - A slot is physical_block * block_size + offset (int64); a negative slot
+ *    marks a padding token.
+ *  - Ownership: the caller owns every buffer.  The library never allocates or
+ *    frees device memory; scratch for split-K decode ("workspace") and for the
+ *    host-buffer step ("staging") is passed in by the caller.
+ *  - Execution: device work is enqueued asynchronously on `stream` (a
+ *    cudaStream_t passed as void*; NULL is the legacy default stream).  No
+ *    entry point synchronizes.  All device pointers must belong to the
+ *    device that is current on the calling thread.
+ *  - Host-side validation happens before anything is enqueued: a bad scalar or
+ *    a null / misaligned pointer returns PKV_ERR_INVALID_ARG, a valid but
+ *    unbuilt shape returns PKV_ERR_UNSUPPORTED, a launch failure returns
+ *    PKV_ERR_CUDA (pkv_last_cuda_error() gives the CUDA error code).
+ *  - Device-side index errors (values the host cannot see because they live
+ *    in device memory) never fault: the kernel skips the offending access and
+ *    ORs a PKV_DEVERR_* bit into *dev_err when dev_err is not NULL.  Read the
+ *    word after the stream has synchronized; outputs are then unreliable.
+ *  - Alignment: every 16-bit tensor pointer must be 16-byte aligned.
+ *  - Supported shapes: head_dim in {64, 128}, block_size in {16, 32},
+ *    num_heads / num_kv_heads in {1, 2, 4, 8}, dtype fp16 or bf16.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1,   /* bad scalar, null or misaligned pointer      */
+  PKV_ERR_UNSUPPORTED = 2,   /* shape / dtype combination not built         */
+  PKV_ERR_WORKSPACE = 3,     /* workspace or staging buffer too small       */
+  PKV_ERR_CUDA = 4,          /* a CUDA runtime call failed                  */
+  PKV_ERR_OUT_OF_BLOCKS = 5  /* allocator: the free list is empty           */
+} pkv_status;
+
+typedef enum { PKV_FP16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Bits ORed into *dev_err by the kernels. */
+#define PKV_DEVERR_BAD_BLOCK 1u   /* decode: table entry outside [0, num_blocks)          */
+#define PKV_DEVERR_BAD_SLOT 2u    /* reshape_and_cache: slot >= num_blocks * block_size   */
+#define PKV_DEVERR_BAD_PAIR 4u    /* copy_blocks: src or dst outside [0, num_blocks)      */
+#define PKV_DEVERR_BAD_CONTEXT 8u /* decode: context_len < 0, > max_context_len, or more
+                                     blocks than max_blocks_per_seq                        */
+#define PKV_DEVERR_TIMEOUT 16u    /* decode: a bounded wait for an async copy gave up      */
+
+/* Library version string, e.g. "pagedkv 0.1.0 sm_100a". */
+const char* pkv_version(void);
+/* Static English description of a status code. */
+const char* pkv_status_string(int status);
+/* cudaError_t of the most recent PKV_ERR_CUDA on the calling thread (0 if none). */
+int pkv_last_cuda_error(void);
+
+/*
+ * pkv_reshape_and_cache — write the K and V vectors of new tokens into their
+ * cache slots ([csdn] "内存困局的破局者": the cache keeps K and V per token;
+ * [betteryeah] §2.2: pages are filled as a sequence grows).
+ *
+ *   key, value    device, [num_tokens, num_kv_heads, head_dim], 16-bit
+ *   k_cache, v_cache  device caches (layout above), written in place
+ *   slot_mapping  device int64 [num_tokens]; token t goes to
+ *                 block = slot / block_size, offset = slot % block_size;
+ *                 slot < 0 skips the token; slot >= num_blocks*block_size sets
+ *                 PKV_DEVERR_BAD_SLOT and skips it.
+ * Bit-exact copy.  Two tokens with the same slot leave one of them (which
+ * one is unspecified).  num_tokens == 0 is a no-op.
+ */
+pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                 void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                 int num_kv_heads, int head_dim, int block_size,
+                                 int num_blocks, pkv_dtype dtype, unsigned* dev_err,
+                                 void* stream);
+
+/*
+ * pkv_copy_blocks — copy-on-write block copy ([cortexgrid] FAQ on parallel
+ * sampling: shared blocks are reference-counted and copied when several
+ * holders must modify them).
+ *
+ *   block_mapping  device int64 [num_pairs, 2] of (src, dst) physical blocks.
+ *                  For each pair the whole K block and the whole V block (all
+ *                  kv heads, offsets and dims) of src are copied to dst.
+ * Preconditions (what the allocator produces): dst values are distinct and no
+ * dst is also a src in the same call; otherwise the result is unspecified.
+ * A pair with an index outside [0, num_blocks) sets PKV_DEVERR_BAD_PAIR and
+ * is skipped.  Bit-exact.  num_pairs == 0 is a no-op.
+ */
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                           int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, pkv_dtype dtype, unsigned* dev_err, void* stream);
+
+/*
+ * Split-K (partitioned) decode.  For long contexts the context of each
+ * sequence is cut into partitions of partition_size tokens; each partition
+ * produces a (max logit, exp-sum, unnormalised output) triple in the
+ * workspace and a second kernel merges them.  pkv_paged_attn_partition_size
+ * returns the partition size `pkv_paged_attn_decode` will use:
+ *   requested > 0  -> requested (must be a multiple of block_size);
+ *   requested == 0 -> chosen from the shape; a value >= max_context_len
+ *                     means single pass (no workspace needed).
+ */
+int pkv_paged_attn_partition_size(int num_seqs, int num_kv_heads, int block_size,
+                                  int max_context_len, int requested);
+
+/* Workspace bytes pkv_paged_attn_decode needs for these arguments (0 when it
+ * runs single-pass).  Returns 0 too for invalid arguments. */
+size_t pkv_paged_attn_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_dim, int block_size, int max_context_len,
+                                      int partition_size);
+
+/*
+ * pkv_paged_attn_decode — attention of each sequence's one new query token
+ * over its paged KV cache.  The kernel assembles each sequence's keys and
+ * values from the block table across non-contiguous blocks ([csdn]
+ * "分页式KV缓存"; [betteryeah] §2.4), so the result equals
+ *     out[i, h, :] = softmax(scale * q[i, h, :] . K_i^T) . V_i
+ * over the context_lens[i] cached tokens of sequence i, where query head h
+ * reads kv head h / (num_heads / num_kv_heads).  fp32 accumulation, output
+ * rounded to the input dtype (round to nearest even).
+ *
+ *   out            device [num_seqs, num_heads, head_dim], written
+ *   q              device [num_seqs, num_heads, head_dim]
+ *   block_tables   device int32 [num_seqs, max_blocks_per_seq]; entries at or
+ *                  beyond ceil(context_len / block_size) are never read
+ *   context_lens   device int32 [num_seqs]; 0 gives an all-zero output row
+ *   max_context_len  an upper bound of context_lens (sizes the launch)
+ *   partition_size 0 = choose; else force this partition size (see above)
+ *   workspace      device, >= pkv_paged_attn_workspace_bytes(...) bytes,
+ *                  16-byte aligned; may be NULL when that is 0.  Its contents
+ *                  need no initialisation and are scratch afterwards.
+ * A table entry outside [0, num_blocks) sets PKV_DEVERR_BAD_BLOCK and that
+ * block is left out.  num_seqs == 0 is a no-op.
+ */
+pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, int num_seqs,
+                                 int num_heads, int num_kv_heads, int head_dim,
+                                 int block_size, int max_blocks_per_seq, int max_context_len,
+                                 int num_blocks, pkv_dtype dtype, int partition_size,
+                                 void* workspace, size_t workspace_bytes, unsigned* dev_err,
+                                 void* stream);
+
+/*
+ * pkv_decode_step_host — one whole decode step from HOST buffers: copies the
+ * step's inputs host->device, runs copy_blocks (if num_pairs > 0),
+ * reshape_and_cache (if num_new_tokens > 0) and paged_attn_decode, and copies
+ * the output back, all enqueued on `stream`.  The caches stay on the device.
+ *
+ *   *_host     host pointers; page-locked (pinned) memory makes the copies
+ *              asynchronous, pageable memory works but copies synchronously.
+ *              The host buffers must stay valid until the stream has finished.
+ *   staging    device scratch of >= pkv_decode_step_staging_bytes(...) bytes
+ *              (16-byte aligned) that receives the step's inputs and output.
+ *   workspace  as for pkv_paged_attn_decode.
+ * Shapes as for the three calls above.
+ */
+size_t pkv_decode_step_staging_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                     int head_dim, int max_blocks_per_seq, int num_new_tokens,
+                                     int num_pairs);
+pkv_status pkv_decode_step_host(
+    void* out_host, const void* q_host, const void* key_host, const void* value_host,
+    const int64_t* slot_mapping_host, int num_new_tokens, const int64_t* block_mapping_host,
+    int num_pairs, const int32_t* block_tables_host, const int32_t* context_lens_host,
+    void* k_cache, void* v_cache, float scale, int num_seqs, int num_heads, int num_kv_heads,
+    int head_dim, int block_size, int max_blocks_per_seq, int max_context_len, int num_blocks,
+    pkv_dtype dtype, int partition_size, void* staging, size_t staging_bytes, void* workspace,
+    size_t workspace_bytes, unsigned* dev_err, void* stream);
+
+/*
+ * Host block allocator ([csdn] "分页式KV缓存" and "典型工作流程拆解" step 7;
+ * [betteryeah] §2.2; [cortexgrid] FAQ on parallel sampling).  Host memory
+ * only; not thread-safe (one allocator per scheduler thread).
+ *
+ *  - The free list is a FIFO queue: allocation takes the front, release
+ *    appends at the back.  Its initial order is `free_order` (a permutation of
+ *    0..num_blocks-1, copied) or the identity when NULL.
+ *  - add_seq takes ceil(num_tokens / block_size) blocks, or none if short.
+ *  - fork makes `child` share all of `parent`'s blocks (refcount + 1 each).
+ *  - append_slot reserves the slot of the sequence's next token.  At a block
+ *    boundary it takes a fresh block.  Inside a block whose refcount exceeds
+ *    one it copies on write: it takes a fresh block, returns (old, new) in
+ *    *cow_src / *cow_dst for pkv_copy_blocks, decrements the old block's
+ *    refcount and points the table at the new block.  Otherwise both are -1.
+ *    The last holder of a block (refcount 1) writes in place.
+ *  - free_seq drops one reference per block, front to back; a block that
+ *    reaches zero is appended to the free queue.
+ * Errors: unknown / duplicate ids or bad sizes -> PKV_ERR_INVALID_ARG;
+ * empty free list -> PKV_ERR_OUT_OF_BLOCKS (the state is left unchanged).
+ */
+typedef struct pkv_alloc pkv_alloc;
+
+/* NULL on bad arguments (num_blocks <= 0, block_size <= 0, free_order not a permutation). */
+pkv_alloc* pkv_alloc_create(int num_blocks, int block_size, const int32_t* free_order);
+void pkv_alloc_destroy(pkv_alloc* a);
+pkv_status pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id, int64_t num_tokens);
+pkv_status pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child);
+pkv_status pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_t* slot,
+                                 int64_t* cow_src, int64_t* cow_dst);
+/* Appends one token to each of seq_ids[0..n) in order.  slots[n] receives the
+ * slots; cow_pairs[2*k], cow_pairs[2*k+1] the k-th copy pair (capacity n
+ * pairs); *num_cow their count; *num_done how many appends succeeded (all n
+ * unless an error status is returned). */
+pkv_status pkv_alloc_append_slots(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots,
+                                  int64_t* cow_pairs, int* num_cow, int* num_done);
+pkv_status pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id);
+/* table_out: host int32 [n, max_blocks], padded with -1. */
+pkv_status pkv_alloc_block_table(const pkv_alloc* a, const int64_t* seq_ids, int n,
+                                 int max_blocks, int32_t* table_out);
+/* lens_out: host int32 [n], each sequence's token count. */
+pkv_status pkv_alloc_context_lens(const pkv_alloc* a, const int64_t* seq_ids, int n,
+                                  int32_t* lens_out);
+int pkv_alloc_num_free(const pkv_alloc* a);
+/* -1 for an out-of-range block. */
+int pkv_alloc_refcount(const pkv_alloc* a, int block);
+/* -1 for an unknown sequence. */
+int64_t pkv_alloc_seq_len(const pkv_alloc* a, int64_t seq_id);
+int pkv_alloc_seq_num_blocks(const pkv_alloc* a, int64_t seq_id);
+/* Cached tokens and allocated blocks, each physical block counted once (a
+ * block's fill is the most slots any holder has filled); utilization is
+ * cached_tokens / (used_blocks * block_size). */
+pkv_status pkv_alloc_usage(const pkv_alloc* a, int64_t* cached_tokens, int64_t* used_blocks);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

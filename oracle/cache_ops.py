@@ -27,16 +27,17 @@ import numpy as np
 
 
 def reshape_and_cache(key_bits, value_bits, k_cache_bits, v_cache_bits, slot_mapping,
-                      block_size):
-    """Scatter new tokens' K/V into copies of the caches.
+                      block_size, inplace=False):
+    """Scatter new tokens' K/V into copies of the caches (or into the given
+    arrays when ``inplace``, which spares a copy of very large pools).
 
     key_bits, value_bits: uint16 ``[T, H_kv, D]``; caches uint16
     ``[num_blocks, H_kv, block_size, D]``; slot_mapping int64 ``[T]``.
     Returns ``(k_cache, v_cache, out_of_range)`` where ``out_of_range`` lists
     the token indices whose slot lay beyond the pool (those are skipped).
     """
-    k_out = np.array(k_cache_bits, copy=True)
-    v_out = np.array(v_cache_bits, copy=True)
+    k_out = k_cache_bits if inplace else np.array(k_cache_bits, copy=True)
+    v_out = v_cache_bits if inplace else np.array(v_cache_bits, copy=True)
     num_slots = k_out.shape[0] * block_size
     bad = []
     for t, slot in enumerate(np.asarray(slot_mapping, dtype=np.int64)):
@@ -51,14 +52,15 @@ def reshape_and_cache(key_bits, value_bits, k_cache_bits, v_cache_bits, slot_map
     return k_out, v_out, bad
 
 
-def copy_blocks(k_cache_bits, v_cache_bits, block_mapping):
-    """Copy whole physical blocks, K and V, for each (src, dst) pair in order.
+def copy_blocks(k_cache_bits, v_cache_bits, block_mapping, inplace=False):
+    """Copy whole physical blocks, K and V, for each (src, dst) pair in order
+    (into copies of the caches, or into the given arrays when ``inplace``).
 
     Returns ``(k_cache, v_cache, out_of_range)``; pairs with an index outside
     the pool are skipped and listed.
     """
-    k_out = np.array(k_cache_bits, copy=True)
-    v_out = np.array(v_cache_bits, copy=True)
+    k_out = k_cache_bits if inplace else np.array(k_cache_bits, copy=True)
+    v_out = v_cache_bits if inplace else np.array(v_cache_bits, copy=True)
     num_blocks = k_out.shape[0]
     bad = []
     for p, (src, dst) in enumerate(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2)):

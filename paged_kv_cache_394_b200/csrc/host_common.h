@@ -1,0 +1,22 @@
+// host_common.h — host-side helpers shared by the pagedkv entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pagedkv.h"
+
+namespace pkv {
+
+// Records `e` as the calling thread's last CUDA error and maps it to a status.
+pkv_status cuda_status(cudaError_t e);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool head_dim_supported(int d) { return d == 64 || d == 128; }
+inline bool block_size_supported(int bs) { return bs == 16 || bs == 32; }
+inline bool dtype_valid(int dt) { return dt == PKV_FP16 || dt == PKV_BF16; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace pkv

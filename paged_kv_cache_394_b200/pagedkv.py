@@ -1,0 +1,309 @@
+"""Thin ctypes binding of ``libpagedkv.so`` (declared in include/pagedkv.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  Device tensors are torch tensors (torch supplies device memory
+and streams); their pointers, shapes and the current CUDA stream are passed
+through the C ABI.  Importing this module loads the library and raises
+``ImportError`` if it has not been built — there is no fallback.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libpagedkv.so is not built (run `python -m paged_kv_cache_394_b200.build`)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_OUT_OF_BLOCKS = range(6)
+FP16, BF16 = 0, 1
+DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_PAIR, DEVERR_BAD_CONTEXT, DEVERR_TIMEOUT = (
+    1, 2, 4, 8, 16)
+
+_vp, _i, _i64, _f, _sz, _u = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                              ctypes.c_size_t, ctypes.c_uint)
+
+
+def _proto(name, restype, *argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+_lib_version = _proto("pkv_version", ctypes.c_char_p)
+_status_string = _proto("pkv_status_string", ctypes.c_char_p, _i)
+_last_cuda_error = _proto("pkv_last_cuda_error", _i)
+_reshape_and_cache = _proto("pkv_reshape_and_cache", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                            _i, _i, _vp, _vp)
+_copy_blocks = _proto("pkv_copy_blocks", _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp)
+_partition_size = _proto("pkv_paged_attn_partition_size", _i, _i, _i, _i, _i, _i)
+_workspace_bytes = _proto("pkv_paged_attn_workspace_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
+_paged_attn_decode = _proto("pkv_paged_attn_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i,
+                            _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
+_staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
+_decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
+                           _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
+                           _vp, _sz, _vp, _vp)
+_alloc_create = _proto("pkv_alloc_create", _vp, _i, _i, _vp)
+_alloc_destroy = _proto("pkv_alloc_destroy", None, _vp)
+_alloc_add_seq = _proto("pkv_alloc_add_seq", _i, _vp, _i64, _i64)
+_alloc_fork = _proto("pkv_alloc_fork", _i, _vp, _i64, _i64)
+_alloc_append_slot = _proto("pkv_alloc_append_slot", _i, _vp, _i64, _vp, _vp, _vp)
+_alloc_append_slots = _proto("pkv_alloc_append_slots", _i, _vp, _vp, _i, _vp, _vp, _vp, _vp)
+_alloc_free_seq = _proto("pkv_alloc_free_seq", _i, _vp, _i64)
+_alloc_block_table = _proto("pkv_alloc_block_table", _i, _vp, _vp, _i, _i, _vp)
+_alloc_context_lens = _proto("pkv_alloc_context_lens", _i, _vp, _vp, _i, _vp)
+_alloc_num_free = _proto("pkv_alloc_num_free", _i, _vp)
+_alloc_refcount = _proto("pkv_alloc_refcount", _i, _vp, _i)
+_alloc_seq_len = _proto("pkv_alloc_seq_len", _i64, _vp, _i64)
+_alloc_seq_num_blocks = _proto("pkv_alloc_seq_num_blocks", _i, _vp, _i64)
+_alloc_usage = _proto("pkv_alloc_usage", _i, _vp, _vp, _vp)
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status, where):
+        msg = "%s: %s" % (where, _status_string(status).decode())
+        if status == ERR_CUDA:
+            msg += " (cudaError %d)" % _last_cuda_error()
+        super().__init__(msg)
+        self.status = status
+
+
+def _check(status, where):
+    if status != OK:
+        raise PagedKVError(status, where)
+
+
+def version():
+    return _lib_version().decode()
+
+
+def library_path():
+    return LIB_PATH
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float16:
+        return FP16
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("expected float16 or bfloat16, got %s" % t.dtype)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, name, dtype=None):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, dev_err=None, stream=None):
+    """Write the new tokens' K/V ([T, Hkv, D]) into their slots of the caches."""
+    for n, t in (("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    num_blocks, hkv, bs, d = k_cache.shape
+    t = key.shape[0]
+    if key.shape != (t, hkv, d) or value.shape != key.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if slot_mapping.shape != (t,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    _check(_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                              _ptr(slot_mapping), t, hkv, d, bs, num_blocks,
+                              _dtype_code(k_cache), _ptr(dev_err), _stream(stream)),
+           "reshape_and_cache")
+
+
+def copy_blocks(k_cache, v_cache, block_mapping, dev_err=None, stream=None):
+    """Copy whole blocks (K and V) for each (src, dst) row of block_mapping [P, 2]."""
+    _dev(k_cache, "k_cache")
+    _dev(v_cache, "v_cache")
+    _dev(block_mapping, "block_mapping", torch.int64)
+    num_blocks, hkv, bs, d = k_cache.shape
+    p = block_mapping.shape[0] if block_mapping.numel() else 0
+    if block_mapping.numel() and block_mapping.shape != (p, 2):
+        raise ValueError("block_mapping must be [num_pairs, 2]")
+    _check(_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), p, hkv, d, bs,
+                        num_blocks, _dtype_code(k_cache), _ptr(dev_err), _stream(stream)),
+           "copy_blocks")
+
+
+def partition_size(num_seqs, num_kv_heads, block_size, max_context_len, requested=0):
+    return _partition_size(num_seqs, num_kv_heads, block_size, max_context_len, requested)
+
+
+def workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                    partition_size=0):
+    return _workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_context_len, partition_size)
+
+
+def alloc_workspace(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                    partition_size=0, device=None):
+    n = workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                        max_context_len, partition_size)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                      block_size, max_context_len, partition_size=0, workspace=None,
+                      dev_err=None, stream=None):
+    """Paged decode attention; writes out [S, H, D].  See include/pagedkv.h."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    s, h, d = q.shape
+    num_blocks, hkv, bs, dk = k_cache.shape
+    if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if q.dtype != k_cache.dtype or out.dtype != q.dtype:
+        raise TypeError("q, out and caches must share a dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    if workspace is None:
+        need = workspace_bytes(s, h, hkv, d, bs, max_context_len, partition_size)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if need else None
+    ws_ptr = _ptr(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_paged_attn_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                              _ptr(block_tables), _ptr(context_lens), float(scale), s, h, hkv, d,
+                              bs, block_tables.shape[1], max_context_len, num_blocks,
+                              _dtype_code(q), partition_size, ws_ptr, ws_bytes, _ptr(dev_err),
+                              _stream(stream)),
+           "paged_attn_decode")
+
+
+def staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                  num_new_tokens, num_pairs):
+    return _staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                          num_new_tokens, num_pairs)
+
+
+def decode_step_host(out_host, q_host, key_host, value_host, slot_mapping_host,
+                     block_mapping_host, block_tables_host, context_lens_host, k_cache, v_cache,
+                     scale, max_context_len, staging, workspace=None, partition_size=0,
+                     dev_err=None, stream=None):
+    """One whole step from host tensors (pinned for async copies); see the header."""
+    _dev(k_cache, "k_cache")
+    _dev(v_cache, "v_cache")
+    _dev(staging, "staging")
+    for n, t in (("out_host", out_host), ("q_host", q_host), ("key_host", key_host),
+                 ("value_host", value_host), ("slot_mapping_host", slot_mapping_host),
+                 ("block_mapping_host", block_mapping_host),
+                 ("block_tables_host", block_tables_host),
+                 ("context_lens_host", context_lens_host)):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous host tensor" % n)
+    s, h, d = q_host.shape
+    num_blocks, hkv, bs, _ = k_cache.shape
+    t = key_host.shape[0]
+    p = block_mapping_host.shape[0] if block_mapping_host.numel() else 0
+    ws_ptr = _ptr(workspace)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(_decode_step_host(_ptr(out_host), _ptr(q_host), _ptr(key_host), _ptr(value_host),
+                             _ptr(slot_mapping_host), t, _ptr(block_mapping_host), p,
+                             _ptr(block_tables_host), _ptr(context_lens_host), _ptr(k_cache),
+                             _ptr(v_cache), float(scale), s, h, hkv, d, bs,
+                             block_tables_host.shape[1], max_context_len, num_blocks,
+                             _dtype_code(k_cache), partition_size, _ptr(staging),
+                             staging.numel(), ws_ptr, ws_bytes, _ptr(dev_err), _stream(stream)),
+           "decode_step_host")
+
+
+class BlockAllocator:
+    """Host block allocator (free list, refcounts, fork, copy-on-write)."""
+
+    def __init__(self, num_blocks, block_size, free_order=None):
+        self._order = None
+        if free_order is not None:
+            self._order = (ctypes.c_int32 * num_blocks)(*[int(b) for b in free_order])
+        self._h = _alloc_create(num_blocks, block_size, self._order)
+        if not self._h:
+            raise PagedKVError(ERR_INVALID_ARG, "BlockAllocator")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if self._h:
+            _alloc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id, num_tokens):
+        _check(_alloc_add_seq(self._h, seq_id, num_tokens), "add_seq")
+
+    def fork(self, parent, child):
+        _check(_alloc_fork(self._h, parent, child), "fork")
+
+    def append_slot(self, seq_id):
+        slot, src, dst = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(_alloc_append_slot(self._h, seq_id, ctypes.byref(slot), ctypes.byref(src),
+                                  ctypes.byref(dst)), "append_slot")
+        return slot.value, src.value, dst.value
+
+    def append_slots(self, seq_ids):
+        n = len(seq_ids)
+        ids = (ctypes.c_int64 * max(n, 1))(*seq_ids)
+        slots = (ctypes.c_int64 * max(n, 1))()
+        pairs = (ctypes.c_int64 * max(2 * n, 2))()
+        ncow, done = ctypes.c_int(), ctypes.c_int()
+        _check(_alloc_append_slots(self._h, ids, n, slots, pairs, ctypes.byref(ncow),
+                                   ctypes.byref(done)), "append_slots")
+        return list(slots[:n]), [(pairs[2 * k], pairs[2 * k + 1]) for k in range(ncow.value)]
+
+    def free_seq(self, seq_id):
+        _check(_alloc_free_seq(self._h, seq_id), "free_seq")
+
+    def block_table(self, seq_ids, max_blocks):
+        n = len(seq_ids)
+        ids = (ctypes.c_int64 * max(n, 1))(*seq_ids)
+        out = (ctypes.c_int32 * max(n * max_blocks, 1))()
+        _check(_alloc_block_table(self._h, ids, n, max_blocks, out), "block_table")
+        flat = list(out[:n * max_blocks])
+        return [flat[i * max_blocks:(i + 1) * max_blocks] for i in range(n)]
+
+    def context_lens(self, seq_ids):
+        n = len(seq_ids)
+        ids = (ctypes.c_int64 * max(n, 1))(*seq_ids)
+        out = (ctypes.c_int32 * max(n, 1))()
+        _check(_alloc_context_lens(self._h, ids, n, out), "context_lens")
+        return list(out[:n])
+
+    def num_free(self):
+        return _alloc_num_free(self._h)
+
+    def refcount(self, block):
+        return _alloc_refcount(self._h, block)
+
+    def seq_len(self, seq_id):
+        return _alloc_seq_len(self._h, seq_id)
+
+    def seq_num_blocks(self, seq_id):
+        return _alloc_seq_num_blocks(self._h, seq_id)
+
+    def usage(self):
+        tokens, blocks = ctypes.c_int64(), ctypes.c_int64()
+        _check(_alloc_usage(self._h, ctypes.byref(tokens), ctypes.byref(blocks)), "usage")
+        return tokens.value, blocks.value

@@ -1,0 +1,102 @@
+"""The C ABI library loads, exports every symbol include/pagedkv.h declares,
+and validates arguments on the host (no GPU needed: every case below is
+rejected before anything is enqueued)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names.update(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_394_b200 import pagedkv
+    return ctypes.CDLL(pagedkv.LIB_PATH)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 20
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_version_and_status_strings():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    assert "sm_100a" in pk.version()
+    for s in range(6):
+        assert pk._status_string(s).decode() != "unknown status"
+    assert pk._status_string(99).decode() == "unknown status"
+
+
+def test_host_validation_without_gpu():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    null = None
+    # reshape_and_cache: unsupported head_dim, negative tokens, null pointers
+    assert pk._reshape_and_cache(null, null, null, null, null, 4, 2, 96, 16, 8, 0, null, null) == pk.ERR_UNSUPPORTED
+    assert pk._reshape_and_cache(null, null, null, null, null, -1, 2, 64, 16, 8, 0, null, null) == pk.ERR_INVALID_ARG
+    assert pk._reshape_and_cache(null, null, null, null, null, 4, 2, 64, 16, 8, 0, null, null) == pk.ERR_INVALID_ARG
+    assert pk._reshape_and_cache(null, null, null, null, null, 0, 2, 64, 16, 8, 0, null, null) == pk.OK
+    assert pk._reshape_and_cache(null, null, null, null, null, 4, 2, 64, 16, 8, 7, null, null) == pk.ERR_INVALID_ARG
+    # misaligned pointers
+    bad = ctypes.c_void_p(0x1008)
+    good = ctypes.c_void_p(0x1000)
+    assert pk._reshape_and_cache(bad, good, good, good, good, 4, 2, 64, 16, 8, 0, null, null) == pk.ERR_INVALID_ARG
+    # copy_blocks
+    assert pk._copy_blocks(null, null, null, 0, 2, 64, 16, 8, 0, null, null) == pk.OK
+    assert pk._copy_blocks(null, null, null, 3, 2, 64, 16, 8, 0, null, null) == pk.ERR_INVALID_ARG
+    assert pk._copy_blocks(good, good, good, 3, 2, 64, 24, 8, 0, null, null) == pk.ERR_UNSUPPORTED
+    # decode: group 3 unsupported, heads not a multiple, partition not a multiple
+    args = lambda **kw: dict(dict(s=2, h=6, hkv=2, d=64, bs=16, mb=4, mc=64, n=8, part=0), **kw)
+
+    def dec(a, ptr=good, ws=None, wsb=0):
+        return pk._paged_attn_decode(ptr, ptr, ptr, ptr, ptr, ptr, 0.125, a["s"], a["h"], a["hkv"],
+                                     a["d"], a["bs"], a["mb"], a["mc"], a["n"], 0, a["part"], ws,
+                                     wsb, null, null)
+    assert dec(args()) == pk.ERR_UNSUPPORTED              # G = 3
+    assert dec(args(h=5)) == pk.ERR_INVALID_ARG            # 5 % 2 != 0
+    assert dec(args(h=4, part=24)) == pk.ERR_INVALID_ARG   # not a multiple of 16
+    assert dec(args(h=4, mc=65)) == pk.ERR_INVALID_ARG     # > max_blocks * block_size
+    assert dec(args(h=4, s=0)) == pk.OK
+    assert dec(args(h=4), ptr=null) == pk.ERR_INVALID_ARG
+    assert dec(args(h=4), ptr=bad) == pk.ERR_INVALID_ARG
+    assert dec(args(h=4, part=16)) == pk.ERR_WORKSPACE     # split needs a workspace
+    # non-finite scale
+    assert pk._paged_attn_decode(good, good, good, good, good, good, float("nan"), 2, 4, 2, 64, 16,
+                                 4, 64, 8, 0, 0, null, 0, null, null) == pk.ERR_INVALID_ARG
+
+
+def test_partition_and_workspace_queries():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    # short contexts over many (sequence, kv head) units: single pass
+    assert pk.partition_size(64, 32, 16, 2048) >= 2048
+    assert pk.workspace_bytes(64, 32, 32, 128, 16, 2048) == 0
+    # long contexts: 512-token partitions
+    assert pk.partition_size(8, 40, 16, 32768) == 512
+    n = 8 * 40 * 64
+    assert pk.workspace_bytes(8, 40, 40, 128, 16, 32768) >= n * (128 + 2) * 4
+    # an explicit request is honoured
+    assert pk.partition_size(64, 32, 16, 2048, 256) == 256
+    assert pk.workspace_bytes(64, 32, 32, 128, 16, 2048, 256) >= 64 * 32 * 8 * 130 * 4
+    assert pk.workspace_bytes(64, 32, 32, 128, 16, 2048, 24) == 0   # invalid request
+
+
+def test_staging_bytes_covers_inputs():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    s, h, hkv, d, mb, t, p = 64, 32, 32, 128, 128, 64, 3
+    need = 2 * s * h * d * 2 + 2 * t * hkv * d * 2 + t * 8 + p * 16 + s * mb * 4 + s * 4
+    assert pk.staging_bytes(s, h, hkv, d, mb, t, p) >= need

@@ -1,0 +1,120 @@
+"""The C++ host block allocator against the oracle block manager: identical
+slots, copy pairs, tables, refcounts and free counts (bit-exact integer work)
+on random operation traces, plus its error statuses."""
+
+import numpy as np
+import pytest
+
+from oracle.block_manager import AllocError, BlockManager
+
+pk = pytest.importorskip("paged_kv_cache_394_b200.pagedkv")
+
+STATUS = {"INVALID_ARG": 1, "OUT_OF_BLOCKS": 5}
+
+
+def both(oracle_call, lib_call):
+    """Run one operation on both; they must agree on success, result and error."""
+    try:
+        expect = oracle_call()
+        err = None
+    except AllocError as e:
+        expect, err = None, STATUS[e.status]
+    try:
+        got = lib_call()
+        got_err = None
+    except pk.PagedKVError as e:
+        got, got_err = None, e.status
+    assert got_err == err
+    assert got == expect
+    return err is None
+
+
+@pytest.mark.parametrize("seed,num_blocks,bs", [(1, 40, 16), (2, 97, 32), (3, 12, 16), (4, 300, 16)])
+def test_random_traces_match_oracle(seed, num_blocks, bs):
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(num_blocks)
+    ref = BlockManager(num_blocks, bs, free_order=order)
+    lib = pk.BlockAllocator(num_blocks, bs, free_order=order)
+    live, next_id = [], 0
+    for _ in range(1500):
+        op = int(rng.integers(0, 12))
+        if op < 2 or not live:
+            n = int(rng.integers(0, 5 * bs))
+            if both(lambda: ref.add_seq(next_id, n), lambda: lib.add_seq(next_id, n)):
+                live.append(next_id)
+            next_id += 1
+        elif op < 4:
+            parent = live[int(rng.integers(len(live)))]
+            if both(lambda: ref.fork(parent, next_id), lambda: lib.fork(parent, next_id)):
+                live.append(next_id)
+            next_id += 1
+        elif op < 9:
+            s = live[int(rng.integers(len(live)))]
+            both(lambda: ref.append_slot(s), lambda: lib.append_slot(s))
+        elif op < 10:
+            batch = [live[int(i)] for i in rng.integers(0, len(live), size=int(rng.integers(1, 6)))]
+
+            def ref_batch():
+                slots, pairs = [], []
+                for s in batch:
+                    slot, a, b = ref.append_slot(s)
+                    slots.append(slot)
+                    if a >= 0:
+                        pairs.append((a, b))
+                return slots, pairs
+            # a batch that runs out part-way leaves both in the same partial state
+            try:
+                expect = ref_batch()
+            except AllocError as e:
+                expect = e.status
+            try:
+                got = lib.append_slots(batch)
+            except pk.PagedKVError as e:
+                got = {1: "INVALID_ARG", 5: "OUT_OF_BLOCKS"}[e.status]
+            assert got == expect
+        elif op < 11:
+            s = live.pop(int(rng.integers(len(live))))
+            both(lambda: ref.free_seq(s), lambda: lib.free_seq(s))
+        else:
+            bogus = next_id + 1000
+            both(lambda: ref.free_seq(bogus), lambda: lib.free_seq(bogus))
+        # full state comparison
+        assert lib.num_free() == ref.num_free()
+        if live:
+            mb = max(1, max(len(ref.seq_blocks(s)) for s in live))
+            assert lib.block_table(live, mb) == ref.block_table(live, mb)
+            assert lib.context_lens(live) == [ref.seq_len(s) for s in live]
+    assert [lib.refcount(b) for b in range(num_blocks)] == ref.refcount
+    tokens, blocks = lib.usage()
+    if blocks:
+        assert tokens / (blocks * bs) == pytest.approx(ref.physical_utilization(), abs=1e-15)
+
+
+def test_parallel_sampling_scenario():
+    lib = pk.BlockAllocator(200, 16)
+    lib.add_seq(0, 1020)
+    for c in range(1, 8):
+        lib.fork(0, c)
+    slots, pairs = lib.append_slots(list(range(8)))
+    assert len(pairs) == 7 and len(set(d for _, d in pairs)) == 7
+    assert all(s % 16 == 1020 % 16 for s in slots)
+    assert lib.num_free() == 200 - 64 - 7
+
+
+def test_error_statuses():
+    with pytest.raises(pk.PagedKVError):
+        pk.BlockAllocator(0, 16)
+    with pytest.raises(pk.PagedKVError):
+        pk.BlockAllocator(4, 16, free_order=[0, 0, 1, 2])
+    a = pk.BlockAllocator(2, 16)
+    a.add_seq(7, 20)
+    with pytest.raises(pk.PagedKVError) as e:
+        a.add_seq(8, 1)
+    assert e.value.status == pk.ERR_OUT_OF_BLOCKS
+    with pytest.raises(pk.PagedKVError) as e:
+        a.add_seq(7, 1)
+    assert e.value.status == pk.ERR_INVALID_ARG
+    with pytest.raises(pk.PagedKVError):
+        a.block_table([7], 1)
+    assert a.refcount(5) == -1 and a.seq_len(99) == -1
+    assert a.seq_num_blocks(7) == 2

@@ -149,10 +149,12 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
         time.sleep(0.3)
+        self.t_start = time.time()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.t_stop = time.time()
         time.sleep(0.25)
         self.proc.terminate()
         try:
@@ -172,9 +174,12 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
         power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(power) if power else None}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+               "reasons": reasons, "samples": len(rows),
+               "power_w_max": max(power) if power else None}
+        if self.t_stop - self.t_start < 0.6:
+            out["note"] = "timed region shorter than the 200 ms sampling period"
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -458,8 +463,8 @@ def run_reference(args):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--partition", type=int, default=None,

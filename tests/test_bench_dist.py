@@ -1,0 +1,93 @@
+"""Multi-process plumbing of bench.py on CPU: gloo, world size 2.
+
+Each rank runs its own replica batch (weak scaling, no collective on the data
+path); the ranks only meet at the barrier and in the max / sum of timings.
+"""
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w = bench.init_dist("gloo", timeout_s=60)
+    bench.barrier()
+    # a per-rank "step time" and byte count, as the bench aggregates them
+    t = bench.max_over_ranks(1.0 + r)
+    b = bench.sum_over_ranks(100.0 * (r + 1))
+    seed = bench.replica_seed(395, r)
+    from paged_kv_cache_394_b200 import workloads as W
+    wl = W.make("tiny", seed=seed)
+    out.put((r, w, t, b, seed, int(wl.q.view("int16").astype("int64").sum())))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_rank_plumbing():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r for r, *_ in res] == [0, 1]
+    assert all(w == 2 for _, w, *_ in res)
+    assert all(t == 2.0 for _, _, t, *_ in res)        # max over ranks
+    assert all(x[3] == 300.0 for x in res)            # sum over ranks
+    seeds = {x[4] for x in res}
+    assert len(seeds) == 2                              # independent replicas
+    assert res[0][5] != res[1][5]
+
+
+def test_single_process_is_identity():
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.sum_over_ranks(2.0) == 2.0
+
+
+def test_step_bytes_counts_kv_q_out_and_writes():
+    from paged_kv_cache_394_b200 import workloads as W
+    w = W.make("tiny")
+    kv = 2 * int(w.context_lens.sum()) * w.num_kv_heads * w.head_dim * 2
+    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * 2
+    assert bench.decode_bytes(w) == kv + qo
+    assert bench.write_bytes(w) == 4 * len(w.slot_mapping) * w.num_kv_heads * w.head_dim * 2 \
+        + 8 * len(w.slot_mapping)
+    assert bench.step_bytes(w) == bench.decode_bytes(w) + bench.write_bytes(w)
+
+
+def test_reference_arm_non_zero_rank_does_nothing(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.run_reference(bench.parse_args(["--impl", "reference", "--steps", "1"]))
+    assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("name", ["tiny"])
+def test_reference_arm_prints_one_line(monkeypatch, capsys, name):
+    import json
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    bench.run_reference(bench.parse_args(["--impl", "reference", "--workload", name,
+                                          "--steps", "2", "--warmup", "3",
+                                          "--cpu-seconds", "1"]))
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"

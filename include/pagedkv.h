@@ -23,7 +23,9 @@
  *    marks a padding token.
  *  - Ownership: the caller owns every buffer.  The library never allocates or
  *    frees device memory; scratch for split-K decode ("workspace") and for the
- *    host-buffer step ("staging") is passed in by the caller.
+ *    host-buffer step ("staging") is passed in by the caller (except for
+ *    pkv_paged_attn_decode_static_ws, whose scratch is a fixed array inside
+ *    the library).
  *  - Execution: device work is enqueued asynchronously on `stream` (a
  *    cudaStream_t passed as void*; NULL is the legacy default stream).  No
  *    entry point synchronizes.  All device pointers must belong to the
@@ -163,6 +165,39 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
                                  int num_blocks, pkv_dtype dtype, int partition_size,
                                  void* workspace, size_t workspace_bytes, unsigned* dev_err,
                                  void* stream);
+
+/*
+ * pkv_paged_attn_decode_static_ws — pkv_paged_attn_decode without a caller
+ * workspace.  No counterpart in the source pages: it exists for callers that
+ * cannot allocate device memory, such as a plugin inside a host application
+ * that owns all device allocations, or a serving loop that must not call
+ * cudaMalloc after start-up (cudaMalloc can synchronise the device).
+ *
+ * Arguments and results are those of pkv_paged_attn_decode; only the split-K
+ * scratch differs.  It is a fixed array of PKV_STATIC_WORKSPACE_BYTES inside
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  This entry point allocates and frees nothing.
+ *  - If the call would need more scratch than that (see
+ *    pkv_paged_attn_workspace_bytes), it returns PKV_ERR_WORKSPACE and
+ *    enqueues nothing.  16 MiB holds, e.g., 8 sequences x 40 heads x 64
+ *    partitions of head_dim 128.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.  Later calls on the device only read the cache.
+ *  - All calls on a device share the one array, and it keeps whatever the
+ *    last call left there.  Nothing in it needs to start at zero: every value
+ *    a call reads back was written earlier in the same call.  Calls that
+ *    overlap on the GPU (different streams, or different host threads without
+ *    ordering between them) race on the array; serialise them.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_tables,
+                                           const int32_t* context_lens, float scale,
+                                           int num_seqs, int num_heads, int num_kv_heads,
+                                           int head_dim, int block_size, int max_blocks_per_seq,
+                                           int max_context_len, int num_blocks, pkv_dtype dtype,
+                                           int partition_size, unsigned* dev_err, void* stream);
 
 /*
  * pkv_decode_step_host — one whole decode step from HOST buffers: copies the

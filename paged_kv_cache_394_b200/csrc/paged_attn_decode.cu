@@ -717,3 +717,70 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
   rcfg.dynamicSmemBytes = 0;
   return cuda_status(cudaLaunchKernelEx(&rcfg, reduce_entry(head_dim, dtype), p));
 }
+
+// ---------------------------------------------------------------------------
+// Decode whose split-K scratch lives in a fixed device array.
+//
+// For callers that cannot allocate device memory: a plugin loaded into a host
+// application that owns every device allocation and hands out none, or a
+// serving loop that must not call cudaMalloc once it is running, because
+// cudaMalloc can synchronise the device and stall every stream in flight.
+// The caller still passes all inputs and outputs; only the scratch is fixed.
+// ---------------------------------------------------------------------------
+
+// The split-K scratch of pkv_paged_attn_decode_static_ws.  Every GPU on which
+// this library is loaded keeps these PKV_STATIC_WORKSPACE_BYTES until the
+// process exits.  In host code this name is only a stand-in for the device
+// symbol, never a device address: the kernels get the address that
+// cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char pkv_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+#include <mutex>
+
+namespace pkv {
+namespace {
+constexpr int kMaxStaticWsDevices = 64;
+void* g_static_ws_addr[kMaxStaticWsDevices] = {};
+std::mutex g_static_ws_mutex;
+
+// Device address of pkv_static_workspace on the current device, looked up
+// once per device (with that device current) and cached.
+pkv_status static_workspace_address(void** addr) {
+  int dev = 0;
+  pkv_status st = cuda_status(cudaGetDevice(&dev));
+  if (st != PKV_OK) return st;
+  if (dev < 0 || dev >= kMaxStaticWsDevices) return PKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (g_static_ws_addr[dev] == nullptr) {
+    void* p = nullptr;
+    st = cuda_status(cudaGetSymbolAddress(&p, pkv_static_workspace));
+    if (st != PKV_OK) return st;
+    g_static_ws_addr[dev] = p;
+  }
+  *addr = g_static_ws_addr[dev];
+  return PKV_OK;
+}
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attn_decode_static_ws(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, float scale, int num_seqs,
+    int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+    int max_context_len, int num_blocks, pkv_dtype dtype, int partition_size, unsigned* dev_err,
+    void* stream) {
+  using namespace pkv;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || block_size <= 0 ||
+      max_context_len < 0 || partition_size < 0)
+    return PKV_ERR_INVALID_ARG;
+  const size_t need = pkv_paged_attn_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                     block_size, max_context_len, partition_size);
+  if (need > PKV_STATIC_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const pkv_status st = static_workspace_address(&ws);
+  if (st != PKV_OK) return st;
+  return pkv_paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                               num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                               max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                               partition_size, ws, PKV_STATIC_WORKSPACE_BYTES, dev_err, stream);
+}

@@ -45,6 +45,10 @@ _partition_size = _proto("pkv_paged_attn_partition_size", _i, _i, _i, _i, _i, _i
 _workspace_bytes = _proto("pkv_paged_attn_workspace_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
 _paged_attn_decode = _proto("pkv_paged_attn_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i,
                             _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
+_paged_attn_decode_static_ws = _proto("pkv_paged_attn_decode_static_ws", _i, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                     _vp)
+STATIC_WORKSPACE_BYTES = 16 << 20
 _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
 _decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
                            _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
@@ -188,6 +192,30 @@ def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scal
                               _dtype_code(q), partition_size, ws_ptr, ws_bytes, _ptr(dev_err),
                               _stream(stream)),
            "paged_attn_decode")
+
+
+def paged_attn_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                num_kv_heads, block_size, max_context_len, partition_size=0,
+                                dev_err=None, stream=None):
+    """paged_attn_decode with its split-K scratch in the library's fixed device
+    array (no allocation anywhere).  For callers that cannot allocate device
+    memory; see include/pagedkv.h for the size limit and the sharing rules."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    s, h, d = q.shape
+    num_blocks, hkv, bs, dk = k_cache.shape
+    if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if q.dtype != k_cache.dtype or out.dtype != q.dtype:
+        raise TypeError("q, out and caches must share a dtype")
+    _check(_paged_attn_decode_static_ws(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(block_tables), _ptr(context_lens), float(scale), s,
+                                        h, hkv, d, bs, block_tables.shape[1], max_context_len,
+                                        num_blocks, _dtype_code(q), partition_size,
+                                        _ptr(dev_err), _stream(stream)),
+           "paged_attn_decode_static_ws")
 
 
 def staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,

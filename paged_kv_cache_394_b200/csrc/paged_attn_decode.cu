@@ -32,9 +32,12 @@
 //    unnormalised output) to the workspace and a reduce kernel merges them;
 //    a sequence with a single partition is written directly.
 //  * No waits on other CTAs anywhere; mbarrier waits are bounded in time.
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "host_common.h"
@@ -244,6 +247,55 @@ __device__ __forceinline__ void process_block(WarpState<Tr>& st, const typename 
   }
 }
 
+// Merges the W warps' (max, sum, unnormalised output) of one CTA and stores
+// the result: the normalised output when the sequence has one partition,
+// else the partition's (m, l, o) triple in the workspace.
+//   cm, cl: [W][G] per-warp running max and exp-sum (base-2 logits)
+//   cacc:   [W][G][D] per-warp unnormalised outputs
+template <int W, int G, int D, class DT>
+__device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, const float* cm,
+                                                      const float* cl, const float* cacc,
+                                                      int seq, int kvh, int part, bool direct) {
+  using T = typename DT::T;
+  constexpr int NC = D / 8;
+  for (int idx = threadIdx.x; idx < G * NC; idx += W * 32) {
+    const int g = idx / NC;
+    const int cc = idx % NC;
+    float big_m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < W; ++w) big_m = fmaxf(big_m, cm[w * G + g]);
+    float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float den = 0.f;
+    if (big_m != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const float f = exp2_approx(cm[w * G + g] - big_m);
+        den = fmaf(f, cl[w * G + g], den);
+        const float* a = cacc + (w * G + g) * D + cc * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) num[e] = fmaf(f, a[e], num[e]);
+      }
+    }
+    const int head = kvh * G + g;
+    if (direct) {
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) num[e] *= inv;
+      T* o = static_cast<T*>(p.out) + (static_cast<size_t>(seq) * p.num_heads + head) * D + cc * 8;
+      *reinterpret_cast<uint4*>(o) = pack8(num, DT());
+    } else {
+      const size_t slot = (static_cast<size_t>(seq) * p.num_heads + head) * p.max_parts + part;
+      float4* o = reinterpret_cast<float4*>(p.ws_out + slot * D + cc * 8);
+      o[0] = make_float4(num[0], num[1], num[2], num[3]);
+      o[1] = make_float4(num[4], num[5], num[6], num[7]);
+      if (cc == 0) {
+        p.ws_max[slot] = big_m;
+        p.ws_sum[slot] = den;
+      }
+    }
+  }
+}
+
 template <class Tr>
 __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeParams p) {
   using T = typename Tr::T;
@@ -402,42 +454,313 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
     }
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < G * NC; idx += Tr::THREADS) {
-    const int g = idx / NC;
-    const int cc = idx % NC;
-    float big_m = -INFINITY;
+  merge_warps_and_store<W, G, D, typename Tr::DT>(p, cm, cl, cacc, seq, kvh, part, direct);
+}
+
+// ---------------------------------------------------------------------------
+// Grouped-query decode on the tensor cores (G >= 2).
+//
+// With G query heads per kv head, q.K and P.V carry G multiply-adds per
+// cached element; on the CUDA cores that makes the kernel instruction-bound
+// (about 1,700 warp instructions per 16 tokens at G = 8).  Here each warp runs
+// them as mma.sync m16n8k16 with the 16 tokens of a sub-block as M and the
+// heads as N (N = 8 covers G <= 8 with no padding at G = 8):
+//   q.K:  S^T[t][n] = sum_d K[t][d] q[n][d]      A = K   (ldmatrix)
+//   P.V:  O^T[d][n] += sum_t V[t][d] P[n][t]     A = V^T (ldmatrix.trans),
+//                                                B = P, transposed in registers
+//                                                from the S^T accumulator by movmatrix
+// K and V of a (block, kv head) reach shared memory by 2-D tiled TMA loads
+// with the 128-byte swizzle: boxes of 16 rows x 64 elements, so ldmatrix rows
+// fall in distinct banks.  A stage is one 16-token sub-block (a block of 32
+// is two stages).  The ring, the table slice, the bounded waits, the split-K
+// partitions and the final merge are as in paged_decode_kernel.
+// ---------------------------------------------------------------------------
+template <int D_, int BS_, int G_, class DT_, int W_, int NS_>
+struct MmaTraits {
+  static constexpr int D = D_, BS = BS_, G = G_, W = W_, NS = NS_;
+  using DT = DT_;
+  using T = typename DT::T;
+  static constexpr int SUB = 16;                   // tokens per stage (the mma M)
+  static constexpr int SUBS_PER_BLOCK = BS / SUB;
+  static constexpr int BOXES = D / 64;             // 128-byte-wide boxes per row
+  static constexpr int BOX_BYTES = SUB * 128;      // one 16 x 64 box
+  static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
+  static constexpr int KSTEPS = D / 16;            // q.K k-steps = P.V m-tiles
+  static constexpr int THREADS = W * 32;
+  static constexpr int RING_BYTES = W * NS * STAGE_BYTES;
+  static constexpr int BAR_BYTES = W * NS * 8;
+  static constexpr int COMBINE_BYTES = W * G * (D + 2) * 4;
+  static_assert(G >= 2 && G <= 8, "tensor-core path serves 2..8 heads per kv head");
+  static_assert(BS % SUB == 0 && D % 64 == 0, "shape");
+  static_assert(COMBINE_BYTES <= RING_BYTES, "combine scratch reuses the ring");
+  static size_t smem_bytes(int part_blocks) {
+    return 1024 + static_cast<size_t>(RING_BYTES) + BAR_BYTES +
+           static_cast<size_t>(part_blocks) * 4;
+  }
+};
+
+// Byte offset of 16-byte chunk `ch` of row `t` in a tile of BOXES swizzled
+// 16 x 128-byte boxes (chunk index XOR row % 8, per 1024-byte swizzle atom).
+__device__ __forceinline__ uint32_t swizzled(int t, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * 2048 + t * 128 + (((ch & 7) ^ (t & 7)) << 4));
+}
+
+template <class Tr>
+__device__ __forceinline__ void mma_sub_block(uint32_t kt, uint32_t vt, int valid,
+                                              const uint32_t (&qf)[Tr::KSTEPS][2],
+                                              float (&acc)[Tr::KSTEPS][4], float (&m)[2],
+                                              float (&l)[2], float qscale, int lane) {
+  constexpr int KS = Tr::KSTEPS;
+  const int j = lane >> 3;  // which 8x8 matrix this lane addresses
+  const int r = lane & 7;
+  // ---- q.K: S^T (16 tokens x 8 heads) ----------------------------------------
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const int t = ((j & 1) << 3) + r;
 #pragma unroll
-    for (int w = 0; w < W; ++w) big_m = fmaxf(big_m, cm[w * G + g]);
-    float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float den = 0.f;
-    if (big_m != -INFINITY) {
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(kt + swizzled(t, 2 * ks + (j >> 1)), a);
+      mma_16816(s, a, qf[ks][0], qf[ks][1], typename Tr::DT());
+    }
+  }
+  // lane holds tokens t0 = lane/4 and t0 + 8, heads 2(lane%4) and 2(lane%4)+1
+  const int t0 = lane >> 2;
+  float x0 = s[0] * qscale, x1 = s[1] * qscale, x2 = s[2] * qscale, x3 = s[3] * qscale;
+  if (valid < Tr::SUB) {
+    if (t0 >= valid) x0 = x1 = -INFINITY;
+    if (t0 + 8 >= valid) x2 = x3 = -INFINITY;
+  }
+  // ---- online softmax per head: reduce over the 8 lanes sharing lane % 4 ------
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        const float f = exp2_approx(cm[w * G + g] - big_m);
-        den = fmaf(f, cl[w * G + g], den);
-        const float* a = cacc + (w * G + g) * D + cc * 8;
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
+  }
+  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+  const float a0 = exp2_approx(m[0] - mn0), a1 = exp2_approx(m[1] - mn1);
+  const float p0 = exp2_approx(x0 - mn0), p1 = exp2_approx(x1 - mn1);
+  const float p2 = exp2_approx(x2 - mn0), p3 = exp2_approx(x3 - mn1);
+  float s0 = p0 + p2, s1 = p1 + p3;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) num[e] = fmaf(f, a[e], num[e]);
+  for (int o = 4; o < 32; o <<= 1) {
+    s0 += __shfl_xor_sync(kFullMask, s0, o);
+    s1 += __shfl_xor_sync(kFullMask, s1, o);
+  }
+  l[0] = l[0] * a0 + s0;
+  l[1] = l[1] * a1 + s1;
+  m[0] = mn0;
+  m[1] = mn1;
+  if (__any_sync(kFullMask, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      acc[mt][0] *= a0;
+      acc[mt][1] *= a1;
+      acc[mt][2] *= a0;
+      acc[mt][3] *= a1;
+    }
+  }
+  // ---- P as the B operand: transpose the S^T fragments in registers -----------
+  // bf16 keeps 8 mantissa bits, too few for p near 1 at the required accuracy,
+  // so bf16 P is split as hi + lo (both bf16, |P - hi - lo| <= 2^-18 P) and
+  // P.V runs twice; fp16 P (11 bits) is used as is.
+  constexpr bool kSplitP = std::is_same<typename Tr::DT, Bf16>::value;
+  const uint32_t h01 = pack2(p0, p1, typename Tr::DT());
+  const uint32_t h23 = pack2(p2, p3, typename Tr::DT());
+  const uint32_t b0 = movmatrix_trans(h01);
+  const uint32_t b1 = movmatrix_trans(h23);
+  uint32_t b0_lo = 0, b1_lo = 0;
+  if constexpr (kSplitP) {
+    b0_lo = movmatrix_trans(pack2(p0 - __uint_as_float(h01 << 16),
+                                  p1 - __uint_as_float(h01 & 0xffff0000u), Bf16()));
+    b1_lo = movmatrix_trans(pack2(p2 - __uint_as_float(h23 << 16),
+                                  p3 - __uint_as_float(h23 & 0xffff0000u), Bf16()));
+  }
+  // ---- rows past the context hold stale data (maybe NaN): zero them in V so
+  //      that 0 * V stays 0 inside the tensor-core sum
+  if (valid < Tr::SUB) {
+    const int chunks = (Tr::SUB - valid) * Tr::BOXES * 8;
+    for (int i = lane; i < chunks; i += 32) {
+      const int row = valid + i / (Tr::BOXES * 8);
+      const int rem = i % (Tr::BOXES * 8);
+      const uint32_t at = vt + (rem >> 3) * 2048 + row * 128 + ((rem & 7) << 4);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(at), "r"(0u) : "memory");
+    }
+    __syncwarp();
+  }
+  // ---- P.V: O^T (D dims x 8 heads) -------------------------------------------
+  {
+    const int t = ((j >> 1) << 3) + r;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_trans(vt + swizzled(t, 2 * mt + (j & 1)), a);
+      mma_16816(acc[mt], a, b0, b1, typename Tr::DT());
+      if constexpr (kSplitP) mma_16816(acc[mt], a, b0_lo, b1_lo, typename Tr::DT());
+    }
+  }
+}
+
+template <class Tr>
+__global__ void __launch_bounds__(Tr::THREADS)
+    paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
+                            const __grid_constant__ CUtensorMap vmap) {
+  using T = typename Tr::T;
+  constexpr int W = Tr::W, NS = Tr::NS, G = Tr::G, D = Tr::D, BS = Tr::BS, KS = Tr::KSTEPS;
+  constexpr int SPB = Tr::SUBS_PER_BLOCK;
+  extern __shared__ unsigned char smem_raw[];
+  // the 128-byte swizzle needs 1024-byte-aligned boxes
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
+  int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
+
+  const int part = blockIdx.x % p.max_parts;
+  const int unit = blockIdx.x / p.max_parts;
+  const int kvh = unit % p.num_kv_heads;
+  const int seq = unit / p.num_kv_heads;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  grid_dependency_wait();
+  trigger_dependents();
+
+  const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
+  int ctx = p.context_lens[seq];
+  if (ctx < 0 || ctx > ctx_cap) {
+    if (threadIdx.x == 0 && part == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
+    ctx = min(max(ctx, 0), ctx_cap);
+  }
+  const int nblk = (ctx + BS - 1) / BS;
+  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
+  if (part >= max(nparts, 1)) return;
+  const bool direct = nparts <= 1;
+  const int blk_begin = part * p.part_blocks;
+  const int nb = min(nblk, blk_begin + p.part_blocks) - blk_begin;
+  const int sb_begin = blk_begin * SPB;
+  const int nsb = max(0, min((ctx + Tr::SUB - 1) / Tr::SUB, (blk_begin + nb) * SPB) - sb_begin);
+
+  const int32_t* trow =
+      p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq + blk_begin;
+  for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = trow[i];
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) mbar_init(smem_addr(bars + warp * NS + s), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) + {0,1,8,9}
+  uint32_t qf[KS][2];
+  {
+    const int n = lane >> 2;
+    const int c = lane & 3;
+    const T* qrow = static_cast<const T*>(p.q) +
+                    (static_cast<size_t>(seq) * p.num_heads + kvh * G + min(n, G - 1)) * D;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qf[ks][0] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
+      qf[ks][1] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+    }
+  }
+  float acc[KS][4];
+#pragma unroll
+  for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY};
+  float l[2] = {0.f, 0.f};
+
+  const int nbw = nsb > warp ? (nsb - warp + W - 1) / W : 0;
+  const uint32_t ring0 = smem_addr(smem) + warp * NS * Tr::STAGE_BYTES;
+  const uint32_t bar0 = smem_addr(bars + warp * NS);
+
+  auto table_entry = [&](int k) {  // physical block of this warp's k-th sub-block
+    const int sb = sb_begin + warp + k * W;
+    return tbl[sb / SPB - blk_begin];
+  };
+  auto issue = [&](int k) {  // lane 0 only
+    const int stage = k % NS;
+    const int sb = sb_begin + warp + k * W;
+    const int pb = tbl[sb / SPB - blk_begin];
+    const uint32_t bar = bar0 + stage * 8;
+    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
+      const int y = (pb * p.num_kv_heads + kvh) * BS + (sb % SPB) * Tr::SUB;
+      const uint32_t kdst = ring0 + stage * Tr::STAGE_BYTES;
+      mbar_arrive_expect_tx(bar, Tr::STAGE_BYTES);
+#pragma unroll
+      for (int b = 0; b < Tr::BOXES; ++b) {
+        tma_load_2d(kdst + b * Tr::BOX_BYTES, &kmap, b * 64, y, bar);
+        tma_load_2d(kdst + Tr::TILE_BYTES + b * Tr::BOX_BYTES, &vmap, b * 64, y, bar);
+      }
+    } else {
+      set_err(p.err, PKV_DEVERR_BAD_BLOCK);
+      mbar_arrive(bar);
+    }
+  };
+
+  if (lane == 0) {
+    for (int k = 0; k < min(NS, nbw); ++k) issue(k);
+  }
+  for (int k = 0; k < nbw; ++k) {
+    const int stage = k % NS;
+    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1);
+    if (!__all_sync(kFullMask, ok)) {
+      if (lane == 0) {
+        set_err(p.err, PKV_DEVERR_TIMEOUT);
+        for (int jj = k; jj < min(k + NS, nbw); ++jj)
+          (void)mbar_wait_bounded(bar0 + (jj % NS) * 8, (jj / NS) & 1);
+      }
+      __syncwarp();
+      break;
+    }
+    const int pb = table_entry(k);
+    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
+      const int sb = sb_begin + warp + k * W;
+      const int valid = min(Tr::SUB, ctx - sb * Tr::SUB);
+      const uint32_t kt = ring0 + stage * Tr::STAGE_BYTES;
+      mma_sub_block<Tr>(kt, kt + Tr::TILE_BYTES, valid, qf, acc, m, l, p.qscale, lane);
+    }
+    __syncwarp();
+    if (lane == 0 && k + NS < nbw) {
+      fence_proxy_async_smem();
+      issue(k + NS);
+    }
+  }
+
+  // ---- merge the warps -------------------------------------------------------
+  __syncthreads();
+  float* cm = reinterpret_cast<float*>(smem);
+  float* cl = cm + W * G;
+  float* cacc = cl + W * G;
+  {
+    const int c = lane & 3;
+    const int d_lo = lane >> 2;
+    if (lane < 4) {
+      if (2 * c < G) {
+        cm[warp * G + 2 * c] = m[0];
+        cl[warp * G + 2 * c] = l[0];
+      }
+      if (2 * c + 1 < G) {
+        cm[warp * G + 2 * c + 1] = m[1];
+        cl[warp * G + 2 * c + 1] = l[1];
       }
     }
-    const int head = kvh * G + g;
-    if (direct) {
-      const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) num[e] *= inv;
-      T* o = static_cast<T*>(p.out) + (static_cast<size_t>(seq) * p.num_heads + head) * D + cc * 8;
-      *reinterpret_cast<uint4*>(o) = pack8(num, typename Tr::DT());
-    } else {
-      const size_t slot = (static_cast<size_t>(seq) * p.num_heads + head) * p.max_parts + part;
-      float4* o = reinterpret_cast<float4*>(p.ws_out + slot * D + cc * 8);
-      o[0] = make_float4(num[0], num[1], num[2], num[3]);
-      o[1] = make_float4(num[4], num[5], num[6], num[7]);
-      if (cc == 0) {
-        p.ws_max[slot] = big_m;
-        p.ws_sum[slot] = den;
+    for (int mt = 0; mt < KS; ++mt) {
+      const int d = 16 * mt + d_lo;
+      if (2 * c < G) {
+        cacc[(warp * G + 2 * c) * D + d] = acc[mt][0];
+        cacc[(warp * G + 2 * c) * D + d + 8] = acc[mt][2];
+      }
+      if (2 * c + 1 < G) {
+        cacc[(warp * G + 2 * c + 1) * D + d] = acc[mt][1];
+        cacc[(warp * G + 2 * c + 1) * D + d + 8] = acc[mt][3];
       }
     }
   }
+  __syncthreads();
+  merge_warps_and_store<W, G, D, typename Tr::DT>(p, cm, cl, cacc, seq, kvh, part, direct);
 }
 
 // Context length as the kernels use it: negative or oversized values are
@@ -534,13 +857,8 @@ KernelEntry make_entry() {
 
 template <int D, int BS, class DT>
 KernelEntry entry_for_group(int g) {
-  switch (g) {
-    case 1: return make_entry<D, BS, 1, DT>();
-    case 2: return make_entry<D, BS, 2, DT>();
-    case 4: return make_entry<D, BS, 4, DT>();
-    case 8: return make_entry<D, BS, 8, DT>();
-    default: return KernelEntry{nullptr, 0, 0};
-  }
+  // one query head per kv head: the CUDA-core kernel (G >= 2 uses the tensor cores)
+  return g == 1 ? make_entry<D, BS, 1, DT>() : KernelEntry{nullptr, 0, 0};
 }
 
 template <class DT>
@@ -554,6 +872,115 @@ KernelEntry entry_for(int d, int bs, int g) {
 
 KernelEntry decode_entry(int d, int bs, int g, pkv_dtype dt) {
   return dt == PKV_FP16 ? entry_for<Fp16>(d, bs, g) : entry_for<Bf16>(d, bs, g);
+}
+
+// ---- tensor-core kernel dispatch -------------------------------------------
+using MmaKernelFn = void (*)(const DecodeParams, const CUtensorMap, const CUtensorMap);
+
+struct MmaEntry {
+  MmaKernelFn fn;
+  int threads;
+  size_t smem_fixed;
+};
+
+// 4 warps; about 96 KiB of ring per CTA (2 CTAs per SM).
+template <int D>
+struct MmaShape {
+  static constexpr int W = 4;
+  static constexpr int STAGE = 2 * (D / 64) * 16 * 128;
+  static constexpr int NS = cmax(2, cmin(6, (96 * 1024) / (W * STAGE)));
+};
+
+template <int D, int BS, int G, class DT>
+MmaEntry make_mma_entry() {
+  using Tr = MmaTraits<D, BS, G, DT, MmaShape<D>::W, MmaShape<D>::NS>;
+  return MmaEntry{paged_decode_mma_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(0)};
+}
+
+template <int D, int BS, class DT>
+MmaEntry mma_for_group(int g) {
+  switch (g) {
+    case 2: return make_mma_entry<D, BS, 2, DT>();
+    case 4: return make_mma_entry<D, BS, 4, DT>();
+    case 8: return make_mma_entry<D, BS, 8, DT>();
+    default: return MmaEntry{nullptr, 0, 0};
+  }
+}
+
+template <class DT>
+MmaEntry mma_for(int d, int bs, int g) {
+  if (d == 128 && bs == 16) return mma_for_group<128, 16, DT>(g);
+  if (d == 128 && bs == 32) return mma_for_group<128, 32, DT>(g);
+  if (d == 64 && bs == 16) return mma_for_group<64, 16, DT>(g);
+  if (d == 64 && bs == 32) return mma_for_group<64, 32, DT>(g);
+  return MmaEntry{nullptr, 0, 0};
+}
+
+MmaEntry mma_entry(int d, int bs, int g, pkv_dtype dt) {
+  return dt == PKV_FP16 ? mma_for<Fp16>(d, bs, g) : mma_for<Bf16>(d, bs, g);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Tensor map over a cache viewed as rows of head_dim elements
+// ([num_blocks * num_kv_heads * block_size, head_dim]); boxes of 16 rows x 64
+// elements (128 bytes) with the 128-byte swizzle.  Encoded maps are cached per
+// thread, keyed by everything they depend on.
+pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, int hkv, int bs,
+                            int d, pkv_dtype dt) {
+  struct Slot {
+    const void* base;
+    int num_blocks, hkv, bs, d, dt;
+    CUtensorMap map;
+  };
+  thread_local Slot slots[4] = {};
+  thread_local int next = 0;
+  for (const Slot& sl : slots) {
+    if (sl.base == base && sl.num_blocks == num_blocks && sl.hkv == hkv && sl.bs == bs &&
+        sl.d == d && sl.dt == dt) {
+      *out = sl.map;
+      return PKV_OK;
+    }
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return cuda_status(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d),
+                        static_cast<cuuint64_t>(num_blocks) * hkv * bs};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  Slot& sl = slots[next];
+  next = (next + 1) % 4;
+  const CUresult r =
+      enc(&sl.map, dt == PKV_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+          2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    sl.base = nullptr;
+    return cuda_status(cudaErrorInvalidValue);
+  }
+  sl.base = base;
+  sl.num_blocks = num_blocks;
+  sl.hkv = hkv;
+  sl.bs = bs;
+  sl.d = d;
+  sl.dt = dt;
+  *out = sl.map;
+  return PKV_OK;
 }
 
 KernelFn reduce_entry(int d, pkv_dtype dt) {
@@ -664,12 +1091,25 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
   const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * max_parts;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
-  const KernelEntry ke = decode_entry(head_dim, block_size, group, dtype);
-  if (ke.fn == nullptr) return PKV_ERR_UNSUPPORTED;
-  const size_t smem = ke.smem_fixed + static_cast<size_t>(part_blocks) * 4;
+  const bool use_mma = group >= 2;
+  const KernelEntry ke = use_mma ? KernelEntry{nullptr, 0, 0}
+                                 : decode_entry(head_dim, block_size, group, dtype);
+  const MmaEntry me = use_mma ? mma_entry(head_dim, block_size, group, dtype)
+                              : MmaEntry{nullptr, 0, 0};
+  if (ke.fn == nullptr && me.fn == nullptr) return PKV_ERR_UNSUPPORTED;
+  const size_t smem = (use_mma ? me.smem_fixed : ke.smem_fixed) + static_cast<size_t>(part_blocks) * 4;
+  const void* kernel_ptr = use_mma ? reinterpret_cast<const void*>(me.fn)
+                                   : reinterpret_cast<const void*>(ke.fn);
   pkv_status st = cuda_status(cudaFuncSetAttribute(
-      ke.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+      kernel_ptr, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
   if (st != PKV_OK) return st;
+  CUtensorMap kmap, vmap;
+  if (use_mma) {
+    st = cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
+    if (st != PKV_OK) return st;
+    st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
+    if (st != PKV_OK) return st;
+  }
 
   DecodeParams p;
   p.out = out;
@@ -702,12 +1142,13 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(ke.threads);
+  cfg.blockDim = dim3(use_mma ? me.threads : ke.threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = as_stream(stream);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  st = cuda_status(cudaLaunchKernelEx(&cfg, ke.fn, p));
+  st = use_mma ? cuda_status(cudaLaunchKernelEx(&cfg, me.fn, p, kmap, vmap))
+               : cuda_status(cudaLaunchKernelEx(&cfg, ke.fn, p));
   if (st != PKV_OK || max_parts <= 1) return st;
 
   const long long warps = static_cast<long long>(num_seqs) * num_heads;
@@ -735,7 +1176,6 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
 // cudaGetSymbolAddress returns for the current device.
 static __device__ __align__(256) unsigned char pkv_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
 
-#include <mutex>
 
 namespace pkv {
 namespace {

@@ -196,12 +196,12 @@ def hbm_peak():
 
 
 def kernel_source_hash():
+    """Hash of the device code (the decode kernels and their helpers)."""
     csrc = os.path.join(ROOT, "paged_kv_cache_394_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in ("common.cuh", "paged_attn_kernels.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 

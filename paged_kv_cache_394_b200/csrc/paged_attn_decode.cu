@@ -1,37 +1,6 @@
-// paged_attn_decode.cu — PagedAttention decode for B200 (sm_100a).
-//
-// What it computes.  Each sequence's one new query token attends over the
-// sequence's cached keys and values, which live in fixed-size blocks scattered
-// through a physical pool and are found through the sequence's block table;
-// the kernel assembles the data from the page table across non-contiguous
-// regions, transparently to the model ([csdn] "分页式KV缓存：让显存利用接近理论
-// 极限"; [betteryeah] §2.2 and §2.4 "技术实现细节").  So, for sequence i and
-// query head h (kv head g = h / G, G = num_heads / num_kv_heads):
-//     out[i,h,:] = softmax(scale * q[i,h,:] . K^T) . V  over context_lens[i] tokens.
-//
-// How (B200 design).  The work is HBM-bound: every cached K/V byte is read
-// once, and there are G multiply-adds per byte at most.  So:
-//  * One CTA per (sequence, kv head, partition).  It serves all G query heads
-//    of that kv head, so each K/V byte leaves HBM once.
-//  * The partition's slice of the block table is staged in shared memory.
-//  * Each warp owns a ring of NS stages in shared memory and streams its own
-//    blocks (blocks w, w+W, w+2W, ... of the partition) with the TMA engine's
-//    1-D bulk copy: one (block, kv head) of K is one contiguous block_size *
-//    head_dim run (4 KiB at block 16 / dim 128), likewise V, so a stage is two
-//    bulk copies completing on one mbarrier.  Lane 0 refills a stage as soon
-//    as the warp has consumed it, so NS blocks per warp are always in flight.
-//  * q·K: lane (c, r) holds 8 dims (chunk c) of q for all G heads and reads
-//    8 dims of R rows at a time (conflict-free 16-byte shared loads); the
-//    partial dot products are summed across the NC = D/8 lanes of a row by a
-//    butterfly reduce-scatter, which leaves each lane one finished logit.
-//  * Online softmax in base 2 (q is pre-scaled by scale*log2(e)); running max
-//    and sum per head; the accumulator is rescaled only when the max moves.
-//  * P·V with fp32 accumulators, 8 dims x G heads per lane.
-//  * Warps merge their (max, sum, acc) in shared memory at the end.
-//  * Long contexts: partitions of partition_size tokens write (max, sum,
-//    unnormalised output) to the workspace and a reduce kernel merges them;
-//    a sequence with a single partition is written directly.
-//  * No waits on other CTAs anywhere; mbarrier waits are bounded in time.
+// paged_attn_decode.cu — host side of PagedAttention decode: shape dispatch,
+// partition choice, workspace layout, TMA tensor maps and the C entry points.
+// The kernels are in paged_attn_kernels.cuh.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -39,793 +8,10 @@
 #include <mutex>
 #include <type_traits>
 
-#include "common.cuh"
 #include "host_common.h"
+#include "paged_attn_kernels.cuh"
 
 namespace pkv {
-
-struct DecodeParams {
-  void* out;
-  const void* q;
-  const void* k_cache;
-  const void* v_cache;
-  const int32_t* block_tables;
-  const int32_t* context_lens;
-  float qscale;  // scale * log2(e)
-  int num_seqs;
-  int num_heads;
-  int num_kv_heads;
-  int max_blocks_per_seq;
-  int max_context_len;
-  int num_blocks;
-  int block_size;
-  int part_blocks;  // blocks per partition
-  int max_parts;    // partitions per sequence at max_context_len
-  float* ws_out;    // [S, H, max_parts, D]
-  float* ws_max;    // [S, H, max_parts]
-  float* ws_sum;    // [S, H, max_parts]
-  unsigned* err;
-};
-
-__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
-__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
-__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
-
-template <int D_, int BS_, int G_, class DT_, int W_, int NS_>
-struct DecodeTraits {
-  static constexpr int D = D_, BS = BS_, G = G_, W = W_, NS = NS_;
-  using DT = DT_;
-  using T = typename DT::T;
-  static constexpr int NC = D / 8;                // 16-byte chunks per row
-  static constexpr int LOG2_NC = ilog2(NC);
-  static constexpr int R = 32 / NC;               // rows per warp-wide load
-  static constexpr int ROWS_PER_LANE = BS / R;
-  // rows per lane per sub-tile: keeps G * JS partial logits <= NC per lane
-  static constexpr int JS = cmin(ROWS_PER_LANE, cmax(1, NC / G));
-  static constexpr int TS = R * JS;               // tokens per sub-tile
-  static constexpr int NSUB = BS / TS;
-  static constexpr int NV = G * JS;               // partial logits per lane
-  static constexpr int LOG2_NV = ilog2(NV);
-  static constexpr int REP = NC / NV;             // lanes holding each logit
-  static constexpr int SEG = JS * REP;            // lanes of one head within a row group
-  static constexpr int CHUNK_ELEMS = BS * D;
-  static constexpr int CHUNK_BYTES = CHUNK_ELEMS * 2;
-  static constexpr int STAGE_BYTES = 2 * CHUNK_BYTES;
-  static constexpr int THREADS = W * 32;
-  static constexpr int PB_FLOATS = R * NV + 8;    // p values + per-head alpha (G <= 8)
-  static constexpr int RING_BYTES = W * NS * STAGE_BYTES;
-  static constexpr int BAR_BYTES = W * NS * 8;
-  static constexpr int PBUF_BYTES = W * 2 * PB_FLOATS * 4;
-  static constexpr int COMBINE_BYTES = W * G * (D + 2) * 4;
-  static_assert(NV <= NC && NC % NV == 0, "logit layout");
-  static_assert(BS % TS == 0, "sub-tiles must tile a block");
-  static_assert(COMBINE_BYTES <= RING_BYTES, "combine scratch reuses the ring");
-  static_assert(G <= 8, "alpha slots");
-
-  static size_t smem_bytes(int part_blocks) {
-    return static_cast<size_t>(RING_BYTES) + BAR_BYTES + PBUF_BYTES +
-           static_cast<size_t>(part_blocks) * 4;
-  }
-};
-
-// Butterfly reduce-scatter of NV values over the NC lanes of a row group.
-// Afterwards lane l holds the full sum of value index (l % NC) / (NC / NV).
-template <int NV, int NC>
-__device__ __forceinline__ float reduce_scatter(float (&v)[NV], int lane) {
-  constexpr int LOG2_NC = ilog2(NC);
-  constexpr int LOG2_NV = ilog2(NV);
-#pragma unroll
-  for (int step = 0; step < LOG2_NC; ++step) {
-    const int mask = NC >> (step + 1);
-    if (step < LOG2_NV) {
-      const int half = NV >> (step + 1);
-      const bool upper = (lane & mask) != 0;
-#pragma unroll
-      for (int k = 0; k < half; ++k) {
-        const float send = upper ? v[k] : v[k + half];
-        const float keep = upper ? v[k + half] : v[k];
-        v[k] = keep + __shfl_xor_sync(kFullMask, send, mask);
-      }
-    } else {
-      v[0] += __shfl_xor_sync(kFullMask, v[0], mask);
-    }
-  }
-  return v[0];
-}
-
-// Max / sum over the lanes that hold logits of one head: SEG lanes in each
-// row group (skipping replica lanes for the sum) times the R row groups.
-template <class Tr>
-__device__ __forceinline__ float segment_max(float x) {
-#pragma unroll
-  for (int m = Tr::REP; m < Tr::SEG; m <<= 1) x = fmaxf(x, __shfl_xor_sync(kFullMask, x, m));
-#pragma unroll
-  for (int m = Tr::NC; m < 32; m <<= 1) x = fmaxf(x, __shfl_xor_sync(kFullMask, x, m));
-  return x;
-}
-
-template <class Tr>
-__device__ __forceinline__ float segment_sum(float x) {
-#pragma unroll
-  for (int m = Tr::REP; m < Tr::SEG; m <<= 1) x += __shfl_xor_sync(kFullMask, x, m);
-#pragma unroll
-  for (int m = Tr::NC; m < 32; m <<= 1) x += __shfl_xor_sync(kFullMask, x, m);
-  return x;
-}
-
-// Per-warp running state of the online softmax.
-template <class Tr>
-struct WarpState {
-  float q[Tr::G][8];    // q chunk of each head, pre-scaled
-  float acc[Tr::G][8];  // unnormalised output chunk, rows r (mod R) of this lane
-  float m;              // running max of this lane's head (base-2 logits)
-  float l;              // running exp-sum of this lane's head
-};
-
-// Consumes one block (K and V chunks in shared memory): `valid` leading
-// tokens of it belong to the sequence.
-template <class Tr, bool kFull>
-__device__ __forceinline__ void process_block(WarpState<Tr>& st, const typename Tr::T* kch,
-                                              const typename Tr::T* vch, int valid, float* pbuf,
-                                              int& buf, int lane) {
-  constexpr int NC = Tr::NC, R = Tr::R, JS = Tr::JS, TS = Tr::TS, NV = Tr::NV, G = Tr::G;
-  const int c = lane & (NC - 1);
-  const int r0 = lane >> Tr::LOG2_NC;
-  const int li = (lane & (NC - 1)) / Tr::REP;  // logit index held after the reduce
-  const int lg = li / JS;                      // its head
-  const int lj = li % JS;                      // its row within the lane's rows
-  const int ltok = r0 + R * lj;                // its token within the sub-tile
-#pragma unroll
-  for (int sub = 0; sub < Tr::NSUB; ++sub) {
-    const int tb = sub * TS;
-    if (!kFull && tb >= valid) break;
-    // ---- q . K for TS tokens --------------------------------------------
-    float part[NV];
-#pragma unroll
-    for (int j = 0; j < JS; ++j) {
-      const int row = tb + r0 + R * j;
-      const uint4 raw = *reinterpret_cast<const uint4*>(kch + row * Tr::D + c * 8);
-      float kf[8];
-      unpack8(raw, kf, typename Tr::DT());
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float s = st.q[g][0] * kf[0];
-#pragma unroll
-        for (int e = 1; e < 8; ++e) s = fmaf(st.q[g][e], kf[e], s);
-        part[g * JS + j] = s;
-      }
-    }
-    float x = reduce_scatter<NV, NC>(part, lane);
-    const bool in_seq = kFull || (tb + ltok) < valid;
-    x = in_seq ? x : -INFINITY;
-    // ---- online softmax update of this lane's head ----------------------
-    const float m_new = fmaxf(st.m, segment_max<Tr>(x));
-    const float alpha = exp2_approx(st.m - m_new);
-    const float p = in_seq ? exp2_approx(x - m_new) : 0.f;
-    st.l = st.l * alpha + segment_sum<Tr>(p);
-    st.m = m_new;
-    float* pb = pbuf + buf * Tr::PB_FLOATS;
-    if ((lane & (Tr::REP - 1)) == 0) {
-      pb[r0 * NV + li] = p;
-      if (r0 == 0 && lj == 0) pb[R * NV + lg] = alpha;
-    }
-    __syncwarp();
-    // ---- P . V ------------------------------------------------------------
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float a = pb[R * NV + g];
-      if (a != 1.f) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) st.acc[g][e] *= a;
-      }
-    }
-    float pv[NV];
-#pragma unroll
-    for (int k = 0; k < NV; k += 4) {
-      const float4 f = *reinterpret_cast<const float4*>(pb + r0 * NV + k);
-      pv[k] = f.x;
-      pv[k + 1] = f.y;
-      pv[k + 2] = f.z;
-      pv[k + 3] = f.w;
-    }
-#pragma unroll
-    for (int j = 0; j < JS; ++j) {
-      const int row = tb + r0 + R * j;
-      if (kFull || row < valid) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(vch + row * Tr::D + c * 8);
-        float vf[8];
-        unpack8(raw, vf, typename Tr::DT());
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pg = pv[g * JS + j];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) st.acc[g][e] = fmaf(pg, vf[e], st.acc[g][e]);
-        }
-      }
-    }
-    buf ^= 1;
-  }
-}
-
-// Merges the W warps' (max, sum, unnormalised output) of one CTA and stores
-// the result: the normalised output when the sequence has one partition,
-// else the partition's (m, l, o) triple in the workspace.
-//   cm, cl: [W][G] per-warp running max and exp-sum (base-2 logits)
-//   cacc:   [W][G][D] per-warp unnormalised outputs
-template <int W, int G, int D, class DT>
-__device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, const float* cm,
-                                                      const float* cl, const float* cacc,
-                                                      int seq, int kvh, int part, bool direct) {
-  using T = typename DT::T;
-  constexpr int NC = D / 8;
-  for (int idx = threadIdx.x; idx < G * NC; idx += W * 32) {
-    const int g = idx / NC;
-    const int cc = idx % NC;
-    float big_m = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < W; ++w) big_m = fmaxf(big_m, cm[w * G + g]);
-    float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float den = 0.f;
-    if (big_m != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < W; ++w) {
-        const float f = exp2_approx(cm[w * G + g] - big_m);
-        den = fmaf(f, cl[w * G + g], den);
-        const float* a = cacc + (w * G + g) * D + cc * 8;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) num[e] = fmaf(f, a[e], num[e]);
-      }
-    }
-    const int head = kvh * G + g;
-    if (direct) {
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) num[e] *= inv;
-      T* o = static_cast<T*>(p.out) + (static_cast<size_t>(seq) * p.num_heads + head) * D + cc * 8;
-      *reinterpret_cast<uint4*>(o) = pack8(num, DT());
-    } else {
-      const size_t slot = (static_cast<size_t>(seq) * p.num_heads + head) * p.max_parts + part;
-      float4* o = reinterpret_cast<float4*>(p.ws_out + slot * D + cc * 8);
-      o[0] = make_float4(num[0], num[1], num[2], num[3]);
-      o[1] = make_float4(num[4], num[5], num[6], num[7]);
-      if (cc == 0) {
-        p.ws_max[slot] = big_m;
-        p.ws_sum[slot] = den;
-      }
-    }
-  }
-}
-
-template <class Tr>
-__global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeParams p) {
-  using T = typename Tr::T;
-  constexpr int W = Tr::W, NS = Tr::NS, G = Tr::G, D = Tr::D, BS = Tr::BS, NC = Tr::NC;
-  extern __shared__ __align__(128) unsigned char smem[];
-  T* ring = reinterpret_cast<T*>(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
-  float* pbuf_all = reinterpret_cast<float*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
-  int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES + Tr::PBUF_BYTES);
-
-  const int part = blockIdx.x % p.max_parts;
-  const int unit = blockIdx.x / p.max_parts;
-  const int kvh = unit % p.num_kv_heads;
-  const int seq = unit / p.num_kv_heads;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  // Inputs may come from the previous kernel in the stream (e.g. the cache
-  // write); wait for it before reading anything, then let the next one start.
-  grid_dependency_wait();
-  trigger_dependents();
-
-  const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
-  int ctx = p.context_lens[seq];
-  if (ctx < 0 || ctx > ctx_cap) {
-    if (threadIdx.x == 0 && part == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
-    ctx = min(max(ctx, 0), ctx_cap);
-  }
-  const int nblk = (ctx + BS - 1) / BS;
-  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
-  if (part >= max(nparts, 1)) return;
-  const bool direct = nparts <= 1;
-  const int blk_begin = part * p.part_blocks;
-  const int nb = min(nblk, blk_begin + p.part_blocks) - blk_begin;
-
-  // ---- stage the block-table slice; initialise this warp's barriers --------
-  const int32_t* trow =
-      p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq + blk_begin;
-  for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = trow[i];
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < NS; ++s) mbar_init(smem_addr(bars + warp * NS + s), 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  // ---- this lane's q chunk for the G heads, pre-scaled ---------------------
-  WarpState<Tr> st;
-  const int c = lane & (NC - 1);
-  {
-    const T* qrow = static_cast<const T*>(p.q) +
-                    (static_cast<size_t>(seq) * p.num_heads + kvh * G) * D + c * 8;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(qrow + g * D);
-      unpack8(raw, st.q[g], typename Tr::DT());
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        st.q[g][e] *= p.qscale;
-        st.acc[g][e] = 0.f;
-      }
-    }
-  }
-  st.m = -INFINITY;
-  st.l = 0.f;
-
-  // ---- stream this warp's blocks through its ring ---------------------------
-  const int nbw = nb > warp ? (nb - warp + W - 1) / W : 0;
-  T* wring = ring + static_cast<size_t>(warp) * NS * 2 * Tr::CHUNK_ELEMS;
-  const uint32_t bar0 = smem_addr(bars + warp * NS);
-  const T* kbase = static_cast<const T*>(p.k_cache);
-  const T* vbase = static_cast<const T*>(p.v_cache);
-  const size_t head_off = static_cast<size_t>(kvh) * Tr::CHUNK_ELEMS;
-  const size_t block_stride = static_cast<size_t>(p.num_kv_heads) * Tr::CHUNK_ELEMS;
-
-  auto issue = [&](int k) {  // lane 0 only
-    const int stage = k % NS;
-    const int pb = tbl[warp + k * W];
-    const uint32_t bar = bar0 + stage * 8;
-    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
-      const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
-      mbar_arrive_expect_tx(bar, 2 * Tr::CHUNK_BYTES);
-      bulk_copy_g2s(smem_addr(wring + (2 * stage) * Tr::CHUNK_ELEMS), kbase + off,
-                    Tr::CHUNK_BYTES, bar);
-      bulk_copy_g2s(smem_addr(wring + (2 * stage + 1) * Tr::CHUNK_ELEMS), vbase + off,
-                    Tr::CHUNK_BYTES, bar);
-    } else {
-      set_err(p.err, PKV_DEVERR_BAD_BLOCK);
-      mbar_arrive(bar);  // complete the phase with no data; consumers skip it
-    }
-  };
-
-  if (lane == 0) {
-    for (int k = 0; k < min(NS, nbw); ++k) issue(k);
-  }
-  float* pbuf = pbuf_all + warp * 2 * Tr::PB_FLOATS;
-  int buf = 0;
-  for (int k = 0; k < nbw; ++k) {
-    const int stage = k % NS;
-    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1);
-    if (!__all_sync(kFullMask, ok)) {
-      // Give up on this warp's blocks: report, then wait (bounded) for the
-      // copies still in flight so none lands after the CTA has exited.
-      if (lane == 0) {
-        set_err(p.err, PKV_DEVERR_TIMEOUT);
-        for (int j = k; j < min(k + NS, nbw); ++j)
-          (void)mbar_wait_bounded(bar0 + (j % NS) * 8, (j / NS) & 1);
-      }
-      __syncwarp();
-      break;
-    }
-    const int pb = tbl[warp + k * W];
-    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
-      const T* kch = wring + (2 * stage) * Tr::CHUNK_ELEMS;
-      const T* vch = kch + Tr::CHUNK_ELEMS;
-      const int lb = blk_begin + warp + k * W;
-      const int valid = min(BS, ctx - lb * BS);
-      if (valid == BS)
-        process_block<Tr, true>(st, kch, vch, BS, pbuf, buf, lane);
-      else
-        process_block<Tr, false>(st, kch, vch, valid, pbuf, buf, lane);
-    }
-    __syncwarp();
-    if (lane == 0 && k + NS < nbw) {
-      fence_proxy_async_smem();  // the warp's reads of this stage precede the refill
-      issue(k + NS);
-    }
-  }
-
-  // ---- merge the row groups, then the warps ---------------------------------
-#pragma unroll
-  for (int m = NC; m < 32; m <<= 1)
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) st.acc[g][e] += __shfl_xor_sync(kFullMask, st.acc[g][e], m);
-
-  __syncthreads();  // every warp is done with the ring; reuse it
-  float* cm = reinterpret_cast<float*>(smem);  // [W][G]
-  float* cl = cm + W * G;                      // [W][G]
-  float* cacc = cl + W * G;                    // [W][G][D]
-  {
-    const int li = (lane & (NC - 1)) / Tr::REP;
-    const int r0 = lane >> Tr::LOG2_NC;
-    if ((lane & (Tr::REP - 1)) == 0 && r0 == 0 && li % Tr::JS == 0) {
-      cm[warp * G + li / Tr::JS] = st.m;
-      cl[warp * G + li / Tr::JS] = st.l;
-    }
-    if (r0 == 0) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float4* dst = reinterpret_cast<float4*>(cacc + (warp * G + g) * D + c * 8);
-        dst[0] = make_float4(st.acc[g][0], st.acc[g][1], st.acc[g][2], st.acc[g][3]);
-        dst[1] = make_float4(st.acc[g][4], st.acc[g][5], st.acc[g][6], st.acc[g][7]);
-      }
-    }
-  }
-  __syncthreads();
-  merge_warps_and_store<W, G, D, typename Tr::DT>(p, cm, cl, cacc, seq, kvh, part, direct);
-}
-
-// ---------------------------------------------------------------------------
-// Grouped-query decode on the tensor cores (G >= 2).
-//
-// With G query heads per kv head, q.K and P.V carry G multiply-adds per
-// cached element; on the CUDA cores that makes the kernel instruction-bound
-// (about 1,700 warp instructions per 16 tokens at G = 8).  Here each warp runs
-// them as mma.sync m16n8k16 with the 16 tokens of a sub-block as M and the
-// heads as N (N = 8 covers G <= 8 with no padding at G = 8):
-//   q.K:  S^T[t][n] = sum_d K[t][d] q[n][d]      A = K   (ldmatrix)
-//   P.V:  O^T[d][n] += sum_t V[t][d] P[n][t]     A = V^T (ldmatrix.trans),
-//                                                B = P, transposed in registers
-//                                                from the S^T accumulator by movmatrix
-// K and V of a (block, kv head) reach shared memory by 2-D tiled TMA loads
-// with the 128-byte swizzle: boxes of 16 rows x 64 elements, so ldmatrix rows
-// fall in distinct banks.  A stage is one 16-token sub-block (a block of 32
-// is two stages).  The ring, the table slice, the bounded waits, the split-K
-// partitions and the final merge are as in paged_decode_kernel.
-// ---------------------------------------------------------------------------
-template <int D_, int BS_, int G_, class DT_, int W_, int NS_>
-struct MmaTraits {
-  static constexpr int D = D_, BS = BS_, G = G_, W = W_, NS = NS_;
-  using DT = DT_;
-  using T = typename DT::T;
-  static constexpr int SUB = 16;                   // tokens per stage (the mma M)
-  static constexpr int SUBS_PER_BLOCK = BS / SUB;
-  static constexpr int BOXES = D / 64;             // 128-byte-wide boxes per row
-  static constexpr int BOX_BYTES = SUB * 128;      // one 16 x 64 box
-  static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
-  static constexpr int KSTEPS = D / 16;            // q.K k-steps = P.V m-tiles
-  static constexpr int THREADS = W * 32;
-  static constexpr int RING_BYTES = W * NS * STAGE_BYTES;
-  static constexpr int BAR_BYTES = W * NS * 8;
-  static constexpr int COMBINE_BYTES = W * G * (D + 2) * 4;
-  static_assert(G >= 2 && G <= 8, "tensor-core path serves 2..8 heads per kv head");
-  static_assert(BS % SUB == 0 && D % 64 == 0, "shape");
-  static_assert(COMBINE_BYTES <= RING_BYTES, "combine scratch reuses the ring");
-  static size_t smem_bytes(int part_blocks) {
-    return 1024 + static_cast<size_t>(RING_BYTES) + BAR_BYTES +
-           static_cast<size_t>(part_blocks) * 4;
-  }
-};
-
-// Byte offset of 16-byte chunk `ch` of row `t` in a tile of BOXES swizzled
-// 16 x 128-byte boxes (chunk index XOR row % 8, per 1024-byte swizzle atom).
-__device__ __forceinline__ uint32_t swizzled(int t, int ch) {
-  return static_cast<uint32_t>((ch >> 3) * 2048 + t * 128 + (((ch & 7) ^ (t & 7)) << 4));
-}
-
-template <class Tr>
-__device__ __forceinline__ void mma_sub_block(uint32_t kt, uint32_t vt, int valid,
-                                              const uint32_t (&qf)[Tr::KSTEPS][2],
-                                              float (&acc)[Tr::KSTEPS][4], float (&m)[2],
-                                              float (&l)[2], float qscale, int lane) {
-  constexpr int KS = Tr::KSTEPS;
-  const int j = lane >> 3;  // which 8x8 matrix this lane addresses
-  const int r = lane & 7;
-  // ---- q.K: S^T (16 tokens x 8 heads) ----------------------------------------
-  float s[4] = {0.f, 0.f, 0.f, 0.f};
-  {
-    const int t = ((j & 1) << 3) + r;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      uint32_t a[4];
-      ldsm_x4(kt + swizzled(t, 2 * ks + (j >> 1)), a);
-      mma_16816(s, a, qf[ks][0], qf[ks][1], typename Tr::DT());
-    }
-  }
-  // lane holds tokens t0 = lane/4 and t0 + 8, heads 2(lane%4) and 2(lane%4)+1
-  const int t0 = lane >> 2;
-  float x0 = s[0] * qscale, x1 = s[1] * qscale, x2 = s[2] * qscale, x3 = s[3] * qscale;
-  if (valid < Tr::SUB) {
-    if (t0 >= valid) x0 = x1 = -INFINITY;
-    if (t0 + 8 >= valid) x2 = x3 = -INFINITY;
-  }
-  // ---- online softmax per head: reduce over the 8 lanes sharing lane % 4 ------
-  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
-  }
-  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-  const float a0 = exp2_approx(m[0] - mn0), a1 = exp2_approx(m[1] - mn1);
-  const float p0 = exp2_approx(x0 - mn0), p1 = exp2_approx(x1 - mn1);
-  const float p2 = exp2_approx(x2 - mn0), p3 = exp2_approx(x3 - mn1);
-  float s0 = p0 + p2, s1 = p1 + p3;
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    s0 += __shfl_xor_sync(kFullMask, s0, o);
-    s1 += __shfl_xor_sync(kFullMask, s1, o);
-  }
-  l[0] = l[0] * a0 + s0;
-  l[1] = l[1] * a1 + s1;
-  m[0] = mn0;
-  m[1] = mn1;
-  if (__any_sync(kFullMask, a0 != 1.f || a1 != 1.f)) {
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      acc[mt][0] *= a0;
-      acc[mt][1] *= a1;
-      acc[mt][2] *= a0;
-      acc[mt][3] *= a1;
-    }
-  }
-  // ---- P as the B operand: transpose the S^T fragments in registers -----------
-  // bf16 keeps 8 mantissa bits, too few for p near 1 at the required accuracy,
-  // so bf16 P is split as hi + lo (both bf16, |P - hi - lo| <= 2^-18 P) and
-  // P.V runs twice; fp16 P (11 bits) is used as is.
-  constexpr bool kSplitP = std::is_same<typename Tr::DT, Bf16>::value;
-  const uint32_t h01 = pack2(p0, p1, typename Tr::DT());
-  const uint32_t h23 = pack2(p2, p3, typename Tr::DT());
-  const uint32_t b0 = movmatrix_trans(h01);
-  const uint32_t b1 = movmatrix_trans(h23);
-  uint32_t b0_lo = 0, b1_lo = 0;
-  if constexpr (kSplitP) {
-    b0_lo = movmatrix_trans(pack2(p0 - __uint_as_float(h01 << 16),
-                                  p1 - __uint_as_float(h01 & 0xffff0000u), Bf16()));
-    b1_lo = movmatrix_trans(pack2(p2 - __uint_as_float(h23 << 16),
-                                  p3 - __uint_as_float(h23 & 0xffff0000u), Bf16()));
-  }
-  // ---- rows past the context hold stale data (maybe NaN): zero them in V so
-  //      that 0 * V stays 0 inside the tensor-core sum
-  if (valid < Tr::SUB) {
-    const int chunks = (Tr::SUB - valid) * Tr::BOXES * 8;
-    for (int i = lane; i < chunks; i += 32) {
-      const int row = valid + i / (Tr::BOXES * 8);
-      const int rem = i % (Tr::BOXES * 8);
-      const uint32_t at = vt + (rem >> 3) * 2048 + row * 128 + ((rem & 7) << 4);
-      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(at), "r"(0u) : "memory");
-    }
-    __syncwarp();
-  }
-  // ---- P.V: O^T (D dims x 8 heads) -------------------------------------------
-  {
-    const int t = ((j >> 1) << 3) + r;
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      uint32_t a[4];
-      ldsm_x4_trans(vt + swizzled(t, 2 * mt + (j & 1)), a);
-      mma_16816(acc[mt], a, b0, b1, typename Tr::DT());
-      if constexpr (kSplitP) mma_16816(acc[mt], a, b0_lo, b1_lo, typename Tr::DT());
-    }
-  }
-}
-
-template <class Tr>
-__global__ void __launch_bounds__(Tr::THREADS)
-    paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
-                            const __grid_constant__ CUtensorMap vmap) {
-  using T = typename Tr::T;
-  constexpr int W = Tr::W, NS = Tr::NS, G = Tr::G, D = Tr::D, BS = Tr::BS, KS = Tr::KSTEPS;
-  constexpr int SPB = Tr::SUBS_PER_BLOCK;
-  extern __shared__ unsigned char smem_raw[];
-  // the 128-byte swizzle needs 1024-byte-aligned boxes
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
-  int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
-
-  const int part = blockIdx.x % p.max_parts;
-  const int unit = blockIdx.x / p.max_parts;
-  const int kvh = unit % p.num_kv_heads;
-  const int seq = unit / p.num_kv_heads;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  grid_dependency_wait();
-  trigger_dependents();
-
-  const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
-  int ctx = p.context_lens[seq];
-  if (ctx < 0 || ctx > ctx_cap) {
-    if (threadIdx.x == 0 && part == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
-    ctx = min(max(ctx, 0), ctx_cap);
-  }
-  const int nblk = (ctx + BS - 1) / BS;
-  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
-  if (part >= max(nparts, 1)) return;
-  const bool direct = nparts <= 1;
-  const int blk_begin = part * p.part_blocks;
-  const int nb = min(nblk, blk_begin + p.part_blocks) - blk_begin;
-  const int sb_begin = blk_begin * SPB;
-  const int nsb = max(0, min((ctx + Tr::SUB - 1) / Tr::SUB, (blk_begin + nb) * SPB) - sb_begin);
-
-  const int32_t* trow =
-      p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq + blk_begin;
-  for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = trow[i];
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < NS; ++s) mbar_init(smem_addr(bars + warp * NS + s), 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) + {0,1,8,9}
-  uint32_t qf[KS][2];
-  {
-    const int n = lane >> 2;
-    const int c = lane & 3;
-    const T* qrow = static_cast<const T*>(p.q) +
-                    (static_cast<size_t>(seq) * p.num_heads + kvh * G + min(n, G - 1)) * D;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qf[ks][0] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
-      qf[ks][1] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
-    }
-  }
-  float acc[KS][4];
-#pragma unroll
-  for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-  float m[2] = {-INFINITY, -INFINITY};
-  float l[2] = {0.f, 0.f};
-
-  const int nbw = nsb > warp ? (nsb - warp + W - 1) / W : 0;
-  const uint32_t ring0 = smem_addr(smem) + warp * NS * Tr::STAGE_BYTES;
-  const uint32_t bar0 = smem_addr(bars + warp * NS);
-
-  auto table_entry = [&](int k) {  // physical block of this warp's k-th sub-block
-    const int sb = sb_begin + warp + k * W;
-    return tbl[sb / SPB - blk_begin];
-  };
-  auto issue = [&](int k) {  // lane 0 only
-    const int stage = k % NS;
-    const int sb = sb_begin + warp + k * W;
-    const int pb = tbl[sb / SPB - blk_begin];
-    const uint32_t bar = bar0 + stage * 8;
-    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
-      const int y = (pb * p.num_kv_heads + kvh) * BS + (sb % SPB) * Tr::SUB;
-      const uint32_t kdst = ring0 + stage * Tr::STAGE_BYTES;
-      mbar_arrive_expect_tx(bar, Tr::STAGE_BYTES);
-#pragma unroll
-      for (int b = 0; b < Tr::BOXES; ++b) {
-        tma_load_2d(kdst + b * Tr::BOX_BYTES, &kmap, b * 64, y, bar);
-        tma_load_2d(kdst + Tr::TILE_BYTES + b * Tr::BOX_BYTES, &vmap, b * 64, y, bar);
-      }
-    } else {
-      set_err(p.err, PKV_DEVERR_BAD_BLOCK);
-      mbar_arrive(bar);
-    }
-  };
-
-  if (lane == 0) {
-    for (int k = 0; k < min(NS, nbw); ++k) issue(k);
-  }
-  for (int k = 0; k < nbw; ++k) {
-    const int stage = k % NS;
-    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1);
-    if (!__all_sync(kFullMask, ok)) {
-      if (lane == 0) {
-        set_err(p.err, PKV_DEVERR_TIMEOUT);
-        for (int jj = k; jj < min(k + NS, nbw); ++jj)
-          (void)mbar_wait_bounded(bar0 + (jj % NS) * 8, (jj / NS) & 1);
-      }
-      __syncwarp();
-      break;
-    }
-    const int pb = table_entry(k);
-    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
-      const int sb = sb_begin + warp + k * W;
-      const int valid = min(Tr::SUB, ctx - sb * Tr::SUB);
-      const uint32_t kt = ring0 + stage * Tr::STAGE_BYTES;
-      mma_sub_block<Tr>(kt, kt + Tr::TILE_BYTES, valid, qf, acc, m, l, p.qscale, lane);
-    }
-    __syncwarp();
-    if (lane == 0 && k + NS < nbw) {
-      fence_proxy_async_smem();
-      issue(k + NS);
-    }
-  }
-
-  // ---- merge the warps -------------------------------------------------------
-  __syncthreads();
-  float* cm = reinterpret_cast<float*>(smem);
-  float* cl = cm + W * G;
-  float* cacc = cl + W * G;
-  {
-    const int c = lane & 3;
-    const int d_lo = lane >> 2;
-    if (lane < 4) {
-      if (2 * c < G) {
-        cm[warp * G + 2 * c] = m[0];
-        cl[warp * G + 2 * c] = l[0];
-      }
-      if (2 * c + 1 < G) {
-        cm[warp * G + 2 * c + 1] = m[1];
-        cl[warp * G + 2 * c + 1] = l[1];
-      }
-    }
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      const int d = 16 * mt + d_lo;
-      if (2 * c < G) {
-        cacc[(warp * G + 2 * c) * D + d] = acc[mt][0];
-        cacc[(warp * G + 2 * c) * D + d + 8] = acc[mt][2];
-      }
-      if (2 * c + 1 < G) {
-        cacc[(warp * G + 2 * c + 1) * D + d] = acc[mt][1];
-        cacc[(warp * G + 2 * c + 1) * D + d + 8] = acc[mt][3];
-      }
-    }
-  }
-  __syncthreads();
-  merge_warps_and_store<W, G, D, typename Tr::DT>(p, cm, cl, cacc, seq, kvh, part, direct);
-}
-
-// Context length as the kernels use it: negative or oversized values are
-// clamped (and reported by the partition kernel).
-__device__ __forceinline__ int clamped_context(const DecodeParams& p, int seq) {
-  const int cap = min(p.max_context_len, p.max_blocks_per_seq * p.block_size);
-  return min(max(p.context_lens[seq], 0), cap);
-}
-
-// Merges the partitions of each (sequence, head): M = max_p m_p,
-// out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.  One warp per
-// (sequence, head); sequences with a single partition were written directly
-// by the partition kernel and are skipped here.
-template <int D, class DT>
-__global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeParams p) {
-  using T = typename DT::T;
-  constexpr int PER_LANE = D / 32;
-  grid_dependency_wait();
-  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (gw >= p.num_seqs * p.num_heads) return;
-  const int seq = gw / p.num_heads;
-  const int head = gw % p.num_heads;
-  const int ctx = clamped_context(p, seq);
-  const int nblk = (ctx + p.block_size - 1) / p.block_size;
-  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
-  if (nparts <= 1) return;
-  const size_t base = static_cast<size_t>(gw) * p.max_parts;
-  float big_m = -INFINITY;
-  for (int q = lane; q < nparts; q += 32) big_m = fmaxf(big_m, p.ws_max[base + q]);
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) big_m = fmaxf(big_m, __shfl_xor_sync(kFullMask, big_m, m));
-  float num[PER_LANE];
-#pragma unroll
-  for (int e = 0; e < PER_LANE; ++e) num[e] = 0.f;
-  float den = 0.f;
-#pragma unroll 4
-  for (int q = 0; q < nparts; ++q) {
-    const float f = exp2_approx(p.ws_max[base + q] - big_m);
-    den = fmaf(f, p.ws_sum[base + q], den);
-    const float* o = p.ws_out + (base + q) * D + lane * PER_LANE;
-    if constexpr (PER_LANE == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(o);
-      num[0] = fmaf(f, v.x, num[0]);
-      num[1] = fmaf(f, v.y, num[1]);
-      num[2] = fmaf(f, v.z, num[2]);
-      num[3] = fmaf(f, v.w, num[3]);
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(o);
-      num[0] = fmaf(f, v.x, num[0]);
-      num[1] = fmaf(f, v.y, num[1]);
-    }
-  }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  T* out = static_cast<T*>(p.out) + static_cast<size_t>(gw) * D + lane * PER_LANE;
-  T vals[PER_LANE];
-#pragma unroll
-  for (int e = 0; e < PER_LANE; ++e) vals[e] = static_cast<T>(num[e] * inv);
-  if constexpr (PER_LANE == 4)
-    *reinterpret_cast<uint2*>(out) = *reinterpret_cast<const uint2*>(vals);
-  else
-    *reinterpret_cast<uint32_t*>(out) = *reinterpret_cast<const uint32_t*>(vals);
-  (void)seq;
-  (void)head;
-}
 
 // ---------------------------------------------------------------------------
 // Host side: shape dispatch, partition choice, workspace layout, launch.
@@ -991,19 +177,26 @@ KernelFn reduce_entry(int d, pkv_dtype dt) {
 }
 
 constexpr int kMaxPartitionBlocks = 4096;  // block-table slice kept in shared memory
-constexpr int kSplitAbove = 4096;          // tokens: longer contexts are always split
-constexpr int kDefaultPartition = 512;     // tokens per partition when split
+constexpr int kSlots = 2 * 148;            // resident decode CTAs: two per SM, 148 SMs
 
+// Partition size in tokens.  With enough (sequence, kv head) units to fill the
+// GPU and contexts of at most 2048 tokens, one pass (no reduce) is fastest.
+// Otherwise contexts are cut so there are about four CTAs per resident slot,
+// in partitions of 256..1024 tokens: measured on B200, 512-token partitions
+// are 4-8 % slower than 1024 (a CTA's start-up is not amortised) and one
+// pass over 4096-token contexts leaves an 8 % tail.
 int choose_partition(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
                      int requested) {
   if (requested > 0) return requested;
-  const int whole = std::max(block_size, (max_context_len + block_size - 1) / block_size * block_size);
-  const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
-  // Few (sequence, kv head) units cannot fill 148 SMs, and very long
-  // contexts leave a long tail: split those into partitions.
-  if (max_context_len > kSplitAbove || (units < 2 * 148 && max_context_len > 2 * kDefaultPartition))
-    return std::min(whole, kDefaultPartition);
-  return whole;
+  const int whole =
+      std::max(block_size, (max_context_len + block_size - 1) / block_size * block_size);
+  const long long units = std::max(1LL, static_cast<long long>(num_seqs) * num_kv_heads);
+  if (units >= kSlots && max_context_len <= 2048) return whole;
+  const long long parts = std::max(1LL, (4LL * kSlots + units - 1) / units);
+  const long long want = (max_context_len + parts - 1) / parts;
+  int part = 256;
+  while (part < want && part < 1024) part <<= 1;
+  return std::min(whole, part);
 }
 
 struct WorkspaceLayout {

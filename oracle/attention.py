@@ -167,3 +167,43 @@ def paged_attention_decode_partitioned(q_bits, k_cache_bits, v_cache_bits,
                      for a in starts]
         out[s, h] = combine_partitions(summaries) if summaries else np.zeros(head_dim)
     return out
+
+
+def paged_attention_prefill(q_bits, k_cache_bits, v_cache_bits, block_tables, context_lens,
+                            query_start, scale, num_kv_heads, block_size, dtype, rows=None):
+    """Chunked-prefill attention over the paged cache, in float64.
+
+    Sequence i contributes q_len_i = query_start[i+1] - query_start[i] query
+    tokens: the last q_len_i of its context_lens[i] cached tokens (the step
+    has already written their K/V).  Its j-th query sits at position
+    p = C_i - q_len_i + j and attends causally to tokens 0..p, as every token of
+    an autoregressive model does when its own K/V are computed ([csdn]
+    "内存困局的破局者": each generated token's K and V join the cache).
+
+    q_bits: uint16 [T, H, D] with T = query_start[-1] (queries of all sequences
+    packed in order).  Returns float64 [T, H, D]; ``rows`` (iterable of
+    (token, head)) restricts the computation, other rows are NaN.
+    """
+    total, num_heads, head_dim = q_bits.shape
+    if num_heads % num_kv_heads:
+        raise ValueError("num_heads must be a multiple of num_kv_heads")
+    query_start = np.asarray(query_start, dtype=np.int64)
+    seq_of = np.repeat(np.arange(len(query_start) - 1), np.diff(query_start))
+    if rows is None:
+        rows = [(t, h) for t in range(total) for h in range(num_heads)]
+    out = np.full((total, num_heads, head_dim), np.nan, dtype=np.float64)
+    gathered = {}
+    for t, h in rows:
+        s = int(seq_of[t])
+        c = int(context_lens[s])
+        q_len = int(query_start[s + 1] - query_start[s])
+        pos = c - q_len + (t - int(query_start[s]))
+        g = kv_head_of(h, num_heads, num_kv_heads)
+        if (s, g) not in gathered:
+            gathered[(s, g)] = (
+                gather_kv(k_cache_bits, block_tables[s], c, g, block_size, dtype),
+                gather_kv(v_cache_bits, block_tables[s], c, g, block_size, dtype),
+            )
+        keys, values = gathered[(s, g)]
+        out[t, h] = attend(widen(q_bits[t, h], dtype), keys[:pos + 1], values[:pos + 1], scale)
+    return out

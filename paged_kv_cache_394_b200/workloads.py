@@ -32,6 +32,7 @@ import numpy as np
 NAN_BITS = {"fp16": np.uint16(0x7E00), "bf16": np.uint16(0x7FC0)}
 SEED_BASE = 394
 NAMES = ("tiny", "llama7b", "gqa_chat", "long_splitk", "prefix_share")
+PREFILL_NAMES = ("llama7b_prefill", "gqa_prefill")
 
 
 @dataclass
@@ -54,6 +55,7 @@ class Workload:
     cow_pairs: np.ndarray             # int64 [P, 2]
     partition_size: int = 0           # 0: the library chooses
     notes: dict = field(default_factory=dict)
+    query_start: np.ndarray = None    # int32 [S+1] for prefill (q is [T, H, D]); None for decode
 
     @property
     def num_seqs(self):
@@ -248,6 +250,52 @@ def build_prefix_share_workload(num_prompts, samples, prompt_len, div_low, div_h
                            "prompt_blocks": n_prompt_blocks})
 
 
+def build_prefill_workload(hist_lens, new_lens, num_heads, num_kv_heads, head_dim, block_size,
+                           dtype, seed, pool_factor=1.2, name="prefill"):
+    """One chunked-prefill step: sequence i already caches hist_lens[i] tokens
+    and this step appends new_lens[i] more, whose K/V it writes and whose
+    queries then attend causally over the whole context.
+
+    q is [T, H, D] with T = sum(new_lens), packed sequence by sequence;
+    ``query_start`` holds the offsets.  Slots of the new tokens hold NaN until
+    the step writes them.
+    """
+    rng = np.random.default_rng(seed)
+    hist = np.asarray(hist_lens, dtype=np.int64)
+    new = np.asarray(new_lens, dtype=np.int64)
+    lens = hist + new
+    s = len(lens)
+    need = [_blocks_for(c, block_size) for c in lens]
+    num_blocks = max(1, int(math.ceil(pool_factor * sum(need))))
+    perm = rng.permutation(num_blocks)
+    mb = max(1, max(need))
+    tables = np.full((s, mb), -1, dtype=np.int32)
+    filled = {}
+    slots = []
+    pos = 0
+    for i in range(s):
+        blocks = perm[pos:pos + need[i]]
+        pos += need[i]
+        tables[i, :need[i]] = blocks
+        for k, b in enumerate(blocks):
+            filled[int(b)] = int(max(0, min(block_size, hist[i] - k * block_size)))
+        for t in range(int(hist[i]), int(lens[i])):
+            slots.append(int(blocks[t // block_size]) * block_size + t % block_size)
+    kc, vc = _fill_pool(rng, num_blocks, num_kv_heads, block_size, head_dim, dtype, filled)
+    t_new = int(new.sum())
+    q = _normal_bits(rng, (t_new, num_heads, head_dim), dtype)
+    key = _normal_bits(rng, (t_new, num_kv_heads, head_dim), dtype)
+    value = _normal_bits(rng, (t_new, num_kv_heads, head_dim), dtype)
+    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    return Workload(name=name, dtype=dtype, num_heads=num_heads, num_kv_heads=num_kv_heads,
+                    head_dim=head_dim, block_size=block_size, num_blocks=num_blocks,
+                    context_lens=lens.astype(np.int32), block_tables=tables, q=q,
+                    k_cache=kc, v_cache=vc, key=key, value=value,
+                    slot_mapping=np.asarray(slots, dtype=np.int64),
+                    cow_pairs=np.zeros((0, 2), dtype=np.int64), query_start=qs,
+                    notes={"seed": seed})
+
+
 def chat_lengths(rng, n, median=600.0, sigma=1.0, low=16, high=4096):
     """Lognormal lengths with the given median, clipped and rounded."""
     x = rng.lognormal(mean=math.log(median), sigma=sigma, size=n)
@@ -255,10 +303,19 @@ def chat_lengths(rng, n, median=600.0, sigma=1.0, low=16, high=4096):
 
 
 def make(name, seed=None):
-    """The named workload.  ``seed`` defaults to 394 + its index in ``NAMES``."""
-    idx = NAMES.index(name)
+    """The named workload.  ``seed`` defaults to 394 + its index in
+    ``NAMES + PREFILL_NAMES``."""
+    idx = (NAMES + PREFILL_NAMES).index(name)
     seed = SEED_BASE + idx if seed is None else seed
     rng = np.random.default_rng(seed + 1000)   # lengths; values use ``seed``
+    if name == "llama7b_prefill":
+        # a chunked-prefill batch of 2048 new tokens (the batched-token budget
+        # of the vLLM examples), 512 per sequence, on top of 0..3072 cached
+        return build_prefill_workload(rng.integers(0, 3072 + 1, size=4), [512] * 4, 32, 32, 128,
+                                      16, "fp16", seed, name=name)
+    if name == "gqa_prefill":
+        return build_prefill_workload(rng.integers(0, 3072 + 1, size=4), [512] * 4, 32, 8, 128,
+                                      32, "bf16", seed, name=name)
     if name == "tiny":
         return build_decode_workload([5, 17, 32, 100], 4, 4, 64, 16, "fp16", seed,
                                      num_blocks=64, name=name)
@@ -287,4 +344,7 @@ def describe(w):
         "sum_context": int(w.context_lens.astype(np.int64).sum()),
         "max_context": w.max_context_len, "new_tokens": int(len(w.slot_mapping)),
         "cow_pairs": int(len(w.cow_pairs)), "partition_size": w.partition_size,
+        **({"query_tokens": int(w.query_start[-1]),
+            "max_query_len": int(np.diff(w.query_start).max())}
+           if w.query_start is not None else {}),
     }

@@ -125,6 +125,26 @@ def step_bytes(w):
     return decode_bytes(w) + write_bytes(w) + copy_bytes(w)
 
 
+def prefill_flops(w):
+    """Algorithmic FLOPs of one prefill call: for every query row, q.K and P.V
+    over the keys it sees (position + 1 of them), 2 FLOPs per multiply-add."""
+    import numpy as np
+    q_len = np.diff(w.query_start).astype(np.int64)
+    hist = w.context_lens.astype(np.int64) - q_len
+    # sum over sequences of sum_{j<q_len} (hist + j + 1)
+    keys = int((q_len * hist + q_len * (q_len + 1) // 2).sum())
+    return 4 * keys * w.num_heads * w.head_dim
+
+
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -223,6 +243,9 @@ def committed_traffic(workload):
 # our arm
 # ---------------------------------------------------------------------------
 def run_ours(args):
+    from paged_kv_cache_394_b200 import workloads as W
+    if args.workload in W.PREFILL_NAMES:
+        return run_ours_prefill(args)
     import numpy as np
     import torch
 
@@ -380,6 +403,144 @@ def run_ours(args):
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     del ws, staging
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def run_ours_prefill(args):
+    """One chunked-prefill step: reshape_and_cache of the new tokens, then
+    paged prefill attention.  Metric: attention TFLOP/s (tensor-bound)."""
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    from paged_kv_cache_394_b200 import workloads as W
+
+    rank, world = init_dist("nccl") if dist_env()[1] > 1 else (0, 1)
+    local = dist_env()[2]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = W.SEED_BASE + (W.NAMES + W.PREFILL_NAMES).index(args.workload)
+    w = W.make(args.workload, seed=replica_seed(base, rank))
+    tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(tdt)
+
+    q, kc, vc, key, val = up(w.q), up(w.k_cache), up(w.v_cache), up(w.key), up(w.value)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    lens = torch.from_numpy(w.context_lens).to(dev)
+    qstart = torch.from_numpy(w.query_start).to(dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    max_q = int(np.diff(w.query_start).max())
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(ev_a=None, ev_b=None):
+        pk.reshape_and_cache(key, val, kc, vc, slots, dev_err=err, stream=stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        pk.paged_attn_prefill(out, q, kc, vc, tables, lens, qstart, w.scale, w.num_kv_heads,
+                              w.block_size, w.max_context_len, max_q, dev_err=err, stream=stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError("device error word %d during warm-up" % int(err.item()))
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(*ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clk = clocks.stop()
+    ms_per_step = max_over_ranks(t0.elapsed_time(t1), dev) / args.steps
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = prefill_flops(w)
+    all_flops = sum_over_ranks(flops, dev)
+    value = all_flops / (ms_per_step * 1e-3) / 1e12
+    achieved = flops / (kern_ms * 1e-3) / 1e12
+    peak, peak_kind = tensor_peak()
+
+    # end to end through the Python API: pinned host inputs in, output back
+    def pinned(a, view=None):
+        return torch.from_numpy(np.ascontiguousarray(a if view is None else a.view(view))).pin_memory()
+    hq, hk, hv = pinned(w.q, np.int16), pinned(w.key, np.int16), pinned(w.value, np.int16)
+    hs, ht, hl, hqs = (pinned(w.slot_mapping), pinned(w.block_tables), pinned(w.context_lens),
+                       pinned(w.query_start))
+    hout = torch.empty(w.q.shape, dtype=torch.int16).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(key), torch.empty_like(val)
+    ds, dt_, dl, dqs = (torch.empty_like(slots), torch.empty_like(tables), torch.empty_like(lens),
+                        torch.empty_like(qstart))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, ht, hl, hqs))
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            dq.view(torch.int16).copy_(hq, non_blocking=True)
+            dk.view(torch.int16).copy_(hk, non_blocking=True)
+            dv.view(torch.int16).copy_(hv, non_blocking=True)
+            ds.copy_(hs, non_blocking=True)
+            dt_.copy_(ht, non_blocking=True)
+            dl.copy_(hl, non_blocking=True)
+            dqs.copy_(hqs, non_blocking=True)
+        pk.reshape_and_cache(dk, dv, kc, vc, ds, dev_err=err, stream=stream)
+        pk.paged_attn_prefill(out, dq, kc, vc, dt_, dl, dqs, w.scale, w.num_kv_heads,
+                              w.block_size, w.max_context_len, max_q, dev_err=err, stream=stream)
+        with torch.cuda.stream(stream):
+            hout.copy_(out.view(torch.int16), non_blocking=True)
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    if int(err.item()) != 0:
+        raise RuntimeError("device error word %d" % int(err.item()))
+    if rank == 0:
+        line = {
+            "metric": "paged-prefill attention TFLOP/s",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": dict(W.describe(w), parallelism="replicas%d" % world,
+                           l2="no flush: each step rewrites the new tokens' K/V"),
+            "tokens_per_s": round(world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": "paged_prefill_kernel",
+                         "algorithmic_flops_per_launch": flops,
+                         "avg_launch_ms": round(kern_ms, 5),
+                         "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same "
+                                        "dense rate)" % peak_kind},
+            "e2e": {"value": round(all_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "api": "pagedkv.reshape_and_cache + paged_attn_prefill"},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()

@@ -167,6 +167,35 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
                                  void* stream);
 
 /*
+ * pkv_paged_attn_prefill — chunked-prefill attention over the paged cache.
+ * Sequence i appends q_len_i = query_start[i+1] - query_start[i] tokens in
+ * this step; their K/V must already be in the cache (pkv_reshape_and_cache),
+ * so the sequence caches context_lens[i] tokens and its j-th new token sits at
+ * position p = context_lens[i] - q_len_i + j.  That token's query attends
+ * causally to tokens 0..p, gathered through the block table as in decode
+ * ([csdn] "分页式KV缓存"; [betteryeah] §2.2, §2.4):
+ *     out[t, h, :] = softmax(scale * q[t, h, :] . K[0..p]^T) . V[0..p]
+ * with query head h reading kv head h / (num_heads / num_kv_heads).  fp32
+ * accumulation on the tensor cores; output rounded to nearest even.
+ *
+ *   q, out        device [T, num_heads, head_dim] with T = query_start[num_seqs]:
+ *                 the queries of all sequences, packed in order
+ *   query_start   device int32 [num_seqs + 1], non-decreasing, starting at 0
+ *   max_query_len an upper bound of q_len_i (sizes the launch); <= max_context_len
+ * A sequence whose q_len is negative, above its context length or above
+ * max_query_len, or whose context length is out of range, sets
+ * PKV_DEVERR_BAD_CONTEXT and its rows are left unwritten.  A table entry
+ * outside [0, num_blocks) sets PKV_DEVERR_BAD_BLOCK.  No workspace is needed.
+ */
+pkv_status pkv_paged_attn_prefill(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, const int32_t* query_start,
+                                  float scale, int num_seqs, int num_heads, int num_kv_heads,
+                                  int head_dim, int block_size, int max_blocks_per_seq,
+                                  int max_context_len, int max_query_len, int num_blocks,
+                                  pkv_dtype dtype, unsigned* dev_err, void* stream);
+
+/*
  * pkv_paged_attn_decode_static_ws — pkv_paged_attn_decode without a caller
  * workspace.  No counterpart in the source pages: it exists for callers that
  * cannot allocate device memory, such as a plugin inside a host application

@@ -1,6 +1,7 @@
 // host_common.h — host-side helpers shared by the pagedkv entry points.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,5 +19,10 @@ inline bool block_size_supported(int bs) { return bs == 16 || bs == 32; }
 inline bool dtype_valid(int dt) { return dt == PKV_FP16 || dt == PKV_BF16; }
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// 2-D TMA tensor map over a cache viewed as [num_blocks * hkv * bs, d] rows,
+// boxes of 16 rows x 64 elements with the 128-byte swizzle (cached per thread).
+pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, int hkv, int bs,
+                            int d, pkv_dtype dt);
 
 }  // namespace pkv

@@ -1,0 +1,346 @@
+// paged_prefill_kernels.cuh — chunked-prefill attention over the paged KV
+// cache for B200 (sm_100a).
+//
+// What it computes.  Sequence i appends q_len_i tokens in this step; their
+// K/V are already in the cache (written by reshape_and_cache), so the
+// sequence caches C_i tokens and its j-th new token sits at position
+// p = C_i - q_len_i + j.  That token's query attends causally to tokens 0..p,
+// gathered through the block table like decode does ([csdn] "分页式KV缓存";
+// [betteryeah] §2.2, §2.4): out = softmax(scale * q . K[0..p]^T) . V[0..p].
+//
+// How.  One CTA per (sequence, kv head, tile of 64 query rows), a row being a
+// (new token, query head of this kv head) pair.  Four consumer warps own 16
+// rows each and run FlashAttention-style on the tensor cores:
+//   S = Q K^T   mma.sync m16n8k16, rows x 16 keys (two n-tiles), K by ldmatrix
+//   P = online softmax of S (base 2), straight from the S accumulator layout
+//   O += P V    V by ldmatrix.trans, D/8 n-tiles
+// A fifth warp produces: it streams the sequence's keys 16 at a time into a
+// ring of NS stages (2-D tiled TMA with the 128-byte swizzle, one full and one
+// empty mbarrier per stage) and reads the block table 32 entries at a time.
+// Every wait is bounded.  Causal masking uses -inf before the max; keys past
+// the context are zeroed in the V fragments so stale NaN never enters a sum.
+#pragma once
+
+#include <math.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace pkv {
+
+struct PrefillParams {
+  void* out;  // [T, H, D]
+  const void* q;  // [T, H, D]
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start;  // [S + 1]
+  float qscale;  // scale * log2(e)
+  int num_seqs;
+  int num_heads;
+  int num_kv_heads;
+  int max_blocks_per_seq;
+  int max_context_len;
+  int max_query_len;
+  int num_blocks;
+  int q_tiles;  // query tiles per (sequence, kv head) at max_query_len
+  unsigned* err;
+};
+
+template <int D_, int BS_, int G_, class DT_, int NS_>
+struct PrefillTraits {
+  static constexpr int D = D_, BS = BS_, G = G_, NS = NS_;
+  using DT = DT_;
+  using T = typename DT::T;
+  static constexpr int CW = 4;                       // consumer warps
+  static constexpr int THREADS = (CW + 1) * 32;      // + the producer warp
+  static constexpr int ROWS = CW * 16;               // query rows per CTA
+  static constexpr int SUB = 16;                     // keys per stage
+  static constexpr int SUBS_PER_BLOCK = BS / SUB;
+  static constexpr int BOXES = D / 64;
+  static constexpr int BOX_BYTES = SUB * 128;
+  static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int NTD = D / 8;                  // output n-tiles
+  static constexpr int RING_BYTES = NS * STAGE_BYTES;
+  static_assert(BS % SUB == 0 && D % 64 == 0 && G >= 1 && G <= 8, "shape");
+  static size_t smem_bytes() { return 1024 + static_cast<size_t>(RING_BYTES) + NS * 16 + NS * 4; }
+};
+
+// Byte offset of 16-byte chunk `ch` of row `t` in a tile of swizzled
+// 16 x 128-byte boxes (the 128-byte TMA swizzle: chunk XOR row % 8).
+__device__ __forceinline__ uint32_t prefill_swz(int t, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * 2048 + t * 128 + (((ch & 7) ^ (t & 7)) << 4));
+}
+
+template <class Tr>
+__global__ void __launch_bounds__(Tr::THREADS)
+    paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap) {
+  using T = typename Tr::T;
+  using DT = typename Tr::DT;
+  constexpr int NS = Tr::NS, G = Tr::G, D = Tr::D, BS = Tr::BS, KS = Tr::KSTEPS;
+  constexpr int NTD = Tr::NTD, ROWS = Tr::ROWS, CW = Tr::CW, SPB = Tr::SUBS_PER_BLOCK;
+  constexpr bool kSplitP = std::is_same<DT, Bf16>::value;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
+  uint64_t* empty = full + NS;
+  int* stage_ok = reinterpret_cast<int*>(empty + NS);
+
+  // heavier tiles (later queries see more keys) are launched first
+  const int tile = p.q_tiles - 1 - static_cast<int>(blockIdx.x % p.q_tiles);
+  const int unit = blockIdx.x / p.q_tiles;
+  const int kvh = unit % p.num_kv_heads;
+  const int seq = unit / p.num_kv_heads;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  grid_dependency_wait();
+  trigger_dependents();
+
+  const int ctx = p.context_lens[seq];
+  const int q0 = p.query_start[seq];
+  const int q_len = p.query_start[seq + 1] - q0;
+  const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
+  if (ctx < 0 || ctx > cap || q_len < 0 || q_len > ctx || q_len > p.max_query_len) {
+    if (threadIdx.x == 0 && tile == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
+    return;
+  }
+  const int rows_total = q_len * G;
+  if (tile * ROWS >= rows_total) return;
+  const int last_tok = (min(rows_total, (tile + 1) * ROWS) - 1) / G;
+  const int nkv = ctx - q_len + last_tok + 1;  // keys this tile needs: 0 .. nkv-1
+  const int nsub = (nkv + Tr::SUB - 1) / Tr::SUB;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_addr(full + s), 1);
+      mbar_init(smem_addr(empty + s), CW);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const uint32_t ring0 = smem_addr(smem);
+
+  if (warp == CW) {
+    // ---- producer: keys 16 at a time through the ring ----------------------
+    const int32_t* trow = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
+    const int nblk = (nkv + BS - 1) / BS;
+    int chunk = -1, entry = -1;
+    for (int k = 0; k < nsub; ++k) {
+      const int blk = k / SPB;
+      if ((blk >> 5) != chunk) {
+        chunk = blk >> 5;
+        const int i = (chunk << 5) + lane;
+        entry = i < nblk ? trow[i] : -1;
+      }
+      const int pb = __shfl_sync(kFullMask, entry, blk & 31);
+      bool ok = true;
+      if (lane == 0) {
+        const int stage = k % NS;
+        ok = mbar_wait_bounded(smem_addr(empty + stage), ((k / NS) & 1) ^ 1);
+        if (!ok) {
+          set_err(p.err, PKV_DEVERR_TIMEOUT);
+        } else if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
+          stage_ok[stage] = 1;
+          const int y = (pb * p.num_kv_heads + kvh) * BS + (k % SPB) * Tr::SUB;
+          const uint32_t dst = ring0 + stage * Tr::STAGE_BYTES;
+          const uint32_t bar = smem_addr(full + stage);
+          mbar_arrive_expect_tx(bar, Tr::STAGE_BYTES);
+#pragma unroll
+          for (int b = 0; b < Tr::BOXES; ++b) {
+            tma_load_2d(dst + b * Tr::BOX_BYTES, &kmap, b * 64, y, bar);
+            tma_load_2d(dst + Tr::TILE_BYTES + b * Tr::BOX_BYTES, &vmap, b * 64, y, bar);
+          }
+        } else {
+          set_err(p.err, PKV_DEVERR_BAD_BLOCK);
+          stage_ok[stage] = 0;
+          mbar_arrive(smem_addr(full + stage));
+        }
+      }
+      if (!__shfl_sync(kFullMask, ok, 0)) break;
+    }
+    return;
+  }
+
+  // ---- consumers ---------------------------------------------------------
+  const int c = lane & 3;
+  const int rbase = tile * ROWS + warp * 16 + (lane >> 2);  // this lane's rows: rbase, rbase + 8
+  int pos[2];
+  const T* qrow[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = rbase + 8 * h;
+    const bool active = r < rows_total;
+    const int j = active ? r / G : 0;
+    const int g = active ? r % G : 0;
+    pos[h] = active ? ctx - q_len + j : -1;
+    qrow[h] = static_cast<const T*>(p.q) +
+              (static_cast<size_t>(q0 + j) * p.num_heads + kvh * G + g) * D;
+  }
+  // Q as A fragments: a0 (row lo, d 2c..), a1 (row hi), a2 (row lo, d 8+2c..), a3 (row hi)
+  uint32_t qa[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    qa[ks][0] = pos[0] >= 0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + 16 * ks + 2 * c) : 0u;
+    qa[ks][1] = pos[1] >= 0 ? *reinterpret_cast<const uint32_t*>(qrow[1] + 16 * ks + 2 * c) : 0u;
+    qa[ks][2] =
+        pos[0] >= 0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + 16 * ks + 8 + 2 * c) : 0u;
+    qa[ks][3] =
+        pos[1] >= 0 ? *reinterpret_cast<const uint32_t*>(qrow[1] + 16 * ks + 8 + 2 * c) : 0u;
+  }
+  float acc[NTD][4];
+#pragma unroll
+  for (int n = 0; n < NTD; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY};
+  float l[2] = {0.f, 0.f};
+
+  // keys this warp can see: up to the position of its last active row
+  const int wfirst = tile * ROWS + warp * 16;
+  const int wlast = min(rows_total, wfirst + 16) - 1;
+  const int warp_max_pos = wlast >= wfirst ? ctx - q_len + wlast / G : -1;
+  const int warp_min_pos = ctx - q_len + wfirst / G;
+  const int j8 = lane >> 3, r8 = lane & 7;
+
+  for (int k = 0; k < nsub; ++k) {
+    const int stage = k % NS;
+    const bool ok = mbar_wait_bounded(smem_addr(full + stage), (k / NS) & 1);
+    if (!__all_sync(kFullMask, ok)) {
+      if (lane == 0) {
+        set_err(p.err, PKV_DEVERR_TIMEOUT);
+        for (int jj = k; jj < min(k + NS, nsub); ++jj)
+          (void)mbar_wait_bounded(smem_addr(full + jj % NS), (jj / NS) & 1);
+      }
+      __syncwarp();
+      break;
+    }
+    const int kv0 = k * Tr::SUB;
+    if (stage_ok[stage] && kv0 <= warp_max_pos) {
+      const uint32_t kt = ring0 + stage * Tr::STAGE_BYTES;
+      const uint32_t vt = kt + Tr::TILE_BYTES;
+      // ---- S = Q K^T for 16 keys (two n-tiles) -------------------------------
+      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int t = ((j8 >> 1) << 3) + r8;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t b[4];
+          ldsm_x4(kt + prefill_swz(t, 2 * ks + (j8 & 1)), b);
+          mma_16816(s[0], qa[ks], b[0], b[1], DT());
+          mma_16816(s[1], qa[ks], b[2], b[3], DT());
+        }
+      }
+      float x[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[nt][e] = s[nt][e] * p.qscale;
+      if (kv0 + Tr::SUB - 1 > warp_min_pos) {  // the causal boundary crosses this stage
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = kv0 + nt * 8 + 2 * c + (e & 1);
+            if (key > pos[e >> 1]) x[nt][e] = -INFINITY;
+          }
+      }
+      // ---- online softmax per row (rows lo, hi; a quad of lanes shares a row)
+      float pr[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float mx = fmaxf(fmaxf(x[0][2 * h], x[0][2 * h + 1]), fmaxf(x[1][2 * h], x[1][2 * h + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
+        const float m_new = fmaxf(m[h], mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;  // fully masked row so far
+        const float alpha = exp2_approx(m[h] - m_use);
+        float sum = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            pr[nt][2 * h + e] = exp2_approx(x[nt][2 * h + e] - m_use);
+            sum += pr[nt][2 * h + e];
+          }
+        sum += __shfl_xor_sync(kFullMask, sum, 1);
+        sum += __shfl_xor_sync(kFullMask, sum, 2);
+        l[h] = l[h] * alpha + sum;
+        m[h] = m_new;
+        if (__any_sync(kFullMask, alpha != 1.f)) {
+#pragma unroll
+          for (int n = 0; n < NTD; ++n) {
+            acc[n][2 * h] *= alpha;
+            acc[n][2 * h + 1] *= alpha;
+          }
+        }
+      }
+      // ---- P as A fragments, straight from the S layout ----------------------
+      uint32_t pa[4], pl[4];
+      pa[0] = pack2(pr[0][0], pr[0][1], DT());
+      pa[1] = pack2(pr[0][2], pr[0][3], DT());
+      pa[2] = pack2(pr[1][0], pr[1][1], DT());
+      pa[3] = pack2(pr[1][2], pr[1][3], DT());
+      if constexpr (kSplitP) {
+        // bf16 P as hi + lo so P.V keeps ~16 mantissa bits
+        pl[0] = pack2(pr[0][0] - __uint_as_float(pa[0] << 16),
+                      pr[0][1] - __uint_as_float(pa[0] & 0xffff0000u), Bf16());
+        pl[1] = pack2(pr[0][2] - __uint_as_float(pa[1] << 16),
+                      pr[0][3] - __uint_as_float(pa[1] & 0xffff0000u), Bf16());
+        pl[2] = pack2(pr[1][0] - __uint_as_float(pa[2] << 16),
+                      pr[1][1] - __uint_as_float(pa[2] & 0xffff0000u), Bf16());
+        pl[3] = pack2(pr[1][2] - __uint_as_float(pa[3] << 16),
+                      pr[1][3] - __uint_as_float(pa[3] & 0xffff0000u), Bf16());
+      }
+      // keys past the context may hold stale data: zero them in the V fragments
+      const int vkeep = ctx - kv0;  // keys of this stage inside the context
+      uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+      if (vkeep < Tr::SUB) {
+        const int t0 = 2 * c, t1 = 8 + 2 * c;
+        keep_lo = (t0 < vkeep ? 0x0000ffffu : 0u) | (t0 + 1 < vkeep ? 0xffff0000u : 0u);
+        keep_hi = (t1 < vkeep ? 0x0000ffffu : 0u) | (t1 + 1 < vkeep ? 0xffff0000u : 0u);
+      }
+      // ---- O += P V -------------------------------------------------------------
+      {
+        const int t = ((j8 & 1) << 3) + r8;
+#pragma unroll
+        for (int pair = 0; pair < NTD / 2; ++pair) {
+          uint32_t b[4];
+          ldsm_x4_trans(vt + prefill_swz(t, 2 * pair + (j8 >> 1)), b);
+          b[0] &= keep_lo;
+          b[1] &= keep_hi;
+          b[2] &= keep_lo;
+          b[3] &= keep_hi;
+          mma_16816(acc[2 * pair], pa, b[0], b[1], DT());
+          mma_16816(acc[2 * pair + 1], pa, b[2], b[3], DT());
+          if constexpr (kSplitP) {
+            mma_16816(acc[2 * pair], pl, b[0], b[1], DT());
+            mma_16816(acc[2 * pair + 1], pl, b[2], b[3], DT());
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(empty + stage));
+  }
+
+  // ---- normalise and store this lane's rows -------------------------------------
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (pos[h] < 0) continue;
+    const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
+    T* orow = static_cast<T*>(p.out) + (qrow[h] - static_cast<const T*>(p.q));
+#pragma unroll
+    for (int n = 0; n < NTD; ++n) {
+      *reinterpret_cast<uint32_t*>(orow + n * 8 + 2 * c) =
+          pack2(acc[n][2 * h] * inv, acc[n][2 * h + 1] * inv, DT());
+    }
+  }
+}
+
+}  // namespace pkv

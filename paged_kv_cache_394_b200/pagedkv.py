@@ -49,6 +49,8 @@ _paged_attn_decode_static_ws = _proto("pkv_paged_attn_decode_static_ws", _i, _vp
                                      _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                      _vp)
 STATIC_WORKSPACE_BYTES = 16 << 20
+_paged_attn_prefill = _proto("pkv_paged_attn_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i,
+                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp)
 _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
 _decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
                            _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
@@ -216,6 +218,33 @@ def paged_attn_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_
                                         num_blocks, _dtype_code(q), partition_size,
                                         _ptr(dev_err), _stream(stream)),
            "paged_attn_decode_static_ws")
+
+
+def paged_attn_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start, scale,
+                       num_kv_heads, block_size, max_context_len, max_query_len, dev_err=None,
+                       stream=None):
+    """Chunked-prefill attention; q/out are [T, H, D], query_start [S+1].  See
+    include/pagedkv.h."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    _dev(query_start, "query_start", torch.int32)
+    t, h, d = q.shape
+    num_blocks, hkv, bs, dk = k_cache.shape
+    s = context_lens.shape[0]
+    if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if query_start.shape != (s + 1,) or block_tables.shape[0] != s:
+        raise ValueError("query_start must be [S+1], block_tables [S, max_blocks]")
+    if q.dtype != k_cache.dtype or out.dtype != q.dtype:
+        raise TypeError("q, out and caches must share a dtype")
+    _check(_paged_attn_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                               _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
+                               float(scale), s, h, hkv, d, bs, block_tables.shape[1],
+                               max_context_len, max_query_len, num_blocks, _dtype_code(q),
+                               _ptr(dev_err), _stream(stream)),
+           "paged_attn_prefill")
 
 
 def staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,

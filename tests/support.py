@@ -46,6 +46,8 @@ class DeviceWorkload:
         self.lens = torch.from_numpy(w.context_lens).cuda()
         self.out = torch.empty_like(self.q)
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.qstart = (torch.from_numpy(w.query_start).cuda()
+                       if w.query_start is not None else None)
 
 
 def run_step(pk, dw, partition_size=None, decode=True):
@@ -62,6 +64,23 @@ def run_step(pk, dw, partition_size=None, decode=True):
                              partition_size=part, dev_err=dw.err)
     torch.cuda.synchronize()
     return int(dw.err.item())
+
+
+def run_prefill_step(pk, dw):
+    """reshape_and_cache of the new tokens, then chunked-prefill attention."""
+    w = dw.w
+    pk.reshape_and_cache(dw.key, dw.value, dw.k_cache, dw.v_cache, dw.slots, dev_err=dw.err)
+    pk.paged_attn_prefill(dw.out, dw.q, dw.k_cache, dw.v_cache, dw.tables, dw.lens, dw.qstart,
+                          w.scale, w.num_kv_heads, w.block_size, w.max_context_len,
+                          int(np.diff(w.query_start).max()), dev_err=dw.err)
+    torch.cuda.synchronize()
+    return int(dw.err.item())
+
+
+def oracle_prefill(w, kc, vc, rows=None):
+    return OA.paged_attention_prefill(w.q, kc, vc, w.block_tables, w.context_lens,
+                                      w.query_start, w.scale, w.num_kv_heads, w.block_size,
+                                      w.dtype, rows=rows)
 
 
 def oracle_caches(w, inplace=False):

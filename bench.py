@@ -588,6 +588,77 @@ def cpu_baseline(w, seconds):
                       "heads), %.1f s on the host cores" % (n, w.num_seqs, w.num_heads, dt)}
 
 
+def replay_trace(mgr, trace, cached, max_live=64):
+    """Admits the trace's requests in order, up to max_live at a time; every
+    iteration appends one generated token to each live request and frees those
+    that are done.  Works on the C++ allocator and on the oracle alike."""
+    import collections
+    live = collections.OrderedDict()
+    prompt_tokens = cached_tokens = peak = 0
+    ops = 0
+    for rid, (toks, out_len) in enumerate(trace):
+        while len(live) >= max_live:
+            for sid in list(live):
+                mgr.append_slot(sid)
+                ops += 1
+                live[sid] -= 1
+                if live[sid] == 0:
+                    mgr.free_seq(sid)
+                    ops += 1
+                    del live[sid]
+        if cached:
+            cached_tokens += mgr.add_seq_cached(rid, toks)
+        else:
+            mgr.add_seq(rid, len(toks))
+        ops += 1
+        prompt_tokens += len(toks)
+        live[rid] = out_len
+        peak = max(peak, mgr.num_blocks - mgr.num_free() - (mgr.num_evictable() if cached else 0))
+    for sid in list(live):
+        mgr.free_seq(sid)
+        ops += 1
+    return prompt_tokens, cached_tokens, peak, ops
+
+
+def run_prefix_cache_trace(args):
+    """Host measurement of prefix caching on a seeded chat trace."""
+    from oracle.block_manager import BlockManager
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    from paged_kv_cache_394_b200 import workloads as W
+    trace = W.chat_trace(W.SEED_BASE + 50)
+    nb, bs = 16384, 16
+    res = {}
+    for cached in (True, False):
+        mgr = pk.BlockAllocator(nb, bs)
+        t0 = time.perf_counter()
+        prompt, hit_tokens, peak, ops = replay_trace(mgr, trace, cached)
+        dt = time.perf_counter() - t0
+        res[cached] = (prompt, hit_tokens, peak, ops, dt, mgr.cache_stats())
+    ref = BlockManager(nb, bs)
+    t0 = time.perf_counter()
+    _, ref_hit, ref_peak, ref_ops, = replay_trace(ref, trace, True)
+    ref_dt = time.perf_counter() - t0
+    prompt, hit_tokens, peak, ops, dt, stats = res[True]
+    q, h, _, ev = stats
+    if (ref_hit, ref_peak) != (hit_tokens, peak) or ref.cache_stats()[:2] != (q, h):
+        raise RuntimeError("allocator and oracle disagree on the trace")
+    line = {
+        "metric": "prefix-cache hit rate on a shared-system-prompt chat trace",
+        "value": round(h / q, 4), "unit": "fraction", "higher_is_better": True,
+        "config": {"workload": "prefix_cache_trace", "requests": len(trace), "system_prompts": 8,
+                   "zipf_a": 1.2, "num_blocks": nb, "block_size": bs, "max_live": 64},
+        "prefill_tokens_saved": round(hit_tokens / prompt, 4),
+        "peak_blocks": {"cached": peak, "uncached": res[False][2],
+                        "saved": round(1 - peak / res[False][2], 4)},
+        "evicted_blocks": ev,
+        "allocator_ops_per_s": round(ops / dt, 1),
+        "cpu_baseline": {"value": round(ref_ops / ref_dt, 1), "unit": "ops/s", "cores": 1,
+                         "kind": "oracle", "sample": "the same trace through oracle.block_manager"},
+        "data": "synthetic",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -639,7 +710,9 @@ def main(argv=None):
     args = parse_args(argv)
     # at least three untimed warm-up steps, whatever was asked
     args.warmup = max(3, args.warmup)
-    if args.impl == "reference":
+    if args.workload == "prefix_cache_trace":
+        run_prefix_cache_trace(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -298,6 +298,8 @@ pkv_status pkv_alloc_block_table(const pkv_alloc* a, const int64_t* seq_ids, int
 pkv_status pkv_alloc_context_lens(const pkv_alloc* a, const int64_t* seq_ids, int n,
                                   int32_t* lens_out);
 int pkv_alloc_num_free(const pkv_alloc* a);
+/* Cached blocks with refcount 0 (kept for reuse, evicted when the free list is empty). */
+int pkv_alloc_num_evictable(const pkv_alloc* a);
 /* -1 for an out-of-range block. */
 int pkv_alloc_refcount(const pkv_alloc* a, int block);
 /* -1 for an unknown sequence. */
@@ -307,6 +309,33 @@ int pkv_alloc_seq_num_blocks(const pkv_alloc* a, int64_t seq_id);
  * block's fill is the most slots any holder has filled); utilization is
  * cached_tokens / (used_blocks * block_size). */
 pkv_status pkv_alloc_usage(const pkv_alloc* a, int64_t* cached_tokens, int64_t* used_blocks);
+
+/*
+ * Prefix caching ([csdn] API example: `enable_prefix_caching`, and the
+ * `cache_hit_rate` it recommends monitoring; sequences with a common prompt
+ * point at the same first pages, [csdn] "分页式KV缓存").
+ *
+ * pkv_alloc_add_seq_cached admits a sequence whose prompt is token_ids[0..n).
+ * A full block is identified by its whole token prefix.  The prompt's full
+ * blocks are looked up in order; the cached ones are reused (refcount + 1) up
+ * to the first miss, the rest are taken fresh, and each fresh full block is
+ * registered under its prefix (the caller writes its K/V in the same step).
+ * Partial blocks are never cached.  *num_cached_tokens receives the number of
+ * leading prompt tokens whose K/V are already in the cache.
+ *
+ * A cached block whose refcount drops to zero stays cached and is evictable,
+ * least recently released first; an allocation that finds the free list empty
+ * evicts the oldest one.  Prefixes are compared through a 64-bit chain hash
+ * plus the block's own tokens, so two different prefixes are confused only
+ * on a 64-bit hash collision.  OUT_OF_BLOCKS leaves the state unchanged.
+ */
+pkv_status pkv_alloc_add_seq_cached(pkv_alloc* a, int64_t seq_id, const int32_t* token_ids,
+                                    int64_t num_tokens, int64_t* num_cached_tokens);
+/* Full blocks looked up, hits among them, blocks cached now, blocks evicted so far.
+ * cache_hit_rate = hit_blocks / queried_blocks.  Any output may be NULL. */
+pkv_status pkv_alloc_cache_stats(const pkv_alloc* a, int64_t* queried_blocks,
+                                 int64_t* hit_blocks, int64_t* cached_blocks,
+                                 int64_t* evicted_blocks);
 
 #ifdef __cplusplus
 }

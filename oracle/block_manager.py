@@ -34,6 +34,23 @@ Readings taken where the pages are silent:
 * An append at a block boundary takes a fresh block and needs no copy.
 * Freeing walks the sequence's blocks front to back; each block whose
   refcount reaches zero is appended to the free queue.
+
+Prefix caching (the ``enable_prefix_caching`` switch and the ``cache_hit_rate``
+metric of [csdn]; sequences with a common prompt pointing at the same first
+pages, [csdn] "分页式KV缓存"):
+
+* A full block is identified by the exact token sequence from the start of
+  its sequence through its last token.  ``add_seq_cached`` looks the prompt's
+  full blocks up in order and reuses the cached ones up to the first miss;
+  every freshly taken full block is registered under its prefix unless that
+  prefix is already cached (a prefix keeps its first registered block while
+  that block stays cached; such a block becomes unreachable when an earlier
+  block of its prefix is evicted, and reachable again once that earlier
+  prefix is re-registered).  Partial blocks are never cached.
+* A cached block whose refcount drops to zero stays cached and becomes
+  evictable, least recently released first.  Allocation takes the free queue
+  first, then evicts the oldest evictable block (dropping its cache entry).
+* Hit rate = full blocks found / full blocks looked up.
 """
 
 from collections import deque
@@ -64,10 +81,19 @@ class BlockManager:
         self.free = deque(order)
         self.refcount = [0] * num_blocks
         self.seqs = {}  # seq_id -> {"blocks": [..], "tokens": n}
+        self.cache = {}         # full token prefix (tuple) -> block
+        self.cache_key = {}     # block -> its prefix key
+        self.evictable = []     # cached blocks with refcount 0, oldest first
+        self.queried = 0
+        self.hits = 0
+        self.evicted = 0
 
     # -- queries ---------------------------------------------------------
     def num_free(self):
         return len(self.free)
+
+    def num_evictable(self):
+        return len(self.evictable)
 
     def seq_blocks(self, seq_id):
         return list(self.seqs[seq_id]["blocks"])
@@ -77,18 +103,34 @@ class BlockManager:
 
     # -- operations ------------------------------------------------------
     def _take(self):
-        if not self.free:
+        if self.free:
+            b = self.free.popleft()
+        elif self.evictable:
+            b = self.evictable.pop(0)
+            del self.cache[self.cache_key.pop(b)]
+            self.evicted += 1
+        else:
             raise AllocError("OUT_OF_BLOCKS", "pool exhausted")
-        b = self.free.popleft()
         self.refcount[b] = 1
         return b
+
+    def _available(self):
+        return len(self.free) + len(self.evictable)
+
+    def _release(self, b):
+        self.refcount[b] -= 1
+        if self.refcount[b] == 0:
+            if b in self.cache_key:
+                self.evictable.append(b)
+            else:
+                self.free.append(b)
 
     def add_seq(self, seq_id, num_tokens):
         if seq_id in self.seqs or num_tokens < 0:
             raise AllocError("INVALID_ARG", "bad seq id or length")
         need = blocks_for(num_tokens, self.block_size)
-        if need > len(self.free):
-            raise AllocError("OUT_OF_BLOCKS", "need %d, have %d" % (need, len(self.free)))
+        if need > self._available():
+            raise AllocError("OUT_OF_BLOCKS", "need %d, have %d" % (need, self._available()))
         self.seqs[seq_id] = {"blocks": [self._take() for _ in range(need)],
                              "tokens": num_tokens}
 
@@ -113,10 +155,14 @@ class BlockManager:
         offset = pos % self.block_size
         cow_src = cow_dst = -1
         if offset == 0:
+            if not self._available():
+                raise AllocError("OUT_OF_BLOCKS", "pool exhausted")
             seq["blocks"].append(self._take())
         else:
             last = seq["blocks"][-1]
             if self.refcount[last] > 1:
+                if not self._available():
+                    raise AllocError("OUT_OF_BLOCKS", "pool exhausted")
                 fresh = self._take()
                 self.refcount[last] -= 1
                 seq["blocks"][-1] = fresh
@@ -128,9 +174,49 @@ class BlockManager:
         if seq_id not in self.seqs:
             raise AllocError("INVALID_ARG", "unknown seq id")
         for b in self.seqs.pop(seq_id)["blocks"]:
-            self.refcount[b] -= 1
+            self._release(b)
+
+    def add_seq_cached(self, seq_id, tokens):
+        """Admit a sequence whose prompt is ``tokens``, reusing cached full
+        blocks of its longest cached prefix.  Returns the number of prompt
+        tokens whose K/V are already cached."""
+        tokens = [int(t) for t in tokens]
+        if seq_id in self.seqs:
+            raise AllocError("INVALID_ARG", "bad seq id")
+        bs = self.block_size
+        n = len(tokens)
+        nfull = n // bs
+        need = blocks_for(n, bs)
+        hits = []
+        for k in range(nfull):
+            b = self.cache.get(tuple(tokens[:(k + 1) * bs]))
+            if b is None:
+                break
+            hits.append(b)
+        reclaimed = sum(1 for b in hits if self.refcount[b] == 0)
+        if need - len(hits) > self._available() - reclaimed:
+            raise AllocError("OUT_OF_BLOCKS", "pool exhausted")
+        self.queried += nfull
+        self.hits += len(hits)
+        for b in hits:
             if self.refcount[b] == 0:
-                self.free.append(b)
+                self.evictable.remove(b)
+            self.refcount[b] += 1
+        blocks = list(hits)
+        for k in range(len(hits), need):
+            b = self._take()
+            if k < nfull:
+                key = tuple(tokens[:(k + 1) * bs])
+                if key not in self.cache:
+                    self.cache[key] = b
+                    self.cache_key[b] = key
+            blocks.append(b)
+        self.seqs[seq_id] = {"blocks": blocks, "tokens": n}
+        return len(hits) * bs
+
+    def cache_stats(self):
+        """(full blocks looked up, hits, blocks cached now, blocks evicted)."""
+        return self.queried, self.hits, len(self.cache), self.evicted
 
     def block_table(self, seq_ids, max_blocks):
         """Rows of physical block ids, padded with -1."""

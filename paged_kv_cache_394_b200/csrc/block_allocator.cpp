@@ -11,9 +11,20 @@
 // with a caller-given initial order; copy-on-write only on an append into a
 // partly filled last block whose refcount exceeds one; the last holder writes
 // in place.  Every failing call leaves the state unchanged.
+//
+// Prefix caching ([csdn] API example `enable_prefix_caching` and its
+// `cache_hit_rate` metric): a full prompt block is known by its whole token
+// prefix.  Here that prefix is represented by a chain hash,
+// h_k = mix(h_{k-1}, tokens of block k), with splitmix64 as the mixer
+// (Steele, Lea and Flood, "Fast splittable pseudorandom number generators",
+// 2014); a candidate block must also carry the same parent hash and the same
+// block tokens, so two prefixes are confused only on a 64-bit collision of the
+// parent chain.  Cached blocks whose refcount drops to zero stay cached on an
+// LRU list and are evicted only when the free queue is empty.
 #include <algorithm>
 #include <climits>
 #include <deque>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -25,23 +36,78 @@ struct pkv_alloc {
     std::vector<int> blocks;
     int64_t tokens = 0;
   };
+  struct CacheEntry {
+    bool cached = false;
+    uint64_t hash = 0;         // chain hash of the block's prefix
+    uint64_t parent_hash = 0;  // chain hash of the prefix before it
+    std::vector<int32_t> tokens;
+    std::list<int>::iterator lru;  // valid while the block is evictable
+    bool evictable = false;
+  };
   int num_blocks = 0;
   int block_size = 0;
   std::deque<int> free_q;
   std::vector<int> refcount;
   std::unordered_map<int64_t, Seq> seqs;
+  std::vector<CacheEntry> entry;                 // per physical block
+  std::unordered_map<uint64_t, int> cache;       // chain hash -> block
+  std::list<int> evictable;                      // refcount-0 cached blocks, oldest first
+  int64_t queried = 0, hits = 0, evicted = 0;
 
+  int available() const { return static_cast<int>(free_q.size() + evictable.size()); }
+
+  // A block with refcount 1: the free queue first, else the oldest evictable
+  // cached block (its cache entry is dropped).  The caller checked available().
   int take() {
-    const int b = free_q.front();
-    free_q.pop_front();
+    int b;
+    if (!free_q.empty()) {
+      b = free_q.front();
+      free_q.pop_front();
+    } else {
+      b = evictable.front();
+      evictable.pop_front();
+      CacheEntry& e = entry[b];
+      cache.erase(e.hash);
+      e.cached = false;
+      e.evictable = false;
+      e.tokens.clear();
+      ++evicted;
+    }
     refcount[b] = 1;
     return b;
+  }
+
+  void release(int b) {
+    if (--refcount[b] == 0) {
+      CacheEntry& e = entry[b];
+      if (e.cached) {
+        e.lru = evictable.insert(evictable.end(), b);
+        e.evictable = true;
+      } else {
+        free_q.push_back(b);
+      }
+    }
   }
 };
 
 namespace {
 
 int64_t blocks_for(int64_t tokens, int bs) { return (tokens + bs - 1) / bs; }
+
+uint64_t splitmix64(uint64_t x) {
+  x += 0x9e3779b97f4a7c15ull;
+  x = (x ^ (x >> 30)) * 0xbf58476d1ce4e5b9ull;
+  x = (x ^ (x >> 27)) * 0x94d049bb133111ebull;
+  return x ^ (x >> 31);
+}
+
+constexpr uint64_t kRootHash = 0x243f6a8885a308d3ull;  // chain hash of the empty prefix
+
+uint64_t chain_hash(uint64_t parent, const int32_t* tokens, int n) {
+  uint64_t h = splitmix64(parent);
+  for (int i = 0; i < n; ++i) h = splitmix64(h ^ static_cast<uint32_t>(tokens[i]));
+  return h;
+}
 
 }  // namespace
 
@@ -53,6 +119,7 @@ extern "C" pkv_alloc* pkv_alloc_create(int num_blocks, int block_size,
   a->num_blocks = num_blocks;
   a->block_size = block_size;
   a->refcount.assign(num_blocks, 0);
+  a->entry.resize(num_blocks);
   if (free_order == nullptr) {
     for (int b = 0; b < num_blocks; ++b) a->free_q.push_back(b);
   } else {
@@ -75,7 +142,7 @@ extern "C" void pkv_alloc_destroy(pkv_alloc* a) { delete a; }
 extern "C" pkv_status pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id, int64_t num_tokens) {
   if (a == nullptr || num_tokens < 0 || a->seqs.count(seq_id)) return PKV_ERR_INVALID_ARG;
   const int64_t need = blocks_for(num_tokens, a->block_size);
-  if (need > static_cast<int64_t>(a->free_q.size())) return PKV_ERR_OUT_OF_BLOCKS;
+  if (need > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
   pkv_alloc::Seq s;
   s.tokens = num_tokens;
   s.blocks.reserve(static_cast<size_t>(need));
@@ -104,12 +171,12 @@ extern "C" pkv_status pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_
   const int offset = static_cast<int>(pos % a->block_size);
   int64_t src = -1, dst = -1;
   if (offset == 0) {
-    if (a->free_q.empty()) return PKV_ERR_OUT_OF_BLOCKS;
+    if (a->available() == 0) return PKV_ERR_OUT_OF_BLOCKS;
     s.blocks.push_back(a->take());
   } else {
     const int last = s.blocks.back();
     if (a->refcount[last] > 1) {
-      if (a->free_q.empty()) return PKV_ERR_OUT_OF_BLOCKS;
+      if (a->available() == 0) return PKV_ERR_OUT_OF_BLOCKS;
       const int fresh = a->take();
       a->refcount[last] -= 1;
       s.blocks.back() = fresh;
@@ -153,11 +220,86 @@ extern "C" pkv_status pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id) {
   if (a == nullptr) return PKV_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
-  for (int b : it->second.blocks) {
-    if (--a->refcount[b] == 0) a->free_q.push_back(b);
-  }
+  for (int b : it->second.blocks) a->release(b);
   a->seqs.erase(it);
   return PKV_OK;
+}
+
+extern "C" pkv_status pkv_alloc_add_seq_cached(pkv_alloc* a, int64_t seq_id,
+                                               const int32_t* token_ids, int64_t num_tokens,
+                                               int64_t* num_cached_tokens) {
+  if (a == nullptr || num_tokens < 0 || a->seqs.count(seq_id) ||
+      (num_tokens > 0 && token_ids == nullptr))
+    return PKV_ERR_INVALID_ARG;
+  const int bs = a->block_size;
+  const int64_t nfull = num_tokens / bs;
+  const int64_t need = blocks_for(num_tokens, bs);
+  // look the full blocks up in order, up to the first miss
+  std::vector<int> hit;
+  std::vector<uint64_t> hashes;
+  uint64_t parent = kRootHash;
+  for (int64_t k = 0; k < nfull; ++k) {
+    const int32_t* tok = token_ids + k * bs;
+    const uint64_t h = chain_hash(parent, tok, bs);
+    hashes.push_back(h);
+    if (static_cast<int64_t>(hit.size()) == k) {
+      auto f = a->cache.find(h);
+      if (f != a->cache.end()) {
+        const pkv_alloc::CacheEntry& e = a->entry[f->second];
+        if (e.parent_hash == parent && std::equal(e.tokens.begin(), e.tokens.end(), tok))
+          hit.push_back(f->second);
+      }
+    }
+    parent = h;
+  }
+  int reclaimed = 0;
+  for (int b : hit) reclaimed += a->refcount[b] == 0 ? 1 : 0;
+  if (need - static_cast<int64_t>(hit.size()) > a->available() - reclaimed)
+    return PKV_ERR_OUT_OF_BLOCKS;
+  a->queried += nfull;
+  a->hits += static_cast<int64_t>(hit.size());
+  pkv_alloc::Seq s;
+  s.tokens = num_tokens;
+  s.blocks.reserve(static_cast<size_t>(need));
+  for (int b : hit) {
+    pkv_alloc::CacheEntry& e = a->entry[b];
+    if (a->refcount[b] == 0) {
+      a->evictable.erase(e.lru);
+      e.evictable = false;
+    }
+    a->refcount[b] += 1;
+    s.blocks.push_back(b);
+  }
+  for (int64_t k = static_cast<int64_t>(hit.size()); k < need; ++k) {
+    const int b = a->take();
+    if (k < nfull && a->cache.find(hashes[k]) == a->cache.end()) {
+      pkv_alloc::CacheEntry& e = a->entry[b];
+      e.cached = true;
+      e.hash = hashes[k];
+      e.parent_hash = k == 0 ? kRootHash : hashes[k - 1];
+      e.tokens.assign(token_ids + k * bs, token_ids + (k + 1) * bs);
+      a->cache.emplace(hashes[k], b);
+    }
+    s.blocks.push_back(b);
+  }
+  a->seqs.emplace(seq_id, std::move(s));
+  if (num_cached_tokens) *num_cached_tokens = static_cast<int64_t>(hit.size()) * bs;
+  return PKV_OK;
+}
+
+extern "C" pkv_status pkv_alloc_cache_stats(const pkv_alloc* a, int64_t* queried_blocks,
+                                            int64_t* hit_blocks, int64_t* cached_blocks,
+                                            int64_t* evicted_blocks) {
+  if (a == nullptr) return PKV_ERR_INVALID_ARG;
+  if (queried_blocks) *queried_blocks = a->queried;
+  if (hit_blocks) *hit_blocks = a->hits;
+  if (cached_blocks) *cached_blocks = static_cast<int64_t>(a->cache.size());
+  if (evicted_blocks) *evicted_blocks = a->evicted;
+  return PKV_OK;
+}
+
+extern "C" int pkv_alloc_num_evictable(const pkv_alloc* a) {
+  return a ? static_cast<int>(a->evictable.size()) : -1;
 }
 
 extern "C" pkv_status pkv_alloc_block_table(const pkv_alloc* a, const int64_t* seq_ids, int n,

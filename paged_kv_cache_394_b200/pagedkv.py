@@ -69,6 +69,9 @@ _alloc_refcount = _proto("pkv_alloc_refcount", _i, _vp, _i)
 _alloc_seq_len = _proto("pkv_alloc_seq_len", _i64, _vp, _i64)
 _alloc_seq_num_blocks = _proto("pkv_alloc_seq_num_blocks", _i, _vp, _i64)
 _alloc_usage = _proto("pkv_alloc_usage", _i, _vp, _vp, _vp)
+_alloc_add_seq_cached = _proto("pkv_alloc_add_seq_cached", _i, _vp, _i64, _vp, _i64, _vp)
+_alloc_cache_stats = _proto("pkv_alloc_cache_stats", _i, _vp, _vp, _vp, _vp, _vp)
+_alloc_num_evictable = _proto("pkv_alloc_num_evictable", _i, _vp)
 
 
 class PagedKVError(RuntimeError):
@@ -364,3 +367,21 @@ class BlockAllocator:
         tokens, blocks = ctypes.c_int64(), ctypes.c_int64()
         _check(_alloc_usage(self._h, ctypes.byref(tokens), ctypes.byref(blocks)), "usage")
         return tokens.value, blocks.value
+
+    def add_seq_cached(self, seq_id, token_ids):
+        """Admit a prompt, reusing cached full blocks; returns cached token count."""
+        n = len(token_ids)
+        arr = (ctypes.c_int32 * max(n, 1))(*[int(t) for t in token_ids])
+        cached = ctypes.c_int64()
+        _check(_alloc_add_seq_cached(self._h, seq_id, arr, n, ctypes.byref(cached)),
+               "add_seq_cached")
+        return cached.value
+
+    def cache_stats(self):
+        """(full blocks looked up, hits, blocks cached now, blocks evicted)."""
+        vals = [ctypes.c_int64() for _ in range(4)]
+        _check(_alloc_cache_stats(self._h, *[ctypes.byref(v) for v in vals]), "cache_stats")
+        return tuple(v.value for v in vals)
+
+    def num_evictable(self):
+        return _alloc_num_evictable(self._h)

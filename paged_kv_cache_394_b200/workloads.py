@@ -296,6 +296,25 @@ def build_prefill_workload(hist_lens, new_lens, num_heads, num_kv_heads, head_di
                     notes={"seed": seed})
 
 
+def chat_trace(seed, num_requests=2000, num_system=8, zipf_a=1.2, system_len=(256, 1024),
+               user_len=(32, 512), output_len=(16, 128), vocab=32000):
+    """Synthetic chat requests sharing system prompts, for prefix caching.
+
+    Each request = one of ``num_system`` system prompts (chosen with a Zipf
+    law, so a few are popular) + a random user turn, and generates a random
+    number of tokens.  Returns a list of (prompt token ids, output length).
+    """
+    rng = np.random.default_rng(seed)
+    systems = [rng.integers(0, vocab, int(rng.integers(*system_len))).tolist()
+               for _ in range(num_system)]
+    ranks = np.minimum(rng.zipf(zipf_a, num_requests), num_system) - 1
+    reqs = []
+    for r in ranks:
+        user = rng.integers(0, vocab, int(rng.integers(*user_len))).tolist()
+        reqs.append((systems[int(r)] + user, int(rng.integers(*output_len))))
+    return reqs
+
+
 def chat_lengths(rng, n, median=600.0, sigma=1.0, low=16, high=4096):
     """Lognormal lengths with the given median, clipped and rounded."""
     x = rng.lognormal(mean=math.log(median), sigma=sigma, size=n)

@@ -118,3 +118,43 @@ def test_error_statuses():
         a.block_table([7], 1)
     assert a.refcount(5) == -1 and a.seq_len(99) == -1
     assert a.seq_num_blocks(7) == 2
+
+
+@pytest.mark.parametrize("seed,num_blocks,bs", [(11, 48, 4), (12, 120, 16), (13, 20, 2)])
+def test_prefix_cache_traces_match_oracle(seed, num_blocks, bs):
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(num_blocks)
+    ref = BlockManager(num_blocks, bs, free_order=order)
+    lib = pk.BlockAllocator(num_blocks, bs, free_order=order)
+    # a few "system prompts" so that prefixes repeat, plus random tails
+    bases = [list(rng.integers(0, 7, int(rng.integers(0, 6 * bs)))) for _ in range(5)]
+    live, next_id = [], 0
+    for _ in range(1200):
+        op = int(rng.integers(0, 10))
+        if op < 4 or not live:
+            toks = bases[int(rng.integers(len(bases)))] + \
+                list(rng.integers(0, 7, int(rng.integers(0, 2 * bs))))
+            if both(lambda: ref.add_seq_cached(next_id, toks),
+                    lambda: lib.add_seq_cached(next_id, toks)):
+                live.append(next_id)
+            next_id += 1
+        elif op < 5:
+            parent = live[int(rng.integers(len(live)))]
+            if both(lambda: ref.fork(parent, next_id), lambda: lib.fork(parent, next_id)):
+                live.append(next_id)
+            next_id += 1
+        elif op < 7:
+            s = live[int(rng.integers(len(live)))]
+            both(lambda: ref.append_slot(s), lambda: lib.append_slot(s))
+        else:
+            s = live.pop(int(rng.integers(len(live))))
+            both(lambda: ref.free_seq(s), lambda: lib.free_seq(s))
+        assert lib.num_free() == ref.num_free()
+        assert lib.num_evictable() == ref.num_evictable()
+        assert lib.cache_stats() == ref.cache_stats()
+        if live:
+            mb = max(1, max(len(ref.seq_blocks(s)) for s in live))
+            assert lib.block_table(live, mb) == ref.block_table(live, mb)
+    assert [lib.refcount(b) for b in range(num_blocks)] == ref.refcount
+    q, h, _, ev = lib.cache_stats()
+    assert h > 0 and ev > 0          # the trace exercised hits and evictions

@@ -160,3 +160,79 @@ def test_invalid_arguments():
         mgr.block_table([0], 0)
     with pytest.raises(AllocError):
         BlockManager(4, 16, free_order=[0, 1, 1, 2])
+
+
+# ---------------------------------------------------------------------------
+# prefix caching
+# ---------------------------------------------------------------------------
+def test_shared_system_prompt_hit_rate_closed_form():
+    # n requests = k-block system prompt + a distinct 3-block suffix each:
+    # the first misses everything, each later one hits exactly the k prompt blocks
+    bs, k, n = 16, 5, 7
+    rng = np.random.default_rng(0)
+    system = list(rng.integers(0, 1000, k * bs))
+    mgr = BlockManager(200, bs)
+    for i in range(n):
+        suffix = list(rng.integers(1000, 2000, 3 * bs))
+        cached = mgr.add_seq_cached(i, system + suffix)
+        assert cached == (0 if i == 0 else k * bs)
+    queried, hits, cached_blocks, evicted = mgr.cache_stats()
+    assert queried == n * (k + 3) and hits == (n - 1) * k
+    assert hits / queried == pytest.approx((n - 1) * k / (n * (k + 3)))
+    assert cached_blocks == k + 3 * n and evicted == 0
+    # sharing: n sequences hold n*(k+3) logical blocks in k + 3n physical ones
+    assert 200 - mgr.num_free() == k + 3 * n
+
+
+def test_freed_prompt_stays_cached_then_hits():
+    mgr = BlockManager(10, 4)
+    toks = list(range(10))                  # 2 full blocks + 2 tokens
+    assert mgr.add_seq_cached(0, toks) == 0
+    mgr.free_seq(0)
+    assert mgr.num_evictable() == 2 and mgr.num_free() == 8   # the partial block is not cached
+    assert mgr.add_seq_cached(1, toks) == 8
+    assert mgr.num_evictable() == 0
+
+
+def test_lru_eviction_breaks_the_chain():
+    mgr = BlockManager(4, 2)
+    a = [1, 2, 3, 4]
+    mgr.add_seq_cached(0, a)                # blocks 0, 1 cached
+    mgr.free_seq(0)                         # evictable: 0 (older), 1
+    mgr.add_seq_cached(1, [5, 6, 7, 8])     # takes free blocks 2, 3
+    mgr.add_seq_cached(2, [9, 10])          # free list empty: evicts block 0 (a's first)
+    assert mgr.seq_blocks(2) == [0]
+    _, _, cached, evicted = mgr.cache_stats()
+    assert evicted == 1 and cached == 4 - 1 + 1   # a's 2nd block, [5..8]'s two, [9,10]
+    mgr.free_seq(2)
+    # a's first block is gone, so its second (still cached) cannot be reached
+    assert mgr.add_seq_cached(3, a) == 0
+
+
+def test_prefix_cache_keeps_refcounts_and_blocks_consistent():
+    rng = np.random.default_rng(9)
+    bs = 4
+    mgr = BlockManager(40, bs, free_order=rng.permutation(40))
+    prompts = [list(rng.integers(0, 5, int(rng.integers(1, 30)))) for _ in range(6)]
+    live = []
+    for step in range(400):
+        op = rng.integers(0, 4)
+        try:
+            if op == 0 or not live:
+                p = prompts[int(rng.integers(len(prompts)))]
+                p = p + list(rng.integers(0, 5, int(rng.integers(0, 6))))
+                mgr.add_seq_cached(step, p)
+                live.append(step)
+            elif op == 1:
+                mgr.append_slot(live[int(rng.integers(len(live)))])
+            else:
+                mgr.free_seq(live.pop(int(rng.integers(len(live)))))
+        except AllocError as e:
+            assert e.status == "OUT_OF_BLOCKS"
+        held = [b for s in live for b in mgr.seq_blocks(s)]
+        assert sum(mgr.refcount) == len(held)
+        assert len(set(held)) + mgr.num_free() + mgr.num_evictable() == 40
+        for b in mgr.evictable:
+            assert mgr.refcount[b] == 0 and b in mgr.cache_key
+        for key, b in mgr.cache.items():
+            assert mgr.cache_key[b] == key and len(key) % bs == 0

@@ -176,10 +176,12 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
  * ([csdn] "分页式KV缓存"; [betteryeah] §2.2, §2.4):
  *     out[t, h, :] = softmax(scale * q[t, h, :] . K[0..p]^T) . V[0..p]
  * with query head h reading kv head h / (num_heads / num_kv_heads).  fp32
- * accumulation on the tensor cores; output rounded to nearest even.
+ * accumulation on the tensor cores (tcgen05 with TMEM accumulators for
+ * head_dim 128, mma.sync for 64); output rounded to nearest even.
  *
  *   q, out        device [T, num_heads, head_dim] with T = query_start[num_seqs]:
  *                 the queries of all sequences, packed in order
+ *   num_tokens    T (the extent of q and out)
  *   query_start   device int32 [num_seqs + 1], non-decreasing, starting at 0
  *   max_query_len an upper bound of q_len_i (sizes the launch); <= max_context_len
  * A sequence whose q_len is negative, above its context length or above
@@ -190,7 +192,8 @@ pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
 pkv_status pkv_paged_attn_prefill(void* out, const void* q, const void* k_cache,
                                   const void* v_cache, const int32_t* block_tables,
                                   const int32_t* context_lens, const int32_t* query_start,
-                                  float scale, int num_seqs, int num_heads, int num_kv_heads,
+                                  float scale, int num_seqs, int num_tokens, int num_heads,
+                                  int num_kv_heads,
                                   int head_dim, int block_size, int max_blocks_per_seq,
                                   int max_context_len, int max_query_len, int num_blocks,
                                   pkv_dtype dtype, unsigned* dev_err, void* stream);

@@ -1,10 +1,14 @@
 // paged_attn_prefill.cu — host side of chunked-prefill attention: validation,
 // shape dispatch and the C entry point.  The kernel is in
 // paged_prefill_kernels.cuh.
+#include <cudaTypedefs.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "host_common.h"
 #include "paged_prefill_kernels.cuh"
+#include "paged_prefill_tc_kernels.cuh"
 
 namespace pkv {
 namespace {
@@ -46,17 +50,81 @@ PrefillEntry prefill_for(int d, int bs, int g) {
   return PrefillEntry{nullptr, 0, 0, 0};
 }
 
+// ---- tcgen05 kernel (head_dim 128) -----------------------------------------------
+using TcPrefillFn = void (*)(const PrefillParams, const CUtensorMap, const CUtensorMap,
+                             const CUtensorMap);
+
+struct TcEntry {
+  TcPrefillFn fn;
+  int threads;
+  size_t smem;
+};
+
+template <int BS, int G, class DT>
+TcEntry make_tc() {
+  using Tr = TcPrefillTraits<BS, G, DT>;
+  return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes()};
+}
+
+template <int BS, class DT>
+TcEntry tc_group(int g) {
+  switch (g) {
+    case 1: return make_tc<BS, 1, DT>();
+    case 2: return make_tc<BS, 2, DT>();
+    case 4: return make_tc<BS, 4, DT>();
+    case 8: return make_tc<BS, 8, DT>();
+    default: return TcEntry{nullptr, 0, 0};
+  }
+}
+
+template <class DT>
+TcEntry tc_for(int bs, int g) {
+  if (bs == 16) return tc_group<16, DT>(g);
+  if (bs == 32) return tc_group<32, DT>(g);
+  return TcEntry{nullptr, 0, 0};
+}
+
+// 3-D tensor map over q [T, H, 128]: boxes of (128/G tokens) x (G heads) x 64 dims,
+// i.e. a tile's 128 rows ordered (token, head), 128-byte swizzle.
+pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num_heads, int group,
+                        pkv_dtype dt) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  if (enc == nullptr) return cuda_status(cudaErrorNotSupported);
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(num_heads),
+                        static_cast<cuuint64_t>(num_tokens)};
+  cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(num_heads) * 128 * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      enc(out, dt == PKV_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+          3, const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : cuda_status(cudaErrorInvalidValue);
+}
+
 }  // namespace
 }  // namespace pkv
 
 extern "C" pkv_status pkv_paged_attn_prefill(
     void* out, const void* q, const void* k_cache, const void* v_cache,
     const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
-    float scale, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    float scale, int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim,
+    int block_size,
     int max_blocks_per_seq, int max_context_len, int max_query_len, int num_blocks,
     pkv_dtype dtype, unsigned* dev_err, void* stream) {
   using namespace pkv;
-  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
+  if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+      max_blocks_per_seq <= 0 ||
       max_context_len < 0 || max_query_len < 0 || num_blocks <= 0 || !dtype_valid(dtype) ||
       num_heads % num_kv_heads != 0 || !isfinite(scale) || max_query_len > max_context_len)
     return PKV_ERR_INVALID_ARG;
@@ -67,28 +135,40 @@ extern "C" pkv_status pkv_paged_attn_prefill(
   if (static_cast<long long>(max_context_len) >
       static_cast<long long>(max_blocks_per_seq) * block_size)
     return PKV_ERR_INVALID_ARG;
-  if (num_seqs == 0 || max_query_len == 0) return PKV_OK;
+  if (num_seqs == 0 || max_query_len == 0 || num_tokens == 0) return PKV_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
     return PKV_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
-  const PrefillEntry pe = dtype == PKV_FP16 ? prefill_for<Fp16>(head_dim, block_size, group)
-                                            : prefill_for<Bf16>(head_dim, block_size, group);
-  if (pe.fn == nullptr) return PKV_ERR_UNSUPPORTED;
+  const bool use_tc = head_dim == 128;
+  const PrefillEntry pe = use_tc ? PrefillEntry{nullptr, 0, 0, 0}
+                          : dtype == PKV_FP16 ? prefill_for<Fp16>(head_dim, block_size, group)
+                                              : prefill_for<Bf16>(head_dim, block_size, group);
+  const TcEntry te = !use_tc ? TcEntry{nullptr, 0, 0}
+                     : dtype == PKV_FP16 ? tc_for<Fp16>(block_size, group)
+                                         : tc_for<Bf16>(block_size, group);
+  if (pe.fn == nullptr && te.fn == nullptr) return PKV_ERR_UNSUPPORTED;
+  const int tile_rows = use_tc ? 128 : pe.rows;
   const long long rows = static_cast<long long>(max_query_len) * group;
-  const int q_tiles = static_cast<int>((rows + pe.rows - 1) / pe.rows);
+  const int q_tiles = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * q_tiles;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
-  CUtensorMap kmap, vmap;
+  CUtensorMap kmap, vmap, qmap;
   pkv_status st =
       cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
   if (st != PKV_OK) return st;
   st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
   if (st != PKV_OK) return st;
-  st = cuda_status(cudaFuncSetAttribute(reinterpret_cast<const void*>(pe.fn),
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(pe.smem)));
+  if (use_tc) {
+    st = q_tensor_map(&qmap, q, num_tokens, num_heads, group, dtype);
+    if (st != PKV_OK) return st;
+  }
+  const void* fn = use_tc ? reinterpret_cast<const void*>(te.fn)
+                          : reinterpret_cast<const void*>(pe.fn);
+  const size_t smem = use_tc ? te.smem : pe.smem;
+  st = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(smem)));
   if (st != PKV_OK) return st;
 
   PrefillParams p;
@@ -115,10 +195,11 @@ extern "C" pkv_status pkv_paged_attn_prefill(
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(pe.threads);
-  cfg.dynamicSmemBytes = pe.smem;
+  cfg.blockDim = dim3(use_tc ? te.threads : pe.threads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = as_stream(stream);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (use_tc) return cuda_status(cudaLaunchKernelEx(&cfg, te.fn, p, qmap, kmap, vmap));
   return cuda_status(cudaLaunchKernelEx(&cfg, pe.fn, p, kmap, vmap));
 }

@@ -1,0 +1,504 @@
+// paged_prefill_tc_kernels.cuh — chunked-prefill attention on the 5th-generation
+// tensor cores (tcgen05 + TMEM) for head_dim 128 on B200 (sm_100a).
+//
+// Computes what paged_prefill_kernels.cuh computes (causal attention of each
+// new token over its sequence's paged cache) with 128-row tiles:
+//   * warp 0 (producer): TMA loads of the 128-row Q tile (3-D tensor map over
+//     [T, H, D], so a tile's rows are (token, head-of-this-kv-head) pairs) and
+//     of K/V tiles of 64 keys, each gathered from 16-key pieces of the paged
+//     cache through the block table, into a 2-stage ring.
+//   * warp 1 (MMA): allocates 256 TMEM columns; one thread issues
+//       S  = Q K^T   (M=128, N=64,  K=128; A, B K-major)  into TMEM (2 buffers)
+//       O += P V     (M=128, N=128, K=64;  A=P K-major, B=V MN-major) into TMEM
+//     and signals completion with tcgen05.commit on mbarriers.
+//   * warps 2-5 (softmax): thread r owns row r (TMEM lane r): it reads its S
+//     row from TMEM, masks causally, keeps the running max / sum in base 2,
+//     rescales its O row in TMEM when the max moves, and writes P (fp16, or
+//     bf16 split into hi + lo halves) into 128-byte-swizzled shared memory.
+//     At the end it reads O, divides by the sum and stores the row.
+// All operand tiles use the 128-byte swizzle (8-row x 128-byte atoms, stride
+// 1024 bytes).  Keys past the context (or not loaded) are zeroed in the V tile
+// before P.V so stale NaN never enters the tensor-core sum.  Every mbarrier
+// wait is bounded; TMEM is released on every path.
+#pragma once
+
+#include <math.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "paged_prefill_kernels.cuh"
+
+namespace pkv {
+namespace tc {
+
+// ---- tcgen05 wrappers --------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]; issued by one thread.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+// Arrives once on `bar` when all earlier tcgen05.mma of this thread complete.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes (one per thread).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
+// address, leading / stride byte offsets in 16-byte units, version 1, layout 2).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                   uint32_t sbo_bytes) {
+  return (static_cast<uint64_t>((saddr >> 4) & 0x3FFFu)) |
+         (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16, fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int m, int n, bool b_mn_major) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+}  // namespace tc
+
+template <int BS_, int G_, class DT_>
+struct TcPrefillTraits {
+  static constexpr int D = 128, BS = BS_, G = G_;
+  using DT = DT_;
+  using T = typename DT::T;
+  static constexpr bool kBf16 = std::is_same<DT, Bf16>::value;
+  static constexpr int M = 128;                  // query rows per CTA
+  static constexpr int NKEY = 64;                // keys per KV tile
+  static constexpr int NS = 4;                   // KV stages (loads run up to 4 tiles ahead)
+  static constexpr int THREADS = 6 * 32;
+  // shared-memory layout (all 1024-byte aligned)
+  static constexpr int Q_HALF = M * 128;         // [128 rows][64 dims] = 16 KiB
+  static constexpr int KV_HALF = NKEY * 128;     // [64 keys][64 dims] = 8 KiB
+  static constexpr int STAGE = 4 * KV_HALF;      // K0 K1 V0 V1
+  static constexpr int P_BYTES = M * 128;        // [128 rows][64 keys]
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * Q_HALF;
+  static constexpr int OFF_P = OFF_KV + NS * STAGE;          // P buffers 0, 1
+  static constexpr int OFF_PLO = OFF_P + 2 * P_BYTES;        // bf16 lo halves 0, 1
+  static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? 2 * P_BYTES : 0);
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2]; tmem slot
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2;
+  // the softmax reference max moves only when a row max exceeds it by more
+  // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
+  static constexpr float kRescaleThreshold = 8.f;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
+  static constexpr uint32_t TMEM_COLS = 256;     // S buffers at 0 and 64, O at 128
+  static size_t smem_bytes() { return 1024 + static_cast<size_t>(SMEM); }
+};
+
+template <class Tr>
+__global__ void __launch_bounds__(Tr::THREADS, 1)
+    paged_prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap qmap,
+                            const __grid_constant__ CUtensorMap kmap,
+                            const __grid_constant__ CUtensorMap vmap) {
+  using T = typename Tr::T;
+  using DT = typename Tr::DT;
+  constexpr int G = Tr::G, BS = Tr::BS, M = Tr::M, NKEY = Tr::NKEY, NS = Tr::NS;
+  constexpr int ROWS_PER_TOK = G;
+  constexpr uint32_t IDESC_S = tc::idesc_f16(Tr::kBf16, M, NKEY, false);
+  constexpr uint32_t IDESC_O = tc::idesc_f16(Tr::kBf16, M, 128, true);
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
+  const uint32_t bar_q = smem_addr(bars + 0);
+  auto bar_kv_full = [&](int s) { return smem_addr(bars + 1 + s); };
+  auto bar_kv_empty = [&](int s) { return smem_addr(bars + 1 + NS + s); };
+  auto bar_s_full = [&](int b) { return smem_addr(bars + 1 + 2 * NS + b); };
+  auto bar_p = [&](int b) { return smem_addr(bars + 3 + 2 * NS + b); };
+  auto bar_o = [&](int b) { return smem_addr(bars + 5 + 2 * NS + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
+
+  const int tile = p.q_tiles - 1 - static_cast<int>(blockIdx.x % p.q_tiles);
+  const int unit = blockIdx.x / p.q_tiles;
+  const int kvh = unit % p.num_kv_heads;
+  const int seq = unit / p.num_kv_heads;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  grid_dependency_wait();
+  trigger_dependents();
+
+  const int ctx = p.context_lens[seq];
+  const int q0 = p.query_start[seq];
+  const int q_len = p.query_start[seq + 1] - q0;
+  const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
+  if (ctx < 0 || ctx > cap || q_len < 0 || q_len > ctx || q_len > p.max_query_len) {
+    if (threadIdx.x == 0 && tile == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
+    return;
+  }
+  const int rows_total = q_len * ROWS_PER_TOK;
+  if (tile * M >= rows_total) return;
+  const int tok0 = tile * (M / G);  // first query token of this tile
+  const int last_tok = (min(rows_total, (tile + 1) * M) - 1) / G;
+  const int nkv = ctx - q_len + last_tok + 1;
+  const int ntiles = (nkv + NKEY - 1) / NKEY;
+
+  if (threadIdx.x == 0) {
+    // one arrival each (an expect_tx arrive or a tcgen05.commit), except p_full:
+    // one arrival per softmax warp
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_kv_full(s), 1);
+      mbar_init(bar_kv_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_s_full(b), 1);
+      mbar_init(bar_p(b), 4);
+      mbar_init(bar_o(b), 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_addr(tmem_slot), Tr::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---- producer ---------------------------------------------------------------
+    const int32_t* trow = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
+    const int nblk = (nkv + BS - 1) / BS;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, 2 * Tr::Q_HALF);
+      tc::tma_load_3d(sbase + Tr::OFF_Q, &qmap, 0, kvh * G, q0 + tok0, bar_q);
+      tc::tma_load_3d(sbase + Tr::OFF_Q + Tr::Q_HALF, &qmap, 64, kvh * G, q0 + tok0, bar_q);
+    }
+    int chunk = -1, entry = -1;
+    for (int t = 0; t < ntiles; ++t) {
+      const int stage = t % NS;
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait_bounded(bar_kv_empty(stage), ((t / NS) & 1) ^ 1);
+        if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
+      }
+      ok = __shfl_sync(kFullMask, ok, 0);
+      if (!ok) break;
+      // the 16-key pieces of this tile that hold keys this CTA needs
+      int npieces = 0;
+      int pb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int key0 = t * NKEY + i * 16;
+        pb[i] = -1;
+        if (key0 < nkv) {
+          const int blk = key0 / BS;
+          if ((blk >> 5) != chunk) {
+            chunk = blk >> 5;
+            const int idx = (chunk << 5) + lane;
+            entry = idx < nblk ? trow[idx] : -1;
+          }
+          pb[i] = __shfl_sync(kFullMask, entry, blk & 31);
+          npieces = i + 1;
+        }
+      }
+      if (lane == 0) {
+        int bytes = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
+            bytes += 4 * 2048;
+        for (int i = 0; i < npieces; ++i)
+          if (static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks))
+            set_err(p.err, PKV_DEVERR_BAD_BLOCK);
+        const uint32_t bar = bar_kv_full(stage);
+        if (bytes > 0) {
+          mbar_arrive_expect_tx(bar, bytes);
+          const uint32_t st = sbase + Tr::OFF_KV + stage * Tr::STAGE;
+          for (int i = 0; i < npieces; ++i) {
+            if (static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks)) continue;
+            const int key0 = t * NKEY + i * 16;
+            const int y = (pb[i] * p.num_kv_heads + kvh) * BS + (key0 % BS);
+            tma_load_2d(st + 0 * Tr::KV_HALF + i * 2048, &kmap, 0, y, bar);
+            tma_load_2d(st + 1 * Tr::KV_HALF + i * 2048, &kmap, 64, y, bar);
+            tma_load_2d(st + 2 * Tr::KV_HALF + i * 2048, &vmap, 0, y, bar);
+            tma_load_2d(st + 3 * Tr::KV_HALF + i * 2048, &vmap, 64, y, bar);
+          }
+        } else {
+          mbar_arrive(bar);
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer ---------------------------------------------------------------
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(bar_q, 0);
+      const uint32_t q_lo = sbase + Tr::OFF_Q, q_hi = q_lo + Tr::Q_HALF;
+      auto issue_pv = [&](int t) {  // O += P V for tile t (its P is in buffer t & 1)
+        const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
+        const uint32_t v0 = st + 2 * Tr::KV_HALF;
+        const uint32_t pbuf = sbase + Tr::OFF_P + (t & 1) * Tr::P_BYTES;
+        const uint32_t plo = sbase + Tr::OFF_PLO + (t & 1) * Tr::P_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < NKEY / 16; ++kk) {
+          const uint64_t bdesc = tc::smem_desc_sw128(v0 + kk * 2048, Tr::KV_HALF, 1024);
+          const uint64_t adesc = tc::smem_desc_sw128(pbuf + kk * 32, 16, 1024);
+          tc::umma_f16(tmem + 128, adesc, bdesc, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+          if constexpr (Tr::kBf16) {
+            const uint64_t ldesc = tc::smem_desc_sw128(plo + kk * 32, 16, 1024);
+            tc::umma_f16(tmem + 128, ldesc, bdesc, IDESC_O, 1u);
+          }
+        }
+        tc::umma_commit(bar_o(t & 1));
+        tc::umma_commit(bar_kv_empty(t % NS));
+      };
+      for (int t = 0; t < ntiles && ok; ++t) {
+        ok = mbar_wait_bounded(bar_kv_full(t % NS), (t / NS) & 1);
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t qa = (ks < 4 ? q_lo : q_hi) + (ks & 3) * 32;
+          const uint32_t kb = st + (ks < 4 ? 0 : Tr::KV_HALF) + (ks & 3) * 32;
+          tc::umma_f16(tmem + (t & 1) * 64, tc::smem_desc_sw128(qa, 16, 1024),
+                       tc::smem_desc_sw128(kb, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(bar_s_full(t & 1));
+        if (t > 0) {
+          ok = mbar_wait_bounded(bar_p((t - 1) & 1), ((t - 1) >> 1) & 1);
+          if (!ok) break;
+          tc::tc_fence_after();
+          issue_pv(t - 1);
+        }
+      }
+      if (ok && ntiles > 0) {
+        ok = mbar_wait_bounded(bar_p((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1);
+        if (ok) {
+          tc::tc_fence_after();
+          issue_pv(ntiles - 1);
+        }
+      }
+      if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ---- softmax warps: thread <-> row <-> TMEM lane ---------------------------------
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool active = r < rows_total - tile * M;
+    const int j = tok0 + r / G;
+    const int g = r % G;
+    const int pos = active ? ctx - q_len + j : -1;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int kv0 = t * NKEY;
+      ok = mbar_wait_bounded(bar_s_full(t & 1), (t >> 1) & 1);
+      if (!__all_sync(kFullMask, ok)) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      float s[NKEY];
+#pragma unroll
+      for (int c = 0; c < NKEY; c += 16) {
+        float v[16];
+        tc::tmem_ld16(lane_addr + (t & 1) * 64 + c, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[c + i] = v[i];
+      }
+      tc::tmem_wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < NKEY; ++c) {
+        s[c] = (kv0 + c <= pos) ? s[c] * p.qscale : -INFINITY;
+        mx = fmaxf(mx, s[c]);
+      }
+      // move the reference max only when this tile would push P above 2^8
+      float alpha = 1.f;
+      if (active && mx > m + Tr::kRescaleThreshold) {
+        alpha = exp2_approx(m - mx);  // 0 on the first tile (m = -inf)
+        m = mx;
+      }
+      const float m_use = m == -INFINITY ? 0.f : m;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < NKEY; ++c) {
+        s[c] = exp2_approx(s[c] - m_use);
+        sum += s[c];
+      }
+      l = l * alpha + sum;
+      if (t > 0 && __any_sync(kFullMask, alpha != 1.f)) {
+        // O must hold every earlier tile before it is rescaled
+        ok = mbar_wait_bounded(bar_o((t - 1) & 1), ((t - 1) >> 1) & 1);
+        if (!__all_sync(kFullMask, ok)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 16) {
+          float v[16];
+          tc::tmem_ld16(lane_addr + 128 + c, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= alpha;
+          tc::tmem_st16(lane_addr + 128 + c, v);
+        }
+        tc::tmem_wait_st();
+      }
+      if (t >= 2) {  // P buffer t & 1 was last read by P.V of tile t - 2
+        ok = mbar_wait_bounded(bar_o(t & 1), ((t - 2) >> 1) & 1);
+        if (!__all_sync(kFullMask, ok)) {
+          ok = false;
+          break;
+        }
+      }
+      // P (16-bit; bf16 as hi + lo) into the swizzled [128 rows][64 keys] buffers
+      unsigned char* prow = smem + Tr::OFF_P + (t & 1) * Tr::P_BYTES + r * 128;
+      unsigned char* plrow = smem + Tr::OFF_PLO + (t & 1) * Tr::P_BYTES + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[4], wl[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = s[ch * 8 + 2 * e], b = s[ch * 8 + 2 * e + 1];
+          w[e] = pack2(a, b, DT());
+          if constexpr (Tr::kBf16) {
+            wl[e] = pack2(a - __uint_as_float(w[e] << 16), b - __uint_as_float(w[e] & 0xffff0000u),
+                          Bf16());
+          }
+        }
+        const int at = ((ch ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow + at) = make_uint4(w[0], w[1], w[2], w[3]);
+        if constexpr (Tr::kBf16)
+          *reinterpret_cast<uint4*>(plrow + at) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      }
+      // keys past the context, or not loaded, hold stale data: zero their V rows
+      const int loaded_end = min(kv0 + NKEY, ((nkv + 15) / 16) * 16);
+      const int vz = min(ctx, loaded_end) - kv0;  // V rows [vz, 64) must be zero
+      if (vz < NKEY) {
+        unsigned char* vt = smem + Tr::OFF_KV + (t % NS) * Tr::STAGE + 2 * Tr::KV_HALF;
+        const int nrows = NKEY - vz;
+        const int tid = r;  // 128 softmax threads
+        for (int idx = tid; idx < nrows * 16; idx += 128) {
+          const int row = vz + idx / 16;
+          const int part = idx % 16;  // 8 chunks in each of the two dim halves
+          *reinterpret_cast<uint4*>(vt + (part >> 3) * Tr::KV_HALF + row * 128 + (part & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p(t & 1));
+    }
+    // ---- epilogue ------------------------------------------------------------------------
+    if (ok && ntiles > 0) {
+      ok = mbar_wait_bounded(bar_o((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1);
+      ok = __all_sync(kFullMask, ok);
+    }
+    if (ok && ntiles > 0) {
+      tc::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      T* orow = static_cast<T*>(p.out) +
+                (static_cast<size_t>(q0 + j) * p.num_heads + kvh * G + g) * Tr::D;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 16) {
+        float v[16];
+        tc::tmem_ld16(lane_addr + 128 + c, v);
+        tc::tmem_wait_ld();
+        if (active) {
+          float a[8], b[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            a[i] = v[i] * inv;
+            b[i] = v[8 + i] * inv;
+          }
+          *reinterpret_cast<uint4*>(orow + c) = pack8(a, DT());
+          *reinterpret_cast<uint4*>(orow + c + 8) = pack8(b, DT());
+        }
+      }
+    } else if (!ok) {
+      if (lane == 0) set_err(p.err, PKV_DEVERR_TIMEOUT);
+    }
+  }
+  // ---- release TMEM (every path reaches here) ---------------------------------------------
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, Tr::TMEM_COLS);
+  }
+}
+
+}  // namespace pkv

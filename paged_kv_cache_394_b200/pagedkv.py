@@ -50,7 +50,7 @@ _paged_attn_decode_static_ws = _proto("pkv_paged_attn_decode_static_ws", _i, _vp
                                      _vp)
 STATIC_WORKSPACE_BYTES = 16 << 20
 _paged_attn_prefill = _proto("pkv_paged_attn_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i,
-                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp)
+                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp)
 _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
 _decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
                            _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
@@ -244,7 +244,7 @@ def paged_attn_prefill(out, q, k_cache, v_cache, block_tables, context_lens, que
         raise TypeError("q, out and caches must share a dtype")
     _check(_paged_attn_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
-                               float(scale), s, h, hkv, d, bs, block_tables.shape[1],
+                               float(scale), s, t, h, hkv, d, bs, block_tables.shape[1],
                                max_context_len, max_query_len, num_blocks, _dtype_code(q),
                                _ptr(dev_err), _stream(stream)),
            "paged_attn_prefill")

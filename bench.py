@@ -19,12 +19,17 @@ the max over ranks.  `e2e` times the same step through the host-buffer entry
 point, with the step's inputs copied from pinned host memory and the output
 read back inside the timed region.
 
+A workload name with the suffix ``_fp8`` (e.g. ``llama7b_fp8``) runs the
+same batch with E4M3 caches: the quantising cache write and the E4M3 decode.
+
 `--impl reference` times the CPU oracle on the host cores instead (rank 0
 only), each step a bounded sample of the same workload.
 """
 
 import argparse
 import hashlib
+
+import numpy as np
 import json
 import os
 import re
@@ -38,6 +43,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
+# per-cache E4M3 scales of the *_fp8 workloads: N(0,1) values reach about 6
+FP8_K_SCALE = FP8_V_SCALE = 6.0 / 448.0
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -100,29 +107,30 @@ def replica_seed(base_seed, rank):
 # ---------------------------------------------------------------------------
 # bytes
 # ---------------------------------------------------------------------------
-def decode_bytes(w):
+def decode_bytes(w, kv_elem=2):
     """Algorithmic bytes of one decode call: K and V of every cached token of
-    every kv head, q read, out written."""
-    e = 2
-    kv = 2 * int(w.context_lens.astype("int64").sum()) * w.num_kv_heads * w.head_dim * e
-    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * e
+    every kv head (``kv_elem`` bytes per element: 2, or 1 for E4M3), q read
+    and out written (16-bit)."""
+    kv = 2 * int(w.context_lens.astype("int64").sum()) * w.num_kv_heads * w.head_dim * kv_elem
+    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * 2
     return kv + qo
 
 
-def write_bytes(w):
-    """reshape_and_cache: read key and value, write them, read the slots."""
+def write_bytes(w, kv_elem=2):
+    """reshape_and_cache: read key and value (16-bit), write them
+    (``kv_elem`` bytes per element), read the slots."""
     t = len(w.slot_mapping)
-    return 2 * 2 * t * w.num_kv_heads * w.head_dim * 2 + 8 * t
+    return 2 * t * w.num_kv_heads * w.head_dim * (2 + kv_elem) + 8 * t
 
 
-def copy_bytes(w):
+def copy_bytes(w, kv_elem=2):
     """copy_blocks: read and write K and V of every copied block, read the pairs."""
-    blk = w.num_kv_heads * w.block_size * w.head_dim * 2
+    blk = w.num_kv_heads * w.block_size * w.head_dim * kv_elem
     return len(w.cow_pairs) * (2 * 2 * blk + 16)
 
 
-def step_bytes(w):
-    return decode_bytes(w) + write_bytes(w) + copy_bytes(w)
+def step_bytes(w, kv_elem=2):
+    return decode_bytes(w, kv_elem) + write_bytes(w, kv_elem) + copy_bytes(w, kv_elem)
 
 
 def prefill_flops(w):
@@ -256,14 +264,31 @@ def run_ours(args):
     local = dist_env()[2]
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    base = W.SEED_BASE + W.NAMES.index(args.workload)
-    w = W.make(args.workload, seed=replica_seed(base, rank))
+    # "<name>_fp8": the named workload with E4M3 caches (one scale per cache)
+    fp8 = args.workload.endswith("_fp8")
+    name = args.workload[:-4] if fp8 else args.workload
+    base = W.SEED_BASE + W.NAMES.index(name)
+    w = W.make(name, seed=replica_seed(base, rank))
     tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+    kv_elem = 1 if fp8 else 2
 
     def up(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(tdt)
 
     q, kc, vc, key, val = up(w.q), up(w.k_cache), up(w.v_cache), up(w.key), up(w.value)
+    if fp8:
+        # the pool, quantised once by the device's own cache write (setup, untimed)
+        nb, hkv, bs, d = kc.shape
+        ks8 = torch.full((hkv,), FP8_K_SCALE, dtype=torch.float32, device=dev)
+        vs8 = torch.full((hkv,), FP8_V_SCALE, dtype=torch.float32, device=dev)
+        k8 = torch.empty(kc.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty_like(k8)
+        every = torch.arange(nb * bs, dtype=torch.int64, device=dev)
+        tok = lambda c: c.permute(0, 2, 1, 3).reshape(nb * bs, hkv, d).contiguous()
+        pk.reshape_and_cache_fp8(tok(kc), tok(vc), k8, v8, every, ks8, vs8)
+        torch.cuda.synchronize(dev)
+        kc, vc = k8, v8
+        del every
     slots = torch.from_numpy(w.slot_mapping).to(dev)
     pairs = torch.from_numpy(np.ascontiguousarray(w.cow_pairs)).to(dev)
     tables = torch.from_numpy(w.block_tables).to(dev)
@@ -282,12 +307,22 @@ def run_ours(args):
     def step(ev_a=None, ev_b=None):
         if has_pairs:
             pk.copy_blocks(kc, vc, pairs, dev_err=err, stream=stream)
-        pk.reshape_and_cache(key, val, kc, vc, slots, dev_err=err, stream=stream)
+        if fp8:
+            pk.reshape_and_cache_fp8(key, val, kc, vc, slots, ks8, vs8, dev_err=err,
+                                     stream=stream)
+        else:
+            pk.reshape_and_cache(key, val, kc, vc, slots, dev_err=err, stream=stream)
         if ev_a is not None:
             ev_a.record(stream)
-        pk.paged_attn_decode(out, q, kc, vc, tables, lens, w.scale, w.num_kv_heads, w.block_size,
-                             w.max_context_len, partition_size=part_req, workspace=ws,
-                             dev_err=err, stream=stream)
+        if fp8:
+            pk.paged_attn_decode_fp8(out, q, kc, vc, tables, lens, w.scale, ks8, vs8,
+                                     w.num_kv_heads, w.block_size,
+                                     w.max_context_len, partition_size=part_req, workspace=ws,
+                                     dev_err=err, stream=stream)
+        else:
+            pk.paged_attn_decode(out, q, kc, vc, tables, lens, w.scale, w.num_kv_heads,
+                                 w.block_size, w.max_context_len, partition_size=part_req,
+                                 workspace=ws, dev_err=err, stream=stream)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -318,11 +353,11 @@ def run_ours(args):
     dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
     total_ms_max = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms_max / args.steps
-    sbytes = step_bytes(w)
+    sbytes = step_bytes(w, kv_elem)
     all_bytes = sum_over_ranks(sbytes, dev)
     value = all_bytes / (ms_per_step * 1e-3) / 1e9
     dec_avg_ms = statistics.mean(dec_ms)
-    dbytes = decode_bytes(w)
+    dbytes = decode_bytes(w, kv_elem)
     achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
 
@@ -343,9 +378,20 @@ def run_ours(args):
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
-        pk.decode_step_host(h_out, h_q, h_key, h_val, h_slots, h_pairs, h_tables, h_lens, kc, vc,
-                            w.scale, w.max_context_len, staging, workspace=ws,
-                            partition_size=part_req, dev_err=err, stream=stream)
+        if not fp8:
+            pk.decode_step_host(h_out, h_q, h_key, h_val, h_slots, h_pairs, h_tables, h_lens, kc,
+                                vc, w.scale, w.max_context_len, staging, workspace=ws,
+                                partition_size=part_req, dev_err=err, stream=stream)
+            return
+        # E4M3 caches: the same copies through the Python binding's tensors
+        with torch.cuda.stream(stream):
+            for dst, src in ((q, h_q), (key, h_key), (val, h_val), (slots, h_slots),
+                             (tables, h_tables), (lens, h_lens)):
+                dst.copy_(src, non_blocking=True)
+            if has_pairs:
+                pairs.copy_(h_pairs, non_blocking=True)
+            step()
+            h_out.copy_(out, non_blocking=True)
     for _ in range(args.warmup):
         e2e_step()
     torch.cuda.synchronize(dev)
@@ -365,7 +411,7 @@ def run_ours(args):
         raise RuntimeError("device error word %d" % int(err.item()))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
     if rank == 0:
@@ -374,9 +420,13 @@ def run_ours(args):
             "metric": "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s",
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 cache, %s q/out, f32 math" % w.dtype if fp8 else w.dtype,
             "data": "synthetic",
-            "config": dict(W.describe(w), parallelism="replicas%d" % world,
+            "config": dict(W.describe(w), workload=args.workload,
+                           kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
+                           if fp8 else w.dtype,
+                           parallelism="replicas%d" % world,
                            partition_used=part, split_k=split,
                            l2="no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
                               % (dbytes / 1e9)),
@@ -388,14 +438,17 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": committed_traffic(args.workload),
-                         "kernel": "paged_decode_kernel" + (" + reduce" if split else ""),
+                         "kernel": ("paged_decode_mma_kernel" if w.num_heads > w.num_kv_heads
+                                    and not fp8 else "paged_decode_kernel")
+                         + (" + reduce" if split else ""),
                          "algorithmic_bytes_per_launch": dbytes,
                          "avg_launch_ms": round(dec_avg_ms, 5),
                          "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                          if peak_kind == "measured" else "fallback 6.65 TB/s"},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "pkv_decode_step_host"},
+                    "api": "pkv_paged_attn_decode_fp8 etc. via the Python binding, torch "
+                           "copies" if fp8 else "pkv_decode_step_host"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
@@ -659,6 +712,54 @@ def run_prefix_cache_trace(args):
     print(json.dumps(line), flush=True)
 
 
+def run_serving_trace(args):
+    """The continuous-batching driver over a seeded Poisson trace of chat-shaped
+    requests (LLaMA-7B attention-layer shapes).  Reports generated tokens/s of
+    device time and the memory utilization of the allocated pages, the figures
+    the pages quote (over 90 % of the cache used, under 4 % wasted)."""
+    import torch
+
+    from paged_kv_cache_394_b200 import engine as E
+    torch.cuda.set_device(0)
+    b = E.ContinuousBatcher(12000, 16, 32, 32, 128, dtype=torch.float16, max_num_seqs=256,
+                            max_num_batched_tokens=2048, max_model_len=2560, seed=394)
+    trace = E.synthetic_trace(394, 400, mean_interarrival=0.2, prompt_median=300,
+                              prompt_sigma=0.8, output_range=(32, 256), max_prompt=2048)
+    for r in trace:
+        b.submit(r)
+    kern_ms = dec_tokens = pre_tokens = steps = 0
+    utils, live_peak = [], 0
+    t0 = time.perf_counter()
+    while not b.idle():
+        rec = b.step()
+        steps += 1
+        kern_ms += rec.kernel_ms
+        dec_tokens += len(rec.decoded)
+        pre_tokens += rec.prefill_tokens
+        live_peak = max(live_peak, rec.live)
+        if rec.used_blocks:
+            utils.append(rec.cached_tokens / (rec.used_blocks * 16))
+    wall = time.perf_counter() - t0
+    line = {
+        "metric": "continuous-batching decode tokens/s per attention layer (device time)",
+        "value": round(dec_tokens / (kern_ms * 1e-3), 1), "unit": "tokens/s",
+        "higher_is_better": True, "data": "synthetic",
+        "config": {"workload": "serving_trace", "requests": len(trace), "num_heads": 32,
+                   "head_dim": 128, "block_size": 16, "dtype": "fp16", "num_blocks": 12000,
+                   "max_num_seqs": 256, "max_num_batched_tokens": 2048,
+                   "arrivals": "Poisson, mean gap 0.2 steps", "prompt": "lognormal median 300",
+                   "output": "U[32, 256]"},
+        "steps": steps, "decode_tokens": dec_tokens, "prefill_tokens": pre_tokens,
+        "prefill_plus_decode_tokens_per_s": round((dec_tokens + pre_tokens) / (kern_ms * 1e-3), 1),
+        "memory_utilization": {"mean": round(float(np.mean(utils)), 4),
+                               "min": round(float(np.min(utils)), 4),
+                               "waste_mean": round(1 - float(np.mean(utils)), 4)},
+        "peak_live_sequences": live_peak,
+        "host_steps_per_s": round(steps / wall, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -712,6 +813,8 @@ def main(argv=None):
     args.warmup = max(3, args.warmup)
     if args.workload == "prefix_cache_trace":
         run_prefix_cache_trace(args)
+    elif args.workload == "serving_trace":
+        run_serving_trace(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -38,7 +38,7 @@
  *    in device memory) never fault: the kernel skips the offending access and
  *    ORs a PKV_DEVERR_* bit into *dev_err when dev_err is not NULL.  Read the
  *    word after the stream has synchronized; outputs are then unreliable.
- *  - Alignment: every 16-bit tensor pointer must be 16-byte aligned.
+ *  - Alignment: every tensor pointer (16-bit or E4M3) must be 16-byte aligned.
  *  - Supported shapes: head_dim in {64, 128}, block_size in {16, 32},
  *    num_heads / num_kv_heads in {1, 2, 4, 8}, dtype fp16 or bf16.
  */
@@ -61,7 +61,9 @@ typedef enum {
   PKV_ERR_OUT_OF_BLOCKS = 5  /* allocator: the free list is empty           */
 } pkv_status;
 
-typedef enum { PKV_FP16 = 0, PKV_BF16 = 1 } pkv_dtype;
+/* PKV_FP8_E4M3 is a cache element type only (copy_blocks, and the caches of
+ * the *_fp8 entry points); queries and outputs are always 16-bit. */
+typedef enum { PKV_FP16 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
 
 /* Bits ORed into *dev_err by the kernels. */
 #define PKV_DEVERR_BAD_BLOCK 1u   /* decode: table entry outside [0, num_blocks)          */
@@ -70,6 +72,7 @@ typedef enum { PKV_FP16 = 0, PKV_BF16 = 1 } pkv_dtype;
 #define PKV_DEVERR_BAD_CONTEXT 8u /* decode: context_len < 0, > max_context_len, or more
                                      blocks than max_blocks_per_seq                        */
 #define PKV_DEVERR_TIMEOUT 16u    /* decode: a bounded wait for an async copy gave up      */
+#define PKV_DEVERR_BAD_SCALE 32u  /* *_fp8: a scale that is not finite and > 0            */
 
 /* Library version string, e.g. "pagedkv 0.1.0 sm_100a". */
 const char* pkv_version(void);
@@ -109,7 +112,8 @@ pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cac
  * Preconditions (what the allocator produces): dst values are distinct and no
  * dst is also a src in the same call; otherwise the result is unspecified.
  * A pair with an index outside [0, num_blocks) sets PKV_DEVERR_BAD_PAIR and
- * is skipped.  Bit-exact.  num_pairs == 0 is a no-op.
+ * is skipped.  Bit-exact.  num_pairs == 0 is a no-op.  dtype is the cache's
+ * element type: PKV_FP16, PKV_BF16 or PKV_FP8_E4M3 (1-byte codes).
  */
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
                            int num_pairs, int num_kv_heads, int head_dim, int block_size,
@@ -230,6 +234,57 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, const void*
                                            int head_dim, int block_size, int max_blocks_per_seq,
                                            int max_context_len, int num_blocks, pkv_dtype dtype,
                                            int partition_size, unsigned* dev_err, void* stream);
+
+/*
+ * 8-bit (E4M3) cache.  The pages name quantised inference as a way to fit
+ * larger models and batches into the memory ([csdn] "量化模型优先考虑边缘场景";
+ * [betteryeah] §4.2 "启用量化推理") without fixing a format; this library stores
+ * the cache as OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, subnormals, no infinities, 0x7F/0xFF NaN, largest finite
+ * 448) with one float scale per kv head and cache:
+ *     code = E4M3(x / scale[h]),   value = decode(code) * scale[h].
+ * Each cache element is one byte; the layout is that of the 16-bit caches.
+ * k_scales, v_scales: device float32 [num_kv_heads] (the same value in every
+ * entry gives one scale per cache).  They live in device memory so a captured
+ * graph can pick up new scales; a scale that is not finite and > 0 sets
+ * PKV_DEVERR_BAD_SCALE (the write then skips that head's elements; decode
+ * output is unreliable).
+ *
+ * pkv_reshape_and_cache_fp8 — pkv_reshape_and_cache that quantises on the way
+ * in.  key/value are 16-bit of type `dtype` ([num_tokens, num_kv_heads,
+ * head_dim]); k_cache/v_cache hold codes.  Each element of kv head h is
+ * widened to float32, divided by k_scales[h] (keys) or v_scales[h] (values)
+ * in IEEE float32 (round to nearest), and rounded to E4M3 by
+ * round-to-nearest-even; magnitudes that round above 448 become +-448, NaN
+ * becomes a NaN code.  Slots behave as in pkv_reshape_and_cache.  Null
+ * scale pointers give PKV_ERR_INVALID_ARG.
+ */
+pkv_status pkv_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                     void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, pkv_dtype dtype, const float* k_scales,
+                                     const float* v_scales, unsigned* dev_err, void* stream);
+
+/*
+ * pkv_paged_attn_decode_fp8 — pkv_paged_attn_decode over E4M3 caches:
+ *     out[i, h, :] = softmax(scale * q[i, h, :] . K~^T) . V~,
+ *     K~ = decode(k_cache codes) * k_scales[g],  V~ = decode(v_cache codes) * v_scales[g]
+ * with g the kv head of query head h.  q and out are 16-bit of type `dtype`;
+ * every other argument, the workspace (same size as
+ * pkv_paged_attn_workspace_bytes gives) and the error behaviour are those of
+ * pkv_paged_attn_decode.  fp32 accumulation on the CUDA cores for every group
+ * size.  Null scale pointers give PKV_ERR_INVALID_ARG.
+ */
+pkv_status pkv_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, float scale,
+                                     const float* k_scales, const float* v_scales,
+                                     int num_seqs, int num_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int max_blocks_per_seq, int max_context_len,
+                                     int num_blocks, pkv_dtype dtype, int partition_size,
+                                     void* workspace, size_t workspace_bytes,
+                                     unsigned* dev_err, void* stream);
 
 /*
  * pkv_decode_step_host — one whole decode step from HOST buffers: copies the

@@ -4,8 +4,9 @@ The pages mention quantised inference only in passing ([csdn] "é‡åŒ–æ¨¡åž‹ä¼˜å…
 åœºæ™¯"; [betteryeah] Â§4.2 "å¯ç”¨é‡åŒ–æŽ¨ç†"), so the format is the plainest modern
 reading: the OCP 8-bit floating point "E4M3" (sign bit, 4 exponent bits with
 bias 7, 3 mantissa bits; subnormals; no infinities; 0x7F / 0xFF are NaN;
-largest finite value 448), with one float scale per tensor:
-    code = E4M3(x / scale),   value = decode(code) * scale.
+largest finite value 448), with one float scale per kv head of each cache
+(equal entries give one scale per cache):
+    code = E4M3(x / scale[h]),   value = decode(code) * scale[h].
 
 Readings taken:
 * x / scale is computed in float32 (the precision the GPU uses), then
@@ -56,11 +57,67 @@ def e4m3_decode(codes):
 
 
 def quantize(bits16, dtype, scale):
-    """16-bit cache values -> E4M3 codes of value / scale (float32 division)."""
+    """16-bit values -> E4M3 codes of value / scale (float32 division);
+    ``scale`` is a number or an array that broadcasts against the values."""
     from .dtypes import widen
     x32 = widen(bits16, dtype).astype(np.float32)
-    return e4m3_encode(x32 / np.float32(scale))
+    return e4m3_encode(x32 / np.asarray(scale, dtype=np.float32))
 
 
 def dequantize(codes, scale):
-    return e4m3_decode(codes) * float(np.float32(scale))
+    return e4m3_decode(codes) * np.asarray(scale, dtype=np.float32).astype(np.float64)
+
+
+def per_head(scales, num_kv_heads):
+    """A scale per kv head as float32 [num_kv_heads] (a number is repeated)."""
+    s = np.asarray(scales, dtype=np.float32).reshape(-1)
+    return np.repeat(s, num_kv_heads) if s.size == 1 else s
+
+
+def quantize_cache(cache_bits, dtype, scales):
+    """A whole 16-bit cache [N, Hkv, bs, D] -> codes, kv head h by scales[h]."""
+    s = per_head(scales, cache_bits.shape[1])
+    return quantize(cache_bits, dtype, s[None, :, None, None])
+
+
+def quantize_into_cache(key_bits, value_bits, k_codes, v_codes, slot_mapping, block_size, dtype,
+                        k_scales, v_scales):
+    """The quantising cache write: kv head h of token t's K (V) becomes
+    E4M3(x / k_scales[h]) (E4M3(x / v_scales[h])) in slot ``slot_mapping[t]``
+    of copies of the code caches; negative slots are skipped.  Same placement
+    as the 16-bit write (block = slot // block_size, offset = slot % block_size)."""
+    k_out = np.array(k_codes, copy=True)
+    v_out = np.array(v_codes, copy=True)
+    hkv = key_bits.shape[1]
+    kq = quantize(key_bits, dtype, per_head(k_scales, hkv)[None, :, None])
+    vq = quantize(value_bits, dtype, per_head(v_scales, hkv)[None, :, None])
+    for t, slot in enumerate(np.asarray(slot_mapping, dtype=np.int64)):
+        if slot < 0:
+            continue
+        block, offset = divmod(int(slot), block_size)
+        k_out[block, :, offset, :] = kq[t]
+        v_out[block, :, offset, :] = vq[t]
+    return k_out, v_out
+
+
+def paged_attention_decode_fp8(q_bits, k_codes, v_codes, block_tables, context_lens, scale,
+                               k_scales, v_scales, num_kv_heads, block_size, dtype, pairs=None):
+    """Paged decode attention over E4M3 caches: the textbook single-query
+    attention of ``oracle.attention`` over the gathered tokens' values
+    decode(code) * scale of their kv head, in float64.  ``pairs`` as in
+    ``oracle.attention.paged_attention_decode``."""
+    from .attention import attend, kv_head_of, token_location
+    from .dtypes import widen
+    num_seqs, num_heads, head_dim = q_bits.shape
+    ks, vs = per_head(k_scales, num_kv_heads), per_head(v_scales, num_kv_heads)
+    if pairs is None:
+        pairs = [(s, h) for s in range(num_seqs) for h in range(num_heads)]
+    out = np.full((num_seqs, num_heads, head_dim), np.nan, dtype=np.float64)
+    for s, h in pairs:
+        g = kv_head_of(h, num_heads, num_kv_heads)
+        blocks, offsets = token_location(np.asarray(block_tables[s]),
+                                         np.arange(int(context_lens[s])), block_size)
+        keys = dequantize(k_codes[blocks, g, offsets, :], ks[g])
+        values = dequantize(v_codes[blocks, g, offsets, :], vs[g])
+        out[s, h] = attend(widen(q_bits[s, h], dtype), keys, values, scale)
+    return out

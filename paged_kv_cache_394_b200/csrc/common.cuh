@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -28,6 +29,10 @@ struct Fp16 {
 };
 struct Bf16 {
   using T = __nv_bfloat16;
+};
+// 8-bit E4M3 cache element (values are code * scale)
+struct Fp8E4M3 {
+  using T = uint8_t;
 };
 
 __device__ __forceinline__ void set_err(unsigned* err, unsigned bit) {
@@ -159,6 +164,22 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8], Bf16) {
     // a bfloat16 is the upper half of a float32
     f[2 * i] = __uint_as_float(w[i] << 16);
     f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// 8 E4M3 codes -> 8 floats (exact: E4M3 -> fp16 -> fp32).
+__device__ __forceinline__ void unpack8(const uint2& u, float (&f)[8], Fp8E4M3) {
+  const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * j));
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&h));
+      f[4 * i + 2 * j] = x.x;
+      f[4 * i + 2 * j + 1] = x.y;
+    }
   }
 }
 

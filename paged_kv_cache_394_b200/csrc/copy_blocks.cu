@@ -50,14 +50,16 @@ extern "C" pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_
                                       int block_size, int num_blocks, pkv_dtype dtype,
                                       unsigned* dev_err, void* stream) {
   using namespace pkv;
-  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !dtype_valid(dtype))
+  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !cache_dtype_valid(dtype))
     return PKV_ERR_INVALID_ARG;
   if (!head_dim_supported(head_dim) || !block_size_supported(block_size))
     return PKV_ERR_UNSUPPORTED;
   if (num_pairs == 0) return PKV_OK;
   if (!k_cache || !v_cache || !block_mapping) return PKV_ERR_INVALID_ARG;
   if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
-  const int64_t vecs = static_cast<int64_t>(num_kv_heads) * block_size * head_dim / 8;
+  // 16-byte vectors per block: 8 elements of a 16-bit cache, 16 of an E4M3 cache
+  const int64_t vecs = static_cast<int64_t>(num_kv_heads) * block_size * head_dim *
+                       cache_elem_bytes(dtype) / 16;
   dim3 grid(static_cast<unsigned>(num_pairs), 2);
   copy_blocks_kernel<<<grid, 256, 0, as_stream(stream)>>>(
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping, vecs,

@@ -17,6 +17,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline bool head_dim_supported(int d) { return d == 64 || d == 128; }
 inline bool block_size_supported(int bs) { return bs == 16 || bs == 32; }
 inline bool dtype_valid(int dt) { return dt == PKV_FP16 || dt == PKV_BF16; }
+// Element types a cache may hold: the 16-bit ones, or E4M3 codes.
+inline bool cache_dtype_valid(int dt) { return dtype_valid(dt) || dt == PKV_FP8_E4M3; }
+inline int cache_elem_bytes(int dt) { return dt == PKV_FP8_E4M3 ? 1 : 2; }
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 

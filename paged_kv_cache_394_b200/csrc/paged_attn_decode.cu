@@ -19,11 +19,13 @@ namespace pkv {
 
 // Warps per CTA and ring stages per warp for a (head_dim, block_size): about
 // 96 KiB of ring per CTA so two CTAs fit on an SM, 2..4 stages per warp.
-template <int D, int BS>
+// An 8-bit cache moves half the bytes per block, so it may keep up to twice
+// as many stages in flight for the same ring size.
+template <int D, int BS, int KB = 2>
 struct LaunchShape {
   static constexpr int W = 4;
-  static constexpr int STAGE = 2 * BS * D * 2;
-  static constexpr int NS = cmax(2, cmin(4, (96 * 1024) / (W * STAGE)));
+  static constexpr int STAGE = 2 * BS * D * KB;
+  static constexpr int NS = cmax(2, cmin(8 / KB, (96 * 1024) / (W * STAGE)));
 };
 
 using KernelFn = void (*)(const DecodeParams);
@@ -34,10 +36,10 @@ struct KernelEntry {
   size_t smem_fixed;  // bytes before the block-table slice
 };
 
-template <int D, int BS, int G, class DT>
+template <int D, int BS, int G, class DT, class KV = DT>
 KernelEntry make_entry() {
-  using LS = LaunchShape<D, BS>;
-  using Tr = DecodeTraits<D, BS, G, DT, LS::W, LS::NS>;
+  using LS = LaunchShape<D, BS, static_cast<int>(sizeof(typename KV::T))>;
+  using Tr = DecodeTraits<D, BS, G, DT, LS::W, LS::NS, KV>;
   return KernelEntry{paged_decode_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(0)};
 }
 
@@ -58,6 +60,32 @@ KernelEntry entry_for(int d, int bs, int g) {
 
 KernelEntry decode_entry(int d, int bs, int g, pkv_dtype dt) {
   return dt == PKV_FP16 ? entry_for<Fp16>(d, bs, g) : entry_for<Bf16>(d, bs, g);
+}
+
+// E4M3 cache: the CUDA-core kernel for every group size (the codes widen to
+// fp32 in registers; q and out keep their 16-bit type).
+template <int D, int BS, class DT>
+KernelEntry fp8_entry_for_group(int g) {
+  switch (g) {
+    case 1: return make_entry<D, BS, 1, DT, Fp8E4M3>();
+    case 2: return make_entry<D, BS, 2, DT, Fp8E4M3>();
+    case 4: return make_entry<D, BS, 4, DT, Fp8E4M3>();
+    case 8: return make_entry<D, BS, 8, DT, Fp8E4M3>();
+    default: return KernelEntry{nullptr, 0, 0};
+  }
+}
+
+template <class DT>
+KernelEntry fp8_entry_for(int d, int bs, int g) {
+  if (d == 128 && bs == 16) return fp8_entry_for_group<128, 16, DT>(g);
+  if (d == 128 && bs == 32) return fp8_entry_for_group<128, 32, DT>(g);
+  if (d == 64 && bs == 16) return fp8_entry_for_group<64, 16, DT>(g);
+  if (d == 64 && bs == 32) return fp8_entry_for_group<64, 32, DT>(g);
+  return KernelEntry{nullptr, 0, 0};
+}
+
+KernelEntry fp8_decode_entry(int d, int bs, int g, pkv_dtype dt) {
+  return dt == PKV_FP16 ? fp8_entry_for<Fp16>(d, bs, g) : fp8_entry_for<Bf16>(d, bs, g);
 }
 
 // ---- tensor-core kernel dispatch -------------------------------------------
@@ -243,16 +271,19 @@ extern "C" size_t pkv_paged_attn_workspace_bytes(int num_seqs, int num_heads, in
   return workspace_layout(num_seqs, num_heads, head_dim, max_parts).total;
 }
 
-extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
-                                            const void* v_cache, const int32_t* block_tables,
-                                            const int32_t* context_lens, float scale,
-                                            int num_seqs, int num_heads, int num_kv_heads,
-                                            int head_dim, int block_size, int max_blocks_per_seq,
-                                            int max_context_len, int num_blocks, pkv_dtype dtype,
-                                            int partition_size, void* workspace,
-                                            size_t workspace_bytes, unsigned* dev_err,
-                                            void* stream) {
-  using namespace pkv;
+namespace pkv {
+
+// Shared body of the 16-bit and the E4M3 decode entry points.  With fp8 the
+// caches hold E4M3 codes and every value of kv head h is code * k_scales[h]
+// (keys) or code * v_scales[h] (values): the K scale folds into the q
+// pre-scale, the V scale into the output numerator.
+pkv_status decode_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, float scale,
+                         int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                         int block_size, int max_blocks_per_seq, int max_context_len,
+                         int num_blocks, pkv_dtype dtype, int partition_size, void* workspace,
+                         size_t workspace_bytes, unsigned* dev_err, void* stream, bool fp8,
+                         const float* k_scales, const float* v_scales) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0 || num_blocks <= 0 || partition_size < 0 || !dtype_valid(dtype) ||
       num_heads % num_kv_heads != 0 || !isfinite(scale))
@@ -266,7 +297,8 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
     return PKV_ERR_INVALID_ARG;
   if (partition_size % block_size != 0) return PKV_ERR_INVALID_ARG;
   if (num_seqs == 0) return PKV_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
+      (fp8 && (!k_scales || !v_scales)))
     return PKV_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
@@ -284,8 +316,9 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
   const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * max_parts;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
-  const bool use_mma = group >= 2;
+  const bool use_mma = group >= 2 && !fp8;
   const KernelEntry ke = use_mma ? KernelEntry{nullptr, 0, 0}
+                         : fp8   ? fp8_decode_entry(head_dim, block_size, group, dtype)
                                  : decode_entry(head_dim, block_size, group, dtype);
   const MmaEntry me = use_mma ? mma_entry(head_dim, block_size, group, dtype)
                               : MmaEntry{nullptr, 0, 0};
@@ -312,6 +345,8 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   p.qscale = scale * kLog2e;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;
@@ -350,6 +385,39 @@ extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void
   rcfg.blockDim = dim3(128);
   rcfg.dynamicSmemBytes = 0;
   return cuda_status(cudaLaunchKernelEx(&rcfg, reduce_entry(head_dim, dtype), p));
+}
+
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
+                                            const void* v_cache, const int32_t* block_tables,
+                                            const int32_t* context_lens, float scale,
+                                            int num_seqs, int num_heads, int num_kv_heads,
+                                            int head_dim, int block_size, int max_blocks_per_seq,
+                                            int max_context_len, int num_blocks, pkv_dtype dtype,
+                                            int partition_size, void* workspace,
+                                            size_t workspace_bytes, unsigned* dev_err,
+                                            void* stream) {
+  return pkv::decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                            partition_size, workspace, workspace_bytes, dev_err, stream, false,
+                            nullptr, nullptr);
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_fp8(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, float scale,
+    const float* k_scales, const float* v_scales, int num_seqs, int num_heads, int num_kv_heads,
+    int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err,
+    void* stream) {
+  return pkv::decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                            partition_size, workspace, workspace_bytes, dev_err, stream, true,
+                            k_scales, v_scales);
 }
 
 // ---------------------------------------------------------------------------

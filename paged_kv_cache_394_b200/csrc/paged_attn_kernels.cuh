@@ -50,6 +50,8 @@ struct DecodeParams {
   const int32_t* block_tables;
   const int32_t* context_lens;
   float qscale;  // scale * log2(e)
+  const float* k_scales;  // 8-bit cache: per-kv-head K scales [num_kv_heads], else null
+  const float* v_scales;  // 8-bit cache: per-kv-head V scales [num_kv_heads], else null
   int num_seqs;
   int num_heads;
   int num_kv_heads;
@@ -69,11 +71,14 @@ __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-template <int D_, int BS_, int G_, class DT_, int W_, int NS_>
+template <int D_, int BS_, int G_, class DT_, int W_, int NS_, class KV_ = DT_>
 struct DecodeTraits {
   static constexpr int D = D_, BS = BS_, G = G_, W = W_, NS = NS_;
-  using DT = DT_;
+  using DT = DT_;   // q and out
   using T = typename DT::T;
+  using KV = KV_;   // cache elements: 16-bit like q, or 8-bit E4M3
+  using KT = typename KV::T;
+  static constexpr int KV_BYTES = static_cast<int>(sizeof(KT));
   static constexpr int NC = D / 8;                // 16-byte chunks per row
   static constexpr int LOG2_NC = ilog2(NC);
   static constexpr int R = 32 / NC;               // rows per warp-wide load
@@ -87,7 +92,7 @@ struct DecodeTraits {
   static constexpr int REP = NC / NV;             // lanes holding each logit
   static constexpr int SEG = JS * REP;            // lanes of one head within a row group
   static constexpr int CHUNK_ELEMS = BS * D;
-  static constexpr int CHUNK_BYTES = CHUNK_ELEMS * 2;
+  static constexpr int CHUNK_BYTES = CHUNK_ELEMS * KV_BYTES;
   static constexpr int STAGE_BYTES = 2 * CHUNK_BYTES;
   static constexpr int THREADS = W * 32;
   static constexpr int PB_FLOATS = R * NV + 8;    // p values + per-head alpha (G <= 8)
@@ -151,6 +156,16 @@ __device__ __forceinline__ float segment_sum(float x) {
   return x;
 }
 
+// 8 consecutive cache elements of a shared-memory row -> floats.
+template <class KV>
+__device__ __forceinline__ void load_row8(const typename KV::T* at, float (&f)[8]) {
+  if constexpr (sizeof(typename KV::T) == 1) {
+    unpack8(*reinterpret_cast<const uint2*>(at), f, KV());
+  } else {
+    unpack8(*reinterpret_cast<const uint4*>(at), f, KV());
+  }
+}
+
 // Per-warp running state of the online softmax.
 template <class Tr>
 struct WarpState {
@@ -163,8 +178,8 @@ struct WarpState {
 // Consumes one block (K and V chunks in shared memory): `valid` leading
 // tokens of it belong to the sequence.
 template <class Tr, bool kFull>
-__device__ __forceinline__ void process_block(WarpState<Tr>& st, const typename Tr::T* kch,
-                                              const typename Tr::T* vch, int valid, float* pbuf,
+__device__ __forceinline__ void process_block(WarpState<Tr>& st, const typename Tr::KT* kch,
+                                              const typename Tr::KT* vch, int valid, float* pbuf,
                                               int& buf, int lane) {
   constexpr int NC = Tr::NC, R = Tr::R, JS = Tr::JS, TS = Tr::TS, NV = Tr::NV, G = Tr::G;
   const int c = lane & (NC - 1);
@@ -182,9 +197,8 @@ __device__ __forceinline__ void process_block(WarpState<Tr>& st, const typename 
 #pragma unroll
     for (int j = 0; j < JS; ++j) {
       const int row = tb + r0 + R * j;
-      const uint4 raw = *reinterpret_cast<const uint4*>(kch + row * Tr::D + c * 8);
       float kf[8];
-      unpack8(raw, kf, typename Tr::DT());
+      load_row8<typename Tr::KV>(kch + row * Tr::D + c * 8, kf);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float s = st.q[g][0] * kf[0];
@@ -230,9 +244,8 @@ __device__ __forceinline__ void process_block(WarpState<Tr>& st, const typename 
     for (int j = 0; j < JS; ++j) {
       const int row = tb + r0 + R * j;
       if (kFull || row < valid) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(vch + row * Tr::D + c * 8);
         float vf[8];
-        unpack8(raw, vf, typename Tr::DT());
+        load_row8<typename Tr::KV>(vch + row * Tr::D + c * 8, vf);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float pg = pv[g * JS + j];
@@ -275,6 +288,11 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
       }
     }
     const int head = kvh * G + g;
+    if (p.v_scales != nullptr) {
+      const float vs = p.v_scales[kvh];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) num[e] *= vs;
+    }
     if (direct) {
       const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
@@ -297,9 +315,10 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
 template <class Tr>
 __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeParams p) {
   using T = typename Tr::T;
+  using KT = typename Tr::KT;
   constexpr int W = Tr::W, NS = Tr::NS, G = Tr::G, D = Tr::D, BS = Tr::BS, NC = Tr::NC;
   extern __shared__ __align__(128) unsigned char smem[];
-  T* ring = reinterpret_cast<T*>(smem);
+  KT* ring = reinterpret_cast<KT*>(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
   float* pbuf_all = reinterpret_cast<float*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
   int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES + Tr::PBUF_BYTES);
@@ -341,6 +360,16 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   __syncthreads();
 
   // ---- this lane's q chunk for the G heads, pre-scaled ---------------------
+  // (an 8-bit cache's K scale folds into the q pre-scale: q.(code*s) = (s*q).code)
+  float qscale = p.qscale;
+  if (p.k_scales != nullptr) {
+    const float ks = p.k_scales[kvh];
+    const float vs = p.v_scales[kvh];
+    if (!(ks > 0.f && ks < INFINITY && vs > 0.f && vs < INFINITY) && threadIdx.x == 0 &&
+        part == 0)
+      set_err(p.err, PKV_DEVERR_BAD_SCALE);
+    qscale *= ks;
+  }
   WarpState<Tr> st;
   const int c = lane & (NC - 1);
   {
@@ -352,7 +381,7 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
       unpack8(raw, st.q[g], typename Tr::DT());
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        st.q[g][e] *= p.qscale;
+        st.q[g][e] *= qscale;
         st.acc[g][e] = 0.f;
       }
     }
@@ -362,10 +391,10 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
 
   // ---- stream this warp's blocks through its ring ---------------------------
   const int nbw = nb > warp ? (nb - warp + W - 1) / W : 0;
-  T* wring = ring + static_cast<size_t>(warp) * NS * 2 * Tr::CHUNK_ELEMS;
+  KT* wring = ring + static_cast<size_t>(warp) * NS * 2 * Tr::CHUNK_ELEMS;
   const uint32_t bar0 = smem_addr(bars + warp * NS);
-  const T* kbase = static_cast<const T*>(p.k_cache);
-  const T* vbase = static_cast<const T*>(p.v_cache);
+  const KT* kbase = static_cast<const KT*>(p.k_cache);
+  const KT* vbase = static_cast<const KT*>(p.v_cache);
   const size_t head_off = static_cast<size_t>(kvh) * Tr::CHUNK_ELEMS;
   const size_t block_stride = static_cast<size_t>(p.num_kv_heads) * Tr::CHUNK_ELEMS;
 
@@ -407,8 +436,8 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
     }
     const int pb = tbl[warp + k * W];
     if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
-      const T* kch = wring + (2 * stage) * Tr::CHUNK_ELEMS;
-      const T* vch = kch + Tr::CHUNK_ELEMS;
+      const KT* kch = wring + (2 * stage) * Tr::CHUNK_ELEMS;
+      const KT* vch = kch + Tr::CHUNK_ELEMS;
       const int lb = blk_begin + warp + k * W;
       const int valid = min(BS, ctx - lb * BS);
       if (valid == BS)

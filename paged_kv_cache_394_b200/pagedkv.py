@@ -20,9 +20,9 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_OUT_OF_BLOCKS = range(6)
-FP16, BF16 = 0, 1
-DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_PAIR, DEVERR_BAD_CONTEXT, DEVERR_TIMEOUT = (
-    1, 2, 4, 8, 16)
+FP16, BF16, FP8_E4M3 = 0, 1, 2
+(DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_PAIR, DEVERR_BAD_CONTEXT, DEVERR_TIMEOUT,
+ DEVERR_BAD_SCALE) = (1, 2, 4, 8, 16, 32)
 
 _vp, _i, _i64, _f, _sz, _u = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                               ctypes.c_size_t, ctypes.c_uint)
@@ -49,6 +49,11 @@ _paged_attn_decode_static_ws = _proto("pkv_paged_attn_decode_static_ws", _i, _vp
                                      _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                      _vp)
 STATIC_WORKSPACE_BYTES = 16 << 20
+_reshape_and_cache_fp8 = _proto("pkv_reshape_and_cache_fp8", _i, _vp, _vp, _vp, _vp, _vp, _i, _i,
+                                _i, _i, _i, _i, _vp, _vp, _vp, _vp)
+_paged_attn_decode_fp8 = _proto("pkv_paged_attn_decode_fp8", _i, _vp, _vp, _vp, _vp, _vp, _vp, _f,
+                                _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp,
+                                _vp)
 _paged_attn_prefill = _proto("pkv_paged_attn_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i,
                              _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp)
 _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
@@ -104,6 +109,13 @@ def _dtype_code(t):
     raise TypeError("expected float16 or bfloat16, got %s" % t.dtype)
 
 
+def _cache_dtype_code(t):
+    """Element type of a cache: 16-bit, or E4M3 codes held as uint8 / float8_e4m3fn."""
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return FP8_E4M3
+    return _dtype_code(t)
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -148,8 +160,10 @@ def copy_blocks(k_cache, v_cache, block_mapping, dev_err=None, stream=None):
     p = block_mapping.shape[0] if block_mapping.numel() else 0
     if block_mapping.numel() and block_mapping.shape != (p, 2):
         raise ValueError("block_mapping must be [num_pairs, 2]")
+    if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must match")
     _check(_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), p, hkv, d, bs,
-                        num_blocks, _dtype_code(k_cache), _ptr(dev_err), _stream(stream)),
+                        num_blocks, _cache_dtype_code(k_cache), _ptr(dev_err), _stream(stream)),
            "copy_blocks")
 
 
@@ -189,6 +203,8 @@ def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scal
     if workspace is None:
         need = workspace_bytes(s, h, hkv, d, bs, max_context_len, partition_size)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if need else None
+        if workspace is not None and stream is not None:
+            workspace.record_stream(stream)   # the temporary must outlive the launch
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_paged_attn_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
@@ -197,6 +213,87 @@ def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scal
                               _dtype_code(q), partition_size, ws_ptr, ws_bytes, _ptr(dev_err),
                               _stream(stream)),
            "paged_attn_decode")
+
+
+def fp8_scales(scales, num_kv_heads, device=None):
+    """Per-kv-head E4M3 scales as the float32 device tensor [num_kv_heads] the
+    library reads: a number is repeated, a tensor is checked and returned."""
+    if isinstance(scales, torch.Tensor):
+        _dev(scales, "scales", torch.float32)
+        if scales.shape != (num_kv_heads,):
+            raise ValueError("scales must be [num_kv_heads]")
+        return scales
+    return torch.full((num_kv_heads,), float(scales), dtype=torch.float32,
+                      device=device or "cuda")
+
+
+def _scales_for(k_scales, v_scales, hkv, device, stream):
+    ks, vs = fp8_scales(k_scales, hkv, device), fp8_scales(v_scales, hkv, device)
+    if stream is not None:   # a temporary must outlive the launch on that stream
+        ks.record_stream(stream)
+        vs.record_stream(stream)
+    return ks, vs
+
+
+def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scales, v_scales,
+                          dev_err=None, stream=None):
+    """Quantise the new tokens' K/V ([T, Hkv, D], 16-bit) to E4M3 codes of
+    x / scale[h] and write them into their slots of the uint8 caches.
+    ``k_scales`` / ``v_scales``: float32 device tensors [Hkv] (see fp8_scales)."""
+    for n, t in (("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    if _cache_dtype_code(k_cache) != FP8_E4M3 or v_cache.dtype != k_cache.dtype:
+        raise TypeError("E4M3 caches must be uint8 (or float8_e4m3fn)")
+    num_blocks, hkv, bs, d = k_cache.shape
+    t = key.shape[0]
+    if key.shape != (t, hkv, d) or value.shape != key.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if value.dtype != key.dtype:
+        raise TypeError("key and value must share a dtype")
+    if slot_mapping.shape != (t,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    ks, vs = _scales_for(k_scales, v_scales, hkv, key.device, stream)
+    _check(_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(slot_mapping), t, hkv, d, bs, num_blocks, _dtype_code(key),
+                                  _ptr(ks), _ptr(vs), _ptr(dev_err), _stream(stream)),
+           "reshape_and_cache_fp8")
+
+
+def paged_attn_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scales,
+                          v_scales, num_kv_heads, block_size, max_context_len, partition_size=0,
+                          workspace=None, dev_err=None, stream=None):
+    """Paged decode attention over E4M3 caches (values = code * scale of the
+    kv head); q and out are 16-bit.  See include/pagedkv.h."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    s, h, d = q.shape
+    num_blocks, hkv, bs, dk = k_cache.shape
+    if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if _cache_dtype_code(k_cache) != FP8_E4M3 or v_cache.dtype != k_cache.dtype:
+        raise TypeError("E4M3 caches must be uint8 (or float8_e4m3fn)")
+    if out.dtype != q.dtype:
+        raise TypeError("q and out must share a dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    if workspace is None:
+        need = workspace_bytes(s, h, hkv, d, bs, max_context_len, partition_size)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if need else None
+        if workspace is not None and stream is not None:
+            workspace.record_stream(stream)   # the temporary must outlive the launch
+    ws_ptr = _ptr(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    ks, vs = _scales_for(k_scales, v_scales, hkv, q.device, stream)
+    _check(_paged_attn_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(block_tables), _ptr(context_lens), float(scale),
+                                  _ptr(ks), _ptr(vs), s, h, hkv, d, bs,
+                                  block_tables.shape[1], max_context_len, num_blocks,
+                                  _dtype_code(q), partition_size, ws_ptr, ws_bytes,
+                                  _ptr(dev_err), _stream(stream)),
+           "paged_attn_decode_fp8")
 
 
 def paged_attn_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, scale,

@@ -106,3 +106,56 @@ def test_staging_bytes_covers_inputs():
     s, h, hkv, d, mb, t, p = 64, 32, 32, 128, 128, 64, 3
     need = 2 * s * h * d * 2 + 2 * t * hkv * d * 2 + t * 8 + p * 16 + s * mb * 4 + s * 4
     assert pk.staging_bytes(s, h, hkv, d, mb, t, p) >= need
+
+
+def test_fp8_host_validation_without_gpu():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    null = None
+    good = ctypes.c_void_p(0x1000)
+    bad = ctypes.c_void_p(0x1008)
+    rc8 = pk._reshape_and_cache_fp8
+    # 16-bit sources only; E4M3 is a cache type, not an input type
+    assert rc8(good, good, good, good, good, 4, 2, 64, 16, 8, pk.FP8_E4M3, good, good, null,
+               null) == pk.ERR_INVALID_ARG
+    # scale arrays are required
+    assert rc8(good, good, good, good, good, 4, 2, 64, 16, 8, pk.FP16, null, good, null,
+               null) == pk.ERR_INVALID_ARG
+    assert rc8(good, good, good, good, good, 4, 2, 64, 16, 8, pk.FP16, good, null, null,
+               null) == pk.ERR_INVALID_ARG
+    assert rc8(null, null, null, null, null, 0, 2, 64, 16, 8, pk.BF16, null, null, null,
+               null) == pk.OK
+    assert rc8(null, null, null, null, null, 4, 2, 96, 16, 8, pk.FP16, good, good, null,
+               null) == pk.ERR_UNSUPPORTED
+    assert rc8(good, bad, good, good, good, 4, 2, 64, 16, 8, pk.FP16, good, good, null,
+               null) == pk.ERR_INVALID_ARG
+    # copy_blocks accepts the 1-byte cache type; unknown types are rejected
+    assert pk._copy_blocks(null, null, null, 0, 2, 64, 16, 8, pk.FP8_E4M3, null, null) == pk.OK
+    assert pk._copy_blocks(good, good, good, 1, 2, 64, 16, 8, 9, null, null) == pk.ERR_INVALID_ARG
+    # the 16-bit scatter and decode still refuse the 1-byte type
+    assert pk._reshape_and_cache(good, good, good, good, good, 4, 2, 64, 16, 8, pk.FP8_E4M3,
+                                 null, null) == pk.ERR_INVALID_ARG
+
+    def dec8(ks=good, vs=good, h=4, dt=pk.FP16, s=2, ptr=good):
+        return pk._paged_attn_decode_fp8(ptr, ptr, ptr, ptr, ptr, ptr, 0.125, ks, vs, s, h, 2, 64,
+                                         16, 4, 64, 8, dt, 0, null, 0, null, null)
+    assert dec8(ks=null) == pk.ERR_INVALID_ARG
+    assert dec8(vs=null) == pk.ERR_INVALID_ARG
+    assert dec8(dt=pk.FP8_E4M3) == pk.ERR_INVALID_ARG     # q/out must be 16-bit
+    assert dec8(h=6) == pk.ERR_UNSUPPORTED                 # G = 3
+    assert dec8(s=0) == pk.OK
+    assert dec8(ptr=bad) == pk.ERR_INVALID_ARG
+
+
+def test_binding_constants_match_the_header():
+    """Status codes, dtype codes and device error bits of the binding equal
+    the values include/pagedkv.h defines."""
+    import re
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    hdr = open(os.path.join(ROOT, "include", "pagedkv.h")).read()
+    bits = dict((m.group(1), int(m.group(2))) for m in
+                re.finditer(r"#define PKV_DEVERR_(\w+) (\d+)u", hdr))
+    assert bits and all(getattr(pk, "DEVERR_" + k) == v for k, v in bits.items())
+    for name, val in re.findall(r"PKV_((?:ERR_\w+|OK))\s*=\s*(\d+)", hdr):
+        assert getattr(pk, name) == int(val), name
+    for name, val in re.findall(r"PKV_(FP16|BF16|FP8_E4M3)\s*=\s*(\d+)", hdr):
+        assert getattr(pk, name) == int(val), name

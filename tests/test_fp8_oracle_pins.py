@@ -67,3 +67,87 @@ def test_planted_encoding_mistakes_are_caught(monkeypatch, mistake):
     rng = np.random.default_rng(1)
     x = (rng.standard_normal(20000) * 20).astype(np.float32)
     assert not np.array_equal(F.e4m3_encode(x), torch_codes(x))
+
+
+def _exact_fp8_values(rng, shape):
+    """float64 values that E4M3 and fp16 both hold exactly: decode(code) for
+    random finite codes of magnitude <= 8."""
+    codes = rng.integers(0, 256, size=shape).astype(np.uint8)
+    vals = e4m3_decode(codes)
+    vals = np.where(np.isnan(vals) | (np.abs(vals) > 8), 0.25, vals)
+    return vals
+
+
+def test_fp8_decode_reduces_to_16bit_decode_on_exact_values():
+    """With every cached value exactly representable in both formats, the
+    E4M3 decode over codes (scales 1) equals the independently pinned fp16
+    decode over the same values, and a power-of-two k_scale / v_scale equals
+    scaling the softmax scale / the output."""
+    from oracle import attention as OA
+    from oracle.fp8 import paged_attention_decode_fp8
+    rng = np.random.default_rng(7)
+    nb, hkv, bs, d, s, h = 12, 2, 16, 64, 3, 4
+    kv = _exact_fp8_values(rng, (2, nb, hkv, bs, d))
+    codes = e4m3_encode(kv.astype(np.float32))
+    bits = kv.astype(np.float16).view(np.uint16)
+    q = rng.standard_normal((s, h, d)).astype(np.float16).view(np.uint16)
+    tables = np.stack([rng.permutation(nb)[:4] for _ in range(s)]).astype(np.int32)
+    lens = np.array([1, 37, 64], dtype=np.int32)
+    ref = OA.paged_attention_decode(q, bits[0], bits[1], tables, lens, 0.125, hkv, bs, "fp16")
+    got = paged_attention_decode_fp8(q, codes[0], codes[1], tables, lens, 0.125, 1.0, 1.0, hkv,
+                                     bs, "fp16")
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    # K scaled by 2 == softmax scale doubled; V scaled by 4 == output times 4
+    got2 = paged_attention_decode_fp8(q, codes[0], codes[1], tables, lens, 0.125, 2.0, 4.0, hkv,
+                                      bs, "fp16")
+    ref2 = OA.paged_attention_decode(q, bits[0], bits[1], tables, lens, 0.25, hkv, bs, "fp16")
+    np.testing.assert_allclose(got2, 4.0 * ref2, rtol=1e-12, atol=1e-12)
+
+
+def test_quantize_into_cache_places_codes_like_the_16bit_write():
+    from oracle import cache_ops as OC
+    from oracle.fp8 import quantize, quantize_into_cache
+    rng = np.random.default_rng(3)
+    nb, hkv, bs, d, t = 6, 2, 16, 64, 20
+    key = rng.standard_normal((t, hkv, d)).astype(np.float16).view(np.uint16)
+    val = rng.standard_normal((t, hkv, d)).astype(np.float16).view(np.uint16)
+    slots = rng.permutation(nb * bs)[:t].astype(np.int64)
+    slots[3] = -1
+    kc = np.zeros((nb, hkv, bs, d), np.uint8)
+    k8, v8 = quantize_into_cache(key, val, kc, kc, slots, bs, "fp16", 0.5, 2.0)
+    # the same scatter done by the (pinned) 16-bit write on pre-quantised codes
+    kq = quantize(key, "fp16", 0.5).astype(np.uint16)
+    vq = quantize(val, "fp16", 2.0).astype(np.uint16)
+    z = np.zeros((nb, hkv, bs, d), np.uint16)
+    kr, vr, bad = OC.reshape_and_cache(kq, vq, z, z, slots, bs)
+    assert not bad
+    assert np.array_equal(k8, kr.astype(np.uint8)) and np.array_equal(v8, vr.astype(np.uint8))
+    # and scale 0.5 means x / 0.5 = 2x: E4M3 of 2x
+    assert np.array_equal(quantize(key, "fp16", 0.5),
+                          e4m3_encode((key.view(np.float16).astype(np.float32) * 2)))
+
+
+def test_per_head_scales_act_head_by_head():
+    """A per-head scale vector equals running each kv head with its own
+    scalar scale (a mix-up of heads or axes fails)."""
+    from oracle.fp8 import paged_attention_decode_fp8, quantize_cache
+    rng = np.random.default_rng(9)
+    nb, hkv, bs, d, s, g = 10, 3, 16, 64, 2, 2
+    bits = rng.standard_normal((2, nb, hkv, bs, d)).astype(np.float16).view(np.uint16)
+    ks = np.array([0.01, 0.02, 0.05], np.float32)
+    vs = np.array([0.03, 0.004, 0.02], np.float32)
+    kc, vc = quantize_cache(bits[0], "fp16", ks), quantize_cache(bits[1], "fp16", vs)
+    for h in range(hkv):
+        assert np.array_equal(kc[:, h], quantize_cache(bits[0][:, h:h + 1], "fp16", ks[h])[:, 0])
+    q = rng.standard_normal((s, hkv * g, d)).astype(np.float16).view(np.uint16)
+    tables = np.stack([rng.permutation(nb)[:5] for _ in range(s)]).astype(np.int32)
+    lens = np.array([70, 33], np.int32)
+    got = paged_attention_decode_fp8(q, kc, vc, tables, lens, 0.125, ks, vs, hkv, bs, "fp16")
+    for h in range(hkv):
+        sub = paged_attention_decode_fp8(q[:, h * g:(h + 1) * g], kc[:, h:h + 1], vc[:, h:h + 1],
+                                         tables, lens, 0.125, ks[h], vs[h], 1, bs, "fp16")
+        np.testing.assert_array_equal(got[:, h * g:(h + 1) * g], sub)
+    # a different scale per head changes the result (the scales are applied)
+    other = paged_attention_decode_fp8(q, kc, vc, tables, lens, 0.125, ks[::-1].copy(), vs, hkv,
+                                       bs, "fp16")
+    assert not np.allclose(other, got)

@@ -272,8 +272,10 @@ pkv_status pkv_reshape_and_cache_fp8(const void* key, const void* value, void* k
  * with g the kv head of query head h.  q and out are 16-bit of type `dtype`;
  * every other argument, the workspace (same size as
  * pkv_paged_attn_workspace_bytes gives) and the error behaviour are those of
- * pkv_paged_attn_decode.  fp32 accumulation on the CUDA cores for every group
- * size.  Null scale pointers give PKV_ERR_INVALID_ARG.
+ * pkv_paged_attn_decode.  fp32 accumulation; head_dim 128 runs on the tensor
+ * cores (mma.sync with the codes widened exactly to fp16; bf16 queries are
+ * rounded to fp16 there, magnitudes above 65504 saturating), head_dim 64 on
+ * the CUDA cores in fp32.  Null scale pointers give PKV_ERR_INVALID_ARG.
  */
 pkv_status pkv_paged_attn_decode_fp8(void* out, const void* q, const void* k_cache,
                                      const void* v_cache, const int32_t* block_tables,

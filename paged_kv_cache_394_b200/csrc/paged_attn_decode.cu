@@ -17,15 +17,27 @@ namespace pkv {
 // Host side: shape dispatch, partition choice, workspace layout, launch.
 // ---------------------------------------------------------------------------
 
+// E4M3 cache: stages per warp of the tensor-core kernel, and whether G = 1
+// also runs there (else on the CUDA cores).  Measured on B200 (decode kernel
+// GB/s, D = 128): with 2 stages (32 KiB of ring, about five CTAs per SM) the
+// tensor-core kernel reads LLaMA-7B shapes at 5667 (G = 1; the CUDA-core
+// kernel: 5087), GQA chat at 5135 (G = 4), long contexts at 6203; with 3
+// stages 5549 / 4964 / 6162; with 6 stages 4396 / 3457 / 4207.
+constexpr int kFp8MmaStages = 2;
+constexpr bool kFp8G1OnTensorCores = true;
+
 // Warps per CTA and ring stages per warp for a (head_dim, block_size): about
 // 96 KiB of ring per CTA so two CTAs fit on an SM, 2..4 stages per warp.
-// An 8-bit cache moves half the bytes per block, so it may keep up to twice
-// as many stages in flight for the same ring size.
+// An 8-bit cache moves half the bytes per block for about the same
+// instructions per token, so per-warp latency, not the ring, limits it: its
+// CTAs keep 2 stages per warp (32 KiB of ring) and about six fit on an SM.
+// Measured on B200 for LLaMA-7B shapes (D = 128, bs 16, G = 1): 2 stages x 4
+// warps 5050 GB/s, 3 x 4: 4832, 3 x 8: 4762, 6 x 4 (two CTAs per SM): 3500.
 template <int D, int BS, int KB = 2>
 struct LaunchShape {
   static constexpr int W = 4;
   static constexpr int STAGE = 2 * BS * D * KB;
-  static constexpr int NS = cmax(2, cmin(8 / KB, (96 * 1024) / (W * STAGE)));
+  static constexpr int NS = KB == 1 ? 2 : cmax(2, cmin(4, (96 * 1024) / (W * STAGE)));
 };
 
 using KernelFn = void (*)(const DecodeParams);
@@ -62,10 +74,14 @@ KernelEntry decode_entry(int d, int bs, int g, pkv_dtype dt) {
   return dt == PKV_FP16 ? entry_for<Fp16>(d, bs, g) : entry_for<Bf16>(d, bs, g);
 }
 
-// E4M3 cache: the CUDA-core kernel for every group size (the codes widen to
-// fp32 in registers; q and out keep their 16-bit type).
+// E4M3 cache on the CUDA cores (the codes widen to fp32 in registers; q and
+// out keep their 16-bit type): G = 1, and every G at head_dim 64 (head_dim
+// 128 with G >= 2 runs on the tensor cores).
 template <int D, int BS, class DT>
 KernelEntry fp8_entry_for_group(int g) {
+  if constexpr (D == 128) {
+    return g == 1 ? make_entry<D, BS, 1, DT, Fp8E4M3>() : KernelEntry{nullptr, 0, 0};
+  }
   switch (g) {
     case 1: return make_entry<D, BS, 1, DT, Fp8E4M3>();
     case 2: return make_entry<D, BS, 2, DT, Fp8E4M3>();
@@ -98,16 +114,17 @@ struct MmaEntry {
 };
 
 // 4 warps; about 96 KiB of ring per CTA (2 CTAs per SM).
-template <int D>
+template <int D, int KB = 2>
 struct MmaShape {
   static constexpr int W = 4;
-  static constexpr int STAGE = 2 * (D / 64) * 16 * 128;
-  static constexpr int NS = cmax(2, cmin(6, (96 * 1024) / (W * STAGE)));
+  static constexpr int STAGE = 2 * (D * KB / 128) * 16 * 128;
+  static constexpr int NS = KB == 1 ? kFp8MmaStages : cmax(2, cmin(6, (96 * 1024) / (W * STAGE)));
 };
 
-template <int D, int BS, int G, class DT>
+template <int D, int BS, int G, class DT, class KV = DT>
 MmaEntry make_mma_entry() {
-  using Tr = MmaTraits<D, BS, G, DT, MmaShape<D>::W, MmaShape<D>::NS>;
+  using MS = MmaShape<D, static_cast<int>(sizeof(typename KV::T))>;
+  using Tr = MmaTraits<D, BS, G, DT, MS::W, MS::NS, KV>;
   return MmaEntry{paged_decode_mma_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(0)};
 }
 
@@ -132,6 +149,25 @@ MmaEntry mma_for(int d, int bs, int g) {
 
 MmaEntry mma_entry(int d, int bs, int g, pkv_dtype dt) {
   return dt == PKV_FP16 ? mma_for<Fp16>(d, bs, g) : mma_for<Bf16>(d, bs, g);
+}
+
+// E4M3 cache on the tensor cores: head_dim 128 (a row is one 128-byte box).
+template <int BS, class DT>
+MmaEntry fp8_mma_for_group(int g) {
+  switch (g) {
+    case 1: return make_mma_entry<128, BS, 1, DT, Fp8E4M3>();
+    case 2: return make_mma_entry<128, BS, 2, DT, Fp8E4M3>();
+    case 4: return make_mma_entry<128, BS, 4, DT, Fp8E4M3>();
+    case 8: return make_mma_entry<128, BS, 8, DT, Fp8E4M3>();
+    default: return MmaEntry{nullptr, 0, 0};
+  }
+}
+
+MmaEntry fp8_mma_entry(int d, int bs, int g, pkv_dtype dt) {
+  if (d != 128) return MmaEntry{nullptr, 0, 0};
+  if (bs == 16) return dt == PKV_FP16 ? fp8_mma_for_group<16, Fp16>(g) : fp8_mma_for_group<16, Bf16>(g);
+  if (bs == 32) return dt == PKV_FP16 ? fp8_mma_for_group<32, Fp16>(g) : fp8_mma_for_group<32, Bf16>(g);
+  return MmaEntry{nullptr, 0, 0};
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
@@ -173,13 +209,18 @@ pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, 
   if (enc == nullptr) return cuda_status(cudaErrorNotSupported);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d),
                         static_cast<cuuint64_t>(num_blocks) * hkv * bs};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, 16};
+  // 16 rows x 128 bytes: 64 16-bit elements or 128 E4M3 codes
+  const int eb = cache_elem_bytes(dt);
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * eb};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), 16};
   cuuint32_t estr[2] = {1, 1};
   Slot& sl = slots[next];
   next = (next + 1) % 4;
   const CUresult r =
-      enc(&sl.map, dt == PKV_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+      enc(&sl.map,
+          dt == PKV_FP16   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+          : dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                           : CU_TENSOR_MAP_DATA_TYPE_UINT8,
           2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -316,12 +357,14 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * max_parts;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
-  const bool use_mma = group >= 2 && !fp8;
+  // G >= 2 runs on the tensor cores (E4M3: head_dim 128 only), G = 1 on the CUDA cores
+  const bool use_mma = fp8 ? head_dim == 128 && (group >= 2 || kFp8G1OnTensorCores) : group >= 2;
   const KernelEntry ke = use_mma ? KernelEntry{nullptr, 0, 0}
                          : fp8   ? fp8_decode_entry(head_dim, block_size, group, dtype)
                                  : decode_entry(head_dim, block_size, group, dtype);
-  const MmaEntry me = use_mma ? mma_entry(head_dim, block_size, group, dtype)
-                              : MmaEntry{nullptr, 0, 0};
+  const MmaEntry me = !use_mma ? MmaEntry{nullptr, 0, 0}
+                      : fp8    ? fp8_mma_entry(head_dim, block_size, group, dtype)
+                               : mma_entry(head_dim, block_size, group, dtype);
   if (ke.fn == nullptr && me.fn == nullptr) return PKV_ERR_UNSUPPORTED;
   const size_t smem = (use_mma ? me.smem_fixed : ke.smem_fixed) + static_cast<size_t>(part_blocks) * 4;
   const void* kernel_ptr = use_mma ? reinterpret_cast<const void*>(me.fn)
@@ -331,9 +374,10 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   if (st != PKV_OK) return st;
   CUtensorMap kmap, vmap;
   if (use_mma) {
-    st = cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
+    const pkv_dtype cdt = fp8 ? PKV_FP8_E4M3 : dtype;
+    st = cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, head_dim, cdt);
     if (st != PKV_OK) return st;
-    st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
+    st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, head_dim, cdt);
     if (st != PKV_OK) return st;
   }
 

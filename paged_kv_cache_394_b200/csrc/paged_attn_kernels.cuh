@@ -485,7 +485,8 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
 }
 
 // ---------------------------------------------------------------------------
-// Grouped-query decode on the tensor cores (G >= 2).
+// Grouped-query decode on the tensor cores (G >= 2; with an E4M3 cache every G,
+// see mma_sub_block_fp8).
 //
 // With G query heads per kv head, q.K and P.V carry G multiply-adds per
 // cached element; on the CUDA cores that makes the kernel instruction-bound
@@ -502,15 +503,18 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
 // is two stages).  The ring, the table slice, the bounded waits, the split-K
 // partitions and the final merge are as in paged_decode_kernel.
 // ---------------------------------------------------------------------------
-template <int D_, int BS_, int G_, class DT_, int W_, int NS_>
+template <int D_, int BS_, int G_, class DT_, int W_, int NS_, class KV_ = DT_>
 struct MmaTraits {
   static constexpr int D = D_, BS = BS_, G = G_, W = W_, NS = NS_;
   using DT = DT_;
   using T = typename DT::T;
+  using KV = KV_;
+  static constexpr bool kFp8 = std::is_same<KV, Fp8E4M3>::value;
   static constexpr int SUB = 16;                   // tokens per stage (the mma M)
   static constexpr int SUBS_PER_BLOCK = BS / SUB;
-  static constexpr int BOXES = D / 64;             // 128-byte-wide boxes per row
-  static constexpr int BOX_BYTES = SUB * 128;      // one 16 x 64 box
+  static constexpr int ROW_BYTES = D * (kFp8 ? 1 : 2);
+  static constexpr int BOXES = ROW_BYTES / 128;    // 128-byte-wide boxes per row
+  static constexpr int BOX_BYTES = SUB * 128;      // one 16-row x 128-byte box
   static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
   static constexpr int KSTEPS = D / 16;            // q.K k-steps = P.V m-tiles
@@ -518,8 +522,8 @@ struct MmaTraits {
   static constexpr int RING_BYTES = W * NS * STAGE_BYTES;
   static constexpr int BAR_BYTES = W * NS * 8;
   static constexpr int COMBINE_BYTES = W * G * (D + 2) * 4;
-  static_assert(G >= 2 && G <= 8, "tensor-core path serves 2..8 heads per kv head");
-  static_assert(BS % SUB == 0 && D % 64 == 0, "shape");
+  static_assert(G >= (kFp8 ? 1 : 2) && G <= 8, "tensor-core path: up to 8 heads per kv head");
+  static_assert(BS % SUB == 0 && D % 64 == 0 && ROW_BYTES % 128 == 0, "shape");
   static_assert(COMBINE_BYTES <= RING_BYTES, "combine scratch reuses the ring");
   static size_t smem_bytes(int part_blocks) {
     return 1024 + static_cast<size_t>(RING_BYTES) + BAR_BYTES +
@@ -630,6 +634,124 @@ __device__ __forceinline__ void mma_sub_block(uint32_t kt, uint32_t vt, int vali
   }
 }
 
+// Two E4M3 codes (a 16-bit half of x) -> fp16x2, exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// The E4M3 form of mma_sub_block: the tile rows are 128 bytes of codes (one
+// swizzled box), widened to fp16 in registers; the mma runs in fp16.
+//   q.K: ldmatrix (16-bit lanes over byte pairs) gives lane (g, u) the codes of
+//        dims 4u..4u+3 of a 16-dim chunk, so the mma's k order inside each
+//        chunk is permuted (logical 2u+{0,1} = dims 4u+{0,1}, logical
+//        8+2u+{0,1} = dims 4u+2+{0,1}); the q fragments use the same order.
+//   P.V: lane (g, u) reads dims 16g..16g+15 of tokens 2u, 2u+1, 2u+8, 2u+9 and
+//        pairs tokens with byte permutes; mma j covers dims 16g+2j (row g) and
+//        16g+2j+1 (row g+8), so the lane's accumulators hold 16 consecutive dims.
+// Returns nothing; updates acc / m / l like mma_sub_block.  x = s * qscale is
+// the base-2 logit (qscale includes the kv head's K scale).
+template <class Tr>
+__device__ __forceinline__ void mma_sub_block_fp8(uint32_t kt, uint32_t vt, int valid,
+                                                  const uint32_t (&qf)[Tr::KSTEPS][2],
+                                                  float (&acc)[Tr::KSTEPS][4], float (&m)[2],
+                                                  float (&l)[2], float qscale, int lane) {
+  constexpr int KS = Tr::KSTEPS;
+  const int j = lane >> 3;
+  const int r = lane & 7;
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const int t = ((j & 1) << 3) + r;
+#pragma unroll
+    for (int cc = 0; cc < KS / 2; ++cc) {
+      uint32_t w[4];
+      ldsm_x4(kt + swizzled(t, 2 * cc + (j >> 1)), w);
+      uint32_t a[4];
+      e4m3x4_to_f16x2(w[0], a[0], a[2]);
+      e4m3x4_to_f16x2(w[1], a[1], a[3]);
+      mma_16816(s, a, qf[2 * cc][0], qf[2 * cc][1], Fp16());
+      e4m3x4_to_f16x2(w[2], a[0], a[2]);
+      e4m3x4_to_f16x2(w[3], a[1], a[3]);
+      mma_16816(s, a, qf[2 * cc + 1][0], qf[2 * cc + 1][1], Fp16());
+    }
+  }
+  const int t0 = lane >> 2;
+  float x0 = s[0] * qscale, x1 = s[1] * qscale, x2 = s[2] * qscale, x3 = s[3] * qscale;
+  if (valid < Tr::SUB) {
+    if (t0 >= valid) x0 = x1 = -INFINITY;
+    if (t0 + 8 >= valid) x2 = x3 = -INFINITY;
+  }
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
+  }
+  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+  const float a0 = exp2_approx(m[0] - mn0), a1 = exp2_approx(m[1] - mn1);
+  const float p0 = exp2_approx(x0 - mn0), p1 = exp2_approx(x1 - mn1);
+  const float p2 = exp2_approx(x2 - mn0), p3 = exp2_approx(x3 - mn1);
+  float s0 = p0 + p2, s1 = p1 + p3;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    s0 += __shfl_xor_sync(kFullMask, s0, o);
+    s1 += __shfl_xor_sync(kFullMask, s1, o);
+  }
+  l[0] = l[0] * a0 + s0;
+  l[1] = l[1] * a1 + s1;
+  m[0] = mn0;
+  m[1] = mn1;
+  if (__any_sync(kFullMask, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      acc[mt][0] *= a0;
+      acc[mt][1] *= a1;
+      acc[mt][2] *= a0;
+      acc[mt][3] *= a1;
+    }
+  }
+  // P in (0, 1] as fp16 (11 significant bits), transposed into the B operand
+  const uint32_t b0 = movmatrix_trans(pack2(p0, p1, Fp16()));
+  const uint32_t b1 = movmatrix_trans(pack2(p2, p3, Fp16()));
+  // rows past the context hold stale codes (maybe NaN): zero them
+  if (valid < Tr::SUB) {
+    for (int i = lane; i < (Tr::SUB - valid) * 8; i += 32) {
+      const uint32_t at = vt + (valid + i / 8) * 128 + ((i & 7) << 4);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(at), "r"(0u) : "memory");
+    }
+    __syncwarp();
+  }
+  {
+    const int g = lane >> 2, u = lane & 3;
+    uint4 v[4];  // tokens 2u, 2u+1, 2u+8, 2u+9: dims 16g .. 16g+15
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tok = 2 * u + (i & 1) + ((i >> 1) << 3);
+      const uint32_t at = vt + tok * 128 + ((g ^ (tok & 7)) << 4);
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                   : "r"(at));
+    }
+    const uint32_t w0[4] = {v[0].x, v[0].y, v[0].z, v[0].w};
+    const uint32_t w1[4] = {v[1].x, v[1].y, v[1].z, v[1].w};
+    const uint32_t w8[4] = {v[2].x, v[2].y, v[2].z, v[2].w};
+    const uint32_t w9[4] = {v[3].x, v[3].y, v[3].z, v[3].w};
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      // bytes (tok a dim d, tok b dim d, tok a dim d+1, tok b dim d+1), d = 16g + 2mt
+      const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+      const uint32_t lo = __byte_perm(w0[mt >> 1], w1[mt >> 1], sel);
+      const uint32_t hi = __byte_perm(w8[mt >> 1], w9[mt >> 1], sel);
+      uint32_t a[4];
+      e4m3x4_to_f16x2(lo, a[0], a[1]);
+      e4m3x4_to_f16x2(hi, a[2], a[3]);
+      mma_16816(acc[mt], a, b0, b1, Fp16());
+    }
+  }
+}
+
 template <class Tr>
 __global__ void __launch_bounds__(Tr::THREADS)
     paged_decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
@@ -680,7 +802,10 @@ __global__ void __launch_bounds__(Tr::THREADS)
   __syncthreads();
 
   // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) + {0,1,8,9}
+  // (E4M3 cache: dims 16ks + 4(lane%4) + {0,1,2,3}, the permuted k order of
+  // mma_sub_block_fp8, as fp16)
   uint32_t qf[KS][2];
+  float qscale = p.qscale;
   {
     const int n = lane >> 2;
     const int c = lane & 3;
@@ -688,8 +813,31 @@ __global__ void __launch_bounds__(Tr::THREADS)
                     (static_cast<size_t>(seq) * p.num_heads + kvh * G + min(n, G - 1)) * D;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
-      qf[ks][0] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
-      qf[ks][1] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+      if constexpr (Tr::kFp8) {
+        uint2 u = n < G ? *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c) : make_uint2(0, 0);
+        if constexpr (std::is_same<typename Tr::DT, Bf16>::value) {
+          // bf16 -> fp16 for the fp16 mma; magnitudes beyond fp16 saturate
+          auto cv = [](uint32_t w) {
+            const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.f), 65504.f);
+            const float hi = fminf(fmaxf(__uint_as_float(w & 0xffff0000u), -65504.f), 65504.f);
+            return pack2(lo, hi, Fp16());
+          };
+          u = make_uint2(cv(u.x), cv(u.y));
+        }
+        qf[ks][0] = u.x;
+        qf[ks][1] = u.y;
+      } else {
+        qf[ks][0] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
+        qf[ks][1] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
+      }
+    }
+    if constexpr (Tr::kFp8) {
+      const float ks = p.k_scales[kvh];
+      const float vs = p.v_scales[kvh];
+      if (!(ks > 0.f && ks < INFINITY && vs > 0.f && vs < INFINITY) && threadIdx.x == 0 &&
+          part == 0)
+        set_err(p.err, PKV_DEVERR_BAD_SCALE);
+      qscale *= ks;
     }
   }
   float acc[KS][4];
@@ -746,7 +894,10 @@ __global__ void __launch_bounds__(Tr::THREADS)
       const int sb = sb_begin + warp + k * W;
       const int valid = min(Tr::SUB, ctx - sb * Tr::SUB);
       const uint32_t kt = ring0 + stage * Tr::STAGE_BYTES;
-      mma_sub_block<Tr>(kt, kt + Tr::TILE_BYTES, valid, qf, acc, m, l, p.qscale, lane);
+      if constexpr (Tr::kFp8)
+        mma_sub_block_fp8<Tr>(kt, kt + Tr::TILE_BYTES, valid, qf, acc, m, l, qscale, lane);
+      else
+        mma_sub_block<Tr>(kt, kt + Tr::TILE_BYTES, valid, qf, acc, m, l, qscale, lane);
     }
     __syncwarp();
     if (lane == 0 && k + NS < nbw) {
@@ -775,14 +926,16 @@ __global__ void __launch_bounds__(Tr::THREADS)
     }
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) {
-      const int d = 16 * mt + d_lo;
+      // rows g and g+8 of mma mt: dims 16mt + g and +8 (E4M3: 16g + 2mt and +1)
+      const int d = Tr::kFp8 ? 16 * d_lo + 2 * mt : 16 * mt + d_lo;
+      const int d2 = Tr::kFp8 ? d + 1 : d + 8;
       if (2 * c < G) {
         cacc[(warp * G + 2 * c) * D + d] = acc[mt][0];
-        cacc[(warp * G + 2 * c) * D + d + 8] = acc[mt][2];
+        cacc[(warp * G + 2 * c) * D + d2] = acc[mt][2];
       }
       if (2 * c + 1 < G) {
         cacc[(warp * G + 2 * c + 1) * D + d] = acc[mt][1];
-        cacc[(warp * G + 2 * c + 1) * D + d + 8] = acc[mt][3];
+        cacc[(warp * G + 2 * c + 1) * D + d2] = acc[mt][3];
       }
     }
   }

@@ -6,13 +6,16 @@
 //   * warp 0 (producer): TMA loads of the 128-row Q tile (3-D tensor map over
 //     [T, H, D], so a tile's rows are (token, head-of-this-kv-head) pairs) and
 //     of K/V tiles of 64 keys, each gathered from 16-key pieces of the paged
-//     cache through the block table, into a 2-stage ring.
+//     cache through the block table, into a 4-stage ring; the 16 boxes of a
+//     tile are issued by 16 lanes at once.
 //   * warp 1 (MMA): allocates 256 TMEM columns; one thread issues
 //       S  = Q K^T   (M=128, N=64,  K=128; A, B K-major)  into TMEM (2 buffers)
 //       O += P V     (M=128, N=128, K=64;  A=P K-major, B=V MN-major) into TMEM
 //     and signals completion with tcgen05.commit on mbarriers.
 //   * warps 2-5 (softmax): thread r owns row r (TMEM lane r): it reads its S
-//     row from TMEM, masks causally, keeps the running max / sum in base 2,
+//     row from TMEM, masks causally (only on tiles that reach past the row),
+//     keeps the running max / sum in base 2 with the scale folded into the
+//     exponent's FFMA,
 //     rescales its O row in TMEM when the max moves, and writes P (fp16, or
 //     bf16 split into hi + lo halves) into 128-byte-swizzled shared memory.
 //     At the end it reads O, divides by the sum and stores the row.
@@ -268,30 +271,36 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           npieces = i + 1;
         }
       }
-      if (lane == 0) {
-        int bytes = 0;
+      int bytes = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
-            bytes += 4 * 2048;
+      for (int i = 0; i < 4; ++i)
+        if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
+          bytes += 4 * 2048;
+      const uint32_t bar = bar_kv_full(stage);
+      if (lane == 0) {
         for (int i = 0; i < npieces; ++i)
           if (static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks))
             set_err(p.err, PKV_DEVERR_BAD_BLOCK);
-        const uint32_t bar = bar_kv_full(stage);
-        if (bytes > 0) {
+        if (bytes > 0)
           mbar_arrive_expect_tx(bar, bytes);
-          const uint32_t st = sbase + Tr::OFF_KV + stage * Tr::STAGE;
-          for (int i = 0; i < npieces; ++i) {
-            if (static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks)) continue;
-            const int key0 = t * NKEY + i * 16;
-            const int y = (pb[i] * p.num_kv_heads + kvh) * BS + (key0 % BS);
-            tma_load_2d(st + 0 * Tr::KV_HALF + i * 2048, &kmap, 0, y, bar);
-            tma_load_2d(st + 1 * Tr::KV_HALF + i * 2048, &kmap, 64, y, bar);
-            tma_load_2d(st + 2 * Tr::KV_HALF + i * 2048, &vmap, 0, y, bar);
-            tma_load_2d(st + 3 * Tr::KV_HALF + i * 2048, &vmap, 64, y, bar);
-          }
-        } else {
+        else
           mbar_arrive(bar);
+      }
+      __syncwarp();
+      // lanes 0..15 issue the 16 boxes of the tile at once: lane = piece * 4 + kind,
+      // kind = K low dims, K high dims, V low dims, V high dims
+      if (lane < 16) {
+        const int i = lane >> 2, kind = lane & 3;
+        int pbi = pb[0];
+        if (i == 1) pbi = pb[1];
+        if (i == 2) pbi = pb[2];
+        if (i == 3) pbi = pb[3];
+        if (i < npieces && static_cast<unsigned>(pbi) < static_cast<unsigned>(p.num_blocks)) {
+          const uint32_t st = sbase + Tr::OFF_KV + stage * Tr::STAGE;
+          const int key0 = t * NKEY + i * 16;
+          const int y = (pbi * p.num_kv_heads + kvh) * BS + (key0 % BS);
+          tma_load_2d(st + kind * Tr::KV_HALF + i * 2048, kind < 2 ? &kmap : &vmap,
+                      (kind & 1) * 64, y, bar);
         }
       }
       __syncwarp();
@@ -377,25 +386,45 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         for (int i = 0; i < 16; ++i) s[c + i] = v[i];
       }
       tc::tmem_wait_ld();
-      float mx = -INFINITY;
+      // Scaled logits are x = s * qscale.  For qscale > 0 the row max of x is
+      // (max s) * qscale exactly, so s is masked and reduced unscaled and the
+      // scale folds into the exponent's FFMA: p = 2^(s * qscale - m).
+      float mult = p.qscale;
+      const bool needs_mask = kv0 + NKEY - 1 > pos;  // this tile reaches past the row
+      if (mult > 0.f) {
+        if (needs_mask) {
 #pragma unroll
-      for (int c = 0; c < NKEY; ++c) {
-        s[c] = (kv0 + c <= pos) ? s[c] * p.qscale : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+          for (int c = 0; c < NKEY; ++c) s[c] = (kv0 + c <= pos) ? s[c] : -INFINITY;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < NKEY; ++c) s[c] = (kv0 + c <= pos) ? s[c] * mult : -INFINITY;
+        mult = 1.f;
       }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < NKEY; c += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], s[c + u]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * mult;
       // move the reference max only when this tile would push P above 2^8
       float alpha = 1.f;
       if (active && mx > m + Tr::kRescaleThreshold) {
         alpha = exp2_approx(m - mx);  // 0 on the first tile (m = -inf)
         m = mx;
       }
-      const float m_use = m == -INFINITY ? 0.f : m;
-      float sum = 0.f;
+      const float neg_m = m == -INFINITY ? 0.f : -m;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < NKEY; ++c) {
-        s[c] = exp2_approx(s[c] - m_use);
-        sum += s[c];
+      for (int c = 0; c < NKEY; c += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          s[c + u] = exp2_approx(fmaf(s[c + u], mult, neg_m));
+          sum4[u] += s[c + u];
+        }
       }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * alpha + sum;
       if (t > 0 && __any_sync(kFullMask, alpha != 1.f)) {
         // O must hold every earlier tile before it is rescaled

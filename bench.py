@@ -223,26 +223,32 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
-    """Hash of the device code (the decode kernels and their helpers)."""
+DECODE_SOURCES = ("common.cuh", "paged_attn_kernels.cuh")
+PREFILL_SOURCES = ("common.cuh", "paged_prefill_kernels.cuh", "paged_prefill_tc_kernels.cuh")
+
+
+def kernel_source_hash(sources=DECODE_SOURCES):
+    """Hash of the device code of one kernel family (kernels and helpers)."""
     csrc = os.path.join(ROOT, "paged_kv_cache_394_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("common.cuh", "paged_attn_kernels.cuh"):
+    for f in sources:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload):
-    """DRAM bytes per decode launch from profiles/, if taken on the current kernels."""
-    path = os.path.join(ROOT, "profiles", "paged_decode_%s_traffic.md" % workload)
+def committed_traffic(workload, kind="decode"):
+    """DRAM bytes per launch of the workload's dominant kernel from profiles/,
+    if the counters were taken on the current device code."""
+    sources = PREFILL_SOURCES if kind == "prefill" else DECODE_SOURCES
+    path = os.path.join(ROOT, "profiles", "paged_%s_%s_traffic.md" % (kind, workload))
     try:
         text = open(path).read()
     except OSError:
         return None
     m_src = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     m_b = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", text)
-    if not (m_src and m_b) or m_src.group(1) != kernel_source_hash():
+    if not (m_src and m_b) or m_src.group(1) != kernel_source_hash(sources):
         return None
     return float(m_b.group(1))
 
@@ -438,8 +444,10 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": committed_traffic(args.workload),
-                         "kernel": ("paged_decode_mma_kernel" if w.num_heads > w.num_kv_heads
-                                    and not fp8 else "paged_decode_kernel")
+                         "kernel": ("paged_decode_mma_kernel"
+                                    if (fp8 and w.head_dim == 128)
+                                    or (not fp8 and w.num_heads > w.num_kv_heads)
+                                    else "paged_decode_kernel")
                          + (" + reduce" if split else ""),
                          "algorithmic_bytes_per_launch": dbytes,
                          "avg_launch_ms": round(dec_avg_ms, 5),
@@ -581,8 +589,10 @@ def run_ours_prefill(args):
                            l2="no flush: each step rewrites the new tokens' K/V"),
             "tokens_per_s": round(world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                         "kernel": "paged_prefill_kernel",
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": committed_traffic(args.workload, "prefill"),
+                         "kernel": "paged_prefill_tc_kernel" if w.head_dim == 128
+                                   else "paged_prefill_kernel",
                          "algorithmic_flops_per_launch": flops,
                          "avg_launch_ms": round(kern_ms, 5),
                          "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same "

@@ -6,6 +6,8 @@
 
 #include <mutex>
 
+#include <type_traits>
+
 #include "host_common.h"
 #include "paged_prefill_kernels.cuh"
 #include "paged_prefill_tc_kernels.cuh"
@@ -58,12 +60,23 @@ struct TcEntry {
   TcPrefillFn fn;
   int threads;
   size_t smem;
+  int rows;  // query rows per CTA
 };
+
+// Query tiles of 128 rows per CTA.  Two share every K/V tile, which halves the
+// TMA traffic per FLOP (the per-SM TMA engine paces the one-tile kernel).
+// Measured on B200 (kernel TFLOP/s, fp16, one tile -> two): 4 x 512 new tokens
+// on 2048 cached 376 -> 482, 2048 on 8192 cached 419 -> 607, the LLaMA-7B
+// prefill batch 350 -> 411.  bf16 splits P into hi + lo halves, so two tiles
+// leave room for only one P buffer per tile: 4096 new on 4096 cached (G = 4)
+// 445 -> 547, but the 4-sequence GQA prefill batch 331 -> 304; bf16 keeps one.
+template <class DT>
+constexpr int kTcQueryTiles = std::is_same<DT, Bf16>::value ? 1 : 2;
 
 template <int BS, int G, class DT>
 TcEntry make_tc() {
-  using Tr = TcPrefillTraits<BS, G, DT>;
-  return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes()};
+  using Tr = TcPrefillTraits<BS, G, DT, kTcQueryTiles<DT>>;
+  return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(), Tr::ROWS};
 }
 
 template <int BS, class DT>
@@ -73,7 +86,7 @@ TcEntry tc_group(int g) {
     case 2: return make_tc<BS, 2, DT>();
     case 4: return make_tc<BS, 4, DT>();
     case 8: return make_tc<BS, 8, DT>();
-    default: return TcEntry{nullptr, 0, 0};
+    default: return TcEntry{nullptr, 0, 0, 0};
   }
 }
 
@@ -81,7 +94,7 @@ template <class DT>
 TcEntry tc_for(int bs, int g) {
   if (bs == 16) return tc_group<16, DT>(g);
   if (bs == 32) return tc_group<32, DT>(g);
-  return TcEntry{nullptr, 0, 0};
+  return TcEntry{nullptr, 0, 0, 0};
 }
 
 // 3-D tensor map over q [T, H, 128]: boxes of (128/G tokens) x (G heads) x 64 dims,
@@ -144,11 +157,11 @@ extern "C" pkv_status pkv_paged_attn_prefill(
   const PrefillEntry pe = use_tc ? PrefillEntry{nullptr, 0, 0, 0}
                           : dtype == PKV_FP16 ? prefill_for<Fp16>(head_dim, block_size, group)
                                               : prefill_for<Bf16>(head_dim, block_size, group);
-  const TcEntry te = !use_tc ? TcEntry{nullptr, 0, 0}
+  const TcEntry te = !use_tc ? TcEntry{nullptr, 0, 0, 0}
                      : dtype == PKV_FP16 ? tc_for<Fp16>(block_size, group)
                                          : tc_for<Bf16>(block_size, group);
   if (pe.fn == nullptr && te.fn == nullptr) return PKV_ERR_UNSUPPORTED;
-  const int tile_rows = use_tc ? 128 : pe.rows;
+  const int tile_rows = use_tc ? te.rows : pe.rows;
   const long long rows = static_cast<long long>(max_query_len) * group;
   const int q_tiles = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * q_tiles;

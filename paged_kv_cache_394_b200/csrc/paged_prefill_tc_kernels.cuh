@@ -131,33 +131,41 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 
 }  // namespace tc
 
-template <int BS_, int G_, class DT_>
+template <int BS_, int G_, class DT_, int QT_>
 struct TcPrefillTraits {
-  static constexpr int D = 128, BS = BS_, G = G_;
+  static constexpr int D = 128, BS = BS_, G = G_, QT = QT_;
   using DT = DT_;
   using T = typename DT::T;
   static constexpr bool kBf16 = std::is_same<DT, Bf16>::value;
-  static constexpr int M = 128;                  // query rows per CTA
+  static constexpr int M = 128;                  // rows of one query tile (one TMEM lane each)
+  static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
   static constexpr int NKEY = 64;                // keys per KV tile
-  static constexpr int NS = 4;                   // KV stages (loads run up to 4 tiles ahead)
-  static constexpr int THREADS = 6 * 32;
+  // KV stages and P buffers per query tile: what fits beside QT query tiles
+  static constexpr int NS = QT == 1 ? 4 : 3;
+  static constexpr int PB = (QT == 2 && kBf16) ? 1 : 2;
+  static constexpr int THREADS = (2 + 4 * QT) * 32;
   // shared-memory layout (all 1024-byte aligned)
   static constexpr int Q_HALF = M * 128;         // [128 rows][64 dims] = 16 KiB
+  static constexpr int Q_TILE = 2 * Q_HALF;
   static constexpr int KV_HALF = NKEY * 128;     // [64 keys][64 dims] = 8 KiB
   static constexpr int STAGE = 4 * KV_HALF;      // K0 K1 V0 V1
   static constexpr int P_BYTES = M * 128;        // [128 rows][64 keys]
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = 2 * Q_HALF;
-  static constexpr int OFF_P = OFF_KV + NS * STAGE;          // P buffers 0, 1
-  static constexpr int OFF_PLO = OFF_P + 2 * P_BYTES;        // bf16 lo halves 0, 1
-  static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? 2 * P_BYTES : 0);
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2]; tmem slot
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2;
+  static constexpr int OFF_KV = QT * Q_TILE;
+  static constexpr int OFF_P = OFF_KV + NS * STAGE;              // [QT][PB] P buffers
+  static constexpr int OFF_PLO = OFF_P + QT * PB * P_BYTES;      // bf16 lo halves
+  static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? QT * PB * P_BYTES : 0);
+  // barriers: q_full, kv_full[NS], kv_empty[NS], then per query tile
+  // s_full[2], p_full[2], o_done[2]; then the TMEM address slot
+  static constexpr int NBAR = 1 + 2 * NS + 6 * QT;
   // the softmax reference max moves only when a row max exceeds it by more
   // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
   static constexpr float kRescaleThreshold = 8.f;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
-  static constexpr uint32_t TMEM_COLS = 256;     // S buffers at 0 and 64, O at 128
+  // per query tile q: S buffers at 256q and 256q + 64, O at 256q + 128
+  static constexpr uint32_t TMEM_COLS = 256 * QT;
+  static_assert(QT == 1 || QT == 2, "one or two query tiles per CTA");
+  static_assert(1024 + SMEM <= 232448, "shared memory per CTA");
   static size_t smem_bytes() { return 1024 + static_cast<size_t>(SMEM); }
 };
 
@@ -169,7 +177,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   using T = typename Tr::T;
   using DT = typename Tr::DT;
   constexpr int G = Tr::G, BS = Tr::BS, M = Tr::M, NKEY = Tr::NKEY, NS = Tr::NS;
-  constexpr int ROWS_PER_TOK = G;
+  constexpr int QT = Tr::QT, PB = Tr::PB, ROWS = Tr::ROWS;
   constexpr uint32_t IDESC_S = tc::idesc_f16(Tr::kBf16, M, NKEY, false);
   constexpr uint32_t IDESC_O = tc::idesc_f16(Tr::kBf16, M, 128, true);
   extern __shared__ unsigned char smem_raw[];
@@ -180,9 +188,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   const uint32_t bar_q = smem_addr(bars + 0);
   auto bar_kv_full = [&](int s) { return smem_addr(bars + 1 + s); };
   auto bar_kv_empty = [&](int s) { return smem_addr(bars + 1 + NS + s); };
-  auto bar_s_full = [&](int b) { return smem_addr(bars + 1 + 2 * NS + b); };
-  auto bar_p = [&](int b) { return smem_addr(bars + 3 + 2 * NS + b); };
-  auto bar_o = [&](int b) { return smem_addr(bars + 5 + 2 * NS + b); };
+  auto bar_s_full = [&](int q, int b) { return smem_addr(bars + 1 + 2 * NS + 6 * q + b); };
+  auto bar_p = [&](int q, int b) { return smem_addr(bars + 3 + 2 * NS + 6 * q + b); };
+  auto bar_o = [&](int q, int b) { return smem_addr(bars + 5 + 2 * NS + 6 * q + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
 
   const int tile = p.q_tiles - 1 - static_cast<int>(blockIdx.x % p.q_tiles);
@@ -203,25 +211,35 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     if (threadIdx.x == 0 && tile == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
     return;
   }
-  const int rows_total = q_len * ROWS_PER_TOK;
-  if (tile * M >= rows_total) return;
-  const int tok0 = tile * (M / G);  // first query token of this tile
-  const int last_tok = (min(rows_total, (tile + 1) * M) - 1) / G;
-  const int nkv = ctx - q_len + last_tok + 1;
+  const int rows_total = q_len * G;
+  if (tile * ROWS >= rows_total) return;
+  const int tok0 = tile * (ROWS / G);  // first query token of this CTA
+  // KV tiles each query tile needs (later rows see more keys; 0 = no rows)
+  int ntq[QT];
+#pragma unroll
+  for (int q = 0; q < QT; ++q) {
+    const int r0 = tile * ROWS + q * M;
+    const int last = (min(rows_total, r0 + M) - 1) / G;
+    ntq[q] = r0 < rows_total ? (ctx - q_len + last + 1 + NKEY - 1) / NKEY : 0;
+  }
+  const int last_tok = (min(rows_total, (tile + 1) * ROWS) - 1) / G;
+  const int nkv = ctx - q_len + last_tok + 1;  // keys the CTA reads
   const int ntiles = (nkv + NKEY - 1) / NKEY;
 
   if (threadIdx.x == 0) {
     // one arrival each (an expect_tx arrive or a tcgen05.commit), except p_full:
-    // one arrival per softmax warp
+    // one arrival per softmax warp of the query tile
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_kv_full(s), 1);
       mbar_init(bar_kv_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_s_full(b), 1);
-      mbar_init(bar_p(b), 4);
-      mbar_init(bar_o(b), 1);
+    for (int q = 0; q < QT; ++q) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(bar_s_full(q, b), 1);
+        mbar_init(bar_p(q, b), 4);
+        mbar_init(bar_o(q, b), 1);
+      }
     }
     fence_mbar_init();
   }
@@ -239,9 +257,14 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const int32_t* trow = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
     const int nblk = (nkv + BS - 1) / BS;
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, 2 * Tr::Q_HALF);
-      tc::tma_load_3d(sbase + Tr::OFF_Q, &qmap, 0, kvh * G, q0 + tok0, bar_q);
-      tc::tma_load_3d(sbase + Tr::OFF_Q + Tr::Q_HALF, &qmap, 64, kvh * G, q0 + tok0, bar_q);
+      mbar_arrive_expect_tx(bar_q, QT * Tr::Q_TILE);
+#pragma unroll
+      for (int q = 0; q < QT; ++q) {
+        const uint32_t dst = sbase + Tr::OFF_Q + q * Tr::Q_TILE;
+        const int z = q0 + tok0 + q * (M / G);
+        tc::tma_load_3d(dst, &qmap, 0, kvh * G, z, bar_q);
+        tc::tma_load_3d(dst + Tr::Q_HALF, &qmap, 64, kvh * G, z, bar_q);
+      }
     }
     int chunk = -1, entry = -1;
     for (int t = 0; t < ntiles; ++t) {
@@ -309,23 +332,36 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     // ---- MMA issuer ---------------------------------------------------------------
     if (lane == 0) {
       bool ok = mbar_wait_bounded(bar_q, 0);
-      const uint32_t q_lo = sbase + Tr::OFF_Q, q_hi = q_lo + Tr::Q_HALF;
-      auto issue_pv = [&](int t) {  // O += P V for tile t (its P is in buffer t & 1)
+      // O_q += P_q V for tile t (P in buffer t % PB of query tile q)
+      auto issue_pv = [&](int q, int t) {
         const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
         const uint32_t v0 = st + 2 * Tr::KV_HALF;
-        const uint32_t pbuf = sbase + Tr::OFF_P + (t & 1) * Tr::P_BYTES;
-        const uint32_t plo = sbase + Tr::OFF_PLO + (t & 1) * Tr::P_BYTES;
+        const int buf = q * PB + t % PB;
+        const uint32_t pbuf = sbase + Tr::OFF_P + buf * Tr::P_BYTES;
+        const uint32_t plo = sbase + Tr::OFF_PLO + buf * Tr::P_BYTES;
+        const uint32_t o_tmem = tmem + q * 256 + 128;
 #pragma unroll
         for (int kk = 0; kk < NKEY / 16; ++kk) {
           const uint64_t bdesc = tc::smem_desc_sw128(v0 + kk * 2048, Tr::KV_HALF, 1024);
           const uint64_t adesc = tc::smem_desc_sw128(pbuf + kk * 32, 16, 1024);
-          tc::umma_f16(tmem + 128, adesc, bdesc, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+          tc::umma_f16(o_tmem, adesc, bdesc, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
           if constexpr (Tr::kBf16) {
             const uint64_t ldesc = tc::smem_desc_sw128(plo + kk * 32, 16, 1024);
-            tc::umma_f16(tmem + 128, ldesc, bdesc, IDESC_O, 1u);
+            tc::umma_f16(o_tmem, ldesc, bdesc, IDESC_O, 1u);
           }
         }
-        tc::umma_commit(bar_o(t & 1));
+        tc::umma_commit(bar_o(q, t & 1));
+      };
+      // P.V of tile t for every query tile that uses it, then release its stage
+      auto finish_tile = [&](int t) {
+#pragma unroll
+        for (int q = 0; q < QT; ++q) {
+          if (t >= ntq[q]) continue;
+          ok = ok && mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+          if (!ok) return;
+          tc::tc_fence_after();
+          issue_pv(q, t);
+        }
         tc::umma_commit(bar_kv_empty(t % NS));
       };
       for (int t = 0; t < ntiles && ok; ++t) {
@@ -334,44 +370,41 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         tc::tc_fence_after();
         const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t qa = (ks < 4 ? q_lo : q_hi) + (ks & 3) * 32;
-          const uint32_t kb = st + (ks < 4 ? 0 : Tr::KV_HALF) + (ks & 3) * 32;
-          tc::umma_f16(tmem + (t & 1) * 64, tc::smem_desc_sw128(qa, 16, 1024),
-                       tc::smem_desc_sw128(kb, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
+        for (int q = 0; q < QT; ++q) {
+          if (t >= ntq[q]) continue;
+          const uint32_t q_lo = sbase + Tr::OFF_Q + q * Tr::Q_TILE, q_hi = q_lo + Tr::Q_HALF;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t qa = (ks < 4 ? q_lo : q_hi) + (ks & 3) * 32;
+            const uint32_t kb = st + (ks < 4 ? 0 : Tr::KV_HALF) + (ks & 3) * 32;
+            tc::umma_f16(tmem + q * 256 + (t & 1) * 64, tc::smem_desc_sw128(qa, 16, 1024),
+                         tc::smem_desc_sw128(kb, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
+          }
+          tc::umma_commit(bar_s_full(q, t & 1));
         }
-        tc::umma_commit(bar_s_full(t & 1));
-        if (t > 0) {
-          ok = mbar_wait_bounded(bar_p((t - 1) & 1), ((t - 1) >> 1) & 1);
-          if (!ok) break;
-          tc::tc_fence_after();
-          issue_pv(t - 1);
-        }
+        if (t > 0) finish_tile(t - 1);
       }
-      if (ok && ntiles > 0) {
-        ok = mbar_wait_bounded(bar_p((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1);
-        if (ok) {
-          tc::tc_fence_after();
-          issue_pv(ntiles - 1);
-        }
-      }
+      if (ok && ntiles > 0) finish_tile(ntiles - 1);
       if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
     }
     __syncwarp();
   } else {
-    // ---- softmax warps: thread <-> row <-> TMEM lane ---------------------------------
+    // ---- softmax warps: query tile qg, thread <-> row <-> TMEM lane -------------------
+    const int qg = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const bool active = r < rows_total - tile * M;
-    const int j = tok0 + r / G;
-    const int g = r % G;
+    const uint32_t lane_addr = tmem + qg * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int crow = qg * M + r;   // row within the CTA
+    const bool active = crow < rows_total - tile * ROWS;
+    const int j = tok0 + crow / G;
+    const int g = crow % G;
     const int pos = active ? ctx - q_len + j : -1;
+    const int my_tiles = qg == 0 ? ntq[0] : ntq[QT - 1];
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
+    for (int t = 0; t < my_tiles; ++t) {
       const int kv0 = t * NKEY;
-      ok = mbar_wait_bounded(bar_s_full(t & 1), (t >> 1) & 1);
+      ok = mbar_wait_bounded(bar_s_full(qg, t & 1), (t >> 1) & 1);
       if (!__all_sync(kFullMask, ok)) {
         ok = false;
         break;
@@ -428,7 +461,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       l = l * alpha + sum;
       if (t > 0 && __any_sync(kFullMask, alpha != 1.f)) {
         // O must hold every earlier tile before it is rescaled
-        ok = mbar_wait_bounded(bar_o((t - 1) & 1), ((t - 1) >> 1) & 1);
+        ok = mbar_wait_bounded(bar_o(qg, (t - 1) & 1), ((t - 1) >> 1) & 1);
         if (!__all_sync(kFullMask, ok)) {
           ok = false;
           break;
@@ -445,16 +478,17 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         tc::tmem_wait_st();
       }
-      if (t >= 2) {  // P buffer t & 1 was last read by P.V of tile t - 2
-        ok = mbar_wait_bounded(bar_o(t & 1), ((t - 2) >> 1) & 1);
+      if (t >= PB) {  // the P buffer of tile t was last read by P.V of tile t - PB
+        ok = mbar_wait_bounded(bar_o(qg, (t - PB) & 1), ((t - PB) >> 1) & 1);
         if (!__all_sync(kFullMask, ok)) {
           ok = false;
           break;
         }
       }
       // P (16-bit; bf16 as hi + lo) into the swizzled [128 rows][64 keys] buffers
-      unsigned char* prow = smem + Tr::OFF_P + (t & 1) * Tr::P_BYTES + r * 128;
-      unsigned char* plrow = smem + Tr::OFF_PLO + (t & 1) * Tr::P_BYTES + r * 128;
+      const int buf = qg * PB + t % PB;
+      unsigned char* prow = smem + Tr::OFF_P + buf * Tr::P_BYTES + r * 128;
+      unsigned char* plrow = smem + Tr::OFF_PLO + buf * Tr::P_BYTES + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t w[4], wl[4];
@@ -473,13 +507,13 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           *reinterpret_cast<uint4*>(plrow + at) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
       // keys past the context, or not loaded, hold stale data: zero their V rows
+      // (every query tile that uses the stage writes the same zeros)
       const int loaded_end = min(kv0 + NKEY, ((nkv + 15) / 16) * 16);
       const int vz = min(ctx, loaded_end) - kv0;  // V rows [vz, 64) must be zero
       if (vz < NKEY) {
         unsigned char* vt = smem + Tr::OFF_KV + (t % NS) * Tr::STAGE + 2 * Tr::KV_HALF;
         const int nrows = NKEY - vz;
-        const int tid = r;  // 128 softmax threads
-        for (int idx = tid; idx < nrows * 16; idx += 128) {
+        for (int idx = r; idx < nrows * 16; idx += 128) {
           const int row = vz + idx / 16;
           const int part = idx % 16;  // 8 chunks in each of the two dim halves
           *reinterpret_cast<uint4*>(vt + (part >> 3) * Tr::KV_HALF + row * 128 + (part & 7) * 16) =
@@ -489,14 +523,14 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p(t & 1));
+      if (lane == 0) mbar_arrive(bar_p(qg, t & 1));
     }
     // ---- epilogue ------------------------------------------------------------------------
-    if (ok && ntiles > 0) {
-      ok = mbar_wait_bounded(bar_o((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1);
+    if (ok && my_tiles > 0) {
+      ok = mbar_wait_bounded(bar_o(qg, (my_tiles - 1) & 1), ((my_tiles - 1) >> 1) & 1);
       ok = __all_sync(kFullMask, ok);
     }
-    if (ok && ntiles > 0) {
+    if (ok && my_tiles > 0) {
       tc::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       T* orow = static_cast<T*>(p.out) +

@@ -2,23 +2,27 @@
 // tensor cores (tcgen05 + TMEM) for head_dim 128 on B200 (sm_100a).
 //
 // Computes what paged_prefill_kernels.cuh computes (causal attention of each
-// new token over its sequence's paged cache) with 128-row tiles:
-//   * warp 0 (producer): TMA loads of the 128-row Q tile (3-D tensor map over
-//     [T, H, D], so a tile's rows are (token, head-of-this-kv-head) pairs) and
-//     of K/V tiles of 64 keys, each gathered from 16-key pieces of the paged
-//     cache through the block table, into a 4-stage ring; the 16 boxes of a
-//     tile are issued by 16 lanes at once.
-//   * warp 1 (MMA): allocates 256 TMEM columns; one thread issues
+// new token over its sequence's paged cache).  A CTA covers QT query tiles of
+// 128 rows (a row is a (token, head-of-this-kv-head) pair) that share every
+// K/V tile of 64 keys:
+//   * warp 0 (K producer): TMA loads of the query tiles (3-D tensor map over
+//     [T, H, D]) and of the K tiles, gathered from 16-key pieces of the paged
+//     cache through the block table into an NS-stage ring; the 8 boxes of a
+//     tile are issued by 8 lanes at once.
+//   * warp 2 (V producer): the same for the V tiles.  K of a stage is released
+//     once S has read it, V once P.V has, so K loads run further ahead.
+//   * warp 1 (MMA): allocates 256 TMEM columns per query tile; one thread
+//     issues, in whichever order their inputs arrive,
 //       S  = Q K^T   (M=128, N=64,  K=128; A, B K-major)  into TMEM (2 buffers)
 //       O += P V     (M=128, N=128, K=64;  A=P K-major, B=V MN-major) into TMEM
 //     and signals completion with tcgen05.commit on mbarriers.
-//   * warps 2-5 (softmax): thread r owns row r (TMEM lane r): it reads its S
-//     row from TMEM, masks causally (only on tiles that reach past the row),
-//     keeps the running max / sum in base 2 with the scale folded into the
-//     exponent's FFMA,
-//     rescales its O row in TMEM when the max moves, and writes P (fp16, or
-//     bf16 split into hi + lo halves) into 128-byte-swizzled shared memory.
-//     At the end it reads O, divides by the sum and stores the row.
+//   * 4 softmax warps per query tile: thread r owns row r (TMEM lane r): it
+//     reads its S row from TMEM, masks causally (only on tiles that reach past
+//     the row), keeps the running max / sum in base 2 with the scale folded
+//     into the exponent's FFMA, rescales its O row in TMEM when the max moves,
+//     and writes P (fp16, or bf16 split into hi + lo halves) into
+//     128-byte-swizzled shared memory.  At the end it reads O, divides by the
+//     sum and stores the row.
 // All operand tiles use the 128-byte swizzle (8-row x 128-byte atoms, stride
 // 1024 bytes).  Keys past the context (or not loaded) are zeroed in the V tile
 // before P.V so stale NaN never enters the tensor-core sum.  Every mbarrier
@@ -143,7 +147,7 @@ struct TcPrefillTraits {
   // KV stages and P buffers per query tile: what fits beside QT query tiles
   static constexpr int NS = QT == 1 ? 4 : 3;
   static constexpr int PB = (QT == 2 && kBf16) ? 1 : 2;
-  static constexpr int THREADS = (2 + 4 * QT) * 32;
+  static constexpr int THREADS = (3 + 4 * QT) * 32;
   // shared-memory layout (all 1024-byte aligned)
   static constexpr int Q_HALF = M * 128;         // [128 rows][64 dims] = 16 KiB
   static constexpr int Q_TILE = 2 * Q_HALF;
@@ -155,9 +159,9 @@ struct TcPrefillTraits {
   static constexpr int OFF_P = OFF_KV + NS * STAGE;              // [QT][PB] P buffers
   static constexpr int OFF_PLO = OFF_P + QT * PB * P_BYTES;      // bf16 lo halves
   static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? QT * PB * P_BYTES : 0);
-  // barriers: q_full, kv_full[NS], kv_empty[NS], then per query tile
-  // s_full[2], p_full[2], o_done[2]; then the TMEM address slot
-  static constexpr int NBAR = 1 + 2 * NS + 6 * QT;
+  // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
+  // per query tile s_full[2], p_full[2], o_done[2]; then the TMEM address slot
+  static constexpr int NBAR = 1 + 4 * NS + 6 * QT;
   // the softmax reference max moves only when a row max exceeds it by more
   // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
   static constexpr float kRescaleThreshold = 8.f;
@@ -186,11 +190,13 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   const uint32_t sbase = smem_addr(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
   const uint32_t bar_q = smem_addr(bars + 0);
-  auto bar_kv_full = [&](int s) { return smem_addr(bars + 1 + s); };
-  auto bar_kv_empty = [&](int s) { return smem_addr(bars + 1 + NS + s); };
-  auto bar_s_full = [&](int q, int b) { return smem_addr(bars + 1 + 2 * NS + 6 * q + b); };
-  auto bar_p = [&](int q, int b) { return smem_addr(bars + 3 + 2 * NS + 6 * q + b); };
-  auto bar_o = [&](int q, int b) { return smem_addr(bars + 5 + 2 * NS + 6 * q + b); };
+  auto bar_k_full = [&](int s) { return smem_addr(bars + 1 + s); };
+  auto bar_k_empty = [&](int s) { return smem_addr(bars + 1 + NS + s); };
+  auto bar_v_full = [&](int s) { return smem_addr(bars + 1 + 2 * NS + s); };
+  auto bar_v_empty = [&](int s) { return smem_addr(bars + 1 + 3 * NS + s); };
+  auto bar_s_full = [&](int q, int b) { return smem_addr(bars + 1 + 4 * NS + 6 * q + b); };
+  auto bar_p = [&](int q, int b) { return smem_addr(bars + 3 + 4 * NS + 6 * q + b); };
+  auto bar_o = [&](int q, int b) { return smem_addr(bars + 5 + 4 * NS + 6 * q + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
 
   const int tile = p.q_tiles - 1 - static_cast<int>(blockIdx.x % p.q_tiles);
@@ -231,8 +237,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     // one arrival per softmax warp of the query tile
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar_kv_full(s), 1);
-      mbar_init(bar_kv_empty(s), 1);
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_v_empty(s), 1);
     }
     for (int q = 0; q < QT; ++q) {
       for (int b = 0; b < 2; ++b) {
@@ -252,11 +260,14 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---- producer ---------------------------------------------------------------
+  if (warp == 0 || warp == 2) {
+    // ---- producers: warp 0 loads Q and the K tiles, warp 2 the V tiles ---------------
+    // K of a stage is released once S has read it, V once P.V has, so the K
+    // loads can run further ahead than the V loads.
+    const bool is_k = warp == 0;
     const int32_t* trow = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
     const int nblk = (nkv + BS - 1) / BS;
-    if (lane == 0) {
+    if (is_k && lane == 0) {
       mbar_arrive_expect_tx(bar_q, QT * Tr::Q_TILE);
 #pragma unroll
       for (int q = 0; q < QT; ++q) {
@@ -271,7 +282,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       const int stage = t % NS;
       bool ok = true;
       if (lane == 0) {
-        ok = mbar_wait_bounded(bar_kv_empty(stage), ((t / NS) & 1) ^ 1);
+        ok = mbar_wait_bounded(is_k ? bar_k_empty(stage) : bar_v_empty(stage),
+                               ((t / NS) & 1) ^ 1);
         if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
       }
       ok = __shfl_sync(kFullMask, ok, 0);
@@ -298,11 +310,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
-          bytes += 4 * 2048;
-      const uint32_t bar = bar_kv_full(stage);
+          bytes += 2 * 2048;
+      const uint32_t bar = is_k ? bar_k_full(stage) : bar_v_full(stage);
       if (lane == 0) {
         for (int i = 0; i < npieces; ++i)
-          if (static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks))
+          if (is_k && static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks))
             set_err(p.err, PKV_DEVERR_BAD_BLOCK);
         if (bytes > 0)
           mbar_arrive_expect_tx(bar, bytes);
@@ -310,10 +322,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           mbar_arrive(bar);
       }
       __syncwarp();
-      // lanes 0..15 issue the 16 boxes of the tile at once: lane = piece * 4 + kind,
-      // kind = K low dims, K high dims, V low dims, V high dims
-      if (lane < 16) {
-        const int i = lane >> 2, kind = lane & 3;
+      // lanes 0..7 issue the tile's 8 boxes of K (or V) at once: lane = piece * 2 +
+      // half; kind 0 / 1 = K low / high dims, 2 / 3 = V low / high dims
+      if (lane < 8) {
+        const int i = lane >> 1, kind = (is_k ? 0 : 2) + (lane & 1);
         int pbi = pb[0];
         if (i == 1) pbi = pb[1];
         if (i == 2) pbi = pb[2];
@@ -352,22 +364,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         tc::umma_commit(bar_o(q, t & 1));
       };
-      // P.V of tile t for every query tile that uses it, then release its stage
-      auto finish_tile = [&](int t) {
-#pragma unroll
-        for (int q = 0; q < QT; ++q) {
-          if (t >= ntq[q]) continue;
-          ok = ok && mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
-          if (!ok) return;
-          tc::tc_fence_after();
-          issue_pv(q, t);
-        }
-        tc::umma_commit(bar_kv_empty(t % NS));
-      };
-      for (int t = 0; t < ntiles && ok; ++t) {
-        ok = mbar_wait_bounded(bar_kv_full(t % NS), (t / NS) & 1);
-        if (!ok) break;
-        tc::tc_fence_after();
+      // S = Q K^T of tile t for every query tile that uses it
+      auto issue_s = [&](int t) {
         const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
 #pragma unroll
         for (int q = 0; q < QT; ++q) {
@@ -382,15 +380,55 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           }
           tc::umma_commit(bar_s_full(q, t & 1));
         }
-        if (t > 0) finish_tile(t - 1);
+      };
+      // is P of tile t ready in every query tile that uses it?
+      auto p_ready = [&](int t) {
+        bool r = true;
+#pragma unroll
+        for (int q = 0; q < QT; ++q)
+          if (t < ntq[q]) r = r && mbar_test_wait(bar_p(q, t & 1), (t >> 1) & 1);
+        return r;
+      };
+      // Issue S and P.V in whichever order their inputs arrive: S of tile ns
+      // needs its K/V and its S buffers back (P.V of tile ns - 2 issued, so the
+      // softmax has read them); P.V of tile np needs P of every query tile.
+      // A fixed order would hold a ready P.V behind the next tile's load.
+      int ns = 0, np = 0;
+      uint64_t t_idle = 0;
+      uint32_t idle = 0;
+      while (ok && np < ntiles) {
+        bool progress = false;
+        if (ns < ntiles && ns - np < 2 &&
+            mbar_test_wait(bar_k_full(ns % NS), (ns / NS) & 1)) {
+          tc::tc_fence_after();
+          issue_s(ns);
+          tc::umma_commit(bar_k_empty(ns % NS));
+          ++ns;
+          progress = true;
+        }
+        if (np < ns && p_ready(np) && mbar_test_wait(bar_v_full(np % NS), (np / NS) & 1)) {
+          tc::tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < QT; ++q)
+            if (np < ntq[q]) issue_pv(q, np);
+          tc::umma_commit(bar_v_empty(np % NS));
+          ++np;
+          progress = true;
+        }
+        if (progress) {
+          idle = 0;
+        } else if (idle++ == 0) {
+          t_idle = global_timer_ns();
+        } else if ((idle & 255u) == 0u && global_timer_ns() - t_idle > kWaitTimeoutNs) {
+          ok = false;
+        }
       }
-      if (ok && ntiles > 0) finish_tile(ntiles - 1);
       if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
     }
     __syncwarp();
   } else {
     // ---- softmax warps: query tile qg, thread <-> row <-> TMEM lane -------------------
-    const int qg = (warp - 2) >> 2;
+    const int qg = (warp - 3) >> 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + qg * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -511,6 +549,12 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       const int loaded_end = min(kv0 + NKEY, ((nkv + 15) / 16) * 16);
       const int vz = min(ctx, loaded_end) - kv0;  // V rows [vz, 64) must be zero
       if (vz < NKEY) {
+        // V of this tile may still be in flight: let it land before zeroing rows
+        ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
+        if (!__all_sync(kFullMask, ok)) {
+          ok = false;
+          break;
+        }
         unsigned char* vt = smem + Tr::OFF_KV + (t % NS) * Tr::STAGE + 2 * Tr::KV_HALF;
         const int nrows = NKEY - vz;
         for (int idx = r; idx < nrows * 16; idx += 128) {

@@ -271,8 +271,10 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     # "<name>_fp8": the named workload with E4M3 caches (one scale per cache)
+    # "<name>_fp8": E4M3 caches; "prefix_share_cascade": cascade decode
     fp8 = args.workload.endswith("_fp8")
-    name = args.workload[:-4] if fp8 else args.workload
+    cascade = args.workload.endswith("_cascade")
+    name = args.workload[:-4] if fp8 else args.workload[:-8] if cascade else args.workload
     base = W.SEED_BASE + W.NAMES.index(name)
     w = W.make(name, seed=replica_seed(base, rank))
     tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
@@ -304,11 +306,22 @@ def run_ours(args):
     part_req = w.partition_size if args.partition is None else args.partition
     part = pk.partition_size(w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len, part_req)
     split = part < w.max_context_len
-    ws = pk.alloc_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
-                            w.max_context_len, part_req, device=dev)
+    if cascade:
+        gs_np, sb_np = W.cascade_groups(w)
+        gstart = torch.from_numpy(gs_np).to(dev)
+        gshared = torch.from_numpy(sb_np).to(dev)
+        max_group, max_shared = int(np.diff(gs_np).max()), int(sb_np.max())
+        ws = torch.empty(max(16, pk.cascade_workspace_bytes(
+            w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+            w.max_context_len, part_req)), dtype=torch.uint8, device=dev)
+    else:
+        ws = pk.alloc_workspace(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim,
+                                w.block_size, w.max_context_len, part_req, device=dev)
     stream = torch.cuda.Stream(device=dev)
     has_pairs = len(w.cow_pairs) > 0
-    launches_per_step = 1 + 1 + (1 if split else 0) + (1 if has_pairs else 0)
+    # cache write (+ block copy) + decode (+ reduce); cascade: prefix pass + suffix + reduce
+    launches_per_step = (1 + (1 if has_pairs else 0) +
+                         (3 if cascade else 1 + (1 if split else 0)))
 
     inputs = dict(q=q, key=key, val=val, slots=slots, pairs=pairs, tables=tables, lens=lens,
                   out=out)
@@ -329,6 +342,12 @@ def run_ours(args):
                                      ks8, vs8, w.num_kv_heads, w.block_size,
                                      w.max_context_len, partition_size=part_req, workspace=ws,
                                      dev_err=err, stream=stream)
+        elif cascade:
+            pk.paged_attn_decode_cascade(t["out"], t["q"], kc, vc, t["tables"], t["lens"], gstart,
+                                         gshared, w.scale, w.num_kv_heads, w.block_size,
+                                         w.max_context_len, max_group, max_shared,
+                                         partition_size=part_req, workspace=ws, dev_err=err,
+                                         stream=stream)
         else:
             pk.paged_attn_decode(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
                                  w.num_kv_heads, w.block_size, w.max_context_len,
@@ -389,12 +408,12 @@ def run_ours(args):
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
-        if not fp8:
+        if not fp8 and not cascade:
             pk.decode_step_host(h_out, h_q, h_key, h_val, h_slots, h_pairs, h_tables, h_lens, kc,
                                 vc, w.scale, w.max_context_len, staging, workspace=ws,
                                 partition_size=part_req, dev_err=err, stream=stream)
             return
-        # E4M3 caches: the same copies through the Python binding's tensors
+        # E4M3 caches or cascade decode: the same copies through the Python binding's tensors
         with torch.cuda.stream(stream):
             for dst, src in ((q, h_q), (key, h_key), (val, h_val), (slots, h_slots),
                              (tables, h_tables), (lens, h_lens)):
@@ -468,7 +487,7 @@ def run_ours(args):
         raise RuntimeError("device error word %d" % int(err.item()))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8 and not cascade:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
     if rank == 0:
@@ -495,11 +514,12 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": committed_traffic(args.workload),
-                         "kernel": ("paged_decode_mma_kernel"
-                                    if (fp8 and w.head_dim == 128)
-                                    or (not fp8 and w.num_heads > w.num_kv_heads)
-                                    else "paged_decode_kernel")
-                         + (" + reduce" if split else ""),
+                         "kernel": ("paged_prefill_tc_kernel (prefix pass) + " if cascade else "")
+                         + ("paged_decode_mma_kernel"
+                            if (fp8 and w.head_dim == 128)
+                            or (not fp8 and w.num_heads > w.num_kv_heads)
+                            else "paged_decode_kernel")
+                         + (" + reduce" if split or cascade else ""),
                          "algorithmic_bytes_per_launch": dbytes,
                          "avg_launch_ms": round(dec_avg_ms, 5),
                          "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
@@ -508,10 +528,10 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "api": "Python binding (reshape_and_cache%s, paged_attn_decode%s) with "
                            "pinned-host copies on side streams, consecutive steps overlapped"
-                           % (("_fp8", "_fp8") if fp8 else ("", "")),
+                           % (("_fp8", "_fp8") if fp8 else ("", "_cascade" if cascade else "")),
                     "serial": {"value": round(e2e_serial, 2), "ms_per_step": round(e2e_serial_ms, 5),
-                               "api": "Python binding with torch copies on one stream" if fp8
-                               else "pkv_decode_step_host (one call per step)"}},
+                               "api": "Python binding with torch copies on one stream"
+                               if fp8 or cascade else "pkv_decode_step_host (one call per step)"}},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }

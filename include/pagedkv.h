@@ -236,6 +236,46 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, const void*
                                            int partition_size, unsigned* dev_err, void* stream);
 
 /*
+ * pkv_paged_attn_decode_cascade — pkv_paged_attn_decode for sequences that
+ * share a cached prefix, such as the parallel samples of one prompt
+ * ([cortexgrid] FAQ on parallel sampling; [csdn] "分页式KV缓存": sequences
+ * with a common prompt point at the same first pages).  The result is that
+ * of pkv_paged_attn_decode on the same arguments; only the work differs: the
+ * shared blocks are read once per group instead of once per sequence.
+ *
+ *   group_start    device int32 [num_groups + 1], non-decreasing, 0 first and
+ *                  num_seqs last: group g is sequences group_start[g] ..
+ *                  group_start[g+1] - 1 (so members are consecutive)
+ *   shared_blocks  device int32 [num_groups]: the first shared_blocks[g]
+ *                  entries of every member's table row are the same physical
+ *                  blocks (whole blocks only: a partly filled last prompt
+ *                  block is per member after copy-on-write), and every member
+ *                  caches at least shared_blocks[g] * block_size tokens
+ *   max_group_size, max_shared_blocks  upper bounds (size the launch);
+ *                  max_shared_blocks * block_size <= max_context_len
+ *   workspace      >= pkv_paged_attn_cascade_workspace_bytes(...) bytes
+ * The group's table entries are read from its first member.  A member whose
+ * context is shorter than its group's shared tokens sets
+ * PKV_DEVERR_BAD_CONTEXT.  head_dim 128 only (PKV_ERR_UNSUPPORTED otherwise);
+ * 16-bit caches.  Other arguments and errors as in pkv_paged_attn_decode.
+ */
+size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                              int head_dim, int block_size,
+                                              int max_context_len, int partition_size);
+pkv_status pkv_paged_attn_decode_cascade(void* out, const void* q, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         const int32_t* context_lens,
+                                         const int32_t* group_start,
+                                         const int32_t* shared_blocks, float scale,
+                                         int num_seqs, int num_groups, int max_group_size,
+                                         int max_shared_blocks, int num_heads,
+                                         int num_kv_heads, int head_dim, int block_size,
+                                         int max_blocks_per_seq, int max_context_len,
+                                         int num_blocks, pkv_dtype dtype, int partition_size,
+                                         void* workspace, size_t workspace_bytes,
+                                         unsigned* dev_err, void* stream);
+
+/*
  * 8-bit (E4M3) cache.  The pages name quantised inference as a way to fit
  * larger models and batches into the memory ([csdn] "量化模型优先考虑边缘场景";
  * [betteryeah] §4.2 "启用量化推理") without fixing a format; this library stores

@@ -28,4 +28,26 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, int hkv, int bs,
                             int d, pkv_dtype dt);
 
+// Groups of cascade decode (device arrays): group g is sequences
+// group_start[g] .. group_start[g+1]-1, sharing their first shared_blocks[g]
+// blocks.
+struct CascadeGroups {
+  const int32_t* group_start;
+  const int32_t* shared_blocks;
+  int num_groups;
+  int max_group_size;
+  int max_shared_blocks;
+};
+
+// The shared-prefix pass of cascade decode (tcgen05 kernel, head_dim 128):
+// writes each member's prefix partial (m, l, unnormalised o) into slot 0 of
+// its rows of the split-K workspace (max_parts slots per (sequence, head)).
+pkv_status launch_cascade_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 const CascadeGroups& groups, float scale, int num_seqs,
+                                 int num_heads, int num_kv_heads, int block_size,
+                                 int max_blocks_per_seq, int max_context_len, int num_blocks,
+                                 pkv_dtype dtype, float* ws_out, float* ws_max, float* ws_sum,
+                                 int max_parts, unsigned* dev_err, cudaStream_t stream);
+
 }  // namespace pkv

@@ -328,7 +328,8 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
                          int block_size, int max_blocks_per_seq, int max_context_len,
                          int num_blocks, pkv_dtype dtype, int partition_size, void* workspace,
                          size_t workspace_bytes, unsigned* dev_err, void* stream, bool fp8,
-                         const float* k_scales, const float* v_scales) {
+                         const float* k_scales, const float* v_scales,
+                         const CascadeGroups* cascade = nullptr) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0 || num_blocks <= 0 || partition_size < 0 || !dtype_valid(dtype) ||
       num_heads % num_kv_heads != 0 || !isfinite(scale))
@@ -352,13 +353,16 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
       choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
   const int part_blocks = part / block_size;
   if (part_blocks > kMaxPartitionBlocks) return PKV_ERR_UNSUPPORTED;
-  const int max_parts = parts_for(max_context_len, block_size, part);
+  // cascade decode: workspace slot 0 holds the prefix pass's partial and the
+  // kernel's partitions start at slot 1
+  const int grid_parts = parts_for(max_context_len, block_size, part);
+  const int max_parts = grid_parts + (cascade ? 1 : 0);
   const WorkspaceLayout wl = workspace_layout(num_seqs, num_heads, head_dim, max_parts);
   if (wl.total > 0) {
     if (workspace == nullptr || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return PKV_ERR_INVALID_ARG;
   }
-  const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * max_parts;
+  const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * grid_parts;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
   // G >= 2 runs on the tensor cores (E4M3: head_dim 128 only), G = 1 on the CUDA cores
@@ -404,6 +408,10 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   p.block_size = block_size;
   p.part_blocks = part_blocks;
   p.max_parts = max_parts;
+  p.grid_parts = grid_parts;
+  p.group_start = cascade ? cascade->group_start : nullptr;
+  p.shared_blocks = cascade ? cascade->shared_blocks : nullptr;
+  p.num_groups = cascade ? cascade->num_groups : 0;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.ws_out = wl.total ? reinterpret_cast<float*>(ws + wl.out_off) : nullptr;
   p.ws_max = wl.total ? reinterpret_cast<float*>(ws + wl.max_off) : nullptr;
@@ -466,6 +474,91 @@ extern "C" pkv_status pkv_paged_attn_decode_fp8(
                             max_blocks_per_seq, max_context_len, num_blocks, dtype,
                             partition_size, workspace, workspace_bytes, dev_err, stream, true,
                             k_scales, v_scales);
+}
+
+// ---------------------------------------------------------------------------
+// Cascade decode for sequences that share a cached prefix.
+//
+// Parallel samples of one prompt share the prompt's blocks through their
+// block tables ([cortexgrid] FAQ on parallel sampling; [csdn] "分页式KV缓存":
+// common prompts point at the same pages).  Plain decode reads those blocks
+// once per sample; the samples of a prompt run at about the same time, so the
+// repeats come from L2, and L2 bandwidth then bounds the step.  Here the
+// shared blocks are read once per group: the tcgen05 kernel in prefix mode
+// attends every member's query rows to them together (slot 0 of the split-K
+// workspace), the decode kernel covers each member's own blocks (slots 1..),
+// and the reduce merges the partials.  The result is that of plain decode.
+// ---------------------------------------------------------------------------
+extern "C" size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_heads,
+                                                         int num_kv_heads, int head_dim,
+                                                         int block_size, int max_context_len,
+                                                         int partition_size) {
+  using namespace pkv;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_context_len < 0 || partition_size < 0)
+    return 0;
+  const int part =
+      choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
+  if (part % block_size != 0) return 0;
+  return workspace_layout(num_seqs, num_heads, head_dim,
+                          1 + parts_for(max_context_len, block_size, part))
+      .total;
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_cascade(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
+    const int32_t* shared_blocks, float scale, int num_seqs, int num_groups, int max_group_size,
+    int max_shared_blocks, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err,
+    void* stream) {
+  using namespace pkv;
+  if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0 ||
+      num_kv_heads <= 0 || block_size <= 0 ||
+      static_cast<long long>(max_shared_blocks) * block_size > max_context_len ||
+      (num_seqs > 0 && (num_groups == 0 || max_group_size == 0)))
+    return PKV_ERR_INVALID_ARG;
+  if (head_dim != 128) return PKV_ERR_UNSUPPORTED;  // the prefix pass is the tcgen05 kernel
+  if (num_seqs == 0) return PKV_OK;
+  if (!group_start || !shared_blocks || !workspace) return PKV_ERR_INVALID_ARG;
+  const CascadeGroups groups{group_start, shared_blocks, num_groups, max_group_size,
+                             max_shared_blocks};
+  // validate everything (and the workspace) before the first launch
+  const size_t need = pkv_paged_attn_cascade_workspace_bytes(
+      num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size);
+  if (workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !dtype_valid(dtype) ||
+      num_heads <= 0 || num_heads % num_kv_heads != 0 || !isfinite(scale) ||
+      partition_size < 0 || partition_size % block_size != 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0 ||
+      static_cast<long long>(max_context_len) >
+          static_cast<long long>(max_blocks_per_seq) * block_size ||
+      !aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_ERR_INVALID_ARG;
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
+  if (!block_size_supported(block_size)) return PKV_ERR_UNSUPPORTED;
+  const int part =
+      choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
+  if (part / block_size > kMaxPartitionBlocks) return PKV_ERR_UNSUPPORTED;
+  const int max_parts = 1 + parts_for(max_context_len, block_size, part);
+  if (static_cast<long long>(num_seqs) * num_kv_heads * max_parts > 0x7fffffffLL)
+    return PKV_ERR_UNSUPPORTED;
+  const WorkspaceLayout wl = workspace_layout(num_seqs, num_heads, head_dim, max_parts);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (max_shared_blocks > 0) {
+    const pkv_status st = launch_cascade_prefix(
+        q, k_cache, v_cache, block_tables, context_lens, groups, scale, num_seqs, num_heads,
+        num_kv_heads, block_size, max_blocks_per_seq, max_context_len, num_blocks, dtype,
+        reinterpret_cast<float*>(ws + wl.out_off), reinterpret_cast<float*>(ws + wl.max_off),
+        reinterpret_cast<float*>(ws + wl.sum_off), max_parts, dev_err, as_stream(stream));
+    if (st != PKV_OK) return st;
+  }
+  return decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       max_context_len, num_blocks, dtype, partition_size, workspace,
+                       workspace_bytes, dev_err, stream, false, nullptr, nullptr, &groups);
 }
 
 // ---------------------------------------------------------------------------

@@ -60,16 +60,39 @@ struct DecodeParams {
   int num_blocks;
   int block_size;
   int part_blocks;  // blocks per partition
-  int max_parts;    // partitions per sequence at max_context_len
+  int max_parts;    // workspace slots per (sequence, head)
+  int grid_parts;   // partitions per (sequence, kv head) in the grid: max_parts,
+                    // or max_parts - 1 under cascade decode (slot 0 is the prefix)
   float* ws_out;    // [S, H, max_parts, D]
   float* ws_max;    // [S, H, max_parts]
   float* ws_sum;    // [S, H, max_parts]
   unsigned* err;
+  // Cascade decode (else null / 0): sequences come in groups, group g being
+  // sequences group_start[g] .. group_start[g+1]-1, whose first
+  // shared_blocks[g] blocks a separate prefix pass covers (its partial sits in
+  // workspace slot 0).  The decode kernels then read only each sequence's
+  // blocks after them, write partials from slot 1 on, and the reduce merges
+  // every slot.
+  const int32_t* group_start;
+  const int32_t* shared_blocks;
+  int num_groups;
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+// First block a decode kernel reads for `seq`: 0, or under cascade decode the
+// shared blocks of its group (binary search over group_start), at most nblk.
+__device__ __forceinline__ int cascade_start_block(const DecodeParams& p, int seq, int nblk) {
+  if (p.group_start == nullptr) return 0;
+  int lo = 0, hi = p.num_groups;  // invariant: group_start[lo] <= seq < group_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.group_start[mid] <= seq) lo = mid; else hi = mid;
+  }
+  return min(max(p.shared_blocks[lo], 0), nblk);
+}
 
 template <int D_, int BS_, int G_, class DT_, int W_, int NS_, class KV_ = DT_>
 struct DecodeTraits {
@@ -300,7 +323,8 @@ __device__ __forceinline__ void merge_warps_and_store(const DecodeParams& p, con
       T* o = static_cast<T*>(p.out) + (static_cast<size_t>(seq) * p.num_heads + head) * D + cc * 8;
       *reinterpret_cast<uint4*>(o) = pack8(num, DT());
     } else {
-      const size_t slot = (static_cast<size_t>(seq) * p.num_heads + head) * p.max_parts + part;
+      const size_t slot = (static_cast<size_t>(seq) * p.num_heads + head) * p.max_parts + part +
+                          (p.group_start != nullptr ? 1 : 0);
       float4* o = reinterpret_cast<float4*>(p.ws_out + slot * D + cc * 8);
       o[0] = make_float4(num[0], num[1], num[2], num[3]);
       o[1] = make_float4(num[4], num[5], num[6], num[7]);
@@ -323,8 +347,8 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   float* pbuf_all = reinterpret_cast<float*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
   int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES + Tr::PBUF_BYTES);
 
-  const int part = blockIdx.x % p.max_parts;
-  const int unit = blockIdx.x / p.max_parts;
+  const int part = blockIdx.x % p.grid_parts;
+  const int unit = blockIdx.x / p.grid_parts;
   const int kvh = unit % p.num_kv_heads;
   const int seq = unit / p.num_kv_heads;
   const int warp = threadIdx.x >> 5;
@@ -342,10 +366,12 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
     ctx = min(max(ctx, 0), ctx_cap);
   }
   const int nblk = (ctx + BS - 1) / BS;
-  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
-  if (part >= max(nparts, 1)) return;
-  const bool direct = nparts <= 1;
-  const int blk_begin = part * p.part_blocks;
+  const int start_blk = cascade_start_block(p, seq, nblk);
+  const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
+  const bool cascade = p.group_start != nullptr;
+  if (part >= (cascade ? nparts : max(nparts, 1))) return;
+  const bool direct = !cascade && nparts <= 1;
+  const int blk_begin = start_blk + part * p.part_blocks;
   const int nb = min(nblk, blk_begin + p.part_blocks) - blk_begin;
 
   // ---- stage the block-table slice; initialise this warp's barriers --------
@@ -766,8 +792,8 @@ __global__ void __launch_bounds__(Tr::THREADS)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
   int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
 
-  const int part = blockIdx.x % p.max_parts;
-  const int unit = blockIdx.x / p.max_parts;
+  const int part = blockIdx.x % p.grid_parts;
+  const int unit = blockIdx.x / p.grid_parts;
   const int kvh = unit % p.num_kv_heads;
   const int seq = unit / p.num_kv_heads;
   const int warp = threadIdx.x >> 5;
@@ -783,10 +809,12 @@ __global__ void __launch_bounds__(Tr::THREADS)
     ctx = min(max(ctx, 0), ctx_cap);
   }
   const int nblk = (ctx + BS - 1) / BS;
-  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
-  if (part >= max(nparts, 1)) return;
-  const bool direct = nparts <= 1;
-  const int blk_begin = part * p.part_blocks;
+  const int start_blk = cascade_start_block(p, seq, nblk);
+  const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
+  const bool cascade = p.group_start != nullptr;
+  if (part >= (cascade ? nparts : max(nparts, 1))) return;
+  const bool direct = !cascade && nparts <= 1;
+  const int blk_begin = start_blk + part * p.part_blocks;
   const int nb = min(nblk, blk_begin + p.part_blocks) - blk_begin;
   const int sb_begin = blk_begin * SPB;
   const int nsb = max(0, min((ctx + Tr::SUB - 1) / Tr::SUB, (blk_begin + nb) * SPB) - sb_begin);
@@ -966,11 +994,16 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   const int head = gw % p.num_heads;
   const int ctx = clamped_context(p, seq);
   const int nblk = (ctx + p.block_size - 1) / p.block_size;
-  const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
-  if (nparts <= 1) return;
+  const bool cascade = p.group_start != nullptr;
+  const int start_blk = cascade_start_block(p, seq, nblk);
+  const int nsuffix = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
+  // slots [first, last): the prefix partial (slot 0, cascade only) and the suffix partitions
+  const int first = cascade && start_blk == 0 ? 1 : 0;
+  const int last = cascade ? 1 + nsuffix : nsuffix;
+  if (!cascade && nsuffix <= 1) return;
   const size_t base = static_cast<size_t>(gw) * p.max_parts;
   float big_m = -INFINITY;
-  for (int q = lane; q < nparts; q += 32) big_m = fmaxf(big_m, p.ws_max[base + q]);
+  for (int q = first + lane; q < last; q += 32) big_m = fmaxf(big_m, p.ws_max[base + q]);
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) big_m = fmaxf(big_m, __shfl_xor_sync(kFullMask, big_m, m));
   float num[PER_LANE];
@@ -978,7 +1011,7 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   for (int e = 0; e < PER_LANE; ++e) num[e] = 0.f;
   float den = 0.f;
 #pragma unroll 4
-  for (int q = 0; q < nparts; ++q) {
+  for (int q = first; q < last; ++q) {
     const float f = exp2_approx(p.ws_max[base + q] - big_m);
     den = fmaf(f, p.ws_sum[base + q], den);
     const float* o = p.ws_out + (base + q) * D + lane * PER_LANE;

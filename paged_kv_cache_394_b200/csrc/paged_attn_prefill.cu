@@ -97,6 +97,32 @@ TcEntry tc_for(int bs, int g) {
   return TcEntry{nullptr, 0, 0, 0};
 }
 
+// Prefix mode (the shared-prefix pass of cascade decode): one 128-row query
+// tile per CTA; a group's members and their heads are its rows.
+template <int BS, int G, class DT>
+TcEntry make_prefix_tc() {
+  using Tr = TcPrefillTraits<BS, G, DT, 1, true>;
+  return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(), Tr::ROWS};
+}
+
+template <int BS, class DT>
+TcEntry prefix_group(int g) {
+  switch (g) {
+    case 1: return make_prefix_tc<BS, 1, DT>();
+    case 2: return make_prefix_tc<BS, 2, DT>();
+    case 4: return make_prefix_tc<BS, 4, DT>();
+    case 8: return make_prefix_tc<BS, 8, DT>();
+    default: return TcEntry{nullptr, 0, 0, 0};
+  }
+}
+
+template <class DT>
+TcEntry prefix_for(int bs, int g) {
+  if (bs == 16) return prefix_group<16, DT>(g);
+  if (bs == 32) return prefix_group<32, DT>(g);
+  return TcEntry{nullptr, 0, 0, 0};
+}
+
 // 3-D tensor map over q [T, H, 128]: boxes of (128/G tokens) x (G heads) x 64 dims,
 // i.e. a tile's 128 rows ordered (token, head), 128-byte swizzle.
 pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num_heads, int group,
@@ -126,6 +152,75 @@ pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num
 }
 
 }  // namespace
+}  // namespace pkv
+
+namespace pkv {
+
+pkv_status launch_cascade_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* block_tables, const int32_t* context_lens,
+                                 const CascadeGroups& groups, float scale, int num_seqs,
+                                 int num_heads, int num_kv_heads, int block_size,
+                                 int max_blocks_per_seq, int max_context_len, int num_blocks,
+                                 pkv_dtype dtype, float* ws_out, float* ws_max, float* ws_sum,
+                                 int max_parts, unsigned* dev_err, cudaStream_t stream) {
+  const int group = num_heads / num_kv_heads;
+  const TcEntry te = dtype == PKV_FP16 ? prefix_for<Fp16>(block_size, group)
+                                       : prefix_for<Bf16>(block_size, group);
+  if (te.fn == nullptr) return PKV_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(groups.max_group_size) * group;
+  const int q_tiles = static_cast<int>((rows + te.rows - 1) / te.rows);
+  const long long grid = static_cast<long long>(groups.num_groups) * num_kv_heads * q_tiles;
+  if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+  if (grid == 0) return PKV_OK;
+  CUtensorMap kmap, vmap, qmap;
+  pkv_status st =
+      cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, 128, dtype);
+  if (st != PKV_OK) return st;
+  st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, 128, dtype);
+  if (st != PKV_OK) return st;
+  st = q_tensor_map(&qmap, q, num_seqs, num_heads, group, dtype);  // the members' queries
+  if (st != PKV_OK) return st;
+  st = cuda_status(cudaFuncSetAttribute(reinterpret_cast<const void*>(te.fn),
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(te.smem)));
+  if (st != PKV_OK) return st;
+
+  PrefillParams p = {};
+  p.q = q;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.qscale = scale * kLog2e;
+  p.num_seqs = groups.num_groups;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.max_query_len = groups.max_group_size;
+  p.num_blocks = num_blocks;
+  p.q_tiles = q_tiles;
+  p.err = dev_err;
+  p.group_start = groups.group_start;
+  p.shared_blocks = groups.shared_blocks;
+  p.ws_out = ws_out;
+  p.ws_max = ws_max;
+  p.ws_sum = ws_sum;
+  p.max_parts = max_parts;
+
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(te.threads);
+  cfg.dynamicSmemBytes = te.smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, te.fn, p, qmap, kmap, vmap));
+}
+
 }  // namespace pkv
 
 extern "C" pkv_status pkv_paged_attn_prefill(
@@ -184,7 +279,7 @@ extern "C" pkv_status pkv_paged_attn_prefill(
                                         static_cast<int>(smem)));
   if (st != PKV_OK) return st;
 
-  PrefillParams p;
+  PrefillParams p = {};
   p.out = out;
   p.q = q;
   p.k_cache = k_cache;

@@ -47,6 +47,17 @@ struct PrefillParams {
   int num_blocks;
   int q_tiles;  // query tiles per (sequence, kv head) at max_query_len
   unsigned* err;
+  // Shared-prefix pass of cascade decode (tcgen05 kernel in prefix mode): the
+  // units are groups of sequences instead of sequences, the queries are the
+  // members' decode queries, the keys the group's shared_blocks[g] leading
+  // blocks, and the result is a split-K partial (m, l, unnormalised o) in
+  // slot 0 of each member's workspace row.
+  const int32_t* group_start;    // [num_groups + 1] first member of each group
+  const int32_t* shared_blocks;  // [num_groups]
+  float* ws_out;                 // [S, H, max_parts, D]
+  float* ws_max;                 // [S, H, max_parts]
+  float* ws_sum;                 // [S, H, max_parts]
+  int max_parts;
 };
 
 template <int D_, int BS_, int G_, class DT_, int NS_>

@@ -135,9 +135,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 
 }  // namespace tc
 
-template <int BS_, int G_, class DT_, int QT_>
+template <int BS_, int G_, class DT_, int QT_, bool PREFIX_ = false>
 struct TcPrefillTraits {
   static constexpr int D = 128, BS = BS_, G = G_, QT = QT_;
+  // prefix mode: the shared-prefix pass of cascade decode (no causal mask,
+  // split-K partials out; see PrefillParams)
+  static constexpr bool kPrefix = PREFIX_;
   using DT = DT_;
   using T = typename DT::T;
   static constexpr bool kBf16 = std::is_same<DT, Bf16>::value;
@@ -211,16 +214,19 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   grid_dependency_wait();
   trigger_dependents();
 
-  const int ctx = p.context_lens[seq];
-  const int q0 = p.query_start[seq];
-  const int q_len = p.query_start[seq + 1] - q0;
+  // seq is a sequence, or in prefix mode a group whose members are the
+  // "tokens" q0 .. q0 + q_len - 1 and whose keys are its shared blocks
+  const int ctx = Tr::kPrefix ? p.shared_blocks[seq] * BS : p.context_lens[seq];
+  const int q0 = Tr::kPrefix ? p.group_start[seq] : p.query_start[seq];
+  const int q_len = (Tr::kPrefix ? p.group_start[seq + 1] : p.query_start[seq + 1]) - q0;
   const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
-  if (ctx < 0 || ctx > cap || q_len < 0 || q_len > ctx || q_len > p.max_query_len) {
+  if (ctx < 0 || ctx > cap || q_len < 0 || (!Tr::kPrefix && q_len > ctx) ||
+      q_len > p.max_query_len) {
     if (threadIdx.x == 0 && tile == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
     return;
   }
   const int rows_total = q_len * G;
-  if (tile * ROWS >= rows_total) return;
+  if (tile * ROWS >= rows_total || (Tr::kPrefix && ctx == 0)) return;
   const int tok0 = tile * (ROWS / G);  // first query token of this CTA
   // KV tiles each query tile needs (later rows see more keys; 0 = no rows)
   int ntq[QT];
@@ -228,10 +234,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   for (int q = 0; q < QT; ++q) {
     const int r0 = tile * ROWS + q * M;
     const int last = (min(rows_total, r0 + M) - 1) / G;
-    ntq[q] = r0 < rows_total ? (ctx - q_len + last + 1 + NKEY - 1) / NKEY : 0;
+    const int keys = Tr::kPrefix ? ctx : ctx - q_len + last + 1;
+    ntq[q] = r0 < rows_total ? (keys + NKEY - 1) / NKEY : 0;
   }
   const int last_tok = (min(rows_total, (tile + 1) * ROWS) - 1) / G;
-  const int nkv = ctx - q_len + last_tok + 1;  // keys the CTA reads
+  const int nkv = Tr::kPrefix ? ctx : ctx - q_len + last_tok + 1;  // keys the CTA reads
   const int ntiles = (nkv + NKEY - 1) / NKEY;
 
   if (threadIdx.x == 0) {
@@ -267,7 +274,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     // K of a stage is released once S has read it, V once P.V has, so the K
     // loads can run further ahead than the V loads.
     const bool is_k = warp == 0;
-    const int32_t* trow = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
+    // prefix mode: the group's first member holds the shared blocks' ids
+    const int32_t* trow = p.block_tables +
+                          static_cast<size_t>(Tr::kPrefix ? q0 : seq) * p.max_blocks_per_seq;
     const int nblk = (nkv + BS - 1) / BS;
     if (is_k && lane == 0) {
       mbar_arrive_expect_tx(bar_q, QT * Tr::Q_TILE);
@@ -438,7 +447,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const bool active = crow < rows_total - tile * ROWS;
     const int j = tok0 + crow / G;
     const int g = crow % G;
-    const int pos = active ? ctx - q_len + j : -1;
+    const int pos = !active ? -1 : Tr::kPrefix ? ctx - 1 : ctx - q_len + j;
     const int my_tiles = qg == 0 ? ntq[0] : ntq[QT - 1];
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -576,7 +585,27 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       ok = mbar_wait_bounded(bar_o(qg, (my_tiles - 1) & 1), ((my_tiles - 1) >> 1) & 1);
       ok = __all_sync(kFullMask, ok);
     }
-    if (ok && my_tiles > 0) {
+    if (ok && my_tiles > 0 && Tr::kPrefix) {
+      // split-K partial of the prefix: (m, l, unnormalised o) in slot 0
+      tc::tc_fence_after();
+      const size_t slot = (static_cast<size_t>(q0 + j) * p.num_heads + kvh * G + g) * p.max_parts;
+      if (active) {
+        if (p.context_lens[q0 + j] < ctx) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
+        p.ws_max[slot] = m;
+        p.ws_sum[slot] = l;
+      }
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 16) {
+        float v[16];
+        tc::tmem_ld16(lane_addr + 128 + c, v);
+        tc::tmem_wait_ld();
+        if (active) {
+          float4* o = reinterpret_cast<float4*>(p.ws_out + slot * Tr::D + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    } else if (ok && my_tiles > 0) {
       tc::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       T* orow = static_cast<T*>(p.out) +

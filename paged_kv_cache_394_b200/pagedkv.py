@@ -49,6 +49,11 @@ _paged_attn_decode_static_ws = _proto("pkv_paged_attn_decode_static_ws", _i, _vp
                                      _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                      _vp)
 STATIC_WORKSPACE_BYTES = 16 << 20
+_cascade_workspace_bytes = _proto("pkv_paged_attn_cascade_workspace_bytes", _sz, _i, _i, _i, _i,
+                                  _i, _i, _i)
+_paged_attn_decode_cascade = _proto("pkv_paged_attn_decode_cascade", _i, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                    _i, _i, _i, _vp, _sz, _vp, _vp)
 _reshape_and_cache_fp8 = _proto("pkv_reshape_and_cache_fp8", _i, _vp, _vp, _vp, _vp, _vp, _i, _i,
                                 _i, _i, _i, _i, _vp, _vp, _vp, _vp)
 _paged_attn_decode_fp8 = _proto("pkv_paged_attn_decode_fp8", _i, _vp, _vp, _vp, _vp, _vp, _vp, _f,
@@ -233,6 +238,48 @@ def _scales_for(k_scales, v_scales, hkv, device, stream):
         ks.record_stream(stream)
         vs.record_stream(stream)
     return ks, vs
+
+
+def cascade_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_context_len, partition_size=0):
+    return _cascade_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                    max_context_len, partition_size)
+
+
+def paged_attn_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                              shared_blocks, scale, num_kv_heads, block_size, max_context_len,
+                              max_group_size, max_shared_blocks, partition_size=0,
+                              workspace=None, dev_err=None, stream=None):
+    """Decode for groups of sequences sharing their first shared_blocks[g]
+    blocks (members consecutive, group g = group_start[g] .. group_start[g+1]-1).
+    Same result as paged_attn_decode.  See include/pagedkv.h."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    for n, t in (("block_tables", block_tables), ("context_lens", context_lens),
+                 ("group_start", group_start), ("shared_blocks", shared_blocks)):
+        _dev(t, n, torch.int32)
+    s, h, d = q.shape
+    num_blocks, hkv, bs, dk = k_cache.shape
+    if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if q.dtype != k_cache.dtype or out.dtype != q.dtype:
+        raise TypeError("q, out and caches must share a dtype")
+    g = shared_blocks.shape[0]
+    if group_start.shape != (g + 1,):
+        raise ValueError("group_start must be [num_groups + 1]")
+    if workspace is None:
+        need = cascade_workspace_bytes(s, h, hkv, d, bs, max_context_len, partition_size)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        if stream is not None:
+            workspace.record_stream(stream)   # the temporary must outlive the launch
+    _check(_paged_attn_decode_cascade(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(block_tables), _ptr(context_lens), _ptr(group_start),
+                                      _ptr(shared_blocks), float(scale), s, g, max_group_size,
+                                      max_shared_blocks, h, hkv, d, bs, block_tables.shape[1],
+                                      max_context_len, num_blocks, _dtype_code(q), partition_size,
+                                      _ptr(workspace), workspace.numel(), _ptr(dev_err),
+                                      _stream(stream)),
+           "paged_attn_decode_cascade")
 
 
 def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scales, v_scales,

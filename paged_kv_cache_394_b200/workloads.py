@@ -247,7 +247,19 @@ def build_prefix_share_workload(num_prompts, samples, prompt_len, div_low, div_h
                     slot_mapping=np.asarray(slots, dtype=np.int64),
                     cow_pairs=np.asarray(cow, dtype=np.int64).reshape(-1, 2),
                     notes={"seed": seed, "prompt_len": prompt_len,
-                           "prompt_blocks": n_prompt_blocks})
+                           "prompt_blocks": n_prompt_blocks, "samples": samples})
+
+
+def cascade_groups(w, shared_blocks=None):
+    """Groups of a prefix-sharing workload for cascade decode: the samples of
+    each prompt (adjacent sequences) and the whole prompt blocks they share
+    (a partly filled last prompt block is private after copy-on-write).
+    Returns int32 arrays (group_start [G+1], shared_blocks [G])."""
+    samples = w.notes["samples"]
+    n = w.num_seqs // samples
+    full = w.notes["prompt_len"] // w.block_size if shared_blocks is None else shared_blocks
+    group_start = np.arange(0, w.num_seqs + 1, samples, dtype=np.int32)
+    return group_start, np.full(n, full, dtype=np.int32)
 
 
 def build_prefill_workload(hist_lens, new_lens, num_heads, num_kv_heads, head_dim, block_size,

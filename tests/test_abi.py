@@ -159,3 +159,25 @@ def test_binding_constants_match_the_header():
         assert getattr(pk, name) == int(val), name
     for name, val in re.findall(r"PKV_(FP16|BF16|FP8_E4M3)\s*=\s*(\d+)", hdr):
         assert getattr(pk, name) == int(val), name
+
+
+def test_cascade_host_validation_without_gpu():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    null = None
+    good = ctypes.c_void_p(0x1000)
+    bad = ctypes.c_void_p(0x1008)
+    ws = pk.cascade_workspace_bytes(4, 8, 2, 128, 16, 256)
+    assert ws > 0 and ws >= pk.workspace_bytes(4, 8, 2, 128, 16, 256)
+
+    def cas(s=4, g=2, mgs=2, msb=4, d=128, ptr=good, gptr=good, wsb=ws, mc=256, part=0):
+        return pk._paged_attn_decode_cascade(ptr, ptr, ptr, ptr, ptr, ptr, gptr, gptr, 0.125, s, g,
+                                             mgs, msb, 8, 2, d, 16, 16, mc, 64, 0, part, good,
+                                             wsb, null, null)
+    assert cas(s=0) == pk.OK
+    assert cas(d=64) == pk.ERR_UNSUPPORTED                 # the prefix pass is head_dim 128
+    assert cas(g=0) == pk.ERR_INVALID_ARG                  # sequences but no groups
+    assert cas(msb=17) == pk.ERR_INVALID_ARG               # 17 * 16 > max_context_len
+    assert cas(gptr=null) == pk.ERR_INVALID_ARG
+    assert cas(wsb=ws - 16) == pk.ERR_WORKSPACE
+    assert cas(ptr=bad) == pk.ERR_INVALID_ARG
+    assert cas(part=24) == pk.ERR_INVALID_ARG              # not a multiple of block_size

@@ -223,12 +223,14 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-DECODE_SOURCES = ("common.cuh", "paged_attn_kernels.cuh")
-PREFILL_SOURCES = ("common.cuh", "paged_prefill_kernels.cuh", "paged_prefill_tc_kernels.cuh")
+# device code and the host code that picks its launch shapes
+DECODE_SOURCES = ("common.cuh", "paged_attn_kernels.cuh", "paged_attn_decode.cu")
+PREFILL_SOURCES = ("common.cuh", "paged_prefill_kernels.cuh", "paged_prefill_tc_kernels.cuh",
+                   "paged_attn_prefill.cu")
 
 
 def kernel_source_hash(sources=DECODE_SOURCES):
-    """Hash of the device code of one kernel family (kernels and helpers)."""
+    """Hash of one kernel family's sources (kernels, helpers, launch shapes)."""
     csrc = os.path.join(ROOT, "paged_kv_cache_394_b200", "csrc")
     h = hashlib.sha256()
     for f in sources:

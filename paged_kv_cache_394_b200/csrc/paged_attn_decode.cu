@@ -17,14 +17,13 @@ namespace pkv {
 // Host side: shape dispatch, partition choice, workspace layout, launch.
 // ---------------------------------------------------------------------------
 
-// E4M3 cache: stages per warp of the tensor-core kernel, and whether G = 1
-// also runs there (else on the CUDA cores).  Measured on B200 (decode kernel
-// GB/s, D = 128): with 2 stages (32 KiB of ring, about five CTAs per SM) the
-// tensor-core kernel reads LLaMA-7B shapes at 5667 (G = 1; the CUDA-core
-// kernel: 5087), GQA chat at 5135 (G = 4), long contexts at 6203; with 3
-// stages 5549 / 4964 / 6162; with 6 stages 4396 / 3457 / 4207.
+// E4M3 cache at head_dim 128: every group size runs on the tensor-core
+// kernel, with this many stages per warp.  Measured on B200 (decode kernel
+// GB/s): with 2 stages (32 KiB of ring, about five CTAs per SM) it reads
+// LLaMA-7B shapes at 5667 (G = 1; the CUDA-core kernel: 5087), GQA chat at
+// 5135 (G = 4), long contexts at 6203; with 3 stages 5549 / 4964 / 6162;
+// with 6 stages 4396 / 3457 / 4207.
 constexpr int kFp8MmaStages = 2;
-constexpr bool kFp8G1OnTensorCores = true;
 
 // Warps per CTA and ring stages per warp for a (head_dim, block_size): about
 // 96 KiB of ring per CTA so two CTAs fit on an SM, 2..4 stages per warp.
@@ -74,14 +73,10 @@ KernelEntry decode_entry(int d, int bs, int g, pkv_dtype dt) {
   return dt == PKV_FP16 ? entry_for<Fp16>(d, bs, g) : entry_for<Bf16>(d, bs, g);
 }
 
-// E4M3 cache on the CUDA cores (the codes widen to fp32 in registers; q and
-// out keep their 16-bit type): G = 1, and every G at head_dim 64 (head_dim
-// 128 with G >= 2 runs on the tensor cores).
+// E4M3 cache on the CUDA cores at head_dim 64 (the codes widen to fp32 in
+// registers; q and out keep their 16-bit type).
 template <int D, int BS, class DT>
 KernelEntry fp8_entry_for_group(int g) {
-  if constexpr (D == 128) {
-    return g == 1 ? make_entry<D, BS, 1, DT, Fp8E4M3>() : KernelEntry{nullptr, 0, 0};
-  }
   switch (g) {
     case 1: return make_entry<D, BS, 1, DT, Fp8E4M3>();
     case 2: return make_entry<D, BS, 2, DT, Fp8E4M3>();
@@ -93,8 +88,6 @@ KernelEntry fp8_entry_for_group(int g) {
 
 template <class DT>
 KernelEntry fp8_entry_for(int d, int bs, int g) {
-  if (d == 128 && bs == 16) return fp8_entry_for_group<128, 16, DT>(g);
-  if (d == 128 && bs == 32) return fp8_entry_for_group<128, 32, DT>(g);
   if (d == 64 && bs == 16) return fp8_entry_for_group<64, 16, DT>(g);
   if (d == 64 && bs == 32) return fp8_entry_for_group<64, 32, DT>(g);
   return KernelEntry{nullptr, 0, 0};
@@ -365,8 +358,9 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * grid_parts;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
-  // G >= 2 runs on the tensor cores (E4M3: head_dim 128 only), G = 1 on the CUDA cores
-  const bool use_mma = fp8 ? head_dim == 128 && (group >= 2 || kFp8G1OnTensorCores) : group >= 2;
+  // 16-bit: G >= 2 on the tensor cores, G = 1 on the CUDA cores;
+  // E4M3: every G on the tensor cores at head_dim 128, on the CUDA cores at 64
+  const bool use_mma = fp8 ? head_dim == 128 : group >= 2;
   const KernelEntry ke = use_mma ? KernelEntry{nullptr, 0, 0}
                          : fp8   ? fp8_decode_entry(head_dim, block_size, group, dtype)
                                  : decode_entry(head_dim, block_size, group, dtype);

@@ -1,7 +1,9 @@
 /*
  * pagedkv.h — C ABI of libpagedkv.so: PagedAttention decode on NVIDIA B200
  * (sm_100a), the cache-write scatter, the copy-on-write block copy, and a
- * host-side block allocator.
+ * host-side block allocator with prefix caching; beyond the decode path,
+ * chunked-prefill attention, cascade decode over shared prefixes, and an
+ * 8-bit (E4M3) cache.
  *
  * Sources cited by page title and section:
  *   [csdn]       devpress.csdn.net, "vLLM镜像深度优化：PagedAttention助力大模型推理效率飞跃"
@@ -18,7 +20,8 @@
  *  - Layouts are row-major.  The caches are
  *        k_cache, v_cache : [num_blocks, num_kv_heads, block_size, head_dim]
  *    so one (block, kv head) is one contiguous run of block_size*head_dim
- *    elements.  Elements are 16-bit (PKV_FP16 or PKV_BF16).
+ *    elements.  Elements are 16-bit (PKV_FP16 or PKV_BF16), or 1-byte E4M3
+ *    codes for the *_fp8 entry points (and copy_blocks with PKV_FP8_E4M3).
  *  - A slot is physical_block * block_size + offset (int64); a negative slot
  *    marks a padding token.
  *  - Ownership: the caller owns every buffer.  The library never allocates or
@@ -40,7 +43,8 @@
  *    word after the stream has synchronized; outputs are then unreliable.
  *  - Alignment: every tensor pointer (16-bit or E4M3) must be 16-byte aligned.
  *  - Supported shapes: head_dim in {64, 128}, block_size in {16, 32},
- *    num_heads / num_kv_heads in {1, 2, 4, 8}, dtype fp16 or bf16.
+ *    num_heads / num_kv_heads in {1, 2, 4, 8}, q/out dtype fp16 or bf16
+ *    (cascade decode: head_dim 128 only).
  */
 #ifndef PAGEDKV_H_
 #define PAGEDKV_H_

@@ -15,6 +15,9 @@ Before the step every slot the step writes, every slot past a sequence's
 context, and every unused block holds NaN, so a missed write or a stray read
 shows up as NaN in the output.
 
+Prefill workloads (``build_prefill_workload``) instead append several tokens
+per sequence whose queries attend causally over the whole context.
+
 The five named workloads follow the chat-serving shapes described for vLLM
 (LLaMA-7B/13B-sized heads, grouped-query heads, block sizes 16 and 32,
 lengths mixed like chat prompts plus generations, parallel sampling that

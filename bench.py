@@ -689,15 +689,16 @@ def run_ours_prefill(args):
 # ---------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample(w, seconds):
+def oracle_sample(w, seconds, threads=None):
     """Times the oracle's step (cache write, then decode of whole sequences in
-    order, all heads) until `seconds` have passed or the batch is done."""
+    order, all heads) until `seconds` have passed or the batch is done, with
+    BLAS limited to `threads` (default: every core this process may use)."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
     from oracle import attention as OA
     from oracle import cache_ops as OC
-    cores = len(os.sched_getaffinity(0))
+    cores = threads or len(os.sched_getaffinity(0))
     done_seqs = 0
     nbytes = 0
     with threadpool_limits(limits=cores):
@@ -722,10 +723,13 @@ def oracle_sample(w, seconds):
 
 def cpu_baseline(w, seconds):
     nbytes, dt, n, cores = oracle_sample(w, seconds)
+    nb1, dt1, n1, _ = oracle_sample(w, seconds / 3, threads=1)
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
             "sample": "cache write + float64 decode of the first %d of %d sequences (all %d "
-                      "heads), %.1f s on the host cores" % (n, w.num_seqs, w.num_heads, dt)}
+                      "heads), %.1f s on the host cores" % (n, w.num_seqs, w.num_heads, dt),
+            "value_1_thread": round(nb1 / dt1 / 1e9, 4),
+            "sample_1_thread": "the same, BLAS on 1 thread: %d sequences in %.1f s" % (n1, dt1)}
 
 
 def replay_trace(mgr, trace, cached, max_live=64):

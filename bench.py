@@ -230,12 +230,16 @@ PREFILL_SOURCES = ("common.cuh", "paged_prefill_kernels.cuh", "paged_prefill_tc_
 
 
 def kernel_source_hash(sources=DECODE_SOURCES):
-    """Hash of one kernel family's sources (kernels, helpers, launch shapes)."""
+    """Hash of one kernel family's sources (kernels, helpers, launch shapes)
+    with comments and blank lines left out, so that editing a comment does not
+    mark counters taken on the same code as stale."""
     csrc = os.path.join(ROOT, "paged_kv_cache_394_b200", "csrc")
     h = hashlib.sha256()
     for f in sources:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        code = [ln.split("//", 1)[0].rstrip() for ln in text.splitlines()]
+        h.update(f.encode() + b"\0" + "\n".join(ln for ln in code if ln).encode())
     return h.hexdigest()[:16]
 
 

@@ -81,8 +81,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Waits for the phase with the given parity to complete; false after
-// kWaitTimeoutNs.  The clock is read only once the first try has failed.
 // Non-blocking: has the phase with this parity completed?
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
@@ -96,6 +94,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// Waits for the phase with the given parity to complete; false after
+// kWaitTimeoutNs.  The clock is read only once the first try has failed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();

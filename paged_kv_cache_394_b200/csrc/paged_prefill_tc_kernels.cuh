@@ -107,6 +107,33 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- sm_100 packed fp32 pairs and three-input max (fewer softmax instructions)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// (a * b + c) on both halves, each rounded to nearest even as fmaf
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three, with fmaxf's treatment of NaN
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
 // address, leading / stride byte offsets in 16-byte units, version 1, layout 2).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
@@ -355,39 +382,41 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     // ---- MMA issuer ---------------------------------------------------------------
     if (lane == 0) {
       bool ok = mbar_wait_bounded(bar_q, 0);
+      // Operand descriptors as a base plus a start-address step: the 14-bit
+      // start field holds address / 16 and never carries, since shared memory
+      // ends below 2^18 bytes.  This keeps the issuing thread's work per MMA to
+      // one add.
+      const uint64_t d_q = tc::smem_desc_sw128(sbase + Tr::OFF_Q, 16, 1024);
+      const uint64_t d_k = tc::smem_desc_sw128(sbase + Tr::OFF_KV, 16, 1024);
+      const uint64_t d_v = tc::smem_desc_sw128(sbase + Tr::OFF_KV + 2 * Tr::KV_HALF, Tr::KV_HALF, 1024);
+      const uint64_t d_p = tc::smem_desc_sw128(sbase + Tr::OFF_P, 16, 1024);
+      const uint64_t d_plo = tc::smem_desc_sw128(sbase + Tr::OFF_PLO, 16, 1024);
       // O_q += P_q V for tile t (P in buffer t % PB of query tile q)
       auto issue_pv = [&](int q, int t) {
-        const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
-        const uint32_t v0 = st + 2 * Tr::KV_HALF;
-        const int buf = q * PB + t % PB;
-        const uint32_t pbuf = sbase + Tr::OFF_P + buf * Tr::P_BYTES;
-        const uint32_t plo = sbase + Tr::OFF_PLO + buf * Tr::P_BYTES;
+        const uint64_t v0 = d_v + static_cast<uint32_t>((t % NS) * (Tr::STAGE >> 4));
+        const uint32_t pstep = static_cast<uint32_t>((q * PB + t % PB) * (Tr::P_BYTES >> 4));
         const uint32_t o_tmem = tmem + q * 256 + 128;
 #pragma unroll
         for (int kk = 0; kk < NKEY / 16; ++kk) {
-          const uint64_t bdesc = tc::smem_desc_sw128(v0 + kk * 2048, Tr::KV_HALF, 1024);
-          const uint64_t adesc = tc::smem_desc_sw128(pbuf + kk * 32, 16, 1024);
-          tc::umma_f16(o_tmem, adesc, bdesc, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
-          if constexpr (Tr::kBf16) {
-            const uint64_t ldesc = tc::smem_desc_sw128(plo + kk * 32, 16, 1024);
-            tc::umma_f16(o_tmem, ldesc, bdesc, IDESC_O, 1u);
-          }
+          const uint64_t bdesc = v0 + kk * (2048 >> 4);
+          tc::umma_f16(o_tmem, d_p + pstep + kk * 2, bdesc, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+          if constexpr (Tr::kBf16) tc::umma_f16(o_tmem, d_plo + pstep + kk * 2, bdesc, IDESC_O, 1u);
         }
         tc::umma_commit(bar_o(q, t & 1));
       };
       // S = Q K^T of tile t for every query tile that uses it
       auto issue_s = [&](int t) {
-        const uint32_t st = sbase + Tr::OFF_KV + (t % NS) * Tr::STAGE;
+        const uint64_t k0 = d_k + static_cast<uint32_t>((t % NS) * (Tr::STAGE >> 4));
 #pragma unroll
         for (int q = 0; q < QT; ++q) {
           if (t >= ntq[q]) continue;
-          const uint32_t q_lo = sbase + Tr::OFF_Q + q * Tr::Q_TILE, q_hi = q_lo + Tr::Q_HALF;
+          const uint64_t q0d = d_q + q * (Tr::Q_TILE >> 4);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t qa = (ks < 4 ? q_lo : q_hi) + (ks & 3) * 32;
-            const uint32_t kb = st + (ks < 4 ? 0 : Tr::KV_HALF) + (ks & 3) * 32;
-            tc::umma_f16(tmem + q * 256 + (t & 1) * 64, tc::smem_desc_sw128(qa, 16, 1024),
-                         tc::smem_desc_sw128(kb, 16, 1024), IDESC_S, ks > 0 ? 1u : 0u);
+            const uint32_t step = (ks < 4 ? 0 : Tr::Q_HALF >> 4) + (ks & 3) * 2;
+            const uint32_t kstep = (ks < 4 ? 0 : Tr::KV_HALF >> 4) + (ks & 3) * 2;
+            tc::umma_f16(tmem + q * 256 + (t & 1) * 64, q0d + step, k0 + kstep, IDESC_S,
+                         ks > 0 ? 1u : 0u);
           }
           tc::umma_commit(bar_s_full(q, t & 1));
         }
@@ -485,9 +514,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       }
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < NKEY; c += 4) {
+      for (int c = 0; c < NKEY; c += 8) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], s[c + u]);
+        for (int u = 0; u < 4; ++u) mx4[u] = tc::max3(mx4[u], s[c + u], s[c + 4 + u]);
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * mult;
       // move the reference max only when this tile would push P above 2^8
@@ -497,15 +526,24 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         m = mx;
       }
       const float neg_m = m == -INFINITY ? 0.f : -m;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // p = 2^(s * mult - m) in fp32 pairs: the same roundings as fmaf and a
+      // float sum per chain (four chains: lanes of sum2[0] and sum2[1])
+      const uint64_t mult2 = tc::f2_pack(mult, mult), neg_m2 = tc::f2_pack(neg_m, neg_m);
+      uint64_t sum2[2] = {tc::f2_pack(0.f, 0.f), tc::f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < NKEY; c += 4) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          s[c + u] = exp2_approx(fmaf(s[c + u], mult, neg_m));
-          sum4[u] += s[c + u];
+        for (int h = 0; h < 2; ++h) {
+          float x0, x1;
+          tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[c + 2 * h], s[c + 2 * h + 1]), mult2, neg_m2), x0, x1);
+          s[c + 2 * h] = exp2_approx(x0);
+          s[c + 2 * h + 1] = exp2_approx(x1);
+          sum2[h] = tc::f2_add(sum2[h], tc::f2_pack(s[c + 2 * h], s[c + 2 * h + 1]));
         }
       }
+      float sum4[4];
+      tc::f2_unpack(sum2[0], sum4[0], sum4[1]);
+      tc::f2_unpack(sum2[1], sum4[2], sum4[3]);
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * alpha + sum;
       if (t > 0 && __any_sync(kFullMask, alpha != 1.f)) {

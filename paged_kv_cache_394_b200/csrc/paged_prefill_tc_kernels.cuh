@@ -410,22 +410,18 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         tc::umma_commit(bar_o(q, t & 1));
       };
-      // S = Q K^T of tile t for every query tile that uses it
-      auto issue_s = [&](int t) {
+      // S_q = Q_q K^T of tile t
+      auto issue_s = [&](int q, int t) {
         const uint64_t k0 = d_k + static_cast<uint32_t>((t % NS) * (Tr::STAGE >> 4));
+        const uint64_t q0d = d_q + q * (Tr::Q_TILE >> 4);
 #pragma unroll
-        for (int q = 0; q < QT; ++q) {
-          if (t >= ntq[q]) continue;
-          const uint64_t q0d = d_q + q * (Tr::Q_TILE >> 4);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t step = (ks < 4 ? 0 : Tr::Q_HALF >> 4) + (ks & 3) * 2;
-            const uint32_t kstep = (ks < 4 ? 0 : Tr::KV_HALF >> 4) + (ks & 3) * 2;
-            tc::umma_f16(tmem + q * 256 + (t & 1) * 64, q0d + step, k0 + kstep, IDESC_S,
-                         ks > 0 ? 1u : 0u);
-          }
-          tc::umma_commit(bar_s_full(q, t & 1));
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t step = (ks < 4 ? 0 : Tr::Q_HALF >> 4) + (ks & 3) * 2;
+          const uint32_t kstep = (ks < 4 ? 0 : Tr::KV_HALF >> 4) + (ks & 3) * 2;
+          tc::umma_f16(tmem + q * 256 + (t & 1) * 64, q0d + step, k0 + kstep, IDESC_S,
+                       ks > 0 ? 1u : 0u);
         }
+        tc::umma_commit(bar_s_full(q, t & 1));
       };
       if constexpr (Tr::kSplitIssue) {
         // Two issuing threads, each taking its MMAs in order with one wait at a
@@ -433,29 +429,39 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         // read S of tile u - 2 (its P of that tile is out), which frees the S
         // buffer; warp PV_WARP issues P.V of tile t once every query tile's P and
         // the V of that tile are in.
+        // Each query tile's MMAs go out as soon as that tile's inputs are in,
+        // except P.V of the CTA's last KV tile, whose V rows past the context
+        // the softmax warps of every query tile zero: it waits for all of them.
         if (warp == 1) {
           for (int u = 0; ok && u < ntiles; ++u) {
             ok = mbar_wait_bounded(bar_k_full(u % NS), (u / NS) & 1);
 #pragma unroll
-            for (int q = 0; q < QT; ++q)
-              if (ok && u >= 2 && u - 2 < ntq[q])
-                ok = mbar_wait_bounded(bar_p(q, u & 1), ((u - 2) >> 1) & 1);
+            for (int q = 0; q < QT; ++q) {
+              if (!ok || u >= ntq[q]) continue;
+              if (u >= 2) ok = mbar_wait_bounded(bar_p(q, u & 1), ((u - 2) >> 1) & 1);
+              if (!ok) break;
+              tc::tc_fence_after();
+              issue_s(q, u);
+            }
             if (!ok) break;
-            tc::tc_fence_after();
-            issue_s(u);
             tc::umma_commit(bar_k_empty(u % NS));
           }
         } else {
           for (int t = 0; ok && t < ntiles; ++t) {
+            const bool last = t == ntiles - 1;
 #pragma unroll
             for (int q = 0; q < QT; ++q)
-              if (ok && t < ntq[q]) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+              if (ok && last && t < ntq[q]) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
             if (ok) ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
-            if (!ok) break;
-            tc::tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < QT; ++q)
-              if (t < ntq[q]) issue_pv(q, t);
+            for (int q = 0; q < QT; ++q) {
+              if (!ok || t >= ntq[q]) continue;
+              if (!last) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+              if (!ok) break;
+              tc::tc_fence_after();
+              issue_pv(q, t);
+            }
+            if (!ok) break;
             tc::umma_commit(bar_v_empty(t % NS));
           }
         }
@@ -480,7 +486,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           if (ns < ntiles && ns - np < 2 &&
               mbar_test_wait(bar_k_full(ns % NS), (ns / NS) & 1)) {
             tc::tc_fence_after();
-            issue_s(ns);
+#pragma unroll
+            for (int q = 0; q < QT; ++q)
+              if (ns < ntq[q]) issue_s(q, ns);
             tc::umma_commit(bar_k_empty(ns % NS));
             ++ns;
             progress = true;

@@ -116,6 +116,23 @@ def decode_bytes(w, kv_elem=2):
     return kv + qo
 
 
+def unique_decode_bytes(w, kv_elem=2):
+    """decode_bytes with every physical block counted once: each distinct
+    block contributes the most tokens any sequence reads from it.  Equal to
+    decode_bytes when no block is shared (prefix sharing makes it smaller)."""
+    import numpy as np
+    most = {}
+    for i, c in enumerate(w.context_lens.astype(np.int64)):
+        nblk = -(-int(c) // w.block_size)
+        for j, b in enumerate(w.block_tables[i, :nblk]):
+            used = min(w.block_size, int(c) - j * w.block_size)
+            if used > most.get(int(b), 0):
+                most[int(b)] = used
+    kv = 2 * sum(most.values()) * w.num_kv_heads * w.head_dim * kv_elem
+    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * 2
+    return kv + qo
+
+
 def write_bytes(w, kv_elem=2):
     """reshape_and_cache: read key and value (16-bit), write them
     (``kv_elem`` bytes per element), read the slots."""
@@ -397,6 +414,34 @@ def run_ours(args):
     achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
 
+    # ---- shared blocks: unique bytes, and the decode timed with L2 flushed ----
+    ubytes = unique_decode_bytes(w, kv_elem)
+    sharing = None
+    if ubytes < dbytes:
+        l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20)
+        scrub = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+        n_fl = min(args.steps, 50)
+        fl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(n_fl)]
+        with torch.cuda.stream(stream):
+            for i in range(n_fl):
+                scrub.zero_()             # evict the previous step's blocks from L2
+                step(*fl_ev[i])
+        torch.cuda.synchronize(dev)
+        fl_ms = statistics.mean(a.elapsed_time(b) for a, b in fl_ev)
+        del scrub
+        traffic = committed_traffic(args.workload)
+        sharing = {
+            "unique_bytes_per_launch": ubytes,
+            "logical_over_unique": round(dbytes / ubytes, 3),
+            "unique_gbs": round(ubytes / (dec_avg_ms * 1e-3) / 1e9, 2),
+            "dram_over_logical": None if traffic is None else round(traffic / dbytes, 4),
+            "l2_flushed": {"achieved": round(dbytes / (fl_ms * 1e-3) / 1e9, 2),
+                           "unique_gbs": round(ubytes / (fl_ms * 1e-3) / 1e9, 2),
+                           "avg_launch_ms": round(fl_ms, 5), "launches": n_fl,
+                           "flush": "%d MB written before each step" % (2 * l2 >> 20)},
+        }
+
     # ---- end to end through the host-buffer entry point ----------------------
     def pinned(a, view=None):
         return torch.from_numpy(np.ascontiguousarray(a if view is None else a.view(view))).pin_memory()
@@ -541,6 +586,8 @@ def run_ours(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
+        if sharing is not None:
+            line["shared_blocks"] = sharing
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

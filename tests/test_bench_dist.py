@@ -114,3 +114,28 @@ def test_reference_arm_prints_one_contract_line():
     assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
     assert line["warmup"] >= 3                      # warm-up is clamped to at least 3
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _slots_read(w):
+    """Every (physical block, slot) the decode reads, by brute force."""
+    seen = set()
+    for i, c in enumerate(w.context_lens):
+        for t in range(int(c)):
+            seen.add((int(w.block_tables[i, t // w.block_size]), t % w.block_size))
+    return seen
+
+
+@pytest.mark.parametrize("kv_elem", [2, 1])
+def test_unique_bytes_count_each_shared_slot_once(kv_elem):
+    from paged_kv_cache_394_b200 import workloads as W
+    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "fp16", seed=5)
+    per_slot = 2 * w.num_kv_heads * w.head_dim * kv_elem
+    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * 2
+    assert bench.unique_decode_bytes(w, kv_elem) == len(_slots_read(w)) * per_slot + qo
+    assert bench.unique_decode_bytes(w, kv_elem) < bench.decode_bytes(w, kv_elem)
+
+
+def test_unique_bytes_equal_logical_without_sharing():
+    from paged_kv_cache_394_b200 import workloads as W
+    w = W.make("tiny")
+    assert bench.unique_decode_bytes(w) == bench.decode_bytes(w)

@@ -68,6 +68,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem desc]: A (M x 16, K-major) sits in tensor
+// memory, row m in lane m, two 16-bit K elements per 32-bit column.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
 // Arrives once on `bar` when all earlier tcgen05.mma of this thread complete.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -98,6 +109,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
       "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
       "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -177,13 +196,18 @@ struct TcPrefillTraits {
   // KV stages and P buffers per query tile: what fits beside QT query tiles.
   // With two query tiles, one P buffer per tile and a fourth KV stage measured
   // 1-2 % faster on B200 than two P buffers and three stages.
-  static constexpr int NS = (QT == 2 && kBf16) ? 3 : 4;
   static constexpr int PB = QT == 2 ? 1 : 2;
   // warps: K producer, MMA issuer, V producer, 4 softmax warps per query
   // tile; with two query tiles a last warp issues P.V while warp 1 issues S
   // (measured on B200: 540 -> 603 TFLOP/s on the LLaMA-7B prefill batch; with
   // one query tile the single polling issuer measured 2 % faster)
   static constexpr bool kSplitIssue = QT == 2;
+  // with the split issuers P goes to TMEM over the S it replaces (P.V reads
+  // its A operand from there), so no shared-memory P buffers are needed and
+  // the softmax never waits for a P buffer; S of tile t + 2 waits instead for
+  // P.V of tile t to finish
+  static constexpr bool kPInTmem = kSplitIssue;
+  static constexpr int NS = kPInTmem ? (kBf16 ? 5 : 5) : ((QT == 2 && kBf16) ? 3 : 4);
   static constexpr int PV_WARP = kSplitIssue ? 3 + 4 * QT : 1;
   static constexpr int THREADS = (3 + 4 * QT + (kSplitIssue ? 1 : 0)) * 32;
   // shared-memory layout (all 1024-byte aligned)
@@ -195,8 +219,9 @@ struct TcPrefillTraits {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QT * Q_TILE;
   static constexpr int OFF_P = OFF_KV + NS * STAGE;              // [QT][PB] P buffers
-  static constexpr int OFF_PLO = OFF_P + QT * PB * P_BYTES;      // bf16 lo halves
-  static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? QT * PB * P_BYTES : 0);
+  static constexpr int P_SMEM = kPInTmem ? 0 : QT * PB * P_BYTES;
+  static constexpr int OFF_PLO = OFF_P + P_SMEM;                 // bf16 lo halves
+  static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? P_SMEM : 0);
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
   // per query tile s_full[2], p_full[2], o_done[2]; then the TMEM address slot
   static constexpr int NBAR = 1 + 4 * NS + 6 * QT;
@@ -402,11 +427,19 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         const uint64_t v0 = d_v + static_cast<uint32_t>((t % NS) * (Tr::STAGE >> 4));
         const uint32_t pstep = static_cast<uint32_t>((q * PB + t % PB) * (Tr::P_BYTES >> 4));
         const uint32_t o_tmem = tmem + q * 256 + 128;
+        // P in TMEM: columns 0..31 of the tile's S buffer (bf16 lo halves in 32..63)
+        const uint32_t p_tmem = tmem + q * 256 + (t & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < NKEY / 16; ++kk) {
           const uint64_t bdesc = v0 + kk * (2048 >> 4);
-          tc::umma_f16(o_tmem, d_p + pstep + kk * 2, bdesc, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
-          if constexpr (Tr::kBf16) tc::umma_f16(o_tmem, d_plo + pstep + kk * 2, bdesc, IDESC_O, 1u);
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          if constexpr (Tr::kPInTmem) {
+            tc::umma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, IDESC_O, acc);
+            if constexpr (Tr::kBf16) tc::umma_f16_ts(o_tmem, p_tmem + 32 + kk * 8, bdesc, IDESC_O, 1u);
+          } else {
+            tc::umma_f16(o_tmem, d_p + pstep + kk * 2, bdesc, IDESC_O, acc);
+            if constexpr (Tr::kBf16) tc::umma_f16(o_tmem, d_plo + pstep + kk * 2, bdesc, IDESC_O, 1u);
+          }
         }
         tc::umma_commit(bar_o(q, t & 1));
       };
@@ -438,7 +471,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll
             for (int q = 0; q < QT; ++q) {
               if (!ok || u >= ntq[q]) continue;
-              if (u >= 2) ok = mbar_wait_bounded(bar_p(q, u & 1), ((u - 2) >> 1) & 1);
+              // the S buffer of tile u - 2 is free once the softmax has read it
+              // (its P is out) or, with P in TMEM over it, once P.V has read P
+              if (u >= 2)
+                ok = Tr::kPInTmem ? mbar_wait_bounded(bar_o(q, u & 1), ((u - 2) >> 1) & 1)
+                                  : mbar_wait_bounded(bar_p(q, u & 1), ((u - 2) >> 1) & 1);
               if (!ok) break;
               tc::tc_fence_after();
               issue_s(q, u);
@@ -613,33 +650,55 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         tc::tmem_wait_st();
       }
-      if (t >= PB) {  // the P buffer of tile t was last read by P.V of tile t - PB
+      if constexpr (Tr::kPInTmem) {
+        // P (16-bit; bf16 as hi + lo) into TMEM over the S just read:
+        // columns 0..31 of the tile's S buffer (bf16 lo halves in 32..63)
+        const uint32_t pt = lane_addr + (t & 1) * 64;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[16], wl[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = s[32 * h + 2 * e], b = s[32 * h + 2 * e + 1];
+            w[e] = pack2(a, b, DT());
+            if constexpr (Tr::kBf16)
+              wl[e] = pack2(a - __uint_as_float(w[e] << 16),
+                            b - __uint_as_float(w[e] & 0xffff0000u), Bf16());
+          }
+          tc::tmem_st16u(pt + 16 * h, w);
+          if constexpr (Tr::kBf16) tc::tmem_st16u(pt + 32 + 16 * h, wl);
+        }
+        tc::tmem_wait_st();
+      }
+      if (!Tr::kPInTmem && t >= PB) {  // the P buffer of tile t was last read by P.V of tile t - PB
         ok = mbar_wait_bounded(bar_o(qg, (t - PB) & 1), ((t - PB) >> 1) & 1);
         if (!__all_sync(kFullMask, ok)) {
           ok = false;
           break;
         }
       }
-      // P (16-bit; bf16 as hi + lo) into the swizzled [128 rows][64 keys] buffers
-      const int buf = qg * PB + t % PB;
-      unsigned char* prow = smem + Tr::OFF_P + buf * Tr::P_BYTES + r * 128;
-      unsigned char* plrow = smem + Tr::OFF_PLO + buf * Tr::P_BYTES + r * 128;
+      if constexpr (!Tr::kPInTmem) {
+        // P (16-bit; bf16 as hi + lo) into the swizzled [128 rows][64 keys] buffers
+        const int buf = qg * PB + t % PB;
+        unsigned char* prow = smem + Tr::OFF_P + buf * Tr::P_BYTES + r * 128;
+        unsigned char* plrow = smem + Tr::OFF_PLO + buf * Tr::P_BYTES + r * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t w[4], wl[4];
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t w[4], wl[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = s[ch * 8 + 2 * e], b = s[ch * 8 + 2 * e + 1];
-          w[e] = pack2(a, b, DT());
-          if constexpr (Tr::kBf16) {
-            wl[e] = pack2(a - __uint_as_float(w[e] << 16), b - __uint_as_float(w[e] & 0xffff0000u),
-                          Bf16());
+          for (int e = 0; e < 4; ++e) {
+            const float a = s[ch * 8 + 2 * e], b = s[ch * 8 + 2 * e + 1];
+            w[e] = pack2(a, b, DT());
+            if constexpr (Tr::kBf16) {
+              wl[e] = pack2(a - __uint_as_float(w[e] << 16), b - __uint_as_float(w[e] & 0xffff0000u),
+                            Bf16());
+            }
           }
+          const int at = ((ch ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(prow + at) = make_uint4(w[0], w[1], w[2], w[3]);
+          if constexpr (Tr::kBf16)
+            *reinterpret_cast<uint4*>(plrow + at) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
         }
-        const int at = ((ch ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow + at) = make_uint4(w[0], w[1], w[2], w[3]);
-        if constexpr (Tr::kBf16)
-          *reinterpret_cast<uint4*>(plrow + at) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       }
       // keys past the context, or not loaded, hold stale data: zero their V rows
       // (every query tile that uses the stage writes the same zeros)

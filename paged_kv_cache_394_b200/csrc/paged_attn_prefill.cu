@@ -67,11 +67,10 @@ struct TcEntry {
 // TMA traffic per FLOP (the per-SM TMA engine paces the one-tile kernel).
 // Measured on B200 (kernel TFLOP/s, fp16, one tile -> two): 4 x 512 new tokens
 // on 2048 cached 376 -> 482, 2048 on 8192 cached 419 -> 607, the LLaMA-7B
-// prefill batch 350 -> 411.  bf16 splits P into hi + lo halves, so two tiles
-// leave room for only one P buffer per tile: 4096 new on 4096 cached (G = 4)
-// 445 -> 547, but the 4-sequence GQA prefill batch 331 -> 304; bf16 keeps one.
+// prefill batch 350 -> 411.  bf16 (P split into hi + lo halves) gained once P
+// moved to TMEM with two query tiles: the GQA prefill batch 388 -> 453.
 template <class DT>
-constexpr int kTcQueryTiles = std::is_same<DT, Bf16>::value ? 1 : 2;
+constexpr int kTcQueryTiles = 2;
 
 template <int BS, int G, class DT>
 TcEntry make_tc() {

@@ -11,18 +11,19 @@
 //     tile are issued by 8 lanes at once.
 //   * warp 2 (V producer): the same for the V tiles.  K of a stage is released
 //     once S has read it, V once P.V has, so K loads run further ahead.
-//   * warp 1 (MMA): allocates 256 TMEM columns per query tile; one thread
-//     issues, in whichever order their inputs arrive,
-//       S  = Q K^T   (M=128, N=64,  K=128; A, B K-major)  into TMEM (2 buffers)
-//       O += P V     (M=128, N=128, K=64;  A=P K-major, B=V MN-major) into TMEM
-//     and signals completion with tcgen05.commit on mbarriers.
+//   * warp 1 (S issuer): allocates 256 TMEM columns per query tile; one thread
+//     issues S = Q K^T (M=128, N=64, K=128; A, B K-major) into one of two TMEM
+//     S buffers per query tile.  The last warp (P.V issuer): one thread issues
+//     O += P V (M=128, N=128, K=64) with A = P read from TMEM (the TS form) and
+//     B = V (MN-major) from shared memory.  Completion goes to mbarriers
+//     through tcgen05.commit; each issuer takes its MMAs in tile order.
 //   * 4 softmax warps per query tile: thread r owns row r (TMEM lane r): it
 //     reads its S row from TMEM, masks causally (only on tiles that reach past
 //     the row), keeps the running max / sum in base 2 with the scale folded
 //     into the exponent's FFMA, rescales its O row in TMEM when the max moves,
-//     and writes P (fp16, or bf16 split into hi + lo halves) into
-//     128-byte-swizzled shared memory.  At the end it reads O, divides by the
-//     sum and stores the row.
+//     and writes P (fp16, or bf16 split into hi + lo halves) into TMEM over
+//     the S it just read.  At the end it reads O, divides by the sum and
+//     stores the row (or, for the cascade prefix pass, writes the partial).
 // All operand tiles use the 128-byte swizzle (8-row x 128-byte atoms, stride
 // 1024 bytes).  Keys past the context (or not loaded) are zeroed in the V tile
 // before P.V so stale NaN never enters the tensor-core sum.  Every mbarrier
@@ -193,35 +194,20 @@ struct TcPrefillTraits {
   static constexpr int M = 128;                  // rows of one query tile (one TMEM lane each)
   static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
   static constexpr int NKEY = 64;                // keys per KV tile
-  // KV stages and P buffers per query tile: what fits beside QT query tiles.
-  // With two query tiles, one P buffer per tile and a fourth KV stage measured
-  // 1-2 % faster on B200 than two P buffers and three stages.
-  static constexpr int PB = QT == 2 ? 1 : 2;
-  // warps: K producer, MMA issuer, V producer, 4 softmax warps per query
-  // tile; with two query tiles a last warp issues P.V while warp 1 issues S
-  // (measured on B200: 540 -> 603 TFLOP/s on the LLaMA-7B prefill batch; with
-  // one query tile the single polling issuer measured 2 % faster)
-  static constexpr bool kSplitIssue = QT == 2;
-  // with the split issuers P goes to TMEM over the S it replaces (P.V reads
-  // its A operand from there), so no shared-memory P buffers are needed and
-  // the softmax never waits for a P buffer; S of tile t + 2 waits instead for
-  // P.V of tile t to finish
-  static constexpr bool kPInTmem = kSplitIssue;
-  static constexpr int NS = kPInTmem ? (kBf16 ? 5 : 5) : ((QT == 2 && kBf16) ? 3 : 4);
-  static constexpr int PV_WARP = kSplitIssue ? 3 + 4 * QT : 1;
-  static constexpr int THREADS = (3 + 4 * QT + (kSplitIssue ? 1 : 0)) * 32;
+  // KV stages: what fits beside QT query tiles (P lives in TMEM, over S)
+  static constexpr int NS = QT == 2 ? 5 : 6;
+  // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
+  // P.V issuer
+  static constexpr int PV_WARP = 3 + 4 * QT;
+  static constexpr int THREADS = (PV_WARP + 1) * 32;
   // shared-memory layout (all 1024-byte aligned)
   static constexpr int Q_HALF = M * 128;         // [128 rows][64 dims] = 16 KiB
   static constexpr int Q_TILE = 2 * Q_HALF;
   static constexpr int KV_HALF = NKEY * 128;     // [64 keys][64 dims] = 8 KiB
   static constexpr int STAGE = 4 * KV_HALF;      // K0 K1 V0 V1
-  static constexpr int P_BYTES = M * 128;        // [128 rows][64 keys]
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QT * Q_TILE;
-  static constexpr int OFF_P = OFF_KV + NS * STAGE;              // [QT][PB] P buffers
-  static constexpr int P_SMEM = kPInTmem ? 0 : QT * PB * P_BYTES;
-  static constexpr int OFF_PLO = OFF_P + P_SMEM;                 // bf16 lo halves
-  static constexpr int OFF_BAR = OFF_PLO + (kBf16 ? P_SMEM : 0);
+  static constexpr int OFF_BAR = OFF_KV + NS * STAGE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
   // per query tile s_full[2], p_full[2], o_done[2]; then the TMEM address slot
   static constexpr int NBAR = 1 + 4 * NS + 6 * QT;
@@ -244,7 +230,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   using T = typename Tr::T;
   using DT = typename Tr::DT;
   constexpr int G = Tr::G, BS = Tr::BS, M = Tr::M, NKEY = Tr::NKEY, NS = Tr::NS;
-  constexpr int QT = Tr::QT, PB = Tr::PB, ROWS = Tr::ROWS;
+  constexpr int QT = Tr::QT, ROWS = Tr::ROWS;
   constexpr uint32_t IDESC_S = tc::idesc_f16(Tr::kBf16, M, NKEY, false);
   constexpr uint32_t IDESC_O = tc::idesc_f16(Tr::kBf16, M, 128, true);
   extern __shared__ unsigned char smem_raw[];
@@ -409,7 +395,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       }
       __syncwarp();
     }
-  } else if (warp == 1 || warp == Tr::PV_WARP) {  // PV_WARP is 1 without a split
+  } else if (warp == 1 || warp == Tr::PV_WARP) {
     // ---- MMA issuers ----------------------------------------------------------------
     if (lane == 0) {
       bool ok = warp != 1 || mbar_wait_bounded(bar_q, 0);  // only S reads Q
@@ -420,12 +406,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       const uint64_t d_q = tc::smem_desc_sw128(sbase + Tr::OFF_Q, 16, 1024);
       const uint64_t d_k = tc::smem_desc_sw128(sbase + Tr::OFF_KV, 16, 1024);
       const uint64_t d_v = tc::smem_desc_sw128(sbase + Tr::OFF_KV + 2 * Tr::KV_HALF, Tr::KV_HALF, 1024);
-      const uint64_t d_p = tc::smem_desc_sw128(sbase + Tr::OFF_P, 16, 1024);
-      const uint64_t d_plo = tc::smem_desc_sw128(sbase + Tr::OFF_PLO, 16, 1024);
-      // O_q += P_q V for tile t (P in buffer t % PB of query tile q)
+      // O_q += P_q V for tile t
       auto issue_pv = [&](int q, int t) {
         const uint64_t v0 = d_v + static_cast<uint32_t>((t % NS) * (Tr::STAGE >> 4));
-        const uint32_t pstep = static_cast<uint32_t>((q * PB + t % PB) * (Tr::P_BYTES >> 4));
         const uint32_t o_tmem = tmem + q * 256 + 128;
         // P in TMEM: columns 0..31 of the tile's S buffer (bf16 lo halves in 32..63)
         const uint32_t p_tmem = tmem + q * 256 + (t & 1) * 64;
@@ -433,13 +416,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         for (int kk = 0; kk < NKEY / 16; ++kk) {
           const uint64_t bdesc = v0 + kk * (2048 >> 4);
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (Tr::kPInTmem) {
-            tc::umma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, IDESC_O, acc);
-            if constexpr (Tr::kBf16) tc::umma_f16_ts(o_tmem, p_tmem + 32 + kk * 8, bdesc, IDESC_O, 1u);
-          } else {
-            tc::umma_f16(o_tmem, d_p + pstep + kk * 2, bdesc, IDESC_O, acc);
-            if constexpr (Tr::kBf16) tc::umma_f16(o_tmem, d_plo + pstep + kk * 2, bdesc, IDESC_O, 1u);
-          }
+          tc::umma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, IDESC_O, acc);
+          if constexpr (Tr::kBf16) tc::umma_f16_ts(o_tmem, p_tmem + 32 + kk * 8, bdesc, IDESC_O, 1u);
         }
         tc::umma_commit(bar_o(q, t & 1));
       };
@@ -456,96 +434,46 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         tc::umma_commit(bar_s_full(q, t & 1));
       };
-      if constexpr (Tr::kSplitIssue) {
-        // Two issuing threads, each taking its MMAs in order with one wait at a
-        // time: warp 1 issues S of tile u once its K has landed and the softmax has
-        // read S of tile u - 2 (its P of that tile is out), which frees the S
-        // buffer; warp PV_WARP issues P.V of tile t once every query tile's P and
-        // the V of that tile are in.
-        // Each query tile's MMAs go out as soon as that tile's inputs are in,
-        // except P.V of the CTA's last KV tile, whose V rows past the context
-        // the softmax warps of every query tile zero: it waits for all of them.
-        if (warp == 1) {
-          for (int u = 0; ok && u < ntiles; ++u) {
-            ok = mbar_wait_bounded(bar_k_full(u % NS), (u / NS) & 1);
+      // Two issuing threads, each taking its MMAs in order with one wait at a
+      // time: warp 1 issues S of tile u once its K has landed and P.V of tile
+      // u - 2 has read the P held in the S buffer it overwrites; warp PV_WARP
+      // issues P.V of tile t once that tile's P and V are in.  (One thread
+      // polling for both measured slower on B200.)
+      // Each query tile's MMAs go out as soon as that tile's inputs are in,
+      // except P.V of the CTA's last KV tile, whose V rows past the context
+      // the softmax warps of every query tile zero: it waits for all of them.
+      if (warp == 1) {
+        for (int u = 0; ok && u < ntiles; ++u) {
+          ok = mbar_wait_bounded(bar_k_full(u % NS), (u / NS) & 1);
 #pragma unroll
-            for (int q = 0; q < QT; ++q) {
-              if (!ok || u >= ntq[q]) continue;
-              // the S buffer of tile u - 2 is free once the softmax has read it
-              // (its P is out) or, with P in TMEM over it, once P.V has read P
-              if (u >= 2)
-                ok = Tr::kPInTmem ? mbar_wait_bounded(bar_o(q, u & 1), ((u - 2) >> 1) & 1)
-                                  : mbar_wait_bounded(bar_p(q, u & 1), ((u - 2) >> 1) & 1);
-              if (!ok) break;
-              tc::tc_fence_after();
-              issue_s(q, u);
-            }
+          for (int q = 0; q < QT; ++q) {
+            if (!ok || u >= ntq[q]) continue;
+            // the S buffer of tile u - 2 holds that tile's P until P.V has read it
+            if (u >= 2) ok = mbar_wait_bounded(bar_o(q, u & 1), ((u - 2) >> 1) & 1);
             if (!ok) break;
-            tc::umma_commit(bar_k_empty(u % NS));
+            tc::tc_fence_after();
+            issue_s(q, u);
           }
-        } else {
-          for (int t = 0; ok && t < ntiles; ++t) {
-            const bool last = t == ntiles - 1;
-#pragma unroll
-            for (int q = 0; q < QT; ++q)
-              if (ok && last && t < ntq[q]) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
-            if (ok) ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
-#pragma unroll
-            for (int q = 0; q < QT; ++q) {
-              if (!ok || t >= ntq[q]) continue;
-              if (!last) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
-              if (!ok) break;
-              tc::tc_fence_after();
-              issue_pv(q, t);
-            }
-            if (!ok) break;
-            tc::umma_commit(bar_v_empty(t % NS));
-          }
+          if (!ok) break;
+          tc::umma_commit(bar_k_empty(u % NS));
         }
       } else {
-        // is P of tile t ready in every query tile that uses it?
-        auto p_ready = [&](int t) {
-          bool r = true;
+        for (int t = 0; ok && t < ntiles; ++t) {
+          const bool last = t == ntiles - 1;
 #pragma unroll
           for (int q = 0; q < QT; ++q)
-            if (t < ntq[q]) r = r && mbar_test_wait(bar_p(q, t & 1), (t >> 1) & 1);
-          return r;
-        };
-        // Issue S and P.V in whichever order their inputs arrive: S of tile ns
-        // needs its K/V and its S buffers back (P.V of tile ns - 2 issued, so the
-        // softmax has read them); P.V of tile np needs P of every query tile.
-        // A fixed order would hold a ready P.V behind the next tile's load.
-        int ns = 0, np = 0;
-        uint64_t t_idle = 0;
-        uint32_t idle = 0;
-        while (ok && np < ntiles) {
-          bool progress = false;
-          if (ns < ntiles && ns - np < 2 &&
-              mbar_test_wait(bar_k_full(ns % NS), (ns / NS) & 1)) {
-            tc::tc_fence_after();
+            if (ok && last && t < ntq[q]) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+          if (ok) ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
 #pragma unroll
-            for (int q = 0; q < QT; ++q)
-              if (ns < ntq[q]) issue_s(q, ns);
-            tc::umma_commit(bar_k_empty(ns % NS));
-            ++ns;
-            progress = true;
-          }
-          if (np < ns && p_ready(np) && mbar_test_wait(bar_v_full(np % NS), (np / NS) & 1)) {
+          for (int q = 0; q < QT; ++q) {
+            if (!ok || t >= ntq[q]) continue;
+            if (!last) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+            if (!ok) break;
             tc::tc_fence_after();
-#pragma unroll
-            for (int q = 0; q < QT; ++q)
-              if (np < ntq[q]) issue_pv(q, np);
-            tc::umma_commit(bar_v_empty(np % NS));
-            ++np;
-            progress = true;
+            issue_pv(q, t);
           }
-          if (progress) {
-            idle = 0;
-          } else if (idle++ == 0) {
-            t_idle = global_timer_ns();
-          } else if ((idle & 255u) == 0u && global_timer_ns() - t_idle > kWaitTimeoutNs) {
-            ok = false;
-          }
+          if (!ok) break;
+          tc::umma_commit(bar_v_empty(t % NS));
         }
       }
       if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
@@ -650,7 +578,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         tc::tmem_wait_st();
       }
-      if constexpr (Tr::kPInTmem) {
+      {
         // P (16-bit; bf16 as hi + lo) into TMEM over the S just read:
         // columns 0..31 of the tile's S buffer (bf16 lo halves in 32..63)
         const uint32_t pt = lane_addr + (t & 1) * 64;
@@ -669,36 +597,6 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           if constexpr (Tr::kBf16) tc::tmem_st16u(pt + 32 + 16 * h, wl);
         }
         tc::tmem_wait_st();
-      }
-      if (!Tr::kPInTmem && t >= PB) {  // the P buffer of tile t was last read by P.V of tile t - PB
-        ok = mbar_wait_bounded(bar_o(qg, (t - PB) & 1), ((t - PB) >> 1) & 1);
-        if (!__all_sync(kFullMask, ok)) {
-          ok = false;
-          break;
-        }
-      }
-      if constexpr (!Tr::kPInTmem) {
-        // P (16-bit; bf16 as hi + lo) into the swizzled [128 rows][64 keys] buffers
-        const int buf = qg * PB + t % PB;
-        unsigned char* prow = smem + Tr::OFF_P + buf * Tr::P_BYTES + r * 128;
-        unsigned char* plrow = smem + Tr::OFF_PLO + buf * Tr::P_BYTES + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t w[4], wl[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = s[ch * 8 + 2 * e], b = s[ch * 8 + 2 * e + 1];
-            w[e] = pack2(a, b, DT());
-            if constexpr (Tr::kBf16) {
-              wl[e] = pack2(a - __uint_as_float(w[e] << 16), b - __uint_as_float(w[e] & 0xffff0000u),
-                            Bf16());
-            }
-          }
-          const int at = ((ch ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(prow + at) = make_uint4(w[0], w[1], w[2], w[3]);
-          if constexpr (Tr::kBf16)
-            *reinterpret_cast<uint4*>(plrow + at) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-        }
       }
       // keys past the context, or not loaded, hold stale data: zero their V rows
       // (every query tile that uses the stage writes the same zeros)

@@ -281,7 +281,7 @@ def committed_traffic(workload, kind="decode"):
 # ---------------------------------------------------------------------------
 def run_ours(args):
     from paged_kv_cache_394_b200 import workloads as W
-    if args.workload in W.PREFILL_NAMES:
+    if args.workload.removesuffix("_fp8") in W.PREFILL_NAMES:
         return run_ours_prefill(args)
     import numpy as np
     import torch
@@ -610,14 +610,46 @@ def run_ours_prefill(args):
     local = dist_env()[2]
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    base = W.SEED_BASE + (W.NAMES + W.PREFILL_NAMES).index(args.workload)
-    w = W.make(args.workload, seed=replica_seed(base, rank))
+    # "<name>_fp8": the named prefill batch over E4M3 caches
+    fp8 = args.workload.endswith("_fp8")
+    name = args.workload.removesuffix("_fp8")
+    base = W.SEED_BASE + (W.NAMES + W.PREFILL_NAMES).index(name)
+    w = W.make(name, seed=replica_seed(base, rank))
     tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
 
     def up(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(tdt)
 
     q, kc, vc, key, val = up(w.q), up(w.k_cache), up(w.v_cache), up(w.key), up(w.value)
+    if fp8:
+        # the pool, quantised once by the device's own cache write (setup, untimed)
+        nb, hkv, bs, d = kc.shape
+        ks8 = torch.full((hkv,), FP8_K_SCALE, dtype=torch.float32, device=dev)
+        vs8 = torch.full((hkv,), FP8_V_SCALE, dtype=torch.float32, device=dev)
+        k8 = torch.empty(kc.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty_like(k8)
+        every = torch.arange(nb * bs, dtype=torch.int64, device=dev)
+        tok = lambda c: c.permute(0, 2, 1, 3).reshape(nb * bs, hkv, d).contiguous()
+        pk.reshape_and_cache_fp8(tok(kc), tok(vc), k8, v8, every, ks8, vs8)
+        torch.cuda.synchronize(dev)
+        kc, vc = k8, v8
+        del every
+
+    def write(k, v, s):
+        if fp8:
+            pk.reshape_and_cache_fp8(k, v, kc, vc, s, ks8, vs8, dev_err=err, stream=stream)
+        else:
+            pk.reshape_and_cache(k, v, kc, vc, s, dev_err=err, stream=stream)
+
+    def attend(o, qq, t, l_, qs):
+        if fp8:
+            pk.paged_attn_prefill_fp8(o, qq, kc, vc, t, l_, qs, w.scale, ks8, vs8, w.num_kv_heads,
+                                      w.block_size, w.max_context_len, max_q, dev_err=err,
+                                      stream=stream)
+        else:
+            pk.paged_attn_prefill(o, qq, kc, vc, t, l_, qs, w.scale, w.num_kv_heads,
+                                  w.block_size, w.max_context_len, max_q, dev_err=err,
+                                  stream=stream)
     slots = torch.from_numpy(w.slot_mapping).to(dev)
     tables = torch.from_numpy(w.block_tables).to(dev)
     lens = torch.from_numpy(w.context_lens).to(dev)
@@ -628,11 +660,10 @@ def run_ours_prefill(args):
     stream = torch.cuda.Stream(device=dev)
 
     def step(ev_a=None, ev_b=None):
-        pk.reshape_and_cache(key, val, kc, vc, slots, dev_err=err, stream=stream)
+        write(key, val, slots)
         if ev_a is not None:
             ev_a.record(stream)
-        pk.paged_attn_prefill(out, q, kc, vc, tables, lens, qstart, w.scale, w.num_kv_heads,
-                              w.block_size, w.max_context_len, max_q, dev_err=err, stream=stream)
+        attend(out, q, tables, lens, qstart)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -691,9 +722,8 @@ def run_ours_prefill(args):
 
     def compute(bufs, o):
         bq, bk, bv, bs, bt, bl, bqs = bufs
-        pk.reshape_and_cache(bk, bv, kc, vc, bs, dev_err=err, stream=stream)
-        pk.paged_attn_prefill(o, bq, kc, vc, bt, bl, bqs, w.scale, w.num_kv_heads,
-                              w.block_size, w.max_context_len, max_q, dev_err=err, stream=stream)
+        write(bk, bv, bs)
+        attend(o, bq, bt, bl, bqs)
 
     def e2e_step():  # serial: copies in, compute, copy out, all on one stream
         upload(dev_in[0], stream)
@@ -750,9 +780,12 @@ def run_ours_prefill(args):
             "metric": "paged-prefill attention TFLOP/s",
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 cache, %s q/out, f32 math" % w.dtype if fp8 else w.dtype,
             "data": "synthetic",
-            "config": dict(W.describe(w), parallelism="replicas%d" % world,
+            "config": dict(W.describe(w), workload=args.workload, parallelism="replicas%d" % world,
+                           kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
+                           if fp8 else w.dtype,
                            l2="no flush: each step rewrites the new tokens' K/V"),
             "tokens_per_s": round(world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
@@ -767,7 +800,9 @@ def run_ours_prefill(args):
             "e2e": {"value": round(all_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                     "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,
-                    "api": "pagedkv.reshape_and_cache + paged_attn_prefill with pinned-host copies "
+                    "api": ("pagedkv.reshape_and_cache_fp8 + paged_attn_prefill_fp8" if fp8 else
+                            "pagedkv.reshape_and_cache + paged_attn_prefill") +
+                           " with pinned-host copies "
                            "on side streams, consecutive steps overlapped",
                     "serial": {"value": round(all_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
                                "ms_per_step": round(e2e_serial_ms, 5),

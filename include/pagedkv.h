@@ -333,6 +333,29 @@ pkv_status pkv_paged_attn_decode_fp8(void* out, const void* q, const void* k_cac
                                      unsigned* dev_err, void* stream);
 
 /*
+ * pkv_paged_attn_prefill_fp8 — pkv_paged_attn_prefill over E4M3 caches:
+ *     out[t, h, :] = softmax(scale * q[t, h, :] . K~[0..p]^T) . V~[0..p]
+ * with K~ and V~ decoded as for pkv_paged_attn_decode_fp8 (codes times the kv
+ * head's k_scales / v_scales entry).  head_dim 128 only (else
+ * PKV_ERR_UNSUPPORTED): the tcgen05 kernel stages each tile's codes by TMA
+ * and widens them exactly to the 16-bit type of q (`dtype`) before the tensor
+ * cores read them; the K scale folds into the logit scale and the V scale
+ * into the final normalisation.  Every other argument and the error
+ * behaviour are those of pkv_paged_attn_prefill; null scale pointers give
+ * PKV_ERR_INVALID_ARG and a scale that is not finite and > 0 sets
+ * PKV_DEVERR_BAD_SCALE.
+ */
+pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* context_lens, const int32_t* query_start,
+                                      float scale, const float* k_scales, const float* v_scales,
+                                      int num_seqs, int num_tokens, int num_heads,
+                                      int num_kv_heads, int head_dim, int block_size,
+                                      int max_blocks_per_seq, int max_context_len,
+                                      int max_query_len, int num_blocks, pkv_dtype dtype,
+                                      unsigned* dev_err, void* stream);
+
+/*
  * pkv_decode_step_host — one whole decode step from HOST buffers: copies the
  * step's inputs host->device, runs copy_blocks (if num_pairs > 0),
  * reshape_and_cache (if num_new_tokens > 0) and paged_attn_decode, and copies

@@ -121,3 +121,34 @@ def paged_attention_decode_fp8(q_bits, k_codes, v_codes, block_tables, context_l
         values = dequantize(v_codes[blocks, g, offsets, :], vs[g])
         out[s, h] = attend(widen(q_bits[s, h], dtype), keys, values, scale)
     return out
+
+
+def paged_attention_prefill_fp8(q_bits, k_codes, v_codes, block_tables, context_lens, query_start,
+                                scale, k_scales, v_scales, num_kv_heads, block_size, dtype,
+                                rows=None):
+    """Chunked-prefill attention over E4M3 caches: for new token j of sequence
+    s, at position p = C_s - q_len_s + j, the textbook attention of
+    ``oracle.attention`` over tokens 0..p with values decode(code) * scale of
+    their kv head, in float64 (the causal reading of
+    ``oracle.attention.paged_attention_prefill``).  ``rows`` (iterable of
+    (token, head)) restricts the computation; other rows are NaN."""
+    from .attention import attend, kv_head_of, token_location
+    from .dtypes import widen
+    total, num_heads, head_dim = q_bits.shape
+    ks, vs = per_head(k_scales, num_kv_heads), per_head(v_scales, num_kv_heads)
+    query_start = np.asarray(query_start, dtype=np.int64)
+    seq_of = np.repeat(np.arange(len(query_start) - 1), np.diff(query_start))
+    if rows is None:
+        rows = [(t, h) for t in range(total) for h in range(num_heads)]
+    out = np.full((total, num_heads, head_dim), np.nan, dtype=np.float64)
+    for t, h in rows:
+        s = int(seq_of[t])
+        c = int(context_lens[s])
+        pos = c - int(query_start[s + 1] - query_start[s]) + (t - int(query_start[s]))
+        g = kv_head_of(h, num_heads, num_kv_heads)
+        blocks, offsets = token_location(np.asarray(block_tables[s]), np.arange(pos + 1),
+                                         block_size)
+        keys = dequantize(k_codes[blocks, g, offsets, :], ks[g])
+        values = dequantize(v_codes[blocks, g, offsets, :], vs[g])
+        out[t, h] = attend(widen(q_bits[t, h], dtype), keys, values, scale)
+    return out

@@ -72,27 +72,28 @@ struct TcEntry {
 template <class DT>
 constexpr int kTcQueryTiles = 2;
 
-template <int BS, int G, class DT>
+template <int BS, int G, class DT, bool FP8>
 TcEntry make_tc() {
-  using Tr = TcPrefillTraits<BS, G, DT, kTcQueryTiles<DT>>;
+  using Tr = TcPrefillTraits<BS, G, DT, kTcQueryTiles<DT>, false, FP8>;
   return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(), Tr::ROWS};
 }
 
-template <int BS, class DT>
+template <int BS, class DT, bool FP8>
 TcEntry tc_group(int g) {
   switch (g) {
-    case 1: return make_tc<BS, 1, DT>();
-    case 2: return make_tc<BS, 2, DT>();
-    case 4: return make_tc<BS, 4, DT>();
-    case 8: return make_tc<BS, 8, DT>();
+    case 1: return make_tc<BS, 1, DT, FP8>();
+    case 2: return make_tc<BS, 2, DT, FP8>();
+    case 4: return make_tc<BS, 4, DT, FP8>();
+    case 8: return make_tc<BS, 8, DT, FP8>();
     default: return TcEntry{nullptr, 0, 0, 0};
   }
 }
 
-template <class DT>
+// (block size, group) -> tcgen05 kernel; fp8: the cache holds E4M3 codes
+template <class DT, bool FP8 = false>
 TcEntry tc_for(int bs, int g) {
-  if (bs == 16) return tc_group<16, DT>(g);
-  if (bs == 32) return tc_group<32, DT>(g);
+  if (bs == 16) return tc_group<16, DT, FP8>(g);
+  if (bs == 32) return tc_group<32, DT, FP8>(g);
   return TcEntry{nullptr, 0, 0, 0};
 }
 
@@ -222,14 +223,18 @@ pkv_status launch_cascade_prefix(const void* q, const void* k_cache, const void*
 
 }  // namespace pkv
 
-extern "C" pkv_status pkv_paged_attn_prefill(
-    void* out, const void* q, const void* k_cache, const void* v_cache,
-    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
-    float scale, int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim,
-    int block_size,
-    int max_blocks_per_seq, int max_context_len, int max_query_len, int num_blocks,
-    pkv_dtype dtype, unsigned* dev_err, void* stream) {
-  using namespace pkv;
+namespace pkv {
+namespace {
+
+// Validates and launches prefill; fp8: the caches hold E4M3 codes (head_dim
+// 128, the tcgen05 kernel) with per-kv-head scales k_scales / v_scales.
+pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          const int32_t* query_start, float scale, int num_seqs, int num_tokens,
+                          int num_heads, int num_kv_heads, int head_dim, int block_size,
+                          int max_blocks_per_seq, int max_context_len, int max_query_len,
+                          int num_blocks, pkv_dtype dtype, bool fp8, const float* k_scales,
+                          const float* v_scales, unsigned* dev_err, void* stream) {
   if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
       max_blocks_per_seq <= 0 ||
       max_context_len < 0 || max_query_len < 0 || num_blocks <= 0 || !dtype_valid(dtype) ||
@@ -239,9 +244,11 @@ extern "C" pkv_status pkv_paged_attn_prefill(
     return PKV_ERR_UNSUPPORTED;
   const int group = num_heads / num_kv_heads;
   if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
+  if (fp8 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
   if (static_cast<long long>(max_context_len) >
       static_cast<long long>(max_blocks_per_seq) * block_size)
     return PKV_ERR_INVALID_ARG;
+  if (fp8 && (!k_scales || !v_scales)) return PKV_ERR_INVALID_ARG;
   if (num_seqs == 0 || max_query_len == 0 || num_tokens == 0) return PKV_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
     return PKV_ERR_INVALID_ARG;
@@ -252,6 +259,8 @@ extern "C" pkv_status pkv_paged_attn_prefill(
                           : dtype == PKV_FP16 ? prefill_for<Fp16>(head_dim, block_size, group)
                                               : prefill_for<Bf16>(head_dim, block_size, group);
   const TcEntry te = !use_tc ? TcEntry{nullptr, 0, 0, 0}
+                     : fp8 ? (dtype == PKV_FP16 ? tc_for<Fp16, true>(block_size, group)
+                                                : tc_for<Bf16, true>(block_size, group))
                      : dtype == PKV_FP16 ? tc_for<Fp16>(block_size, group)
                                          : tc_for<Bf16>(block_size, group);
   if (pe.fn == nullptr && te.fn == nullptr) return PKV_ERR_UNSUPPORTED;
@@ -262,10 +271,11 @@ extern "C" pkv_status pkv_paged_attn_prefill(
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
   CUtensorMap kmap, vmap, qmap;
+  const pkv_dtype cdt = fp8 ? PKV_FP8_E4M3 : dtype;  // element type of the caches
   pkv_status st =
-      cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
+      cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, head_dim, cdt);
   if (st != PKV_OK) return st;
-  st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, head_dim, dtype);
+  st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, head_dim, cdt);
   if (st != PKV_OK) return st;
   if (use_tc) {
     st = q_tensor_map(&qmap, q, num_tokens, num_heads, group, dtype);
@@ -296,6 +306,8 @@ extern "C" pkv_status pkv_paged_attn_prefill(
   p.num_blocks = num_blocks;
   p.q_tiles = q_tiles;
   p.err = dev_err;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
 
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -309,4 +321,32 @@ extern "C" pkv_status pkv_paged_attn_prefill(
   cfg.numAttrs = 1;
   if (use_tc) return cuda_status(cudaLaunchKernelEx(&cfg, te.fn, p, qmap, kmap, vmap));
   return cuda_status(cudaLaunchKernelEx(&cfg, pe.fn, p, kmap, vmap));
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attn_prefill(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+    float scale, int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim,
+    int block_size, int max_blocks_per_seq, int max_context_len, int max_query_len,
+    int num_blocks, pkv_dtype dtype, unsigned* dev_err, void* stream) {
+  return pkv::prefill_launch(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                             scale, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, max_context_len, max_query_len,
+                             num_blocks, dtype, false, nullptr, nullptr, dev_err, stream);
+}
+
+extern "C" pkv_status pkv_paged_attn_prefill_fp8(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+    float scale, const float* k_scales, const float* v_scales, int num_seqs, int num_tokens,
+    int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+    int max_context_len, int max_query_len, int num_blocks, pkv_dtype dtype, unsigned* dev_err,
+    void* stream) {
+  return pkv::prefill_launch(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                             scale, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, max_context_len, max_query_len,
+                             num_blocks, dtype, true, k_scales, v_scales, dev_err, stream);
 }

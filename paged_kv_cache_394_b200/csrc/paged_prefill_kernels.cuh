@@ -47,6 +47,9 @@ struct PrefillParams {
   int num_blocks;
   int q_tiles;  // query tiles per (sequence, kv head) at max_query_len
   unsigned* err;
+  // E4M3 caches (tcgen05 kernel): per-kv-head scales, value = code x scale
+  const float* k_scales;  // [num_kv_heads]
+  const float* v_scales;  // [num_kv_heads]
   // Shared-prefix pass of cascade decode (tcgen05 kernel in prefix mode): the
   // units are groups of sequences instead of sequences, the queries are the
   // members' decode queries, the keys the group's shared_blocks[g] leading

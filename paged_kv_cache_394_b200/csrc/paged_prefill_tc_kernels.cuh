@@ -180,14 +180,32 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Two E4M3 codes (low bytes first) -> two values packed as fp16x2 or bf16x2;
+// exact, since every E4M3 value is an fp16 and a bf16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t two, Fp16) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
+      : "=r"(r)
+      : "r"(two));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t two, Bf16) {
+  const uint32_t h = e4m3x2_to(two, Fp16());
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack2(f.x, f.y, Bf16());
+}
+
 }  // namespace tc
 
-template <int BS_, int G_, class DT_, int QT_, bool PREFIX_ = false>
+template <int BS_, int G_, class DT_, int QT_, bool PREFIX_ = false, bool FP8_ = false>
 struct TcPrefillTraits {
   static constexpr int D = 128, BS = BS_, G = G_, QT = QT_;
   // prefix mode: the shared-prefix pass of cascade decode (no causal mask,
   // split-K partials out; see PrefillParams)
   static constexpr bool kPrefix = PREFIX_;
+  // E4M3 cache: the producer warps stage each tile's codes by TMA and widen
+  // them into the 16-bit stage the MMAs read; K and V scales are per kv head
+  static constexpr bool kFp8 = FP8_;
   using DT = DT_;
   using T = typename DT::T;
   static constexpr bool kBf16 = std::is_same<DT, Bf16>::value;
@@ -195,7 +213,8 @@ struct TcPrefillTraits {
   static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
   static constexpr int NKEY = 64;                // keys per KV tile
   // KV stages: what fits beside QT query tiles (P lives in TMEM, over S)
-  static constexpr int NS = QT == 2 ? 5 : 6;
+  static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : 6;
+  static constexpr int NSTG = kFp8 ? 2 : 0;      // E4M3 staging slots per kind
   // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
   // P.V issuer
   static constexpr int PV_WARP = 3 + 4 * QT;
@@ -207,10 +226,13 @@ struct TcPrefillTraits {
   static constexpr int STAGE = 4 * KV_HALF;      // K0 K1 V0 V1
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QT * Q_TILE;
-  static constexpr int OFF_BAR = OFF_KV + NS * STAGE;
+  static constexpr int STG_TILE = NKEY * 128;   // [64 keys][128 codes], 128-byte swizzle
+  static constexpr int OFF_STG = OFF_KV + NS * STAGE;            // K slots, then V slots
+  static constexpr int OFF_BAR = OFF_STG + 2 * NSTG * STG_TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
-  // per query tile s_full[2], p_full[2], o_done[2]; then the TMEM address slot
-  static constexpr int NBAR = 1 + 4 * NS + 6 * QT;
+  // per query tile s_full[2], p_full[2], o_done[2]; then (E4M3) the staging
+  // slots' stg_full[2][NSTG]; then the TMEM address slot
+  static constexpr int NBAR = 1 + 4 * NS + 6 * QT + 2 * NSTG;
   // the softmax reference max moves only when a row max exceeds it by more
   // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
   static constexpr float kRescaleThreshold = 8.f;
@@ -218,6 +240,7 @@ struct TcPrefillTraits {
   // per query tile q: S buffers at 256q and 256q + 64, O at 256q + 128
   static constexpr uint32_t TMEM_COLS = 256 * QT;
   static_assert(QT == 1 || QT == 2, "one or two query tiles per CTA");
+  static_assert(!(kFp8 && kPrefix), "the cascade prefix pass reads 16-bit caches");
   static_assert(1024 + SMEM <= 232448, "shared memory per CTA");
   static size_t smem_bytes() { return 1024 + static_cast<size_t>(SMEM); }
 };
@@ -246,6 +269,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   auto bar_s_full = [&](int q, int b) { return smem_addr(bars + 1 + 4 * NS + 6 * q + b); };
   auto bar_p = [&](int q, int b) { return smem_addr(bars + 3 + 4 * NS + 6 * q + b); };
   auto bar_o = [&](int q, int b) { return smem_addr(bars + 5 + 4 * NS + 6 * q + b); };
+  auto bar_stg = [&](int kind, int s) {
+    return smem_addr(bars + 1 + 4 * NS + 6 * QT + kind * Tr::NSTG + s);
+  };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
 
   const int tile = p.q_tiles - 1 - static_cast<int>(blockIdx.x % p.q_tiles);
@@ -302,6 +328,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         mbar_init(bar_o(q, b), 1);
       }
     }
+    for (int s = 0; s < Tr::NSTG; ++s) {
+      mbar_init(bar_stg(0, s), 1);
+      mbar_init(bar_stg(1, s), 1);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -333,19 +363,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       }
     }
     int chunk = -1, entry = -1;
-    for (int t = 0; t < ntiles; ++t) {
-      const int stage = t % NS;
-      bool ok = true;
-      if (lane == 0) {
-        ok = mbar_wait_bounded(is_k ? bar_k_empty(stage) : bar_v_empty(stage),
-                               ((t / NS) & 1) ^ 1);
-        if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
-      }
-      ok = __shfl_sync(kFullMask, ok, 0);
-      if (!ok) break;
-      // the 16-key pieces of this tile that hold keys this CTA needs
+    // the 16-key pieces of tile t that hold keys this CTA needs (pb = -1 past
+    // them); t must not decrease from call to call (the table is read in
+    // 32-entry chunks)
+    auto lookup = [&](int t, int (&pb)[4]) {
       int npieces = 0;
-      int pb[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int key0 = t * NKEY + i * 16;
@@ -361,39 +383,162 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           npieces = i + 1;
         }
       }
-      int bytes = 0;
+      return npieces;
+    };
+    auto valid_block = [&](int b) {
+      return static_cast<unsigned>(b) < static_cast<unsigned>(p.num_blocks);
+    };
+    if constexpr (Tr::kFp8) {
+      // E4M3: TMA brings tile t's codes into staging slot t % NSTG (one box of
+      // 16 rows x 128 codes per piece); once a 16-bit stage is free the warp
+      // widens them into it, signals the MMAs, and refills the slot with tile
+      // t + NSTG.
+      const int kind = is_k ? 0 : 1;
+      const uint32_t stg0 = sbase + Tr::OFF_STG + kind * Tr::NSTG * Tr::STG_TILE;
+      auto stage_codes = [&](int t) {  // all lanes (the table lookup is warp-wide)
+        int pb[4];
+        const int npieces = lookup(t, pb);
+        int bytes = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
-          bytes += 2 * 2048;
-      const uint32_t bar = is_k ? bar_k_full(stage) : bar_v_full(stage);
-      if (lane == 0) {
-        for (int i = 0; i < npieces; ++i)
-          if (is_k && static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks))
-            set_err(p.err, PKV_DEVERR_BAD_BLOCK);
-        if (bytes > 0)
-          mbar_arrive_expect_tx(bar, bytes);
-        else
-          mbar_arrive(bar);
-      }
-      __syncwarp();
-      // lanes 0..7 issue the tile's 8 boxes of K (or V) at once: lane = piece * 2 +
-      // half; kind 0 / 1 = K low / high dims, 2 / 3 = V low / high dims
-      if (lane < 8) {
-        const int i = lane >> 1, kind = (is_k ? 0 : 2) + (lane & 1);
-        int pbi = pb[0];
-        if (i == 1) pbi = pb[1];
-        if (i == 2) pbi = pb[2];
-        if (i == 3) pbi = pb[3];
-        if (i < npieces && static_cast<unsigned>(pbi) < static_cast<unsigned>(p.num_blocks)) {
-          const uint32_t st = sbase + Tr::OFF_KV + stage * Tr::STAGE;
-          const int key0 = t * NKEY + i * 16;
-          const int y = (pbi * p.num_kv_heads + kvh) * BS + (key0 % BS);
-          tma_load_2d(st + kind * Tr::KV_HALF + i * 2048, kind < 2 ? &kmap : &vmap,
-                      (kind & 1) * 64, y, bar);
+        for (int i = 0; i < 4; ++i)
+          if (i < npieces && valid_block(pb[i])) bytes += 2048;
+        const uint32_t bar = bar_stg(kind, t % Tr::NSTG);
+        if (lane == 0) {
+          for (int i = 0; i < npieces; ++i)
+            if (is_k && !valid_block(pb[i])) set_err(p.err, PKV_DEVERR_BAD_BLOCK);
+          if (bytes > 0)
+            mbar_arrive_expect_tx(bar, bytes);
+          else
+            mbar_arrive(bar);
         }
+        __syncwarp();
+        if (lane < 4) {
+          int pbi = pb[0];
+          if (lane == 1) pbi = pb[1];
+          if (lane == 2) pbi = pb[2];
+          if (lane == 3) pbi = pb[3];
+          if (lane < npieces && valid_block(pbi)) {
+            const int key0 = t * NKEY + lane * 16;
+            const int y = (pbi * p.num_kv_heads + kvh) * BS + (key0 % BS);
+            tma_load_2d(stg0 + (t % Tr::NSTG) * Tr::STG_TILE + lane * 2048,
+                        is_k ? &kmap : &vmap, 0, y, bar);
+          }
+        }
+        __syncwarp();
+      };
+      for (int t = 0; t < min(Tr::NSTG, ntiles); ++t) stage_codes(t);
+      for (int t = 0; t < ntiles; ++t) {
+        const int stage = t % NS;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(is_k ? bar_k_empty(stage) : bar_v_empty(stage),
+                                 ((t / NS) & 1) ^ 1) &&
+               mbar_wait_bounded(bar_stg(kind, t % Tr::NSTG), (t / Tr::NSTG) & 1);
+          if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
+        }
+        ok = __shfl_sync(kFullMask, ok, 0);
+        if (!ok) break;
+        // 64 rows x 8 chunks of 16 codes; lane takes chunks lane, lane + 32, ...
+        // Chunk c of row r (dims 16c .. 16c + 15) becomes 16-bit chunks 2(c % 4)
+        // and 2(c % 4) + 1 of row r in dim half c / 4; both layouts use the
+        // 128-byte swizzle (16-byte chunk index XOR row % 8).
+        const uint32_t src = stg0 + (t % Tr::NSTG) * Tr::STG_TILE;
+        const uint32_t dst = sbase + Tr::OFF_KV + stage * Tr::STAGE + (is_k ? 0 : 2 * Tr::KV_HALF);
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+          const int idx = lane + 32 * k;
+          const int r = idx >> 3, c = idx & 7;
+          uint32_t w[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                       : "r"(src + r * 128 + ((c ^ (r & 7)) << 4))
+                       : "memory");
+          uint32_t h[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            h[2 * e] = tc::e4m3x2_to(w[e] & 0xffffu, DT());
+            h[2 * e + 1] = tc::e4m3x2_to(w[e] >> 16, DT());
+          }
+          const uint32_t row = dst + (c >> 2) * Tr::KV_HALF + r * 128;
+          const int c0 = (c & 3) * 2;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((c0 ^ (r & 7)) << 4)),
+                       "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           row + (((c0 + 1) ^ (r & 7)) << 4)),
+                       "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                       : "memory");
+        }
+        // the widened tile is for the MMAs (async proxy); the slot's codes are
+        // read, so TMA may refill it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(is_k ? bar_k_full(stage) : bar_v_full(stage));
+        if (t + Tr::NSTG < ntiles) stage_codes(t + Tr::NSTG);
       }
-      __syncwarp();
+    } else {
+      for (int t = 0; t < ntiles; ++t) {
+        const int stage = t % NS;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(is_k ? bar_k_empty(stage) : bar_v_empty(stage),
+                                 ((t / NS) & 1) ^ 1);
+          if (!ok) set_err(p.err, PKV_DEVERR_TIMEOUT);
+        }
+        ok = __shfl_sync(kFullMask, ok, 0);
+        if (!ok) break;
+        // the 16-key pieces of this tile that hold keys this CTA needs
+        int npieces = 0;
+        int pb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int key0 = t * NKEY + i * 16;
+          pb[i] = -1;
+          if (key0 < nkv) {
+            const int blk = key0 / BS;
+            if ((blk >> 5) != chunk) {
+              chunk = blk >> 5;
+              const int idx = (chunk << 5) + lane;
+              entry = idx < nblk ? trow[idx] : -1;
+            }
+            pb[i] = __shfl_sync(kFullMask, entry, blk & 31);
+            npieces = i + 1;
+          }
+        }
+        int bytes = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
+            bytes += 2 * 2048;
+        const uint32_t bar = is_k ? bar_k_full(stage) : bar_v_full(stage);
+        if (lane == 0) {
+          for (int i = 0; i < npieces; ++i)
+            if (is_k && static_cast<unsigned>(pb[i]) >= static_cast<unsigned>(p.num_blocks))
+              set_err(p.err, PKV_DEVERR_BAD_BLOCK);
+          if (bytes > 0)
+            mbar_arrive_expect_tx(bar, bytes);
+          else
+            mbar_arrive(bar);
+        }
+        __syncwarp();
+        // lanes 0..7 issue the tile's 8 boxes of K (or V) at once: lane = piece * 2 +
+        // half; kind 0 / 1 = K low / high dims, 2 / 3 = V low / high dims
+        if (lane < 8) {
+          const int i = lane >> 1, kind = (is_k ? 0 : 2) + (lane & 1);
+          int pbi = pb[0];
+          if (i == 1) pbi = pb[1];
+          if (i == 2) pbi = pb[2];
+          if (i == 3) pbi = pb[3];
+          if (i < npieces && static_cast<unsigned>(pbi) < static_cast<unsigned>(p.num_blocks)) {
+            const uint32_t st = sbase + Tr::OFF_KV + stage * Tr::STAGE;
+            const int key0 = t * NKEY + i * 16;
+            const int y = (pbi * p.num_kv_heads + kvh) * BS + (key0 % BS);
+            tma_load_2d(st + kind * Tr::KV_HALF + i * 2048, kind < 2 ? &kmap : &vmap,
+                        (kind & 1) * 64, y, bar);
+          }
+        }
+        __syncwarp();
+      }
     }
   } else if (warp == 1 || warp == Tr::PV_WARP) {
     // ---- MMA issuers ----------------------------------------------------------------
@@ -491,6 +636,16 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const int g = crow % G;
     const int pos = !active ? -1 : Tr::kPrefix ? ctx - 1 : ctx - q_len + j;
     const int my_tiles = qg == 0 ? ntq[0] : ntq[QT - 1];
+    // E4M3: a cached value is code x scale; the K scale folds into the logit
+    // scale and the V scale into the final normalisation
+    float k_scale = 1.f, v_scale = 1.f;
+    if constexpr (Tr::kFp8) {
+      k_scale = p.k_scales[kvh];
+      v_scale = p.v_scales[kvh];
+      if (!(k_scale > 0.f && k_scale < INFINITY && v_scale > 0.f && v_scale < INFINITY) &&
+          warp == 3 && lane == 0 && tile == 0)
+        set_err(p.err, PKV_DEVERR_BAD_SCALE);
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < my_tiles; ++t) {
@@ -513,7 +668,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       // Scaled logits are x = s * qscale.  For qscale > 0 the row max of x is
       // (max s) * qscale exactly, so s is masked and reduced unscaled and the
       // scale folds into the exponent's FFMA: p = 2^(s * qscale - m).
-      float mult = p.qscale;
+      float mult = p.qscale * k_scale;
       const bool needs_mask = kv0 + NKEY - 1 > pos;  // this tile reaches past the row
       if (mult > 0.f) {
         if (needs_mask) {
@@ -650,7 +805,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       }
     } else if (ok && my_tiles > 0) {
       tc::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? v_scale / l : 0.f;
       T* orow = static_cast<T*>(p.out) +
                 (static_cast<size_t>(q0 + j) * p.num_heads + kvh * G + g) * Tr::D;
 #pragma unroll 1

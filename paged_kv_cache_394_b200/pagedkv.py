@@ -61,6 +61,9 @@ _paged_attn_decode_fp8 = _proto("pkv_paged_attn_decode_fp8", _i, _vp, _vp, _vp, 
                                 _vp)
 _paged_attn_prefill = _proto("pkv_paged_attn_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i,
                              _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp)
+_paged_attn_prefill_fp8 = _proto("pkv_paged_attn_prefill_fp8", _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                 _vp, _vp)
 _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
 _decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
                            _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
@@ -392,6 +395,36 @@ def paged_attn_prefill(out, q, k_cache, v_cache, block_tables, context_lens, que
                                max_context_len, max_query_len, num_blocks, _dtype_code(q),
                                _ptr(dev_err), _stream(stream)),
            "paged_attn_prefill")
+
+
+def paged_attn_prefill_fp8(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                           scale, k_scales, v_scales, num_kv_heads, block_size, max_context_len,
+                           max_query_len, dev_err=None, stream=None):
+    """Chunked-prefill attention over E4M3 caches (values = code * scale of the
+    kv head); q and out are 16-bit, head_dim 128.  See include/pagedkv.h."""
+    for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dev(t, n)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    _dev(query_start, "query_start", torch.int32)
+    t, h, d = q.shape
+    num_blocks, hkv, bs, dk = k_cache.shape
+    s = context_lens.shape[0]
+    if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if query_start.shape != (s + 1,) or block_tables.shape[0] != s:
+        raise ValueError("query_start must be [S+1], block_tables [S, max_blocks]")
+    if _cache_dtype_code(k_cache) != FP8_E4M3 or v_cache.dtype != k_cache.dtype:
+        raise TypeError("E4M3 caches must be uint8 (or float8_e4m3fn)")
+    if out.dtype != q.dtype:
+        raise TypeError("q and out must share a dtype")
+    ks, vs = _scales_for(k_scales, v_scales, hkv, q.device, stream)
+    _check(_paged_attn_prefill_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
+                                   float(scale), _ptr(ks), _ptr(vs), s, t, h, hkv, d, bs,
+                                   block_tables.shape[1], max_context_len, max_query_len,
+                                   num_blocks, _dtype_code(q), _ptr(dev_err), _stream(stream)),
+           "paged_attn_prefill_fp8")
 
 
 def staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,

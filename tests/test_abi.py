@@ -146,6 +146,25 @@ def test_fp8_host_validation_without_gpu():
     assert dec8(ptr=bad) == pk.ERR_INVALID_ARG
 
 
+def test_prefill_fp8_host_validation_without_gpu():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    null = None
+    good = ctypes.c_void_p(0x1000)
+    bad = ctypes.c_void_p(0x1008)
+
+    def pre8(ks=good, vs=good, d=128, h=4, dt=pk.FP16, s=2, ptr=good):
+        # out q k v tables lens qstart scale ks vs S T H Hkv D bs maxblk maxctx maxq nblk dt
+        return pk._paged_attn_prefill_fp8(ptr, ptr, ptr, ptr, ptr, ptr, ptr, 0.125, ks, vs, s, 8,
+                                          h, 2, d, 16, 4, 64, 4, 8, dt, null, null)
+    assert pre8(d=64) == pk.ERR_UNSUPPORTED               # E4M3 prefill: head_dim 128 only
+    assert pre8(h=6) == pk.ERR_UNSUPPORTED                # G = 3
+    assert pre8(ks=null) == pk.ERR_INVALID_ARG
+    assert pre8(vs=null) == pk.ERR_INVALID_ARG
+    assert pre8(dt=pk.FP8_E4M3) == pk.ERR_INVALID_ARG     # q/out must be 16-bit
+    assert pre8(s=0) == pk.OK
+    assert pre8(ptr=bad) == pk.ERR_INVALID_ARG
+
+
 def test_binding_constants_match_the_header():
     """Status codes, dtype codes and device error bits of the binding equal
     the values include/pagedkv.h defines."""

@@ -104,6 +104,52 @@ def test_fp8_decode_reduces_to_16bit_decode_on_exact_values():
     np.testing.assert_allclose(got2, 4.0 * ref2, rtol=1e-12, atol=1e-12)
 
 
+def test_fp8_prefill_reduces_to_16bit_prefill_on_exact_values():
+    """The same reduction for chunked prefill: on values exact in both formats
+    the E4M3 prefill (scales 1) equals the independently pinned 16-bit prefill
+    oracle, including causal rows and a ragged query split, and power-of-two
+    scales act as the softmax scale and an output factor."""
+    from oracle import attention as OA
+    from oracle.fp8 import paged_attention_prefill_fp8
+    rng = np.random.default_rng(8)
+    nb, hkv, bs, d, h = 12, 2, 16, 64, 4
+    kv = _exact_fp8_values(rng, (2, nb, hkv, bs, d))
+    codes = e4m3_encode(kv.astype(np.float32))
+    bits = kv.astype(np.float16).view(np.uint16)
+    tables = np.stack([rng.permutation(nb)[:4] for _ in range(3)]).astype(np.int32)
+    lens = np.array([5, 37, 64], dtype=np.int32)
+    qstart = np.array([0, 5, 8, 20], dtype=np.int32)        # a whole prompt, then chunks
+    q = rng.standard_normal((20, h, d)).astype(np.float16).view(np.uint16)
+    ref = OA.paged_attention_prefill(q, bits[0], bits[1], tables, lens, qstart, 0.125, hkv, bs,
+                                     "fp16")
+    got = paged_attention_prefill_fp8(q, codes[0], codes[1], tables, lens, qstart, 0.125, 1.0,
+                                      1.0, hkv, bs, "fp16")
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+    got2 = paged_attention_prefill_fp8(q, codes[0], codes[1], tables, lens, qstart, 0.125, 2.0,
+                                       4.0, hkv, bs, "fp16")
+    ref2 = OA.paged_attention_prefill(q, bits[0], bits[1], tables, lens, qstart, 0.25, hkv, bs,
+                                      "fp16")
+    np.testing.assert_allclose(got2, 4.0 * ref2, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_prefill_of_one_query_is_decode():
+    """A single new token per sequence is decode (the last cached position)."""
+    from oracle.fp8 import paged_attention_decode_fp8, paged_attention_prefill_fp8
+    rng = np.random.default_rng(9)
+    nb, hkv, bs, d, h = 10, 2, 16, 64, 4
+    codes = rng.integers(0, 256, size=(2, nb, hkv, bs, d)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38                    # no NaN codes
+    tables = np.stack([rng.permutation(nb)[:4] for _ in range(3)]).astype(np.int32)
+    lens = np.array([1, 30, 64], dtype=np.int32)
+    q = rng.standard_normal((3, h, d)).astype(np.float16).view(np.uint16)
+    ks, vs = np.array([0.01, 0.02], np.float32), np.array([0.03, 0.005], np.float32)
+    got = paged_attention_prefill_fp8(q, codes[0], codes[1], tables, lens, np.arange(4), 0.125,
+                                      ks, vs, hkv, bs, "fp16")
+    ref = paged_attention_decode_fp8(q, codes[0], codes[1], tables, lens, 0.125, ks, vs, hkv, bs,
+                                     "fp16")
+    np.testing.assert_array_equal(got, ref)
+
+
 def test_quantize_into_cache_places_codes_like_the_16bit_write():
     from oracle import cache_ops as OC
     from oracle.fp8 import quantize, quantize_into_cache

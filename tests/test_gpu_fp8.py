@@ -90,6 +90,27 @@ class Fp8Device:
         return int(self.err.item())
 
 
+def run_prefill8(pk, dev):
+    """The quantising write of the new tokens, then E4M3 chunked prefill."""
+    w = dev.w
+    pk.reshape_and_cache_fp8(dev.key, dev.value, dev.k8, dev.v8, dev.slots, dev.ks, dev.vs,
+                             dev_err=dev.err)
+    qstart = torch.from_numpy(w.query_start).cuda()
+    pk.paged_attn_prefill_fp8(dev.out, dev.q, dev.k8, dev.v8, dev.tables, dev.lens, qstart,
+                              w.scale, dev.ks, dev.vs, w.num_kv_heads, w.block_size,
+                              w.max_context_len, int(np.diff(w.query_start).max()),
+                              dev_err=dev.err)
+    torch.cuda.synchronize()
+    return int(dev.err.item())
+
+
+def oracle_prefill8(w, kq, vq, rows=None):
+    return OF.paged_attention_prefill_fp8(w.q, kq, vq, w.block_tables, w.context_lens,
+                                          w.query_start, w.scale, k_scales_for(w),
+                                          v_scales_for(w), w.num_kv_heads, w.block_size,
+                                          w.dtype, rows=rows)
+
+
 def oracle_codes(w, k_scales=None, v_scales=None, blocks=None):
     """The oracle's E4M3 caches after the step: the pool quantised, the CoW
     copies, then the new tokens quantised into their slots.  With ``blocks``
@@ -255,4 +276,71 @@ def test_fp8_named_workload_full_size(pk, name):
     assert np.array_equal(dev.k8[bt].cpu().numpy(), kq[blocks])
     assert np.array_equal(dev.v8[bt].cpu().numpy(), vq[blocks])
     assert_close(dev_to_bits(dev.out), oracle_decode8(w, kq, vq, pairs=pairs), w, pairs=pairs)
+    assert torch.isfinite(dev.out.float()).all()
+
+
+PREFILL_HIST = [0, 5, 16, 40, 100, 0]
+PREFILL_NEW = [1, 17, 16, 33, 64, 70]
+PREFILL_SHAPES = [(16, 1, "fp16"), (32, 2, "bf16"), (16, 4, "bf16"), (32, 8, "fp16"),
+                  (16, 8, "bf16"), (32, 1, "fp16"), (16, 2, "fp16"), (32, 4, "bf16")]
+
+
+@pytest.mark.parametrize("bs,g,dtype", PREFILL_SHAPES)
+def test_fp8_prefill_small(pk, bs, g, dtype):
+    """Whole prompts and chunks on short and empty histories, every group size
+    and block size, ragged query tiles (70 new tokens x G heads)."""
+    w = W.build_prefill_workload(PREFILL_HIST, PREFILL_NEW, 2 * g, 2, 128, bs, dtype,
+                                 seed=31 + bs + g)
+    dev = Fp8Device(pk, w)
+    assert run_prefill8(pk, dev) == 0
+    kq, vq = oracle_codes(w)
+    assert np.array_equal(dev.k8.cpu().numpy(), kq)
+    assert np.array_equal(dev.v8.cpu().numpy(), vq)
+    assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq), w)
+
+
+def test_fp8_prefill_long_history_sampled(pk):
+    w = W.build_prefill_workload([3000, 0, 777], [200, 300, 129], 16, 4, 128, 16, "bf16", seed=6)
+    dev = Fp8Device(pk, w)
+    assert run_prefill8(pk, dev) == 0
+    kq, vq = oracle_codes(w)
+    rng = np.random.default_rng(1)
+    rows = sorted({(int(t), int(h)) for t, h in zip(rng.integers(0, 629, 40),
+                                                    rng.integers(0, 16, 40))}
+                  | {(0, 0), (199, 15), (200, 3), (628, 7)})
+    assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq, rows), w, pairs=rows)
+
+
+def test_fp8_prefill_of_one_token_matches_fp8_decode(pk):
+    w = W.build_decode_workload(RAGGED, 8, 2, 128, 16, "fp16", 23)
+    w.query_start = np.arange(w.num_seqs + 1, dtype=np.int32)
+    dev = Fp8Device(pk, w)
+    assert run_prefill8(pk, dev) == 0
+    kq, vq = oracle_codes(w)
+    assert_close(dev_to_bits(dev.out), oracle_decode8(w, kq, vq), w)
+
+
+def test_fp8_prefill_reports_a_bad_scale(pk):
+    w = W.build_prefill_workload([4, 10], [3, 5], 4, 2, 128, 16, "fp16", seed=2)
+    dev = Fp8Device(pk, w)
+    dev.vs = torch.tensor([0.01, 0.0], dtype=torch.float32, device="cuda")
+    assert run_prefill8(pk, dev) & pk.DEVERR_BAD_SCALE
+
+
+def test_fp8_prefill_named_workload_sampled(pk):
+    """The LLaMA-7B prefill batch at full size, on sampled rows."""
+    w = W.make("llama7b_prefill")
+    dev = Fp8Device(pk, w)
+    assert run_prefill8(pk, dev) == 0
+    rng = np.random.default_rng(4)
+    total = int(w.query_start[-1])
+    rows = sorted({(int(t), int(h)) for t, h in zip(rng.integers(0, total, 24),
+                                                    rng.integers(0, w.num_heads, 24))}
+                  | {(0, 0), (total - 1, w.num_heads - 1)})
+    seq_of = np.repeat(np.arange(w.num_seqs), np.diff(w.query_start))
+    seqs = sorted({int(seq_of[t]) for t, _ in rows})
+    blocks = np.unique(np.concatenate(
+        [w.block_tables[s, :-(-int(w.context_lens[s]) // w.block_size)] for s in seqs]))
+    kq, vq = oracle_codes(w, blocks=blocks)
+    assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq, rows), w, pairs=rows)
     assert torch.isfinite(dev.out.float()).all()

@@ -139,3 +139,27 @@ def test_unique_bytes_equal_logical_without_sharing():
     from paged_kv_cache_394_b200 import workloads as W
     w = W.make("tiny")
     assert bench.unique_decode_bytes(w) == bench.decode_bytes(w)
+
+
+@pytest.mark.parametrize("prompt_len,bs", [(37, 16), (64, 16), (100, 32)])
+def test_cascade_groups_share_exactly_their_whole_prompt_blocks(prompt_len, bs):
+    """Every member of a group has the same first shared_blocks[g] table
+    entries (the prompt's whole blocks), those blocks are shared by no other
+    group, and the next entry, if any, differs between members (a partial
+    prompt block is copied on write; divergent tokens get fresh blocks)."""
+    import numpy as np
+    from paged_kv_cache_394_b200 import workloads as W
+    w = W.build_prefix_share_workload(3, 4, prompt_len, 5, 40, 8, 2, 64, bs, "fp16", seed=7)
+    gs, shared = W.cascade_groups(w)
+    assert gs[0] == 0 and gs[-1] == w.num_seqs and (np.diff(gs) > 0).all()
+    seen = set()
+    for g in range(len(shared)):
+        rows = w.block_tables[gs[g]:gs[g + 1]]
+        n = int(shared[g])
+        assert n == prompt_len // bs
+        assert (rows[:, :n] == rows[0, :n]).all()
+        assert not seen & set(rows[0, :n].tolist())
+        seen |= set(rows[0, :n].tolist())
+        if rows.shape[1] > n and len(rows) > 1:
+            assert len(set(rows[:, n].tolist())) == len(rows)
+        assert (w.context_lens[gs[g]:gs[g + 1]] >= n * bs).all()

@@ -15,10 +15,14 @@ Sources, cited by page title and section throughout:
 
 Modules:
 
-* ``attention``      paged decode attention (direct and partitioned forms)
+* ``attention``      paged decode attention (direct and partitioned forms) and
+                     chunked-prefill attention
 * ``cache_ops``      the cache-write scatter and the copy-on-write block copy
-* ``block_manager``  the page allocator: free list, refcounts, sharing, CoW
+* ``block_manager``  the page allocator: free list, refcounts, sharing, CoW,
+                     prefix caching
 * ``dtypes``         exact widening of fp16/bf16 bit patterns to float64
+* ``fp8``            the E4M3 cache: encode / decode, the quantising write,
+                     decode and prefill over dequantised codes
 """
 
-from . import attention, block_manager, cache_ops, dtypes  # noqa: F401
+from . import attention, block_manager, cache_ops, dtypes, fp8  # noqa: F401

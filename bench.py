@@ -981,34 +981,140 @@ def run_serving_trace(args):
     print(json.dumps(line), flush=True)
 
 
+def oracle_sample_fp8(w, seconds, threads=None):
+    """oracle_sample over E4M3 caches: each sequence's blocks are quantised
+    (scale FP8_K_SCALE / FP8_V_SCALE, as in the device runs) and the float64
+    E4M3 decode oracle runs over them; the quantisation is timed too."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import cache_ops as OC
+    from oracle import fp8 as OF
+    cores = threads or len(os.sched_getaffinity(0))
+    done, nbytes = 0, 0
+    with threadpool_limits(limits=cores):
+        t0 = time.perf_counter()
+        kc, vc, _ = OC.copy_blocks(w.k_cache, w.v_cache, w.cow_pairs, inplace=True)
+        kc, vc, _ = OC.reshape_and_cache(w.key, w.value, kc, vc, w.slot_mapping, w.block_size,
+                                         inplace=True)
+        nbytes += write_bytes(w, 1) + copy_bytes(w, 1)
+        for s in range(w.num_seqs):
+            nblk = -(-int(w.context_lens[s]) // w.block_size)
+            blocks = w.block_tables[s, :nblk]
+            k8 = OF.quantize_cache(kc[blocks], w.dtype, FP8_K_SCALE)
+            v8 = OF.quantize_cache(vc[blocks], w.dtype, FP8_V_SCALE)
+            table = np.arange(nblk, dtype=np.int32)[None, :]
+            OF.paged_attention_decode_fp8(w.q[s:s + 1], k8, v8, table, w.context_lens[s:s + 1],
+                                          w.scale, FP8_K_SCALE, FP8_V_SCALE, w.num_kv_heads,
+                                          w.block_size, w.dtype)
+            done += 1
+            nbytes += (2 * int(w.context_lens[s]) * w.num_kv_heads * w.head_dim
+                       + 2 * w.num_heads * w.head_dim * 2)
+            if time.perf_counter() - t0 > seconds:
+                break
+        dt = time.perf_counter() - t0
+    return nbytes, dt, done, cores
+
+
+def oracle_sample_prefill(w, seconds, fp8=False, threads=None):
+    """Times the prefill oracle's step (the new tokens' cache write, then the
+    new tokens of the sequences in order, eight tokens x all heads at a time;
+    over E4M3 codes of each sequence's blocks when ``fp8``) until ``seconds``
+    have passed.  Returns the algorithmic FLOPs of the rows done (4 D per
+    (row, visible key)) and the number of sequences begun."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attention as OA
+    from oracle import cache_ops as OC
+    from oracle import fp8 as OF
+    cores = threads or len(os.sched_getaffinity(0))
+    begun, flops = 0, 0
+    with threadpool_limits(limits=cores):
+        t0 = time.perf_counter()
+        kc, vc, _ = OC.reshape_and_cache(w.key, w.value, w.k_cache, w.v_cache, w.slot_mapping,
+                                         w.block_size, inplace=True)
+        for s in range(w.num_seqs):
+            c = int(w.context_lens[s])
+            nblk = -(-c // w.block_size)
+            blocks = w.block_tables[s, :nblk]
+            table = np.arange(nblk, dtype=np.int32)[None, :]
+            q0, q1 = int(w.query_start[s]), int(w.query_start[s + 1])
+            qs = np.array([0, q1 - q0], dtype=np.int32)
+            if fp8:
+                k8 = OF.quantize_cache(kc[blocks], w.dtype, FP8_K_SCALE)
+                v8 = OF.quantize_cache(vc[blocks], w.dtype, FP8_V_SCALE)
+            begun += 1
+            for j0 in range(0, q1 - q0, 8):
+                rows = [(j, h) for j in range(j0, min(j0 + 8, q1 - q0))
+                        for h in range(w.num_heads)]
+                if fp8:
+                    OF.paged_attention_prefill_fp8(w.q[q0:q1], k8, v8, table,
+                                                   w.context_lens[s:s + 1], qs, w.scale,
+                                                   FP8_K_SCALE, FP8_V_SCALE, w.num_kv_heads,
+                                                   w.block_size, w.dtype, rows=rows)
+                else:
+                    OA.paged_attention_prefill(w.q[q0:q1], kc[blocks], vc[blocks], table,
+                                               w.context_lens[s:s + 1], qs, w.scale,
+                                               w.num_kv_heads, w.block_size, w.dtype, rows=rows)
+                pos0 = c - (q1 - q0)   # position of new token 0
+                flops += sum(4 * w.head_dim * (pos0 + j + 1) for j, _ in rows)
+                if time.perf_counter() - t0 > seconds:
+                    break
+            if time.perf_counter() - t0 > seconds:
+                break
+        dt = time.perf_counter() - t0
+    return flops, dt, begun, cores
+
+
 def run_reference(args):
+    """The reference arm: the float64 oracle, timed on the host cores over a
+    bounded sample of each step, for the same workload, metric and unit as
+    our arm (decode GB/s or prefill TFLOP/s; E4M3 over quantised codes;
+    cascade computes plain decode, so it times the decode oracle)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     from paged_kv_cache_394_b200 import workloads as W
-    w0 = W.make(args.workload)
+    fp8 = args.workload.endswith("_fp8")
+    name = args.workload.removesuffix("_fp8").removesuffix("_cascade")
+    prefill = name in W.PREFILL_NAMES
+    w0 = W.make(name)
+
+    def sample(seconds):
+        w = W.make(name)
+        if prefill:
+            return oracle_sample_prefill(w, seconds, fp8)
+        return oracle_sample_fp8(w, seconds) if fp8 else oracle_sample(w, seconds)
+
     for _ in range(args.warmup):
-        oracle_sample(W.make(args.workload), 0.5)
-    times, total_bytes, n_last, cores = [], 0, 0, 1
+        sample(0.5)
+    times, total, n_last, cores = [], 0, 0, 1
     for _ in range(args.steps):
-        w = W.make(args.workload)
-        nbytes, dt, n_last, cores = oracle_sample(w, args.cpu_seconds)
+        amount, dt, n_last, cores = sample(args.cpu_seconds)
         times.append(dt)
-        total_bytes += nbytes
-    value = total_bytes / sum(times) / 1e9
+        total += amount
+    if prefill:
+        value, unit = total / sum(times) / 1e12, "TFLOP/s"
+        metric = "paged-prefill attention TFLOP/s"
+        what = "the new tokens' cache write + float64 prefill of the new tokens (eight at a time) of the first"
+    else:
+        value, unit = total / sum(times) / 1e9, "GB/s"
+        metric = "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s"
+        what = "cache write + float64 decode of the first"
     line = {
         "impl": "reference",
-        "metric": "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s",
-        "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric,
+        "value": round(value, 6), "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1000 * statistics.mean(times), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": dict(W.describe(w0), parallelism="host cores"),
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+        "data": "synthetic",
+        "config": dict(W.describe(w0), workload=args.workload, parallelism="host cores"),
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores,
                          "kind": "oracle",
-                         "sample": "per step: cache write + float64 decode of the first %d of "
-                                   "%d sequences (all heads), bounded to %.0f s"
-                                   % (n_last, w0.num_seqs, args.cpu_seconds)},
-        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                         "sample": "per step: %s %d of %d sequences (all heads)%s, bounded to "
+                                   "%.0f s" % (what, n_last, w0.num_seqs,
+                                               ", over E4M3 codes" if fp8 else "",
+                                               args.cpu_seconds)},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -78,19 +78,25 @@ def test_reference_arm_non_zero_rank_does_nothing(monkeypatch, capsys):
     assert capsys.readouterr().out == ""
 
 
-@pytest.mark.parametrize("name", ["tiny"])
-def test_reference_arm_prints_one_line(monkeypatch, capsys, name):
+@pytest.mark.parametrize("name,unit", [("tiny", "GB/s"), ("tiny_fp8", "GB/s"),
+                                       ("tiny_cascade", "GB/s"), ("gqa_prefill", "TFLOP/s"),
+                                       ("gqa_prefill_fp8", "TFLOP/s")])
+def test_reference_arm_prints_one_line(monkeypatch, capsys, name, unit):
+    """The reference arm follows each workload's metric and unit (decode
+    GB/s, prefill TFLOP/s; E4M3 over quantised codes) in a bounded sample."""
     import json
     monkeypatch.delenv("RANK", raising=False)
     monkeypatch.delenv("WORLD_SIZE", raising=False)
     bench.run_reference(bench.parse_args(["--impl", "reference", "--workload", name,
                                           "--steps", "2", "--warmup", "3",
-                                          "--cpu-seconds", "1"]))
+                                          "--cpu-seconds", "0.3"]))
     lines = capsys.readouterr().out.strip().splitlines()
     assert len(lines) == 1
     rec = json.loads(lines[0])
-    assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["impl"] == "reference" and rec["unit"] == unit and rec["value"] > 0
+    assert rec["config"]["workload"] == name
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+    assert rec["ms_per_step"] < 30000
 
 
 def test_reference_arm_prints_one_contract_line():

@@ -44,7 +44,7 @@
  *  - Alignment: every tensor pointer (16-bit or E4M3) must be 16-byte aligned.
  *  - Supported shapes: head_dim in {64, 128}, block_size in {16, 32},
  *    num_heads / num_kv_heads in {1, 2, 4, 8}, q/out dtype fp16 or bf16
- *    (cascade decode: head_dim 128 only).
+ *    (cascade decode and E4M3 prefill: head_dim 128 only).
  */
 #ifndef PAGEDKV_H_
 #define PAGEDKV_H_

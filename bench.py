@@ -283,6 +283,11 @@ def run_ours(args):
     from paged_kv_cache_394_b200 import workloads as W
     if args.workload.removesuffix("_fp8") in W.PREFILL_NAMES:
         return run_ours_prefill(args)
+    base_name = args.workload.removesuffix("_fp8").removesuffix("_cascade")
+    if base_name not in W.NAMES:
+        raise ValueError("unknown workload %r" % args.workload)
+    if args.workload.endswith("_cascade") and base_name != "prefix_share":
+        raise ValueError("cascade decode needs the prefix-sharing workload (prefix_share_cascade)")
     import numpy as np
     import torch
 

@@ -169,3 +169,10 @@ def test_cascade_groups_share_exactly_their_whole_prompt_blocks(prompt_len, bs):
         if rows.shape[1] > n and len(rows) > 1:
             assert len(set(rows[:, n].tolist())) == len(rows)
         assert (w.context_lens[gs[g]:gs[g + 1]] >= n * bs).all()
+
+
+@pytest.mark.parametrize("name", ["tiny_cascade", "no_such_workload", "llama7b_cascade"])
+def test_our_arm_rejects_workloads_it_cannot_run(name):
+    """Refused on the host, before any device work."""
+    with pytest.raises(ValueError):
+        bench.run_ours(bench.parse_args(["--workload", name]))

@@ -31,7 +31,9 @@
  *    the library).
  *  - Execution: device work is enqueued asynchronously on `stream` (a
  *    cudaStream_t passed as void*; NULL is the legacy default stream).  No
- *    entry point synchronizes.  All device pointers must belong to the
+ *    entry point synchronizes, with one exception: pkv_decode_step_host
+ *    given pageable (not page-locked) host buffers, whose copies the CUDA
+ *    runtime performs synchronously.  All device pointers must belong to the
  *    device that is current on the calling thread.
  *  - Host-side validation happens before anything is enqueued: a bad scalar or
  *    a null / misaligned pointer returns PKV_ERR_INVALID_ARG, a valid but
@@ -221,10 +223,15 @@ pkv_status pkv_paged_attn_prefill(void* out, const void* q, const void* k_cache,
  *    pkv_paged_attn_workspace_bytes), it returns PKV_ERR_WORKSPACE and
  *    enqueues nothing.  16 MiB holds, e.g., 8 sequences x 40 heads x 64
  *    partitions of head_dim 128.
- *  - The first call on each device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.  Later calls on the device only read the cache.
- *  - All calls on a device share the one array, and it keeps whatever the
+ *  - The array exists once per CUDA context that loads the library: the
+ *    device's primary context, a primary context rebuilt after
+ *    cudaDeviceReset, or a context the application created and made current
+ *    through the driver API each hold their own copy, at their own address.
+ *    The first call made with a context current looks the address up in that
+ *    context (cudaGetSymbolAddress) and caches it under the context's id;
+ *    later calls in the same context only read the cache.  Make the first
+ *    call in each context before any stream capture.
+ *  - All calls in a context share the one array, and it keeps whatever the
  *    last call left there.  Nothing in it needs to start at zero: every value
  *    a call reads back was written earlier in the same call.  Calls that
  *    overlap on the GPU (different streams, or different host threads without
@@ -256,11 +263,14 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, const void*
  *                  block is per member after copy-on-write), and every member
  *                  caches at least shared_blocks[g] * block_size tokens
  *   max_group_size, max_shared_blocks  upper bounds (size the launch);
- *                  max_shared_blocks * block_size <= max_context_len
+ *                  max_shared_blocks * block_size <= max_context_len.  With
+ *                  max_shared_blocks = 0 the shared-prefix pass is skipped
  *   workspace      >= pkv_paged_attn_cascade_workspace_bytes(...) bytes
  * The group's table entries are read from its first member.  A member whose
  * context is shorter than its group's shared tokens sets
- * PKV_DEVERR_BAD_CONTEXT.  head_dim 128 only (PKV_ERR_UNSUPPORTED otherwise);
+ * PKV_DEVERR_BAD_CONTEXT, and so does a shared_blocks[g] above
+ * max_shared_blocks: both passes then treat the group as sharing only
+ * max_shared_blocks blocks.  head_dim 128 only (PKV_ERR_UNSUPPORTED otherwise);
  * 16-bit caches.  Other arguments and errors as in pkv_paged_attn_decode.
  */
 size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,

@@ -406,6 +406,7 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   p.group_start = cascade ? cascade->group_start : nullptr;
   p.shared_blocks = cascade ? cascade->shared_blocks : nullptr;
   p.num_groups = cascade ? cascade->num_groups : 0;
+  p.max_shared_blocks = cascade ? cascade->max_shared_blocks : 0;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.ws_out = wl.total ? reinterpret_cast<float*>(ws + wl.out_off) : nullptr;
   p.ws_max = wl.total ? reinterpret_cast<float*>(ws + wl.max_off) : nullptr;
@@ -566,34 +567,93 @@ extern "C" pkv_status pkv_paged_attn_decode_cascade(
 // ---------------------------------------------------------------------------
 
 // The split-K scratch of pkv_paged_attn_decode_static_ws.  Every GPU on which
-// this library is loaded keeps these PKV_STATIC_WORKSPACE_BYTES until the
-// process exits.  In host code this name is only a stand-in for the device
-// symbol, never a device address: the kernels get the address that
-// cudaGetSymbolAddress returns for the current device.
+// this library is loaded keeps these PKV_STATIC_WORKSPACE_BYTES (once per
+// CUDA context that loads it) until the process exits.  In host code this
+// name is only a stand-in for the device symbol, never a device address: the
+// kernels get the address that cudaGetSymbolAddress returns in the current
+// context.
 static __device__ __align__(256) unsigned char pkv_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
 
 
 namespace pkv {
 namespace {
-constexpr int kMaxStaticWsDevices = 64;
-void* g_static_ws_addr[kMaxStaticWsDevices] = {};
+// The array exists once per CUDA context: every context that loads the
+// library (the device's primary context, one rebuilt after cudaDeviceReset,
+// or a context the application made current through the driver API) holds
+// its own copy at its own address.  So the address is cached per context,
+// keyed by the driver's context id, which is unique for the life of the
+// process (a context rebuilt after a reset gets a new one).
+using CtxGetCurrentFn = CUresult(CUDAAPI*)(CUcontext*);
+using CtxGetIdFn = CUresult(CUDAAPI*)(CUcontext, unsigned long long*);
+
+struct ContextFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+// cuCtxGetCurrent and cuCtxGetId through the runtime's driver entry point
+// (no -lcuda).
+const ContextFns& context_fns() {
+  static ContextFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &ptr, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    ptr = nullptr;
+    q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<CtxGetIdFn>(ptr);
+  });
+  return f;
+}
+
+struct StaticWsEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+constexpr int kStaticWsEntries = 64;
+StaticWsEntry g_static_ws[kStaticWsEntries] = {};
+int g_static_ws_next = 0;
 std::mutex g_static_ws_mutex;
 
-// Device address of pkv_static_workspace on the current device, looked up
-// once per device (with that device current) and cached.
+// Device address of pkv_static_workspace in the context current on this
+// thread, looked up (cudaGetSymbolAddress) the first time a context is seen
+// and cached under its id.
 pkv_status static_workspace_address(void** addr) {
-  int dev = 0;
-  pkv_status st = cuda_status(cudaGetDevice(&dev));
-  if (st != PKV_OK) return st;
-  if (dev < 0 || dev >= kMaxStaticWsDevices) return PKV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (g_static_ws_addr[dev] == nullptr) {
+  const ContextFns& f = context_fns();
+  if (f.get_current == nullptr || f.get_id == nullptr) return cuda_status(cudaErrorNotSupported);
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS) return cuda_status(cudaErrorDeviceUninitialized);
+  if (ctx == nullptr) {
+    // The runtime has not made a context current on this thread yet: the
+    // lookup initialises the current device's primary context.
     void* p = nullptr;
-    st = cuda_status(cudaGetSymbolAddress(&p, pkv_static_workspace));
+    const pkv_status st = cuda_status(cudaGetSymbolAddress(&p, pkv_static_workspace));
     if (st != PKV_OK) return st;
-    g_static_ws_addr[dev] = p;
+    if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+      return cuda_status(cudaErrorDeviceUninitialized);
   }
-  *addr = g_static_ws_addr[dev];
+  unsigned long long id = 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return cuda_status(cudaErrorDeviceUninitialized);
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  for (const StaticWsEntry& e : g_static_ws) {
+    if (e.addr != nullptr && e.ctx_id == id) {
+      *addr = e.addr;
+      return PKV_OK;
+    }
+  }
+  void* p = nullptr;
+  const pkv_status st = cuda_status(cudaGetSymbolAddress(&p, pkv_static_workspace));
+  if (st != PKV_OK) return st;
+  g_static_ws[g_static_ws_next] = StaticWsEntry{id, p};
+  g_static_ws_next = (g_static_ws_next + 1) % kStaticWsEntries;
+  *addr = p;
   return PKV_OK;
 }
 }  // namespace

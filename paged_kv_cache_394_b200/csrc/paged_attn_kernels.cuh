@@ -76,6 +76,7 @@ struct DecodeParams {
   const int32_t* group_start;
   const int32_t* shared_blocks;
   int num_groups;
+  int max_shared_blocks;  // the host's bound on shared_blocks[g]; the prefix pass ran iff > 0
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
@@ -84,14 +85,24 @@ __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 // First block a decode kernel reads for `seq`: 0, or under cascade decode the
 // shared blocks of its group (binary search over group_start), at most nblk.
-__device__ __forceinline__ int cascade_start_block(const DecodeParams& p, int seq, int nblk) {
+// A group's shared_blocks above the host's max_shared_blocks is clamped to it
+// (the prefix pass covered no more; with max_shared_blocks = 0 it did not run
+// and workspace slot 0 holds nothing of this call) and reported as
+// PKV_DEVERR_BAD_CONTEXT by the thread that passes `report`.
+__device__ __forceinline__ int cascade_start_block(const DecodeParams& p, int seq, int nblk,
+                                                   bool report) {
   if (p.group_start == nullptr) return 0;
   int lo = 0, hi = p.num_groups;  // invariant: group_start[lo] <= seq < group_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (p.group_start[mid] <= seq) lo = mid; else hi = mid;
   }
-  return min(max(p.shared_blocks[lo], 0), nblk);
+  int shared = max(p.shared_blocks[lo], 0);
+  if (shared > p.max_shared_blocks) {
+    if (report) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
+    shared = p.max_shared_blocks;
+  }
+  return min(shared, nblk);
 }
 
 template <int D_, int BS_, int G_, class DT_, int W_, int NS_, class KV_ = DT_>
@@ -366,7 +377,8 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
     ctx = min(max(ctx, 0), ctx_cap);
   }
   const int nblk = (ctx + BS - 1) / BS;
-  const int start_blk = cascade_start_block(p, seq, nblk);
+  const int start_blk =
+      cascade_start_block(p, seq, nblk, threadIdx.x == 0 && part == 0 && kvh == 0);
   const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
   const bool cascade = p.group_start != nullptr;
   if (part >= (cascade ? nparts : max(nparts, 1))) return;
@@ -809,7 +821,8 @@ __global__ void __launch_bounds__(Tr::THREADS)
     ctx = min(max(ctx, 0), ctx_cap);
   }
   const int nblk = (ctx + BS - 1) / BS;
-  const int start_blk = cascade_start_block(p, seq, nblk);
+  const int start_blk =
+      cascade_start_block(p, seq, nblk, threadIdx.x == 0 && part == 0 && kvh == 0);
   const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
   const bool cascade = p.group_start != nullptr;
   if (part >= (cascade ? nparts : max(nparts, 1))) return;
@@ -995,7 +1008,7 @@ __global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodePa
   const int ctx = clamped_context(p, seq);
   const int nblk = (ctx + p.block_size - 1) / p.block_size;
   const bool cascade = p.group_start != nullptr;
-  const int start_blk = cascade_start_block(p, seq, nblk);
+  const int start_blk = cascade_start_block(p, seq, nblk, false);
   const int nsuffix = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
   // slots [first, last): the prefix partial (slot 0, cascade only) and the suffix partitions
   const int first = cascade && start_blk == 0 ? 1 : 0;

@@ -203,6 +203,7 @@ pkv_status launch_cascade_prefix(const void* q, const void* k_cache, const void*
   p.err = dev_err;
   p.group_start = groups.group_start;
   p.shared_blocks = groups.shared_blocks;
+  p.max_shared_blocks = groups.max_shared_blocks;
   p.ws_out = ws_out;
   p.ws_max = ws_max;
   p.ws_sum = ws_sum;

@@ -57,6 +57,7 @@ struct PrefillParams {
   // slot 0 of each member's workspace row.
   const int32_t* group_start;    // [num_groups + 1] first member of each group
   const int32_t* shared_blocks;  // [num_groups]
+  int max_shared_blocks;         // host bound on shared_blocks[g]; larger values are clamped
   float* ws_out;                 // [S, H, max_parts, D]
   float* ws_max;                 // [S, H, max_parts]
   float* ws_sum;                 // [S, H, max_parts]

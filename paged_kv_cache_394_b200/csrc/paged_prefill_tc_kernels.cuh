@@ -286,7 +286,18 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 
   // seq is a sequence, or in prefix mode a group whose members are the
   // "tokens" q0 .. q0 + q_len - 1 and whose keys are its shared blocks
-  const int ctx = Tr::kPrefix ? p.shared_blocks[seq] * BS : p.context_lens[seq];
+  int ctx = 0;
+  if constexpr (!Tr::kPrefix) {
+    ctx = p.context_lens[seq];
+  } else {
+    // the decode kernels start after the same clamped count
+    int shared = p.shared_blocks[seq];
+    if (shared > p.max_shared_blocks) {
+      if (threadIdx.x == 0 && tile == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
+      shared = p.max_shared_blocks;
+    }
+    ctx = shared * BS;
+  }
   const int q0 = Tr::kPrefix ? p.group_start[seq] : p.query_start[seq];
   const int q_len = (Tr::kPrefix ? p.group_start[seq + 1] : p.query_start[seq + 1]) - q0;
   const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);

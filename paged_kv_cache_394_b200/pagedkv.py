@@ -275,13 +275,13 @@ def paged_attn_decode_cascade(out, q, k_cache, v_cache, block_tables, context_le
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
         if stream is not None:
             workspace.record_stream(stream)   # the temporary must outlive the launch
+    ws_bytes = workspace.numel() * workspace.element_size()
     _check(_paged_attn_decode_cascade(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                       _ptr(block_tables), _ptr(context_lens), _ptr(group_start),
                                       _ptr(shared_blocks), float(scale), s, g, max_group_size,
                                       max_shared_blocks, h, hkv, d, bs, block_tables.shape[1],
                                       max_context_len, num_blocks, _dtype_code(q), partition_size,
-                                      _ptr(workspace), workspace.numel(), _ptr(dev_err),
-                                      _stream(stream)),
+                                      _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream)),
            "paged_attn_decode_cascade")
 
 
@@ -453,14 +453,14 @@ def decode_step_host(out_host, q_host, key_host, value_host, slot_mapping_host,
     t = key_host.shape[0]
     p = block_mapping_host.shape[0] if block_mapping_host.numel() else 0
     ws_ptr = _ptr(workspace)
-    ws_bytes = workspace.numel() if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(_decode_step_host(_ptr(out_host), _ptr(q_host), _ptr(key_host), _ptr(value_host),
                              _ptr(slot_mapping_host), t, _ptr(block_mapping_host), p,
                              _ptr(block_tables_host), _ptr(context_lens_host), _ptr(k_cache),
                              _ptr(v_cache), float(scale), s, h, hkv, d, bs,
                              block_tables_host.shape[1], max_context_len, num_blocks,
                              _dtype_code(k_cache), partition_size, _ptr(staging),
-                             staging.numel(), ws_ptr, ws_bytes, _ptr(dev_err), _stream(stream)),
+                             staging.numel() * staging.element_size(), ws_ptr, ws_bytes, _ptr(dev_err), _stream(stream)),
            "decode_step_host")
 
 

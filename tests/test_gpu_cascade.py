@@ -111,3 +111,35 @@ def test_cascade_prefix_share_full_size(pk):
     kc, vc = oracle_caches(w, inplace=True)
     assert_close(dev_to_bits(dw.out), oracle_decode(w, kc, vc, pairs=pairs), w, pairs=pairs)
     assert torch.isfinite(dw.out.float()).all()
+
+
+def test_cascade_clamps_device_sharing_to_the_host_bound(pk):
+    """shared_blocks in device memory above the host's max_shared_blocks:
+    with max_shared_blocks = 0 the prefix pass does not run, so the decode
+    kernels must read every block themselves (never the stale workspace
+    slot 0) and report PKV_DEVERR_BAD_CONTEXT; the result is still the
+    plain decode."""
+    w = W.build_prefix_share_workload(3, 4, 70, 5, 40, 8, 2, 128, 16, "fp16", seed=19)
+    dw = DeviceWorkload(w)
+    assert run_step(pk, dw, decode=False) == 0
+    kc, vc = oracle_caches(w)
+    ref = oracle_decode(w, kc, vc)
+    gs, full = W.cascade_groups(w)
+    gs_t = torch.from_numpy(gs).cuda()
+    sb_t = torch.from_numpy(full).cuda()
+    max_group = int(np.diff(gs).max())
+    # a poisoned workspace: a merge that read slot 0 would turn the output NaN
+    ws = torch.empty(pk.cascade_workspace_bytes(w.num_seqs, w.num_heads, w.num_kv_heads,
+                                                w.head_dim, w.block_size, w.max_context_len, 0),
+                     dtype=torch.uint8, device="cuda")
+    ws.view(torch.float32).fill_(float("nan"))
+    for bound in (0, 2):
+        dw.err.zero_()
+        dw.out.zero_()
+        pk.paged_attn_decode_cascade(dw.out, dw.q, dw.k_cache, dw.v_cache, dw.tables, dw.lens,
+                                     gs_t, sb_t, w.scale, w.num_kv_heads, w.block_size,
+                                     w.max_context_len, max_group, bound, workspace=ws,
+                                     dev_err=dw.err)
+        torch.cuda.synchronize()
+        assert int(dw.err.item()) & pk.DEVERR_BAD_CONTEXT
+        assert_close(dev_to_bits(dw.out), ref, w)

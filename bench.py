@@ -31,6 +31,7 @@ import hashlib
 
 import numpy as np
 import json
+import math
 import os
 import re
 import statistics
@@ -279,41 +280,67 @@ def committed_traffic(workload, kind="decode"):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def run_ours(args):
+# Timed beside the headline workload in the default run (one GPU): the other
+# decode configurations (long-context split-K, grouped-query chat, parallel
+# sampling with and without cascade), E4M3 caches and chunked prefill, each a
+# nested object of the headline line with its own value, roofline and clocks.
+OTHER_WORKLOADS = ("llama7b_fp8", "long_splitk", "long_splitk_fp8", "gqa_chat", "gqa_chat_fp8",
+                   "prefix_share", "prefix_share_cascade", "llama7b_prefill",
+                   "llama7b_prefill_fp8", "gqa_prefill", "gqa_prefill_fp8")
+
+
+def split_name(workload):
+    """(base workload, E4M3 cache?, cascade decode?) of a bench workload name."""
     from paged_kv_cache_394_b200 import workloads as W
-    if args.workload.removesuffix("_fp8") in W.PREFILL_NAMES:
-        return run_ours_prefill(args)
-    base_name = args.workload.removesuffix("_fp8").removesuffix("_cascade")
-    if base_name not in W.NAMES:
-        raise ValueError("unknown workload %r" % args.workload)
-    if args.workload.endswith("_cascade") and base_name != "prefix_share":
+    fp8 = workload.endswith("_fp8")
+    cascade = workload.endswith("_cascade")
+    base = workload.removesuffix("_fp8").removesuffix("_cascade")
+    if base not in W.NAMES + W.PREFILL_NAMES:
+        raise ValueError("unknown workload %r" % workload)
+    if cascade and base != "prefix_share":
         raise ValueError("cascade decode needs the prefix-sharing workload (prefix_share_cascade)")
+    if cascade and fp8:
+        raise ValueError("cascade decode reads 16-bit caches")
+    return base, fp8, cascade
+
+
+class Run:
+    """Process-wide state of our arm: ranks, device, and the last workload
+    drawn (a variant of the same base workload reuses it)."""
+
+    def __init__(self, args):
+        import torch
+        self.args = args
+        self.rank, self.world = init_dist("nccl") if dist_env()[1] > 1 else (0, 1)
+        self.local = dist_env()[2]
+        torch.cuda.set_device(self.local)
+        self.dev = torch.device("cuda", self.local)
+        self._cached = (None, None)
+
+    def workload(self, base):
+        from paged_kv_cache_394_b200 import pagedkv as pk
+        from paged_kv_cache_394_b200 import workloads as W
+        if self._cached[0] != base:
+            self._cached = (None, None)    # drop the previous pool before drawing the next
+            seed = replica_seed(W.SEED_BASE + (W.NAMES + W.PREFILL_NAMES).index(base), self.rank)
+            # parallel sampling: the library's C++ allocator lays out the shared
+            # prompt blocks and makes the step's copy-on-write pairs
+            self._cached = (base, W.make(base, seed=seed, allocator=pk.BlockAllocator))
+        return self._cached[1]
+
+
+def device_caches(pk, w, dev, fp8):
+    """q, key, value and the caches on the device; with fp8 the pool is
+    quantised once by the device's own E4M3 cache write (set-up, untimed)."""
     import numpy as np
     import torch
-
-    from paged_kv_cache_394_b200 import pagedkv as pk
-    from paged_kv_cache_394_b200 import workloads as W
-
-    rank, world = init_dist("nccl") if dist_env()[1] > 1 else (0, 1)
-    local = dist_env()[2]
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    # "<name>_fp8": the named workload with E4M3 caches (one scale per cache)
-    # "<name>_fp8": E4M3 caches; "prefix_share_cascade": cascade decode
-    fp8 = args.workload.endswith("_fp8")
-    cascade = args.workload.endswith("_cascade")
-    name = args.workload[:-4] if fp8 else args.workload[:-8] if cascade else args.workload
-    base = W.SEED_BASE + W.NAMES.index(name)
-    w = W.make(name, seed=replica_seed(base, rank))
     tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
-    kv_elem = 1 if fp8 else 2
 
     def up(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(tdt)
-
     q, kc, vc, key, val = up(w.q), up(w.k_cache), up(w.v_cache), up(w.key), up(w.value)
+    scales = None
     if fp8:
-        # the pool, quantised once by the device's own cache write (setup, untimed)
         nb, hkv, bs, d = kc.shape
         ks8 = torch.full((hkv,), FP8_K_SCALE, dtype=torch.float32, device=dev)
         vs8 = torch.full((hkv,), FP8_V_SCALE, dtype=torch.float32, device=dev)
@@ -323,8 +350,63 @@ def run_ours(args):
         tok = lambda c: c.permute(0, 2, 1, 3).reshape(nb * bs, hkv, d).contiguous()
         pk.reshape_and_cache_fp8(tok(kc), tok(vc), k8, v8, every, ks8, vs8)
         torch.cuda.synchronize(dev)
-        kc, vc = k8, v8
-        del every
+        kc, vc, scales = k8, v8, (ks8, vs8)
+    return q, kc, vc, key, val, scales
+
+
+def time_steps(run, stream, step, n):
+    """n back-to-back steps between two CUDA events on `stream`, bracketed by
+    a barrier and a synchronize on both sides; the max over ranks, per step,
+    with the clocks sampled meanwhile."""
+    import torch
+    clocks = ClockSampler(run.local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(run.dev)
+    torch.cuda.synchronize(run.dev)
+    t0.record(stream)
+    for i in range(n):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize(run.dev)
+    barrier(run.dev)
+    clk = clocks.stop()
+    return max_over_ranks(t0.elapsed_time(t1), run.dev) / n, clk
+
+
+def time_kernel(run, stream, launch, est_ms):
+    """The dominant kernel alone, in its own loop after the timed steps: each
+    launch between two CUDA events on `stream`, for about --kernel-seconds
+    (the clocks sampled meanwhile).  Returns (average launch ms, launches,
+    clocks)."""
+    import torch
+    n = int(min(20000, max(50, math.ceil(run.args.kernel_seconds * 1e3 / max(est_ms, 1e-3)))))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    clocks = ClockSampler(run.local)
+    clocks.start()
+    torch.cuda.synchronize(run.dev)
+    for a, b in ev:
+        a.record(stream)
+        launch()
+        b.record(stream)
+    torch.cuda.synchronize(run.dev)
+    clk = clocks.stop()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev), n, clk
+
+
+def bench_decode(run, workload, headline):
+    """One decode step (copy_blocks, the cache write, decode) of `workload`."""
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    from paged_kv_cache_394_b200 import workloads as W
+    args, dev = run.args, run.dev
+    base, fp8, cascade = split_name(workload)
+    w = run.workload(base)
+    kv_elem = 1 if fp8 else 2
+    q, kc, vc, key, val, scales = device_caches(pk, w, dev, fp8)
     slots = torch.from_numpy(w.slot_mapping).to(dev)
     pairs = torch.from_numpy(np.ascontiguousarray(w.cow_pairs)).to(dev)
     tables = torch.from_numpy(w.block_tables).to(dev)
@@ -350,24 +432,13 @@ def run_ours(args):
     # cache write (+ block copy) + decode (+ reduce); cascade: prefix pass + suffix + reduce
     launches_per_step = (1 + (1 if has_pairs else 0) +
                          (3 if cascade else 1 + (1 if split else 0)))
-
     inputs = dict(q=q, key=key, val=val, slots=slots, pairs=pairs, tables=tables, lens=lens,
                   out=out)
 
-    def step(ev_a=None, ev_b=None, t=inputs):
-        if has_pairs:
-            pk.copy_blocks(kc, vc, t["pairs"], dev_err=err, stream=stream)
-        if fp8:
-            pk.reshape_and_cache_fp8(t["key"], t["val"], kc, vc, t["slots"], ks8, vs8,
-                                     dev_err=err, stream=stream)
-        else:
-            pk.reshape_and_cache(t["key"], t["val"], kc, vc, t["slots"], dev_err=err,
-                                 stream=stream)
-        if ev_a is not None:
-            ev_a.record(stream)
+    def decode(t=inputs):
         if fp8:
             pk.paged_attn_decode_fp8(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
-                                     ks8, vs8, w.num_kv_heads, w.block_size,
+                                     scales[0], scales[1], w.num_kv_heads, w.block_size,
                                      w.max_context_len, partition_size=part_req, workspace=ws,
                                      dev_err=err, stream=stream)
         elif cascade:
@@ -381,42 +452,34 @@ def run_ours(args):
                                  w.num_kv_heads, w.block_size, w.max_context_len,
                                  partition_size=part_req, workspace=ws, dev_err=err,
                                  stream=stream)
-        if ev_b is not None:
-            ev_b.record(stream)
+
+    def step(i=0, t=inputs):
+        if has_pairs:
+            pk.copy_blocks(kc, vc, t["pairs"], dev_err=err, stream=stream)
+        if fp8:
+            pk.reshape_and_cache_fp8(t["key"], t["val"], kc, vc, t["slots"], scales[0],
+                                     scales[1], dev_err=err, stream=stream)
+        else:
+            pk.reshape_and_cache(t["key"], t["val"], kc, vc, t["slots"], dev_err=err,
+                                 stream=stream)
+        decode(t)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
     torch.cuda.synchronize(dev)
     if int(err.item()) != 0:
-        raise RuntimeError("device error word %d during warm-up" % int(err.item()))
+        raise RuntimeError("%s: device error word %d during warm-up" % (workload, int(err.item())))
 
-    # ---- timed region: K steps, device events, barrier + sync both sides ----
-    clocks = ClockSampler(local)
-    clocks.start()
-    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(*dec_ev[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    clk = clocks.stop()
-    total_ms = t0.elapsed_time(t1)
-    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
-    total_ms_max = max_over_ranks(total_ms, dev)
-    ms_per_step = total_ms_max / args.steps
+    # ---- timed region: K whole steps, nothing else on the stream -------------
+    ms_per_step, clk = time_steps(run, stream, step, args.steps)
     sbytes = step_bytes(w, kv_elem)
     all_bytes = sum_over_ranks(sbytes, dev)
     value = all_bytes / (ms_per_step * 1e-3) / 1e9
-    dec_avg_ms = statistics.mean(dec_ms)
+    # ---- the decode call alone, for the roofline ------------------------------
+    dec_ms, dec_n, dec_clk = time_kernel(run, stream, decode, ms_per_step)
     dbytes = decode_bytes(w, kv_elem)
-    achieved = dbytes / (dec_avg_ms * 1e-3) / 1e9
+    achieved = dbytes / (dec_ms * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
 
     # ---- shared blocks: unique bytes, and the decode timed with L2 flushed ----
@@ -425,31 +488,70 @@ def run_ours(args):
     if ubytes < dbytes:
         l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20)
         scrub = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-        n_fl = min(args.steps, 50)
+        n_fl = 50
         fl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                  for _ in range(n_fl)]
         with torch.cuda.stream(stream):
-            for i in range(n_fl):
-                scrub.zero_()             # evict the previous step's blocks from L2
-                step(*fl_ev[i])
+            for a, b in fl_ev:
+                scrub.zero_()             # evict the previous launch's blocks from L2
+                a.record(stream)
+                decode()
+                b.record(stream)
         torch.cuda.synchronize(dev)
         fl_ms = statistics.mean(a.elapsed_time(b) for a, b in fl_ev)
         del scrub
-        traffic = committed_traffic(args.workload)
+        traffic = committed_traffic(workload)
         sharing = {
             "unique_bytes_per_launch": ubytes,
             "logical_over_unique": round(dbytes / ubytes, 3),
-            "unique_gbs": round(ubytes / (dec_avg_ms * 1e-3) / 1e9, 2),
+            "unique_gbs": round(ubytes / (dec_ms * 1e-3) / 1e9, 2),
+            "unique_pct_of_hbm_peak": round(100.0 * ubytes / (dec_ms * 1e-3) / 1e9 / peak, 2),
             "dram_over_logical": None if traffic is None else round(traffic / dbytes, 4),
             "l2_flushed": {"achieved": round(dbytes / (fl_ms * 1e-3) / 1e9, 2),
                            "unique_gbs": round(ubytes / (fl_ms * 1e-3) / 1e9, 2),
                            "avg_launch_ms": round(fl_ms, 5), "launches": n_fl,
-                           "flush": "%d MB written before each step" % (2 * l2 >> 20)},
+                           "flush": "%d MB written before each launch" % (2 * l2 >> 20)},
         }
+    kernel = (("paged_prefill_tc_kernel (prefix pass) + " if cascade else "")
+              + ("paged_decode_mma_kernel" if (fp8 and w.head_dim == 128)
+                 or (not fp8 and w.num_heads > w.num_kv_heads) else "paged_decode_kernel")
+              + (" + reduce" if split or cascade else ""))
+    line = {
+        "metric": "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s",
+        "value": round(value, 2), "unit": "GB/s", "ms_per_step": round(ms_per_step, 5),
+        "dtype": "e4m3 cache, %s q/out, f32 math" % w.dtype if fp8 else w.dtype,
+        "config": dict(W.describe(w), workload=workload,
+                       kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
+                       if fp8 else w.dtype,
+                       partition_used=part, split_k=split,
+                       l2=("no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
+                           % (dbytes / 1e9)) if ubytes >= dbytes else
+                          ("no flush between steps: %.2f GB of logical KV reads (%.2f GB of "
+                           "distinct blocks) per step; the launch is also timed with L2 "
+                           "flushed (shared_blocks.l2_flushed)" % (dbytes / 1e9, ubytes / 1e9))),
+        "pct_of_hbm_peak": round(100.0 * value / run.world / peak, 2),
+        "tokens_per_s": round(w.num_seqs * run.world / (ms_per_step * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": committed_traffic(workload), "kernel": kernel,
+                     "algorithmic_bytes_per_launch": dbytes,
+                     "avg_launch_ms": round(dec_ms, 5), "launches_timed": dec_n,
+                     "clocks": dec_clk,
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                     if peak_kind == "measured" else "fallback 6.65 TB/s"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if sharing is not None:
+        line["shared_blocks"] = sharing
+    if not headline:
+        del ws
+        return line
 
-    # ---- end to end through the host-buffer entry point ----------------------
+    # ---- end to end through host buffers --------------------------------------
     def pinned(a, view=None):
         return torch.from_numpy(np.ascontiguousarray(a if view is None else a.view(view))).pin_memory()
+    tdt = q.dtype
     h_q = pinned(w.q, np.int16).view(tdt)
     h_key = pinned(w.key, np.int16).view(tdt)
     h_val = pinned(w.value, np.int16).view(tdt)
@@ -463,7 +565,7 @@ def run_ours(args):
                                                      h_tables, h_lens))
     d2h = h_out.numel() * h_out.element_size()
 
-    def e2e_step():
+    def e2e_step(i=0):
         if not fp8 and not cascade:
             pk.decode_step_host(h_out, h_q, h_key, h_val, h_slots, h_pairs, h_tables, h_lens, kc,
                                 vc, w.scale, w.max_context_len, staging, workspace=ws,
@@ -481,128 +583,90 @@ def run_ours(args):
     for _ in range(args.warmup):
         e2e_step()
     torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    e2e_serial_ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    e2e_serial_ms, _ = time_steps(run, stream, e2e_step, args.steps)
     e2e_serial = all_bytes / (e2e_serial_ms * 1e-3) / 1e9
 
-    # ---- end to end, pipelined: step i+1's inputs cross the host link while
-    # step i computes, and step i's output returns while step i+1 computes.
-    # Every step still copies its own inputs in and its output back inside the
-    # timed region; the cache work stays in order on one stream.
-    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    bufs = [inputs, {k: v.clone() for k, v in inputs.items()}]
+    # pipelined: step i+1's inputs cross the host link while step i computes,
+    # and step i's output returns while step i+1 computes.  Every step still
+    # copies its own inputs in and its output back inside the timed region;
+    # the cache work stays in order on one stream.  16-bit caches: the
+    # library's pipeline (pkv_decode_pipeline_*), one C call per step; E4M3
+    # and cascade: the same overlap built from the binding's calls.
     h_outs = [h_out, torch.empty_like(h_out).pin_memory()]
-    ev_up = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_down = [torch.cuda.Event() for _ in range(2)]
-    h_src = dict(q=h_q, key=h_key, val=h_val, slots=h_slots, pairs=h_pairs, tables=h_tables,
-                 lens=h_lens)
+    if not fp8 and not cascade:
+        pstaging = torch.empty(pk.DecodePipeline.staging_bytes(
+            w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.max_blocks_per_seq,
+            len(w.slot_mapping), len(w.cow_pairs)), dtype=torch.uint8, device=dev)
+        pipe = pk.DecodePipeline(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim,
+                                 w.block_size, w.max_blocks_per_seq, len(w.slot_mapping),
+                                 len(w.cow_pairs), tdt, pstaging, stream=stream)
 
-    def e2e_pipelined(i):
-        b, t = i % 2, bufs[i % 2]
-        up.wait_event(ev_comp[b])          # step i-2 has finished reading buffer b
-        with torch.cuda.stream(up):
-            for k, src in h_src.items():
-                if k != "pairs" or has_pairs:
-                    t[k].copy_(src, non_blocking=True)
-        ev_up[b].record(up)
-        stream.wait_event(ev_up[b])
-        stream.wait_event(ev_down[b])      # step i-2's output has left buffer b
-        step(t=t)
-        ev_comp[b].record(stream)
-        down.wait_event(ev_comp[b])
-        with torch.cuda.stream(down):
-            h_outs[b].copy_(t["out"], non_blocking=True)
-        ev_down[b].record(down)
+        def e2e_pipelined(i):
+            pipe.step(h_outs[i % 2], h_q, h_key, h_val, h_slots, h_pairs, h_tables, h_lens, kc,
+                      vc, w.scale, w.max_context_len, workspace=ws, partition_size=part_req,
+                      dev_err=err)
+            if i == args.steps - 1:
+                pipe.join(stream)          # the timing event waits for the last download
+        e2e_api = "pkv_decode_pipeline_step (one C call per step; upload, compute and " \
+                  "download on three streams, consecutive steps overlapped)"
+    else:
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        bufs = [inputs, {k: v.clone() for k, v in inputs.items()}]
+        ev_up = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_down = [torch.cuda.Event() for _ in range(2)]
+        h_src = dict(q=h_q, key=h_key, val=h_val, slots=h_slots, pairs=h_pairs, tables=h_tables,
+                     lens=h_lens)
 
+        def e2e_pipelined(i):
+            b, t = i % 2, bufs[i % 2]
+            up.wait_event(ev_comp[b])          # step i-2 has finished reading buffer b
+            with torch.cuda.stream(up):
+                for k, src in h_src.items():
+                    if k != "pairs" or has_pairs:
+                        t[k].copy_(src, non_blocking=True)
+            ev_up[b].record(up)
+            stream.wait_event(ev_up[b])
+            stream.wait_event(ev_down[b])      # step i-2's output has left buffer b
+            step(t=t)
+            ev_comp[b].record(stream)
+            down.wait_event(ev_comp[b])
+            with torch.cuda.stream(down):
+                h_outs[b].copy_(t["out"], non_blocking=True)
+            ev_down[b].record(down)
+            if i == args.steps - 1:
+                for bb in range(2):
+                    stream.wait_event(ev_down[bb])
+        e2e_api = ("Python binding (reshape_and_cache%s, paged_attn_decode%s) with "
+                   "pinned-host copies on side streams, consecutive steps overlapped"
+                   % (("_fp8", "_fp8") if fp8 else ("", "_cascade")))
     for i in range(args.warmup):
         e2e_pipelined(i)
     torch.cuda.synchronize(dev)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for i in range(args.steps):
-        e2e_pipelined(i)
-    for b in range(2):
-        stream.wait_event(ev_down[b])
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    e2e_ms, _ = time_steps(run, stream, e2e_pipelined, args.steps)
     e2e_value = all_bytes / (e2e_ms * 1e-3) / 1e9
+    if not fp8 and not cascade:
+        pipe.close()
     if int(err.item()) != 0:
-        raise RuntimeError("device error word %d" % int(err.item()))
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp8 and not cascade:
-        cpu = cpu_baseline(w, args.cpu_seconds)
-
-    if rank == 0:
-        tokens = w.num_seqs * world
-        line = {
-            "metric": "paged-decode KV-read GB/s (% of B200 HBM peak) and attention tokens/s",
-            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 cache, %s q/out, f32 math" % w.dtype if fp8 else w.dtype,
-            "data": "synthetic",
-            "config": dict(W.describe(w), workload=args.workload,
-                           kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
-                           if fp8 else w.dtype,
-                           parallelism="replicas%d" % world,
-                           partition_used=part, split_k=split,
-                           l2="no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
-                              % (dbytes / 1e9)),
-            "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
-            "pct_of_8tbs_nominal": round(100.0 * value / world / 8000.0, 2),
-            "tokens_per_s": round(tokens / (ms_per_step * 1e-3), 1),
-            "context_tokens_per_s": round(world * int(w.context_lens.sum()) / (ms_per_step * 1e-3), 1),
-            "step_bytes": sbytes,
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": committed_traffic(args.workload),
-                         "kernel": ("paged_prefill_tc_kernel (prefix pass) + " if cascade else "")
-                         + ("paged_decode_mma_kernel"
-                            if (fp8 and w.head_dim == 128)
-                            or (not fp8 and w.num_heads > w.num_kv_heads)
-                            else "paged_decode_kernel")
-                         + (" + reduce" if split or cascade else ""),
-                         "algorithmic_bytes_per_launch": dbytes,
-                         "avg_launch_ms": round(dec_avg_ms, 5),
-                         "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
-                         if peak_kind == "measured" else "fallback 6.65 TB/s"},
-            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "Python binding (reshape_and_cache%s, paged_attn_decode%s) with "
-                           "pinned-host copies on side streams, consecutive steps overlapped"
-                           % (("_fp8", "_fp8") if fp8 else ("", "_cascade" if cascade else "")),
-                    "serial": {"value": round(e2e_serial, 2), "ms_per_step": round(e2e_serial_ms, 5),
-                               "api": "Python binding with torch copies on one stream"
-                               if fp8 or cascade else "pkv_decode_step_host (one call per step)"}},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk,
-        }
-        if sharing is not None:
-            line["shared_blocks"] = sharing
-        if cpu is not None:
-            line["cpu_baseline"] = cpu
-        print(json.dumps(line), flush=True)
+        raise RuntimeError("%s: device error word %d" % (workload, int(err.item())))
+    line["context_tokens_per_s"] = round(run.world * int(w.context_lens.sum())
+                                         / (ms_per_step * 1e-3), 1)
+    line["pct_of_8tbs_nominal"] = round(100.0 * value / run.world / 8000.0, 2)
+    line["step_bytes"] = sbytes
+    line["e2e"] = {
+        "value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        "api": e2e_api,
+        "serial": {"value": round(e2e_serial, 2), "ms_per_step": round(e2e_serial_ms, 5),
+                   "api": "Python binding with torch copies on one stream"
+                   if fp8 or cascade else "pkv_decode_step_host (one call per step)"}}
+    if run.rank == 0 and run.world == 1 and not args.no_cpu_baseline and not fp8 and not cascade:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     del ws, staging
-    import torch.distributed as dist
-    if dist.is_initialized():
-        dist.destroy_process_group()
+    return line
 
 
-def run_ours_prefill(args):
+def bench_prefill(run, workload, headline):
     """One chunked-prefill step: reshape_and_cache of the new tokens, then
     paged prefill attention.  Metric: attention TFLOP/s (tensor-bound)."""
     import numpy as np
@@ -610,51 +674,10 @@ def run_ours_prefill(args):
 
     from paged_kv_cache_394_b200 import pagedkv as pk
     from paged_kv_cache_394_b200 import workloads as W
-
-    rank, world = init_dist("nccl") if dist_env()[1] > 1 else (0, 1)
-    local = dist_env()[2]
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    # "<name>_fp8": the named prefill batch over E4M3 caches
-    fp8 = args.workload.endswith("_fp8")
-    name = args.workload.removesuffix("_fp8")
-    base = W.SEED_BASE + (W.NAMES + W.PREFILL_NAMES).index(name)
-    w = W.make(name, seed=replica_seed(base, rank))
-    tdt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
-
-    def up(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(tdt)
-
-    q, kc, vc, key, val = up(w.q), up(w.k_cache), up(w.v_cache), up(w.key), up(w.value)
-    if fp8:
-        # the pool, quantised once by the device's own cache write (setup, untimed)
-        nb, hkv, bs, d = kc.shape
-        ks8 = torch.full((hkv,), FP8_K_SCALE, dtype=torch.float32, device=dev)
-        vs8 = torch.full((hkv,), FP8_V_SCALE, dtype=torch.float32, device=dev)
-        k8 = torch.empty(kc.shape, dtype=torch.uint8, device=dev)
-        v8 = torch.empty_like(k8)
-        every = torch.arange(nb * bs, dtype=torch.int64, device=dev)
-        tok = lambda c: c.permute(0, 2, 1, 3).reshape(nb * bs, hkv, d).contiguous()
-        pk.reshape_and_cache_fp8(tok(kc), tok(vc), k8, v8, every, ks8, vs8)
-        torch.cuda.synchronize(dev)
-        kc, vc = k8, v8
-        del every
-
-    def write(k, v, s):
-        if fp8:
-            pk.reshape_and_cache_fp8(k, v, kc, vc, s, ks8, vs8, dev_err=err, stream=stream)
-        else:
-            pk.reshape_and_cache(k, v, kc, vc, s, dev_err=err, stream=stream)
-
-    def attend(o, qq, t, l_, qs):
-        if fp8:
-            pk.paged_attn_prefill_fp8(o, qq, kc, vc, t, l_, qs, w.scale, ks8, vs8, w.num_kv_heads,
-                                      w.block_size, w.max_context_len, max_q, dev_err=err,
-                                      stream=stream)
-        else:
-            pk.paged_attn_prefill(o, qq, kc, vc, t, l_, qs, w.scale, w.num_kv_heads,
-                                  w.block_size, w.max_context_len, max_q, dev_err=err,
-                                  stream=stream)
+    args, dev = run.args, run.dev
+    base, fp8, _ = split_name(workload)
+    w = run.workload(base)
+    q, kc, vc, key, val, scales = device_caches(pk, w, dev, fp8)
     slots = torch.from_numpy(w.slot_mapping).to(dev)
     tables = torch.from_numpy(w.block_tables).to(dev)
     lens = torch.from_numpy(w.context_lens).to(dev)
@@ -664,41 +687,64 @@ def run_ours_prefill(args):
     max_q = int(np.diff(w.query_start).max())
     stream = torch.cuda.Stream(device=dev)
 
-    def step(ev_a=None, ev_b=None):
+    def write(k, v, s):
+        if fp8:
+            pk.reshape_and_cache_fp8(k, v, kc, vc, s, scales[0], scales[1], dev_err=err,
+                                     stream=stream)
+        else:
+            pk.reshape_and_cache(k, v, kc, vc, s, dev_err=err, stream=stream)
+
+    def attend(o=out, qq=q, t=tables, l_=lens, qs=qstart):
+        if fp8:
+            pk.paged_attn_prefill_fp8(o, qq, kc, vc, t, l_, qs, w.scale, scales[0], scales[1],
+                                      w.num_kv_heads, w.block_size, w.max_context_len, max_q,
+                                      dev_err=err, stream=stream)
+        else:
+            pk.paged_attn_prefill(o, qq, kc, vc, t, l_, qs, w.scale, w.num_kv_heads,
+                                  w.block_size, w.max_context_len, max_q, dev_err=err,
+                                  stream=stream)
+
+    def step(i=0):
         write(key, val, slots)
-        if ev_a is not None:
-            ev_a.record(stream)
-        attend(out, q, tables, lens, qstart)
-        if ev_b is not None:
-            ev_b.record(stream)
+        attend()
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
     torch.cuda.synchronize(dev)
     if int(err.item()) != 0:
-        raise RuntimeError("device error word %d during warm-up" % int(err.item()))
-    clocks = ClockSampler(local)
-    clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(*ev[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    clk = clocks.stop()
-    ms_per_step = max_over_ranks(t0.elapsed_time(t1), dev) / args.steps
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+        raise RuntimeError("%s: device error word %d during warm-up" % (workload, int(err.item())))
+    ms_per_step, clk = time_steps(run, stream, step, args.steps)
+    kern_ms, kern_n, kern_clk = time_kernel(run, stream, attend, ms_per_step)
     flops = prefill_flops(w)
     all_flops = sum_over_ranks(flops, dev)
     value = all_flops / (ms_per_step * 1e-3) / 1e12
     achieved = flops / (kern_ms * 1e-3) / 1e12
     peak, peak_kind = tensor_peak()
+    line = {
+        "metric": "paged-prefill attention TFLOP/s",
+        "value": round(value, 2), "unit": "TFLOP/s", "ms_per_step": round(ms_per_step, 5),
+        "dtype": "e4m3 cache, %s q/out, f32 math" % w.dtype if fp8 else w.dtype,
+        "config": dict(W.describe(w), workload=workload,
+                       kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
+                       if fp8 else w.dtype,
+                       l2="no flush: each step rewrites the new tokens' K/V"),
+        "tokens_per_s": round(run.world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": committed_traffic(workload, "prefill"),
+                     "kernel": "paged_prefill_tc_kernel" if w.head_dim == 128
+                               else "paged_prefill_kernel",
+                     "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": round(kern_ms, 5), "launches_timed": kern_n,
+                     "clocks": kern_clk,
+                     "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same "
+                                    "dense rate)" % peak_kind},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if not headline:
+        return line
 
     # end to end through the Python API: pinned host inputs in, output back
     def pinned(a, view=None):
@@ -730,7 +776,7 @@ def run_ours_prefill(args):
         write(bk, bv, bs)
         attend(o, bq, bt, bl, bqs)
 
-    def e2e_step():  # serial: copies in, compute, copy out, all on one stream
+    def e2e_step(i=0):  # serial: copies in, compute, copy out, all on one stream
         upload(dev_in[0], stream)
         compute(dev_in[0], out)
         with torch.cuda.stream(stream):
@@ -757,65 +803,59 @@ def run_ours_prefill(args):
         with torch.cuda.stream(down_s):
             houts[b].copy_(douts[b].view(torch.int16), non_blocking=True)
         ev_down[b].record(down_s)
+        if i == args.steps - 1:
+            for bb in range(2):
+                stream.wait_event(ev_down[bb])
 
-    def timed(fn, pipelined):
-        for i in range(args.warmup):
-            fn(i) if pipelined else fn()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(dev)
-        torch.cuda.synchronize(dev)
-        e0.record(stream)
-        for i in range(args.steps):
-            fn(i) if pipelined else fn()
-        if pipelined:
-            for b in range(2):
-                stream.wait_event(ev_down[b])
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(dev)
-        return max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
-
-    e2e_serial_ms = timed(e2e_step, False)
-    e2e_ms = timed(e2e_pipelined, True)
+    for i in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_serial_ms, _ = time_steps(run, stream, e2e_step, args.steps)
+    for i in range(args.warmup):
+        e2e_pipelined(i)
+    torch.cuda.synchronize(dev)
+    e2e_ms, _ = time_steps(run, stream, e2e_pipelined, args.steps)
     if int(err.item()) != 0:
-        raise RuntimeError("device error word %d" % int(err.item()))
-    if rank == 0:
-        line = {
-            "metric": "paged-prefill attention TFLOP/s",
-            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 cache, %s q/out, f32 math" % w.dtype if fp8 else w.dtype,
-            "data": "synthetic",
-            "config": dict(W.describe(w), workload=args.workload, parallelism="replicas%d" % world,
-                           kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
-                           if fp8 else w.dtype,
-                           l2="no flush: each step rewrites the new tokens' K/V"),
-            "tokens_per_s": round(world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "traffic": committed_traffic(args.workload, "prefill"),
-                         "kernel": "paged_prefill_tc_kernel" if w.head_dim == 128
-                                   else "paged_prefill_kernel",
-                         "algorithmic_flops_per_launch": flops,
-                         "avg_launch_ms": round(kern_ms, 5),
-                         "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same "
-                                        "dense rate)" % peak_kind},
-            "e2e": {"value": round(all_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                    "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h,
-                    "api": ("pagedkv.reshape_and_cache_fp8 + paged_attn_prefill_fp8" if fp8 else
-                            "pagedkv.reshape_and_cache + paged_attn_prefill") +
-                           " with pinned-host copies "
-                           "on side streams, consecutive steps overlapped",
-                    "serial": {"value": round(all_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
-                               "ms_per_step": round(e2e_serial_ms, 5),
-                               "api": "the same calls with the copies on one stream"}},
-            "gpu_launches": 2 * args.steps,
-            "clocks": clk,
-        }
-        print(json.dumps(line), flush=True)
+        raise RuntimeError("%s: device error word %d" % (workload, int(err.item())))
+    line["e2e"] = {
+        "value": round(all_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        "api": ("pagedkv.reshape_and_cache_fp8 + paged_attn_prefill_fp8" if fp8 else
+                "pagedkv.reshape_and_cache + paged_attn_prefill") +
+               " with pinned-host copies on side streams, consecutive steps overlapped",
+        "serial": {"value": round(all_flops / (e2e_serial_ms * 1e-3) / 1e12, 2),
+                   "ms_per_step": round(e2e_serial_ms, 5),
+                   "api": "the same calls with the copies on one stream"}}
+    return line
+
+
+def run_ours(args):
+    from paged_kv_cache_394_b200 import workloads as W
+    base, _, _ = split_name(args.workload)      # unknown names are refused before any device work
+    run = Run(args)
+
+    def bench(name, headline):
+        return (bench_prefill if split_name(name)[0] in W.PREFILL_NAMES else bench_decode)(
+            run, name, headline)
+
+    line = bench(args.workload, True)
+    # the other configurations, on one GPU only (each rank would hold its GPUs
+    # that much longer under torchrun)
+    others = {}
+    if args.workload == "llama7b" and not args.no_other and run.world == 1:
+        for name in OTHER_WORKLOADS:
+            others[name] = bench(name, False)
+    if run.rank == 0:
+        head = {"metric": line.pop("metric"), "value": line.pop("value"), "unit": line.pop("unit"),
+                "n_gpus": run.world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": line.pop("ms_per_step"), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": line.pop("dtype"),
+                "data": "synthetic"}
+        head["config"] = dict(line.pop("config"), parallelism="replicas%d" % run.world)
+        head.update(line)
+        if others:
+            head["other_workloads"] = others
+        print(json.dumps(head), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
@@ -1082,10 +1122,12 @@ def run_reference(args):
     fp8 = args.workload.endswith("_fp8")
     name = args.workload.removesuffix("_fp8").removesuffix("_cascade")
     prefill = name in W.PREFILL_NAMES
-    w0 = W.make(name)
+    # parallel sampling: the oracle's block manager lays out the blocks
+    from oracle.block_manager import BlockManager
+    w0 = W.make(name, allocator=BlockManager)
 
     def sample(seconds):
-        w = W.make(name)
+        w = W.make(name, allocator=BlockManager)
         if prefill:
             return oracle_sample_prefill(w, seconds, fp8)
         return oracle_sample_fp8(w, seconds) if fp8 else oracle_sample(w, seconds)
@@ -1135,6 +1177,11 @@ def parse_args(argv=None):
     ap.add_argument("--partition", type=int, default=None,
                     help="partition size in tokens (0 = let the library choose)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other", action="store_true",
+                    help="time the named workload only (the default run also times the other "
+                         "configurations as nested objects of the headline line)")
+    ap.add_argument("--kernel-seconds", type=float, default=1.0,
+                    help="length of the loop that times the dominant kernel alone")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args(argv)
 

@@ -209,6 +209,20 @@ pkv_status pkv_paged_attn_prefill(void* out, const void* q, const void* k_cache,
                                   pkv_dtype dtype, unsigned* dev_err, void* stream);
 
 /*
+ * pkv_testing_decode_wait — for tests of failure detection; not for serving.
+ * Every wait of a decode kernel on its own loads is bounded: a warp that waits
+ * longer than wait_ns (2 s by default) gives up, ORs PKV_DEVERR_TIMEOUT into
+ * *dev_err, waits (bounded by 2 s) for its loads still in flight, and lets the
+ * kernel finish, so the CUDA context stays usable.  This call sets wait_ns
+ * for later decode launches from any thread (0 < wait_ns <= 2e9, else
+ * PKV_ERR_INVALID_ARG).  With withhold_first_load non-zero, the first CTA of
+ * every later decode launch skips its first load, so that a wait runs out
+ * and the path above runs; its outputs are then not meaningful.  Restore
+ * with (2000000000, 0).
+ */
+pkv_status pkv_testing_decode_wait(uint64_t wait_ns, int withhold_first_load);
+
+/*
  * pkv_paged_attn_decode_static_ws — pkv_paged_attn_decode without a caller
  * workspace.  No counterpart in the source pages: it exists for callers that
  * cannot allocate device memory, such as a plugin inside a host application
@@ -390,6 +404,56 @@ pkv_status pkv_decode_step_host(
     int head_dim, int block_size, int max_blocks_per_seq, int max_context_len, int num_blocks,
     pkv_dtype dtype, int partition_size, void* staging, size_t staging_bytes, void* workspace,
     size_t workspace_bytes, unsigned* dev_err, void* stream);
+
+/*
+ * pkv_decode_pipeline — consecutive decode steps from HOST buffers, each the
+ * work of pkv_decode_step_host, overlapped across three streams: step i+1's
+ * inputs are copied host->device on an upload stream while step i computes on
+ * the compute stream given at creation, and step i's output is copied back on
+ * a download stream while step i+1 computes.  Every step still copies its
+ * own inputs in and its output out.  No counterpart in the source pages,
+ * which describe the serving loop only in words ([csdn] "典型工作流程拆解").
+ *
+ *   create   staging: device scratch of >= pkv_decode_pipeline_staging_bytes
+ *            bytes (16-byte aligned): two areas, used by alternate steps, each
+ *            sized for max_new_tokens new tokens and max_pairs copy pairs.
+ *            The pipeline creates its two copy streams and six events (no
+ *            device memory) and keeps `stream` as its compute stream.
+ *   step     enqueues one step and returns; the cache work of consecutive
+ *            steps stays in order on the compute stream.  num_new_tokens and
+ *            num_pairs may vary per step up to the maxima.  The step's host
+ *            buffers (pinned memory keeps the copies asynchronous) must stay
+ *            valid and unchanged, and *out_host unread, until the step has
+ *            completed (pkv_decode_pipeline_sync, or work ordered after
+ *            pkv_decode_pipeline_join).  dev_err and workspace as in
+ *            pkv_paged_attn_decode; the workspace is shared by the steps in
+ *            compute-stream order.
+ *   join     makes `stream` wait for every step enqueued so far (no host wait).
+ *   sync     blocks the calling host thread until every step enqueued so far
+ *            has completed.
+ *   destroy  waits for the copy streams, then frees the streams and events.
+ * Shapes and errors as for pkv_decode_step_host; a step beyond the maxima
+ * returns PKV_ERR_INVALID_ARG and enqueues nothing.
+ */
+typedef struct pkv_decode_pipeline pkv_decode_pipeline;
+size_t pkv_decode_pipeline_staging_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int max_blocks_per_seq,
+                                         int max_new_tokens, int max_pairs);
+pkv_status pkv_decode_pipeline_create(pkv_decode_pipeline** pipeline, int num_seqs,
+                                      int num_heads, int num_kv_heads, int head_dim,
+                                      int block_size, int max_blocks_per_seq,
+                                      int max_new_tokens, int max_pairs, pkv_dtype dtype,
+                                      void* staging, size_t staging_bytes, void* stream);
+pkv_status pkv_decode_pipeline_step(
+    pkv_decode_pipeline* pipeline, void* out_host, const void* q_host, const void* key_host,
+    const void* value_host, const int64_t* slot_mapping_host, int num_new_tokens,
+    const int64_t* block_mapping_host, int num_pairs, const int32_t* block_tables_host,
+    const int32_t* context_lens_host, void* k_cache, void* v_cache, float scale,
+    int max_context_len, int num_blocks, int partition_size, void* workspace,
+    size_t workspace_bytes, unsigned* dev_err);
+pkv_status pkv_decode_pipeline_join(pkv_decode_pipeline* pipeline, void* stream);
+pkv_status pkv_decode_pipeline_sync(pkv_decode_pipeline* pipeline);
+void pkv_decode_pipeline_destroy(pkv_decode_pipeline* pipeline);
 
 /*
  * Host block allocator ([csdn] "分页式KV缓存" and "典型工作流程拆解" step 7;

@@ -170,6 +170,16 @@ class BlockManager:
         seq["tokens"] = pos + 1
         return seq["blocks"][-1] * self.block_size + offset, cow_src, cow_dst
 
+    def append_slots(self, seq_ids):
+        """append_slot for each id in order; returns (slots, copy pairs made)."""
+        slots, pairs = [], []
+        for s in seq_ids:
+            slot, src, dst = self.append_slot(s)
+            slots.append(slot)
+            if src >= 0:
+                pairs.append((src, dst))
+        return slots, pairs
+
     def free_seq(self, seq_id):
         if seq_id not in self.seqs:
             raise AllocError("INVALID_ARG", "unknown seq id")

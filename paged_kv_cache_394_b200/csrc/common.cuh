@@ -95,13 +95,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete; false after
-// kWaitTimeoutNs.  The clock is read only once the first try has failed.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// limit_ns.  The clock is read only once the first try has failed.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u && global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    if ((it & 255u) == 0u && global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -125,6 +126,12 @@ __device__ __forceinline__ void bulk_copy_g2s_hint(uint32_t dst, const void* src
       "%2, [%3], %4;" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
+}
+
+// Starts bringing `bytes` (a multiple of 16, 16-byte aligned) of global
+// memory into L2 without waiting for it or using shared memory.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {

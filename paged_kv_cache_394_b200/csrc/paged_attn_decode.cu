@@ -5,6 +5,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 
@@ -242,6 +243,11 @@ KernelFn reduce_entry(int d, pkv_dtype dt) {
                         : paged_decode_reduce_kernel<64, Bf16>;
 }
 
+// The decode kernels' bound on a warp's wait for its own loads, and the
+// testing switch that withholds one load (pkv_testing_decode_wait).
+std::atomic<uint64_t> g_wait_ns{kWaitTimeoutNs};
+std::atomic<int> g_withhold_first_load{0};
+
 constexpr int kMaxPartitionBlocks = 4096;  // block-table slice kept in shared memory
 constexpr int kSlots = 2 * 148;            // resident decode CTAs: two per SM, 148 SMs
 
@@ -407,6 +413,8 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   p.shared_blocks = cascade ? cascade->shared_blocks : nullptr;
   p.num_groups = cascade ? cascade->num_groups : 0;
   p.max_shared_blocks = cascade ? cascade->max_shared_blocks : 0;
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  p.withhold_first_load = g_withhold_first_load.load(std::memory_order_relaxed);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.ws_out = wl.total ? reinterpret_cast<float*>(ws + wl.out_off) : nullptr;
   p.ws_max = wl.total ? reinterpret_cast<float*>(ws + wl.max_off) : nullptr;
@@ -439,6 +447,13 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
 }
 
 }  // namespace pkv
+
+extern "C" pkv_status pkv_testing_decode_wait(uint64_t wait_ns, int withhold_first_load) {
+  if (wait_ns == 0 || wait_ns > pkv::kWaitTimeoutNs) return PKV_ERR_INVALID_ARG;
+  pkv::g_wait_ns.store(wait_ns, std::memory_order_relaxed);
+  pkv::g_withhold_first_load.store(withhold_first_load != 0 ? 1 : 0, std::memory_order_relaxed);
+  return PKV_OK;
+}
 
 extern "C" pkv_status pkv_paged_attn_decode(void* out, const void* q, const void* k_cache,
                                             const void* v_cache, const int32_t* block_tables,

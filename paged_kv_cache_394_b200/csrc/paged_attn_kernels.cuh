@@ -77,7 +77,26 @@ struct DecodeParams {
   const int32_t* shared_blocks;
   int num_groups;
   int max_shared_blocks;  // the host's bound on shared_blocks[g]; the prefix pass ran iff > 0
+  // Bound on a warp's wait for its own loads (kWaitTimeoutNs unless a test
+  // lowers it), and a test switch: CTA 0's warp 0 never issues its first
+  // load, so that its wait runs out and the timeout path runs.
+  uint64_t wait_ns;
+  int withhold_first_load;
 };
+
+// Ring stages (blocks for the CUDA-core kernel, 16-token sub-blocks for the
+// tensor-core kernel) that each warp asks L2 for beyond the ones its ring has
+// in flight (cp.async.bulk.prefetch.L2): more bytes in flight per warp without
+// more shared memory, and the ring's own loads then hit L2.
+#ifndef PKV_L2_AHEAD_CC
+#define PKV_L2_AHEAD_CC 0
+#endif
+#ifndef PKV_L2_AHEAD_MMA16
+#define PKV_L2_AHEAD_MMA16 0
+#endif
+#ifndef PKV_L2_AHEAD_MMA8
+#define PKV_L2_AHEAD_MMA8 0
+#endif
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -129,6 +148,7 @@ struct DecodeTraits {
   static constexpr int CHUNK_BYTES = CHUNK_ELEMS * KV_BYTES;
   static constexpr int STAGE_BYTES = 2 * CHUNK_BYTES;
   static constexpr int THREADS = W * 32;
+  static constexpr int L2_AHEAD = PKV_L2_AHEAD_CC;
   static constexpr int PB_FLOATS = R * NV + 8;    // p values + per-head alpha (G <= 8)
   static constexpr int RING_BYTES = W * NS * STAGE_BYTES;
   static constexpr int BAR_BYTES = W * NS * 8;
@@ -437,6 +457,7 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   const size_t block_stride = static_cast<size_t>(p.num_kv_heads) * Tr::CHUNK_ELEMS;
 
   auto issue = [&](int k) {  // lane 0 only
+    if (p.withhold_first_load && blockIdx.x == 0 && warp == 0 && k == 0) return;
     const int stage = k % NS;
     const int pb = tbl[warp + k * W];
     const uint32_t bar = bar0 + stage * 8;
@@ -453,14 +474,27 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
     }
   };
 
+  auto prefetch = [&](int k) {  // lane 0 only: block k of this warp into L2
+    if (k >= nbw) return;
+    const int pb = tbl[warp + k * W];
+    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
+      const size_t off = static_cast<size_t>(pb) * block_stride + head_off;
+      prefetch_l2(kbase + off, Tr::CHUNK_BYTES);
+      prefetch_l2(vbase + off, Tr::CHUNK_BYTES);
+    }
+  };
+
   if (lane == 0) {
     for (int k = 0; k < min(NS, nbw); ++k) issue(k);
+    if constexpr (Tr::L2_AHEAD > 0) {
+      for (int k = NS; k < NS + Tr::L2_AHEAD; ++k) prefetch(k);
+    }
   }
   float* pbuf = pbuf_all + warp * 2 * Tr::PB_FLOATS;
   int buf = 0;
   for (int k = 0; k < nbw; ++k) {
     const int stage = k % NS;
-    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1);
+    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1, p.wait_ns);
     if (!__all_sync(kFullMask, ok)) {
       // Give up on this warp's blocks: report, then wait (bounded) for the
       // copies still in flight so none lands after the CTA has exited.
@@ -487,6 +521,7 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
     if (lane == 0 && k + NS < nbw) {
       fence_proxy_async_smem();  // the warp's reads of this stage precede the refill
       issue(k + NS);
+      if constexpr (Tr::L2_AHEAD > 0) prefetch(k + NS + Tr::L2_AHEAD);
     }
   }
 
@@ -557,6 +592,7 @@ struct MmaTraits {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
   static constexpr int KSTEPS = D / 16;            // q.K k-steps = P.V m-tiles
   static constexpr int THREADS = W * 32;
+  static constexpr int L2_AHEAD = kFp8 ? PKV_L2_AHEAD_MMA8 : PKV_L2_AHEAD_MMA16;
   static constexpr int RING_BYTES = W * NS * STAGE_BYTES;
   static constexpr int BAR_BYTES = W * NS * 8;
   static constexpr int COMBINE_BYTES = W * G * (D + 2) * 4;
@@ -896,6 +932,7 @@ __global__ void __launch_bounds__(Tr::THREADS)
     return tbl[sb / SPB - blk_begin];
   };
   auto issue = [&](int k) {  // lane 0 only
+    if (p.withhold_first_load && blockIdx.x == 0 && warp == 0 && k == 0) return;
     const int stage = k % NS;
     const int sb = sb_begin + warp + k * W;
     const int pb = tbl[sb / SPB - blk_begin];
@@ -915,12 +952,29 @@ __global__ void __launch_bounds__(Tr::THREADS)
     }
   };
 
+  const unsigned char* kbytes = static_cast<const unsigned char*>(p.k_cache);
+  const unsigned char* vbytes = static_cast<const unsigned char*>(p.v_cache);
+  auto prefetch = [&](int k) {  // lane 0 only: sub-block k of this warp into L2
+    if (k >= nbw) return;
+    const int sb = sb_begin + warp + k * W;
+    const int pb = tbl[sb / SPB - blk_begin];
+    if (static_cast<unsigned>(pb) < static_cast<unsigned>(p.num_blocks)) {
+      const size_t row = (static_cast<size_t>(pb) * p.num_kv_heads + kvh) * BS +
+                         (sb % SPB) * Tr::SUB;
+      prefetch_l2(kbytes + row * Tr::ROW_BYTES, Tr::SUB * Tr::ROW_BYTES);
+      prefetch_l2(vbytes + row * Tr::ROW_BYTES, Tr::SUB * Tr::ROW_BYTES);
+    }
+  };
+
   if (lane == 0) {
     for (int k = 0; k < min(NS, nbw); ++k) issue(k);
+    if constexpr (Tr::L2_AHEAD > 0) {
+      for (int k = NS; k < NS + Tr::L2_AHEAD; ++k) prefetch(k);
+    }
   }
   for (int k = 0; k < nbw; ++k) {
     const int stage = k % NS;
-    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1);
+    const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1, p.wait_ns);
     if (!__all_sync(kFullMask, ok)) {
       if (lane == 0) {
         set_err(p.err, PKV_DEVERR_TIMEOUT);
@@ -944,6 +998,7 @@ __global__ void __launch_bounds__(Tr::THREADS)
     if (lane == 0 && k + NS < nbw) {
       fence_proxy_async_smem();
       issue(k + NS);
+      if constexpr (Tr::L2_AHEAD > 0) prefetch(k + NS + Tr::L2_AHEAD);
     }
   }
 

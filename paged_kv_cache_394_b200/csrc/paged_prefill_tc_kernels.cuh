@@ -37,6 +37,10 @@
 #include "common.cuh"
 #include "paged_prefill_kernels.cuh"
 
+#ifndef PKV_PREFIX_STAGES
+#define PKV_PREFIX_STAGES 6
+#endif
+
 namespace pkv {
 namespace tc {
 
@@ -212,8 +216,9 @@ struct TcPrefillTraits {
   static constexpr int M = 128;                  // rows of one query tile (one TMEM lane each)
   static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
   static constexpr int NKEY = 64;                // keys per KV tile
-  // KV stages: what fits beside QT query tiles (P lives in TMEM, over S)
-  static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : 6;
+  // KV stages: what fits beside QT query tiles (P lives in TMEM, over S); the
+  // cascade prefix pass (one query tile) keeps PKV_PREFIX_STAGES
+  static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : PKV_PREFIX_STAGES;
   static constexpr int NSTG = kFp8 ? 2 : 0;      // E4M3 staging slots per kind
   // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
   // P.V issuer

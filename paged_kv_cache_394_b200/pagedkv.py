@@ -68,6 +68,16 @@ _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i
 _decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
                            _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
                            _vp, _sz, _vp, _vp)
+_testing_decode_wait = _proto("pkv_testing_decode_wait", _i, ctypes.c_uint64, _i)
+_pipeline_staging_bytes = _proto("pkv_decode_pipeline_staging_bytes", _sz, _i, _i, _i, _i, _i, _i,
+                                 _i)
+_pipeline_create = _proto("pkv_decode_pipeline_create", _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                          _vp, _sz, _vp)
+_pipeline_step = _proto("pkv_decode_pipeline_step", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i,
+                        _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _sz, _vp)
+_pipeline_join = _proto("pkv_decode_pipeline_join", _i, _vp, _vp)
+_pipeline_sync = _proto("pkv_decode_pipeline_sync", _i, _vp)
+_pipeline_destroy = _proto("pkv_decode_pipeline_destroy", None, _vp)
 _alloc_create = _proto("pkv_alloc_create", _vp, _i, _i, _vp)
 _alloc_destroy = _proto("pkv_alloc_destroy", None, _vp)
 _alloc_add_seq = _proto("pkv_alloc_add_seq", _i, _vp, _i64, _i64)
@@ -427,6 +437,14 @@ def paged_attn_prefill_fp8(out, q, k_cache, v_cache, block_tables, context_lens,
            "paged_attn_prefill_fp8")
 
 
+def testing_decode_wait(wait_ns, withhold_first_load=False):
+    """Testing hook: the decode kernels' bound on a wait for their own loads,
+    and whether the first CTA withholds its first load so that the wait runs
+    out (see include/pagedkv.h).  Restore with (2_000_000_000, False)."""
+    _check(_testing_decode_wait(int(wait_ns), 1 if withhold_first_load else 0),
+           "testing_decode_wait")
+
+
 def staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                   num_new_tokens, num_pairs):
     return _staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
@@ -460,8 +478,79 @@ def decode_step_host(out_host, q_host, key_host, value_host, slot_mapping_host,
                              _ptr(v_cache), float(scale), s, h, hkv, d, bs,
                              block_tables_host.shape[1], max_context_len, num_blocks,
                              _dtype_code(k_cache), partition_size, _ptr(staging),
-                             staging.numel() * staging.element_size(), ws_ptr, ws_bytes, _ptr(dev_err), _stream(stream)),
+                             staging.numel() * staging.element_size(), ws_ptr, ws_bytes,
+                             _ptr(dev_err), _stream(stream)),
            "decode_step_host")
+
+
+def _host(t, name):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous host tensor" % name)
+
+
+class DecodePipeline:
+    """Consecutive decode steps from host tensors, overlapped across an upload,
+    a compute and a download stream (``pkv_decode_pipeline_*``; see the
+    header).  ``staging`` is a device uint8 tensor of at least
+    ``DecodePipeline.staging_bytes(...)`` bytes; ``stream`` the compute stream."""
+
+    @staticmethod
+    def staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                      max_new_tokens, max_pairs):
+        return _pipeline_staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                       max_blocks_per_seq, max_new_tokens, max_pairs)
+
+    def __init__(self, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                 max_blocks_per_seq, max_new_tokens, max_pairs, dtype, staging, stream=None):
+        _dev(staging, "staging")
+        self._staging = staging                 # kept alive with the pipeline
+        self._stream = torch.cuda.current_stream() if stream is None else stream
+        h = ctypes.c_void_p()
+        _check(_pipeline_create(ctypes.byref(h), num_seqs, num_heads, num_kv_heads, head_dim,
+                                block_size, max_blocks_per_seq, max_new_tokens, max_pairs,
+                                _dtype_code(torch.empty(0, dtype=dtype)), _ptr(staging),
+                                staging.numel() * staging.element_size(),
+                                ctypes.c_void_p(self._stream.cuda_stream)),
+               "decode_pipeline_create")
+        self._h = h
+
+    def step(self, out_host, q_host, key_host, value_host, slot_mapping_host, block_mapping_host,
+             block_tables_host, context_lens_host, k_cache, v_cache, scale, max_context_len,
+             workspace=None, partition_size=0, dev_err=None):
+        for n, t in (("out_host", out_host), ("q_host", q_host), ("key_host", key_host),
+                     ("value_host", value_host), ("slot_mapping_host", slot_mapping_host),
+                     ("block_mapping_host", block_mapping_host),
+                     ("block_tables_host", block_tables_host),
+                     ("context_lens_host", context_lens_host)):
+            _host(t, n)
+        _dev(k_cache, "k_cache")
+        _dev(v_cache, "v_cache")
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        p = block_mapping_host.shape[0] if block_mapping_host.numel() else 0
+        _check(_pipeline_step(self._h, _ptr(out_host), _ptr(q_host), _ptr(key_host),
+                              _ptr(value_host), _ptr(slot_mapping_host), key_host.shape[0],
+                              _ptr(block_mapping_host), p, _ptr(block_tables_host),
+                              _ptr(context_lens_host), _ptr(k_cache), _ptr(v_cache), float(scale),
+                              max_context_len, k_cache.shape[0], partition_size, _ptr(workspace),
+                              ws_bytes, _ptr(dev_err)),
+               "decode_pipeline_step")
+
+    def join(self, stream=None):
+        _check(_pipeline_join(self._h, _stream(stream)), "decode_pipeline_join")
+
+    def sync(self):
+        _check(_pipeline_sync(self._h), "decode_pipeline_sync")
+
+    def close(self):
+        if self._h:
+            _pipeline_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class BlockAllocator:

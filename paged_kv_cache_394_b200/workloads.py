@@ -1,7 +1,10 @@
 """Seeded synthetic workloads for paged decode attention.
 
 This module only draws inputs: sequence lengths, physical block placement,
-N(0, 1) query/key/value values and NaN poison.  It holds none of the
+N(0, 1) query/key/value values and NaN poison.  For parallel sampling the
+placement is a free-list order handed to a block manager that the caller
+supplies (the library's allocator, or the oracle's), which then lays out the
+shared and copied blocks itself.  It holds none of the
 attention arithmetic and is the one module that feeds both the CUDA library
 and the CPU oracle, so both see byte-identical inputs.
 
@@ -191,14 +194,23 @@ def build_decode_workload(context_lens, num_heads, num_kv_heads, head_dim, block
 
 def build_prefix_share_workload(num_prompts, samples, prompt_len, div_low, div_high,
                                 num_heads, num_kv_heads, head_dim, block_size, dtype,
-                                seed, pool_factor=1.2, name="prefix_share"):
+                                seed, allocator, pool_factor=1.2, name="prefix_share"):
     """Parallel sampling: ``samples`` sequences per prompt share the prompt's blocks.
 
-    Each sample appends ``U[div_low, div_high]`` divergent tokens in this step.
-    When the prompt ends inside a block, that partial block is shared too;
-    samples 0..samples-2 get a private copy of it (the step's copy pairs)
-    before the write, and the last sample writes into the original.
-    Sequence order is prompt-major: the samples of a prompt are adjacent.
+    The block layout is not drawn here: ``allocator(num_blocks, block_size,
+    free_order)`` is a block manager (the library's C++ allocator, or the
+    oracle's: ``add_seq``, ``fork``, ``append_slots``, ``block_table``) and
+    this function only drives it, so that the step's block
+    tables, slots and copy pairs are the ones the block manager produces.
+    ``free_order``, a random permutation of the pool, scatters the blocks.
+
+    Each prompt is admitted (``add_seq``) and forked into its other samples,
+    then every sample appends its ``U[div_low, div_high]`` divergent tokens
+    (``append_slots``), prompt by prompt and sample by sample.  When the prompt
+    ends inside a block, the first ``samples - 1`` samples to append copy that
+    shared partial block on write (the step's copy pairs) and the last writes
+    into the original.  Sequence order is prompt-major: the samples of a
+    prompt are adjacent (sequence id = prompt * samples + sample).
     """
     rng = np.random.default_rng(seed)
     bs = block_size
@@ -206,38 +218,30 @@ def build_prefix_share_workload(num_prompts, samples, prompt_len, div_low, div_h
     partial = prompt_len % bs != 0
     div = rng.integers(div_low, div_high + 1, size=num_prompts * samples)
     lens = prompt_len + div
-    first_free_off = prompt_len % bs
     # blocks needed: prompt blocks, copies, and each sample's fresh blocks
-    room_in_partial = (bs - first_free_off) if partial else 0
+    room_in_partial = (bs - prompt_len % bs) if partial else 0
     fresh = [_blocks_for(max(0, int(d) - room_in_partial), bs) for d in div]
     n_copies = num_prompts * (samples - 1) if partial else 0
     total = num_prompts * n_prompt_blocks + n_copies + int(sum(fresh))
     num_blocks = int(math.ceil(pool_factor * total))
-    perm = iter(rng.permutation(num_blocks).tolist())
+    free_order = rng.permutation(num_blocks).astype(np.int32)
+    mgr = allocator(num_blocks, bs, free_order)
     s = num_prompts * samples
-    mb = max(_blocks_for(c, bs) for c in lens)
-    tables = np.full((s, mb), -1, dtype=np.int32)
     filled = {}
-    cow = []
-    slots = []
     for p in range(num_prompts):
-        prompt_blocks = [next(perm) for _ in range(n_prompt_blocks)]
-        for k, b in enumerate(prompt_blocks):
-            filled[b] = min(bs, prompt_len - k * bs)
-        for j in range(samples):
-            i = p * samples + j
-            blocks = list(prompt_blocks)
-            if partial and j < samples - 1:
-                dst = next(perm)
-                cow.append((prompt_blocks[-1], dst))
-                blocks[-1] = dst
-                filled.setdefault(dst, 0)
-            blocks += [next(perm) for _ in range(fresh[i])]
-            for b in blocks[n_prompt_blocks:]:
-                filled.setdefault(b, 0)
-            tables[i, :len(blocks)] = blocks
-            for t in range(prompt_len, int(lens[i])):
-                slots.append(blocks[t // bs] * bs + t % bs)
+        parent = p * samples
+        mgr.add_seq(parent, prompt_len)
+        for k, b in enumerate(mgr.block_table([parent], n_prompt_blocks)[0]):
+            filled[int(b)] = min(bs, prompt_len - k * bs)
+        for j in range(1, samples):
+            mgr.fork(parent, parent + j)
+    slots, cow = [], []
+    for i in range(s):
+        got, pairs = mgr.append_slots([i] * int(div[i]))
+        slots += got
+        cow += pairs
+    mb = max(_blocks_for(c, bs) for c in lens)
+    tables = np.asarray(mgr.block_table(list(range(s)), mb), dtype=np.int32).reshape(s, mb)
     kc, vc = _fill_pool(rng, num_blocks, num_kv_heads, bs, head_dim, dtype, filled)
     t_new = len(slots)
     q = _normal_bits(rng, (s, num_heads, head_dim), dtype)
@@ -250,7 +254,8 @@ def build_prefix_share_workload(num_prompts, samples, prompt_len, div_low, div_h
                     slot_mapping=np.asarray(slots, dtype=np.int64),
                     cow_pairs=np.asarray(cow, dtype=np.int64).reshape(-1, 2),
                     notes={"seed": seed, "prompt_len": prompt_len,
-                           "prompt_blocks": n_prompt_blocks, "samples": samples})
+                           "prompt_blocks": n_prompt_blocks, "samples": samples,
+                           "free_order": free_order})
 
 
 def cascade_groups(w, shared_blocks=None):
@@ -336,9 +341,10 @@ def chat_lengths(rng, n, median=600.0, sigma=1.0, low=16, high=4096):
     return np.clip(np.rint(x), low, high).astype(np.int64)
 
 
-def make(name, seed=None):
+def make(name, seed=None, allocator=None):
     """The named workload.  ``seed`` defaults to 394 + its index in
-    ``NAMES + PREFILL_NAMES``."""
+    ``NAMES + PREFILL_NAMES``.  ``prefix_share`` lays its blocks out with
+    ``allocator`` (see build_prefix_share_workload); the others need none."""
     idx = (NAMES + PREFILL_NAMES).index(name)
     seed = SEED_BASE + idx if seed is None else seed
     rng = np.random.default_rng(seed + 1000)   # lengths; values use ``seed``
@@ -364,8 +370,10 @@ def make(name, seed=None):
         return build_decode_workload(lens, 40, 40, 128, 16, "fp16", seed, name=name,
                                      partition_size=512)
     if name == "prefix_share":
+        if allocator is None:
+            raise ValueError("prefix_share lays out its blocks with a block allocator")
         return build_prefix_share_workload(64, 8, 1020, 64, 256, 64, 8, 128, 16, "bf16",
-                                           seed)
+                                           seed, allocator)
     raise KeyError(name)
 
 

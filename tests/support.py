@@ -18,6 +18,13 @@ ATOL = 2e-3
 RTOL = 1e-2
 
 
+def block_allocator(num_blocks, block_size, free_order):
+    """The library's C++ block allocator: it lays out the shared, copied and
+    fresh blocks of the parallel-sampling workloads."""
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    return pk.BlockAllocator(num_blocks, block_size, free_order)
+
+
 def torch_dtype(w):
     return torch.float16 if w.dtype == "fp16" else torch.bfloat16
 

@@ -200,3 +200,42 @@ def test_cascade_host_validation_without_gpu():
     assert cas(wsb=ws - 16) == pk.ERR_WORKSPACE
     assert cas(ptr=bad) == pk.ERR_INVALID_ARG
     assert cas(part=24) == pk.ERR_INVALID_ARG              # not a multiple of block_size
+
+
+def test_pipeline_staging_and_host_validation_without_gpu():
+    """Two staging areas, each holding a step at the maxima; bad arguments
+    are refused before any stream or event is created."""
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    s, h, hkv, d, mb, t, p = 64, 32, 32, 128, 128, 64, 3
+    one = pk.staging_bytes(s, h, hkv, d, mb, t, p)
+    assert pk.DecodePipeline.staging_bytes(s, h, hkv, d, mb, t, p) >= 2 * one
+    assert pk.DecodePipeline.staging_bytes(s, 0, hkv, d, mb, t, p) == 0
+    lib = ctypes.CDLL(pk.LIB_PATH)
+    lib.pkv_decode_pipeline_create.argtypes = ([ctypes.c_void_p] + [ctypes.c_int] * 9 +
+                                               [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p])
+    h_out = ctypes.c_void_p()
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: every case fails first
+    need = pk.DecodePipeline.staging_bytes(s, h, hkv, d, mb, t, p)
+    args = [s, h, hkv, d, 16, mb, t, p, pk.FP16]
+    assert lib.pkv_decode_pipeline_create(None, *args, fake, need, None) == pk.ERR_INVALID_ARG
+    bad_heads = [s, h, 5, d, 16, mb, t, p, pk.FP16]          # 32 % 5 != 0
+    assert lib.pkv_decode_pipeline_create(ctypes.byref(h_out), *bad_heads, fake, need,
+                                          None) == pk.ERR_INVALID_ARG
+    bad_dim = [s, h, hkv, 96, 16, mb, t, p, pk.FP16]
+    assert lib.pkv_decode_pipeline_create(ctypes.byref(h_out), *bad_dim, fake, need,
+                                          None) == pk.ERR_UNSUPPORTED
+    assert lib.pkv_decode_pipeline_create(ctypes.byref(h_out), *args, None, need,
+                                          None) == pk.ERR_INVALID_ARG
+    assert lib.pkv_decode_pipeline_create(ctypes.byref(h_out), *args, fake, need - 16,
+                                          None) == pk.ERR_WORKSPACE
+    assert h_out.value is None
+    lib.pkv_decode_pipeline_step.restype = ctypes.c_int
+    assert lib.pkv_decode_pipeline_step(None, *([None] * 18)) == pk.ERR_INVALID_ARG
+
+
+def test_testing_wait_hook_validates_on_the_host():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    for bad in (0, 2_000_000_001):
+        with pytest.raises(pk.PagedKVError):
+            pk.testing_decode_wait(bad, False)
+    pk.testing_decode_wait(2_000_000_000, False)      # the default, accepted

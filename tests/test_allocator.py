@@ -158,3 +158,34 @@ def test_prefix_cache_traces_match_oracle(seed, num_blocks, bs):
     assert [lib.refcount(b) for b in range(num_blocks)] == ref.refcount
     q, h, _, ev = lib.cache_stats()
     assert h > 0 and ev > 0          # the trace exercised hits and evictions
+
+
+def test_parallel_sampling_workload_layout_matches_oracle():
+    """The full-size parallel-sampling workload (64 prompts x 8 samples, a
+    1020-token prompt in blocks of 16) laid out by the C++ allocator and by
+    the oracle block manager from the same free order: identical block
+    tables, slots and copy pairs.  Each prompt's shared partial block is
+    copied on write for the first 7 samples to append (the last writes in
+    place), so the step carries 64 x 7 = 448 pairs."""
+    from paged_kv_cache_394_b200 import workloads as W
+    lib = W.make("prefix_share", allocator=pk.BlockAllocator)
+    ref = W.make("prefix_share", allocator=BlockManager)
+    assert np.array_equal(lib.block_tables, ref.block_tables)
+    assert np.array_equal(lib.slot_mapping, ref.slot_mapping)
+    assert np.array_equal(lib.cow_pairs, ref.cow_pairs)
+    assert len(lib.cow_pairs) == 448
+    bs, samples = lib.block_size, lib.notes["samples"]
+    last = lib.notes["prompt_blocks"] - 1            # the partial prompt block
+    for p in range(64):
+        rows = lib.block_tables[p * samples:(p + 1) * samples]
+        src = rows[-1, last]                          # the last sample kept the original
+        pairs = lib.cow_pairs[7 * p:7 * p + 7]
+        assert (pairs[:, 0] == src).all()
+        assert list(pairs[:, 1]) == list(rows[:-1, last])
+    assert len(set(lib.cow_pairs[:, 1].tolist())) == 448
+    assert not set(lib.cow_pairs[:, 1].tolist()) & set(lib.cow_pairs[:, 0].tolist())
+    # every new token lands past its sequence's prompt, in its own table row
+    s = np.repeat(np.arange(lib.num_seqs), lib.context_lens - 1020)
+    pos = np.concatenate([np.arange(1020, c) for c in lib.context_lens])
+    assert np.array_equal(lib.slot_mapping,
+                          lib.block_tables[s, pos // bs].astype(np.int64) * bs + pos % bs)

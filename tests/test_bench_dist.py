@@ -11,6 +11,7 @@ import pytest
 import torch.multiprocessing as mp
 
 import bench
+from support import block_allocator
 
 
 def free_port():
@@ -134,7 +135,8 @@ def _slots_read(w):
 @pytest.mark.parametrize("kv_elem", [2, 1])
 def test_unique_bytes_count_each_shared_slot_once(kv_elem):
     from paged_kv_cache_394_b200 import workloads as W
-    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "fp16", seed=5)
+    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "fp16", seed=5,
+                                      allocator=block_allocator)
     per_slot = 2 * w.num_kv_heads * w.head_dim * kv_elem
     qo = 2 * w.num_seqs * w.num_heads * w.head_dim * 2
     assert bench.unique_decode_bytes(w, kv_elem) == len(_slots_read(w)) * per_slot + qo
@@ -155,7 +157,8 @@ def test_cascade_groups_share_exactly_their_whole_prompt_blocks(prompt_len, bs):
     prompt block is copied on write; divergent tokens get fresh blocks)."""
     import numpy as np
     from paged_kv_cache_394_b200 import workloads as W
-    w = W.build_prefix_share_workload(3, 4, prompt_len, 5, 40, 8, 2, 64, bs, "fp16", seed=7)
+    w = W.build_prefix_share_workload(3, 4, prompt_len, 5, 40, 8, 2, 64, bs, "fp16", seed=7,
+                                      allocator=block_allocator)
     gs, shared = W.cascade_groups(w)
     assert gs[0] == 0 and gs[-1] == w.num_seqs and (np.diff(gs) > 0).all()
     seen = set()

@@ -236,3 +236,19 @@ def test_prefix_cache_keeps_refcounts_and_blocks_consistent():
             assert mgr.refcount[b] == 0 and b in mgr.cache_key
         for key, b in mgr.cache.items():
             assert mgr.cache_key[b] == key and len(key) % bs == 0
+
+
+def test_append_slots_is_append_slot_in_order():
+    """The batched form returns what one append_slot per id returns, in order,
+    with the copy pairs of the appends that made one."""
+    a, b = BlockManager(20, 4), BlockManager(20, 4)
+    for m in (a, b):
+        m.add_seq(1, 6)
+        m.fork(1, 2)
+        m.fork(1, 3)
+    ids = [2, 3, 1, 2, 2, 3]
+    slots, pairs = a.append_slots(ids)
+    expect = [b.append_slot(i) for i in ids]
+    assert slots == [s for s, _, _ in expect]
+    assert pairs == [(s, d) for _, s, d in expect if s >= 0]
+    assert len(pairs) == 2            # sequences 2 and 3 copy; 1, the last holder, writes in place

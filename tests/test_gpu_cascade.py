@@ -10,7 +10,8 @@ import pytest
 import torch
 
 from paged_kv_cache_394_b200 import workloads as W
-from support import DeviceWorkload, assert_close, dev_to_bits, oracle_caches, oracle_decode, run_step
+from support import (DeviceWorkload, assert_close, block_allocator, dev_to_bits, oracle_caches,
+                     oracle_decode, run_step)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +44,7 @@ CASES = [(3, 4, 37, 8, 2, 16, "bf16"), (2, 8, 64, 8, 1, 16, "fp16"), (4, 2, 100,
 @pytest.mark.parametrize("prompts,samples,plen,h,hkv,bs,dtype", CASES)
 def test_cascade_matches_oracle(pk, prompts, samples, plen, h, hkv, bs, dtype):
     w = W.build_prefix_share_workload(prompts, samples, plen, 5, 40, h, hkv, 128, bs, dtype,
-                                      seed=plen + samples)
+                                      seed=plen + samples, allocator=block_allocator)
     dw = DeviceWorkload(w)
     assert run_step(pk, dw, decode=False) == 0
     group_start, shared = W.cascade_groups(w)
@@ -57,7 +58,8 @@ def test_cascade_matches_oracle(pk, prompts, samples, plen, h, hkv, bs, dtype):
 
 def test_cascade_with_fewer_shared_blocks_and_singletons(pk):
     """Declaring less sharing than there is, or none, changes nothing."""
-    w = W.build_prefix_share_workload(3, 4, 70, 5, 40, 8, 2, 128, 16, "fp16", seed=9)
+    w = W.build_prefix_share_workload(3, 4, 70, 5, 40, 8, 2, 128, 16, "fp16", seed=9,
+                                      allocator=block_allocator)
     dw = DeviceWorkload(w)
     assert run_step(pk, dw, decode=False) == 0
     kc, vc = oracle_caches(w)
@@ -86,7 +88,8 @@ def test_cascade_equals_plain_decode_on_independent_sequences(pk):
 
 
 def test_cascade_flags_a_member_shorter_than_its_prefix(pk):
-    w = W.build_prefix_share_workload(2, 4, 64, 5, 40, 8, 2, 128, 16, "fp16", seed=4)
+    w = W.build_prefix_share_workload(2, 4, 64, 5, 40, 8, 2, 128, 16, "fp16", seed=4,
+                                      allocator=block_allocator)
     dw = DeviceWorkload(w)
     assert run_step(pk, dw, decode=False) == 0
     gs, _ = W.cascade_groups(w)
@@ -99,7 +102,7 @@ def test_cascade_flags_a_member_shorter_than_its_prefix(pk):
 def test_cascade_prefix_share_full_size(pk):
     """The parallel-sampling workload at full size (64 prompts x 8 samples),
     on sampled rows including the longest and shortest sequence."""
-    w = W.make("prefix_share")
+    w = W.make("prefix_share", allocator=block_allocator)
     dw = DeviceWorkload(w)
     assert run_step(pk, dw, decode=False) == 0
     gs, shared = W.cascade_groups(w)
@@ -119,7 +122,8 @@ def test_cascade_clamps_device_sharing_to_the_host_bound(pk):
     kernels must read every block themselves (never the stale workspace
     slot 0) and report PKV_DEVERR_BAD_CONTEXT; the result is still the
     plain decode."""
-    w = W.build_prefix_share_workload(3, 4, 70, 5, 40, 8, 2, 128, 16, "fp16", seed=19)
+    w = W.build_prefix_share_workload(3, 4, 70, 5, 40, 8, 2, 128, 16, "fp16", seed=19,
+                                      allocator=block_allocator)
     dw = DeviceWorkload(w)
     assert run_step(pk, dw, decode=False) == 0
     kc, vc = oracle_caches(w)

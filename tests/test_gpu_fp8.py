@@ -15,7 +15,7 @@ import torch
 from oracle import cache_ops as OC
 from oracle import fp8 as OF
 from paged_kv_cache_394_b200 import workloads as W
-from support import assert_close, bits_to_dev, dev_to_bits
+from support import assert_close, bits_to_dev, block_allocator, dev_to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -195,7 +195,8 @@ def test_fp8_write_is_bit_exact_on_edge_values(pk, dtype):
 
 
 def test_fp8_copy_blocks_bit_exact(pk):
-    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "bf16", seed=3)
+    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "bf16", seed=3,
+                                      allocator=block_allocator)
     assert len(w.cow_pairs) == 9
     dev = Fp8Device(pk, w)
     assert dev.step(pk) == 0

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from paged_kv_cache_394_b200 import workloads as W
-from support import (DeviceWorkload, assert_close, dev_to_bits, oracle_caches, oracle_decode,
+from support import (DeviceWorkload, block_allocator, assert_close, dev_to_bits, oracle_caches, oracle_decode,
                      run_step)
 
 pytestmark = pytest.mark.gpu
@@ -49,7 +49,8 @@ def test_cache_write_bit_exact_small(pk, d, bs, dtype):
 
 
 def test_copy_blocks_and_write_bit_exact(pk):
-    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "bf16", seed=3)
+    w = W.build_prefix_share_workload(3, 4, 37, 5, 40, 8, 2, 64, 16, "bf16", seed=3,
+                                      allocator=block_allocator)
     assert len(w.cow_pairs) == 3 * 3
     dw = DeviceWorkload(w)
     assert run_step(pk, dw, decode=False) == 0
@@ -202,7 +203,8 @@ def test_placement_invariance_on_gpu(pk):
 
 
 def test_host_buffer_step_matches_device_step(pk):
-    w = W.build_prefix_share_workload(2, 4, 45, 3, 30, 16, 4, 128, 16, "fp16", seed=8)
+    w = W.build_prefix_share_workload(2, 4, 45, 3, 30, 16, 4, 128, 16, "fp16", seed=8,
+                                      allocator=block_allocator)
     dw = DeviceWorkload(w)
     run_step(pk, dw)
     expect = dev_to_bits(dw.out)
@@ -246,7 +248,8 @@ def sample_pairs(w, n, seed):
 
 @pytest.mark.parametrize("name", W.NAMES)
 def test_named_workload(pk, name):
-    w = W.make(name)
+    # prefix_share: the C++ allocator forks the prompts and makes the copy pairs
+    w = W.make(name, allocator=block_allocator)
     dw = DeviceWorkload(w)
     k_before = dw.k_cache.clone()
     err = run_step(pk, dw)

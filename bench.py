@@ -375,24 +375,35 @@ def time_steps(run, stream, step, n):
 
 
 def time_kernel(run, stream, launch, est_ms):
-    """The dominant kernel alone, in its own loop after the timed steps: each
-    launch between two CUDA events on `stream`, for about --kernel-seconds
-    (the clocks sampled meanwhile).  Returns (average launch ms, launches,
-    clocks)."""
+    """The dominant kernel alone, in its own loops after the timed steps, each
+    launch between two CUDA events on `stream`:
+      * as many launches as the timed region has steps, right after it (the
+        roofline's average launch duration);
+      * a sustained loop of about --kernel-seconds, with the clocks sampled
+        meanwhile (a long HBM- or tensor-bound loop can reach the board's
+        power cap, which lowers the SM clock: reported, not hidden).
+    Returns (average ms, launches, sustained average ms, sustained launches,
+    sustained clocks)."""
     import torch
-    n = int(min(20000, max(50, math.ceil(run.args.kernel_seconds * 1e3 / max(est_ms, 1e-3)))))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(n)]
+
+    def loop(n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        torch.cuda.synchronize(run.dev)
+        for a, b in ev:
+            a.record(stream)
+            launch()
+            b.record(stream)
+        torch.cuda.synchronize(run.dev)
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+    n = max(1, run.args.steps)
+    avg = loop(n)
+    n_long = int(min(20000, max(50, math.ceil(run.args.kernel_seconds * 1e3 / max(est_ms, 1e-3)))))
     clocks = ClockSampler(run.local)
     clocks.start()
-    torch.cuda.synchronize(run.dev)
-    for a, b in ev:
-        a.record(stream)
-        launch()
-        b.record(stream)
-    torch.cuda.synchronize(run.dev)
+    avg_long = loop(n_long)
     clk = clocks.stop()
-    return statistics.mean(a.elapsed_time(b) for a, b in ev), n, clk
+    return avg, n, avg_long, n_long, clk
 
 
 def bench_decode(run, workload, headline):
@@ -477,7 +488,7 @@ def bench_decode(run, workload, headline):
     all_bytes = sum_over_ranks(sbytes, dev)
     value = all_bytes / (ms_per_step * 1e-3) / 1e9
     # ---- the decode call alone, for the roofline ------------------------------
-    dec_ms, dec_n, dec_clk = time_kernel(run, stream, decode, ms_per_step)
+    dec_ms, dec_n, sus_ms, sus_n, sus_clk = time_kernel(run, stream, decode, ms_per_step)
     dbytes = decode_bytes(w, kv_elem)
     achieved = dbytes / (dec_ms * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
@@ -536,7 +547,10 @@ def bench_decode(run, workload, headline):
                      "traffic": committed_traffic(workload), "kernel": kernel,
                      "algorithmic_bytes_per_launch": dbytes,
                      "avg_launch_ms": round(dec_ms, 5), "launches_timed": dec_n,
-                     "clocks": dec_clk,
+                     "sustained": {"achieved": round(dbytes / (sus_ms * 1e-3) / 1e9, 2),
+                                   "frac": round(dbytes / (sus_ms * 1e-3) / 1e9 / peak, 4),
+                                   "avg_launch_ms": round(sus_ms, 5), "launches": sus_n,
+                                   "clocks": sus_clk},
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                      if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "gpu_launches": launches_per_step * args.steps,
@@ -715,7 +729,7 @@ def bench_prefill(run, workload, headline):
     if int(err.item()) != 0:
         raise RuntimeError("%s: device error word %d during warm-up" % (workload, int(err.item())))
     ms_per_step, clk = time_steps(run, stream, step, args.steps)
-    kern_ms, kern_n, kern_clk = time_kernel(run, stream, attend, ms_per_step)
+    kern_ms, kern_n, sus_ms, sus_n, sus_clk = time_kernel(run, stream, attend, ms_per_step)
     flops = prefill_flops(w)
     all_flops = sum_over_ranks(flops, dev)
     value = all_flops / (ms_per_step * 1e-3) / 1e12
@@ -737,7 +751,10 @@ def bench_prefill(run, workload, headline):
                                else "paged_prefill_kernel",
                      "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": round(kern_ms, 5), "launches_timed": kern_n,
-                     "clocks": kern_clk,
+                     "sustained": {"achieved": round(flops / (sus_ms * 1e-3) / 1e12, 2),
+                                   "frac": round(flops / (sus_ms * 1e-3) / 1e12 / peak, 4),
+                                   "avg_launch_ms": round(sus_ms, 5), "launches": sus_n,
+                                   "clocks": sus_clk},
                      "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same "
                                     "dense rate)" % peak_kind},
         "gpu_launches": 2 * args.steps,

@@ -216,6 +216,7 @@ struct TcPrefillTraits {
   static constexpr int M = 128;                  // rows of one query tile (one TMEM lane each)
   static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
   static constexpr int NKEY = 64;                // keys per KV tile
+  static constexpr int kSortUnits = 512;         // (sequence, tile) units ranked per CTA
   // KV stages: what fits beside QT query tiles (P lives in TMEM, over S); the
   // cascade prefix pass (one query tile) keeps PKV_PREFIX_STAGES
   static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : PKV_PREFIX_STAGES;
@@ -279,15 +280,63 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
 
-  const int tile = p.q_tiles - 1 - static_cast<int>(blockIdx.x % p.q_tiles);
-  const int unit = blockIdx.x / p.q_tiles;
-  const int kvh = unit % p.num_kv_heads;
-  const int seq = unit / p.num_kv_heads;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   grid_dependency_wait();
   trigger_dependents();
+
+  // Which (sequence, query tile) this CTA serves.  The kv heads of one unit
+  // are adjacent CTAs.  Units are taken longest first (the most keys to
+  // read), so the long ones do not start last and leave a tail: each CTA
+  // ranks every (sequence, tile) unit by its key count from context_lens and
+  // query_start (staged in the K/V ring before any load uses it) and takes
+  // the unit whose rank is its own index.  Beyond kSortUnits units, or in
+  // prefix mode, later query tiles of a sequence simply come first.
+  const int kvh = static_cast<int>(blockIdx.x % p.num_kv_heads);
+  const int rank = static_cast<int>(blockIdx.x / p.num_kv_heads);
+  int seq = rank / p.q_tiles;
+  int tile = p.q_tiles - 1 - rank % p.q_tiles;
+  if constexpr (!Tr::kPrefix) {
+    if (p.num_seqs * p.q_tiles <= Tr::kSortUnits) {
+      int* keys_of = reinterpret_cast<int*>(smem + Tr::OFF_KV);  // [num_seqs] first key, tiles
+      int* chosen = keys_of + 2 * p.num_seqs;
+      const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
+      for (int i = threadIdx.x; i < p.num_seqs; i += Tr::THREADS) {
+        const int c = min(max(p.context_lens[i], 0), cap);
+        const int ql = p.query_start[i + 1] - p.query_start[i];
+        keys_of[2 * i] = c - ql;   // keys before the sequence's first new token
+        keys_of[2 * i + 1] = ql;
+      }
+      if (threadIdx.x == 0) chosen[0] = rank;
+      __syncthreads();
+      const int units = p.num_seqs * p.q_tiles;
+      // keys CTA-unit u reads (-1: no rows); later tiles see more keys
+      auto unit_keys = [&](int u) {
+        const int s = u / p.q_tiles, t = p.q_tiles - 1 - u % p.q_tiles;
+        const int ql = keys_of[2 * s + 1];
+        const int rows = ql * G;
+        if (ql <= 0 || t * ROWS >= rows) return -1;
+        return keys_of[2 * s] + (min(rows, (t + 1) * ROWS) - 1) / G + 1;
+      };
+      for (int u = threadIdx.x; u < units; u += Tr::THREADS) {
+        const int ku = unit_keys(u);
+        int r = 0;
+        for (int v = 0; v < units; ++v) {
+          const int kv = unit_keys(v);
+          r += (kv > ku || (kv == ku && v < u)) ? 1 : 0;
+        }
+        if (r == rank) chosen[0] = u;
+      }
+      __syncthreads();
+      const int u = chosen[0];
+      seq = u / p.q_tiles;
+      tile = p.q_tiles - 1 - u % p.q_tiles;
+      // the ring is written by TMA (the async proxy) later
+      fence_proxy_async_smem();
+      __syncthreads();
+    }
+  }
 
   // seq is a sequence, or in prefix mode a group whose members are the
   // "tokens" q0 .. q0 + q_len - 1 and whose keys are its shared blocks

@@ -376,9 +376,10 @@ def time_steps(run, stream, step, n):
 
 def time_kernel(run, stream, launch, est_ms):
     """The dominant kernel alone, in its own loops after the timed steps, each
-    launch between two CUDA events on `stream`:
-      * as many launches as the timed region has steps, right after it (the
-        roofline's average launch duration);
+    after --warmup untimed launches, each launch between two CUDA events on
+    `stream`:
+      * as many launches as the timed region has steps (the roofline's
+        average launch duration);
       * a sustained loop of about --kernel-seconds, with the clocks sampled
         meanwhile (a long HBM- or tensor-bound loop can reach the board's
         power cap, which lowers the SM clock: reported, not hidden).
@@ -389,6 +390,8 @@ def time_kernel(run, stream, launch, est_ms):
     def loop(n):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n)]
+        for _ in range(run.args.warmup):   # untimed: the clocks come back up after the pause
+            launch()
         torch.cuda.synchronize(run.dev)
         for a, b in ev:
             a.record(stream)
@@ -443,15 +446,19 @@ def bench_decode(run, workload, headline):
     # cache write (+ block copy) + decode (+ reduce); cascade: prefix pass + suffix + reduce
     launches_per_step = (1 + (1 if has_pairs else 0) +
                          (3 if cascade else 1 + (1 if split else 0)))
+    # the sequences longest first (pkv_decode_order, on the host from the
+    # step's lengths): long sequences do not start last; cascade keeps its groups
+    h_order = None if cascade else pk.decode_order(w.context_lens).pin_memory()
+    order = None if cascade else h_order.to(dev)
     inputs = dict(q=q, key=key, val=val, slots=slots, pairs=pairs, tables=tables, lens=lens,
-                  out=out)
+                  out=out, order=order)
 
     def decode(t=inputs):
         if fp8:
             pk.paged_attn_decode_fp8(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
                                      scales[0], scales[1], w.num_kv_heads, w.block_size,
                                      w.max_context_len, partition_size=part_req, workspace=ws,
-                                     dev_err=err, stream=stream)
+                                     dev_err=err, stream=stream, seq_order=t["order"])
         elif cascade:
             pk.paged_attn_decode_cascade(t["out"], t["q"], kc, vc, t["tables"], t["lens"], gstart,
                                          gshared, w.scale, w.num_kv_heads, w.block_size,
@@ -462,7 +469,7 @@ def bench_decode(run, workload, headline):
             pk.paged_attn_decode(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
                                  w.num_kv_heads, w.block_size, w.max_context_len,
                                  partition_size=part_req, workspace=ws, dev_err=err,
-                                 stream=stream)
+                                 stream=stream, seq_order=t["order"])
 
     def step(i=0, t=inputs):
         if has_pairs:
@@ -535,6 +542,8 @@ def bench_decode(run, workload, headline):
                        kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
                        if fp8 else w.dtype,
                        partition_used=part, split_k=split,
+                       seq_order="index order (cascade groups)" if cascade else
+                       "longest first in 256-token buckets (pkv_decode_order on the host)",
                        l2=("no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
                            % (dbytes / 1e9)) if ubytes >= dbytes else
                           ("no flush between steps: %.2f GB of logical KV reads (%.2f GB of "
@@ -575,8 +584,10 @@ def bench_decode(run, workload, headline):
     staging = torch.empty(pk.staging_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim,
                                            w.max_blocks_per_seq, len(w.slot_mapping),
                                            len(w.cow_pairs)), dtype=torch.uint8, device=dev)
+    # the per-step order (computed on the host from the step's lengths) is uploaded too
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_val, h_slots, h_pairs,
-                                                     h_tables, h_lens))
+                                                     h_tables, h_lens)
+              + ((h_order,) if h_order is not None else ()))
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step(i=0):
@@ -587,8 +598,12 @@ def bench_decode(run, workload, headline):
             return
         # E4M3 caches or cascade decode: the same copies through the Python binding's tensors
         with torch.cuda.stream(stream):
-            for dst, src in ((q, h_q), (key, h_key), (val, h_val), (slots, h_slots),
-                             (tables, h_tables), (lens, h_lens)):
+            srcs = [(q, h_q), (key, h_key), (val, h_val), (slots, h_slots), (tables, h_tables),
+                    (lens, h_lens)]
+            if not cascade:
+                h_order.copy_(pk.decode_order(h_lens))
+                srcs.append((order, h_order))
+            for dst, src in srcs:
                 dst.copy_(src, non_blocking=True)
             if has_pairs:
                 pairs.copy_(h_pairs, non_blocking=True)
@@ -625,19 +640,24 @@ def bench_decode(run, workload, headline):
                   "download on three streams, consecutive steps overlapped)"
     else:
         up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-        bufs = [inputs, {k: v.clone() for k, v in inputs.items()}]
+        bufs = [inputs, {k: None if v is None else v.clone() for k, v in inputs.items()}]
         ev_up = [torch.cuda.Event() for _ in range(2)]
         ev_comp = [torch.cuda.Event() for _ in range(2)]
         ev_down = [torch.cuda.Event() for _ in range(2)]
         h_src = dict(q=h_q, key=h_key, val=h_val, slots=h_slots, pairs=h_pairs, tables=h_tables,
-                     lens=h_lens)
+                     lens=h_lens, order=h_order)
+        h_orders = [h_order, None if cascade else h_order.clone().pin_memory()]
 
         def e2e_pipelined(i):
             b, t = i % 2, bufs[i % 2]
             up.wait_event(ev_comp[b])          # step i-2 has finished reading buffer b
+            if not cascade:
+                ev_up[b].synchronize()         # step i-2's upload has read h_orders[b]
+                h_orders[b].copy_(pk.decode_order(h_lens))
+                h_src["order"] = h_orders[b]
             with torch.cuda.stream(up):
                 for k, src in h_src.items():
-                    if k != "pairs" or has_pairs:
+                    if (k != "pairs" or has_pairs) and src is not None:
                         t[k].copy_(src, non_blocking=True)
             ev_up[b].record(up)
             stream.wait_event(ev_up[b])

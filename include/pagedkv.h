@@ -79,6 +79,7 @@ typedef enum { PKV_FP16 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
                                      blocks than max_blocks_per_seq                        */
 #define PKV_DEVERR_TIMEOUT 16u    /* decode: a bounded wait for an async copy gave up      */
 #define PKV_DEVERR_BAD_SCALE 32u  /* *_fp8: a scale that is not finite and > 0            */
+#define PKV_DEVERR_BAD_ORDER 64u  /* *_ordered: an order entry outside [0, num_seqs)       */
 
 /* Library version string, e.g. "pagedkv 0.1.0 sm_100a". */
 const char* pkv_version(void);
@@ -207,6 +208,42 @@ pkv_status pkv_paged_attn_prefill(void* out, const void* q, const void* k_cache,
                                   int head_dim, int block_size, int max_blocks_per_seq,
                                   int max_context_len, int max_query_len, int num_blocks,
                                   pkv_dtype dtype, unsigned* dev_err, void* stream);
+
+/*
+ * Sequence order for decode.  A decode grid takes its (sequence, kv head,
+ * partition) CTAs in order; with a few waves of CTAs of very different
+ * lengths, a long sequence that starts last leaves the GPU partly idle at the
+ * end.  pkv_decode_order (host only) writes into order[num_seqs] the
+ * sequences longest first, by context length in buckets of 256 tokens, index
+ * order within a bucket (so sequences of about the same length, such as the
+ * samples of one prompt that share its blocks, stay adjacent and share L2).
+ * context_lens and order are host arrays.
+ *
+ * pkv_paged_attn_decode_ordered / pkv_paged_attn_decode_fp8_ordered are
+ * pkv_paged_attn_decode / pkv_paged_attn_decode_fp8 with the CTAs taken in
+ * the order of seq_order (device int32 [num_seqs], a permutation of
+ * 0..num_seqs-1, e.g. pkv_decode_order's); results are identical.  An entry
+ * outside [0, num_seqs) sets PKV_DEVERR_BAD_ORDER and that entry's CTAs do
+ * nothing; a repeated entry leaves the missing sequences' outputs unwritten.
+ * The pages do not order sequences; this is a scheduling choice for B200.
+ */
+pkv_status pkv_decode_order(const int32_t* context_lens, int num_seqs, int32_t* order);
+pkv_status pkv_paged_attn_decode_ordered(void* out, const void* q, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         const int32_t* context_lens, const int32_t* seq_order,
+                                         float scale, int num_seqs, int num_heads,
+                                         int num_kv_heads, int head_dim, int block_size,
+                                         int max_blocks_per_seq, int max_context_len,
+                                         int num_blocks, pkv_dtype dtype, int partition_size,
+                                         void* workspace, size_t workspace_bytes,
+                                         unsigned* dev_err, void* stream);
+pkv_status pkv_paged_attn_decode_fp8_ordered(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    float scale, const float* k_scales, const float* v_scales, int num_seqs, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream);
 
 /*
  * pkv_testing_decode_wait — for tests of failure detection; not for serving.

@@ -13,6 +13,7 @@
 // staging areas alternate between steps; events order each area's reuse.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <new>
 
 #include "host_common.h"
@@ -21,7 +22,7 @@ namespace pkv {
 namespace step {
 
 struct StagingLayout {
-  size_t q, key, value, slots, pairs, tables, lens, out, total;
+  size_t q, key, value, slots, pairs, tables, lens, order, out, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -44,6 +45,7 @@ StagingLayout staging_layout(int num_seqs, int num_heads, int num_kv_heads, int 
   l.pairs = take(static_cast<size_t>(num_pairs) * 16);
   l.tables = take(static_cast<size_t>(num_seqs) * max_blocks_per_seq * 4);
   l.lens = take(static_cast<size_t>(num_seqs) * 4);
+  l.order = take(static_cast<size_t>(num_seqs) * 4);   // pipeline: the sequence order
   l.out = take(qo);
   l.total = off;
   return l;
@@ -139,6 +141,7 @@ struct pkv_decode_pipeline {
   pkv_dtype dtype;
   unsigned char* staging[2];  // two areas of `layout.total` bytes
   pkv::step::StagingLayout layout;  // offsets inside one area, sized for the maxima
+  int32_t* order_host;        // pinned [2][num_seqs]: each area's sequence order
   cudaStream_t compute, up, down;
   cudaEvent_t ev_up[2], ev_comp[2], ev_down[2];
   long long steps;
@@ -163,6 +166,7 @@ void pipeline_release(pkv_decode_pipeline* pl) {
   }
   if (pl->up) cudaStreamDestroy(pl->up);
   if (pl->down) cudaStreamDestroy(pl->down);
+  if (pl->order_host) cudaFreeHost(pl->order_host);
 }
 }  // namespace step
 }  // namespace pkv
@@ -212,7 +216,11 @@ extern "C" pkv_status pkv_decode_pipeline_create(
   pl->layout = staging_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                               max_new_tokens, max_pairs);
   pl->compute = as_stream(stream);
-  pkv_status st = cuda_status(cudaStreamCreateWithFlags(&pl->up, cudaStreamNonBlocking));
+  // pinned host memory for the per-step order (no device memory is allocated)
+  pkv_status st = cuda_status(cudaHostAlloc(reinterpret_cast<void**>(&pl->order_host),
+                                            2 * static_cast<size_t>(std::max(num_seqs, 1)) * 4,
+                                            cudaHostAllocDefault));
+  if (st == PKV_OK) st = cuda_status(cudaStreamCreateWithFlags(&pl->up, cudaStreamNonBlocking));
   if (st == PKV_OK) st = cuda_status(cudaStreamCreateWithFlags(&pl->down, cudaStreamNonBlocking));
   for (int b = 0; b < 2 && st == PKV_OK; ++b) {
     st = cuda_status(cudaEventCreateWithFlags(&pl->ev_up[b], cudaEventDisableTiming));
@@ -251,6 +259,15 @@ extern "C" pkv_status pkv_decode_pipeline_step(
   const int b = static_cast<int>(pl->steps & 1);
   unsigned char* st = pl->staging[b];
   const StagingLayout& l = pl->layout;
+  // the sequence order, longest first, computed on the host from this step's
+  // lengths into the area's pinned buffer once step i-2 has uploaded it
+  int32_t* order_host = pl->order_host + static_cast<size_t>(b) * std::max(S, 1);
+  pkv_status r = cuda_status(cudaEventSynchronize(pl->ev_up[b]));
+  if (r != PKV_OK) return r;
+  if (S > 0) {
+    r = pkv_decode_order(context_lens_host, S, order_host);
+    if (r != PKV_OK) return r;
+  }
   const size_t qo = static_cast<size_t>(S) * H * D * 2;
   const size_t kv = static_cast<size_t>(num_new_tokens) * HKV * D * 2;
   struct Copy {
@@ -265,9 +282,10 @@ extern "C" pkv_status pkv_decode_pipeline_step(
       {l.pairs, block_mapping_host, static_cast<size_t>(num_pairs) * 16},
       {l.tables, block_tables_host, static_cast<size_t>(S) * pl->max_blocks_per_seq * 4},
       {l.lens, context_lens_host, static_cast<size_t>(S) * 4},
+      {l.order, order_host, static_cast<size_t>(S) * 4},
   };
   // upload: once step i-2 has finished reading this area's inputs
-  pkv_status r = cuda_status(cudaStreamWaitEvent(pl->up, pl->ev_comp[b], 0));
+  r = cuda_status(cudaStreamWaitEvent(pl->up, pl->ev_comp[b], 0));
   for (const Copy& c : copies) {
     if (r != PKV_OK) return r;
     if (c.bytes == 0) continue;
@@ -286,11 +304,13 @@ extern "C" pkv_status pkv_decode_pipeline_step(
                               reinterpret_cast<const int64_t*>(st + l.slots), num_new_tokens, HKV,
                               D, pl->block_size, num_blocks, pl->dtype, dev_err, cs);
   if (r == PKV_OK)
-    r = pkv_paged_attn_decode(st + l.out, st + l.q, k_cache, v_cache,
-                              reinterpret_cast<const int32_t*>(st + l.tables),
-                              reinterpret_cast<const int32_t*>(st + l.lens), scale, S, H, HKV, D,
-                              pl->block_size, pl->max_blocks_per_seq, max_context_len, num_blocks,
-                              pl->dtype, partition_size, workspace, workspace_bytes, dev_err, cs);
+    r = pkv_paged_attn_decode_ordered(st + l.out, st + l.q, k_cache, v_cache,
+                                      reinterpret_cast<const int32_t*>(st + l.tables),
+                                      reinterpret_cast<const int32_t*>(st + l.lens),
+                                      reinterpret_cast<const int32_t*>(st + l.order), scale, S,
+                                      H, HKV, D, pl->block_size, pl->max_blocks_per_seq,
+                                      max_context_len, num_blocks, pl->dtype, partition_size,
+                                      workspace, workspace_bytes, dev_err, cs);
   if (r == PKV_OK) r = cuda_status(cudaEventRecord(pl->ev_comp[b], pl->compute));
   // download: once this step's output is written
   if (r == PKV_OK) r = cuda_status(cudaStreamWaitEvent(pl->down, pl->ev_comp[b], 0));

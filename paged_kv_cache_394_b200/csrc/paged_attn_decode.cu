@@ -8,6 +8,7 @@
 #include <atomic>
 #include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "host_common.h"
 #include "paged_attn_kernels.cuh"
@@ -328,7 +329,8 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
                          int num_blocks, pkv_dtype dtype, int partition_size, void* workspace,
                          size_t workspace_bytes, unsigned* dev_err, void* stream, bool fp8,
                          const float* k_scales, const float* v_scales,
-                         const CascadeGroups* cascade = nullptr) {
+                         const CascadeGroups* cascade = nullptr,
+                         const int32_t* seq_order = nullptr) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0 || num_blocks <= 0 || partition_size < 0 || !dtype_valid(dtype) ||
       num_heads % num_kv_heads != 0 || !isfinite(scale))
@@ -413,6 +415,7 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   p.shared_blocks = cascade ? cascade->shared_blocks : nullptr;
   p.num_groups = cascade ? cascade->num_groups : 0;
   p.max_shared_blocks = cascade ? cascade->max_shared_blocks : 0;
+  p.seq_order = cascade ? nullptr : seq_order;  // cascade groups stay together
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   p.withhold_first_load = g_withhold_first_load.load(std::memory_order_relaxed);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -484,6 +487,57 @@ extern "C" pkv_status pkv_paged_attn_decode_fp8(
                             max_blocks_per_seq, max_context_len, num_blocks, dtype,
                             partition_size, workspace, workspace_bytes, dev_err, stream, true,
                             k_scales, v_scales);
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_ordered(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    float scale, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err,
+    void* stream) {
+  if (num_seqs > 0 && seq_order == nullptr) return PKV_ERR_INVALID_ARG;
+  return pkv::decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                            partition_size, workspace, workspace_bytes, dev_err, stream, false,
+                            nullptr, nullptr, nullptr, seq_order);
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_fp8_ordered(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    float scale, const float* k_scales, const float* v_scales, int num_seqs, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream) {
+  if (num_seqs > 0 && seq_order == nullptr) return PKV_ERR_INVALID_ARG;
+  return pkv::decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                            partition_size, workspace, workspace_bytes, dev_err, stream, true,
+                            k_scales, v_scales, nullptr, seq_order);
+}
+
+// Longest-first order of the sequences, in buckets of kOrderBucket tokens
+// (index order within a bucket): a counting sort over the bucket numbers.
+extern "C" pkv_status pkv_decode_order(const int32_t* context_lens, int num_seqs,
+                                       int32_t* order) {
+  constexpr int kOrderBucket = 256;
+  constexpr int kOrderMaxBucket = 4095;  // contexts of 1 Mi tokens or more share one bucket
+  if (num_seqs < 0 || (num_seqs > 0 && (context_lens == nullptr || order == nullptr)))
+    return PKV_ERR_INVALID_ARG;
+  auto bucket = [&](int i) {
+    return std::min(std::max(context_lens[i], 0) / kOrderBucket, kOrderMaxBucket);
+  };
+  int top = 0;
+  for (int i = 0; i < num_seqs; ++i) top = std::max(top, bucket(i));
+  // position k = top - bucket: the longest sequences first
+  std::vector<int> start(static_cast<size_t>(top) + 2, 0);
+  for (int i = 0; i < num_seqs; ++i) ++start[top - bucket(i) + 1];
+  for (int k = 1; k <= top + 1; ++k) start[k] += start[k - 1];
+  for (int i = 0; i < num_seqs; ++i) order[start[top - bucket(i)]++] = i;
+  return PKV_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -82,6 +82,9 @@ struct DecodeParams {
   // load, so that its wait runs out and the timeout path runs.
   uint64_t wait_ns;
   int withhold_first_load;
+  // Optional order of the sequences over the grid (a permutation of
+  // 0 .. num_seqs-1, longest first; see pkv_decode_order), else null.
+  const int32_t* seq_order;
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
@@ -108,89 +111,6 @@ __device__ __forceinline__ int cascade_start_block(const DecodeParams& p, int se
     shared = p.max_shared_blocks;
   }
   return min(shared, nblk);
-}
-
-// The order in which the decode grid takes sequences: longer contexts first,
-// in buckets of kOrderBucket tokens, index order within a bucket.  The grid
-// has a few waves of CTAs of very different lengths; a long sequence that
-// starts last leaves the GPU half idle at the end.  Buckets keep sequences of
-// about the same length in index order, so the samples of one prompt (shared
-// prompt blocks) still run side by side and share L2.  With more than
-// kOrderMaxSeqs sequences, or under cascade decode (whose groups must stay
-// together), the grid keeps index order.
-#ifndef PKV_DECODE_ORDER
-#define PKV_DECODE_ORDER 1
-#endif
-constexpr int kOrderBucket = 256;
-constexpr int kOrderBuckets = 128;  // contexts of 32512 tokens or more share the top bucket
-constexpr int kOrderMaxSeqs = 1024;
-constexpr int kOrderScratchInts = kOrderMaxSeqs + kOrderBuckets + 1;
-
-// The sequence of the given rank in that order.  Called by every thread of
-// the CTA after grid_dependency_wait; `scratch` is kOrderScratchInts ints of
-// shared memory that no async copy has touched yet.
-__device__ __forceinline__ int decode_seq_of_rank(const DecodeParams& p, int rank,
-                                                  int* scratch) {
-  if (!PKV_DECODE_ORDER || p.num_seqs > kOrderMaxSeqs || p.group_start != nullptr) return rank;
-  int* bucket = scratch;                    // [num_seqs], descending-order bucket index
-  int* hist = scratch + kOrderMaxSeqs;      // [kOrderBuckets]
-  int* result = hist + kOrderBuckets;
-  const int cap = min(p.max_context_len, p.max_blocks_per_seq * p.block_size);
-  for (int b = threadIdx.x; b < kOrderBuckets; b += blockDim.x) hist[b] = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < p.num_seqs; i += blockDim.x) {
-    const int c = min(max(p.context_lens[i], 0), cap);
-    const int b = kOrderBuckets - 1 - min(c / kOrderBucket, kOrderBuckets - 1);  // longest: 0
-    bucket[i] = b;
-    atomicAdd(&hist[b], 1);
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    // the bucket holding `rank`: lane l sums buckets 4l .. 4l+3, then a warp scan
-    const int lane = threadIdx.x;
-    const int h0 = hist[4 * lane], h1 = hist[4 * lane + 1], h2 = hist[4 * lane + 2],
-              h3 = hist[4 * lane + 3];
-    const int mine = h0 + h1 + h2 + h3;
-    int incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(kFullMask, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const int excl = incl - mine;
-    const unsigned hit = __ballot_sync(kFullMask, rank >= excl && rank < incl);
-    const int src = __ffs(hit) - 1;             // exactly one lane (rank < num_seqs)
-    int b = 0, k = 0;
-    if (lane == src) {
-      int left = rank - excl, j = 0;
-      const int hs[4] = {h0, h1, h2, h3};
-      while (left >= hs[j]) left -= hs[j++];
-      b = 4 * lane + j;
-      k = left;                                 // the k-th sequence of bucket b, by index
-    }
-    b = __shfl_sync(kFullMask, b, src);
-    k = __shfl_sync(kFullMask, k, src);
-    // the k-th index i with bucket[i] == b, 32 indices per round
-    int found = rank;
-    for (int base = 0; base < p.num_seqs; base += 32) {
-      const int i = base + lane;
-      const unsigned m = __ballot_sync(kFullMask, i < p.num_seqs && bucket[i] == b);
-      const int n = __popc(m);
-      if (k < n) {
-        unsigned mm = m;
-        for (int t = 0; t < k; ++t) mm &= mm - 1;   // drop the k lowest set bits
-        found = base + __ffs(mm) - 1;
-        break;
-      }
-      k -= n;
-    }
-    if (lane == 0) *result = found;
-  }
-  __syncthreads();
-  const int seq = *result;
-  fence_proxy_async_smem();  // the ring's next writers are TMA copies (the async proxy)
-  __syncthreads();
-  return seq;
 }
 
 template <int D_, int BS_, int G_, class DT_, int W_, int NS_, class KV_ = DT_>
@@ -225,7 +145,6 @@ struct DecodeTraits {
   static_assert(NV <= NC && NC % NV == 0, "logit layout");
   static_assert(BS % TS == 0, "sub-tiles must tile a block");
   static_assert(COMBINE_BYTES <= RING_BYTES, "combine scratch reuses the ring");
-  static_assert(kOrderScratchInts * 4 <= RING_BYTES, "the ordering scratch reuses the ring");
   static_assert(G <= 8, "alpha slots");
 
   static size_t smem_bytes(int part_blocks) {
@@ -457,7 +376,13 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   // write); wait for it before reading anything, then let the next one start.
   grid_dependency_wait();
   trigger_dependents();
-  const int seq = decode_seq_of_rank(p, unit / p.num_kv_heads, reinterpret_cast<int*>(smem));
+  // the sequence this CTA serves: in index order, or in the caller's order
+  const int rank = unit / p.num_kv_heads;
+  const int seq = p.seq_order != nullptr ? p.seq_order[rank] : rank;
+  if (static_cast<unsigned>(seq) >= static_cast<unsigned>(p.num_seqs)) {
+    if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
+    return;
+  }
 
   const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
   int ctx = p.context_lens[seq];
@@ -653,7 +578,6 @@ struct MmaTraits {
   static_assert(G >= (kFp8 ? 1 : 2) && G <= 8, "tensor-core path: up to 8 heads per kv head");
   static_assert(BS % SUB == 0 && D % 64 == 0 && ROW_BYTES % 128 == 0, "shape");
   static_assert(COMBINE_BYTES <= RING_BYTES, "combine scratch reuses the ring");
-  static_assert(kOrderScratchInts * 4 <= RING_BYTES, "the ordering scratch reuses the ring");
   static size_t smem_bytes(int part_blocks) {
     return 1024 + static_cast<size_t>(RING_BYTES) + BAR_BYTES +
            static_cast<size_t>(part_blocks) * 4;
@@ -903,7 +827,13 @@ __global__ void __launch_bounds__(Tr::THREADS)
 
   grid_dependency_wait();
   trigger_dependents();
-  const int seq = decode_seq_of_rank(p, unit / p.num_kv_heads, reinterpret_cast<int*>(smem));
+  // the sequence this CTA serves: in index order, or in the caller's order
+  const int rank = unit / p.num_kv_heads;
+  const int seq = p.seq_order != nullptr ? p.seq_order[rank] : rank;
+  if (static_cast<unsigned>(seq) >= static_cast<unsigned>(p.num_seqs)) {
+    if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
+    return;
+  }
 
   const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
   int ctx = p.context_lens[seq];

@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_OUT_OF_BLOCKS = range(6)
 FP16, BF16, FP8_E4M3 = 0, 1, 2
 (DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_PAIR, DEVERR_BAD_CONTEXT, DEVERR_TIMEOUT,
- DEVERR_BAD_SCALE) = (1, 2, 4, 8, 16, 32)
+ DEVERR_BAD_SCALE, DEVERR_BAD_ORDER) = (1, 2, 4, 8, 16, 32, 64)
 
 _vp, _i, _i64, _f, _sz, _u = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                               ctypes.c_size_t, ctypes.c_uint)
@@ -68,6 +68,13 @@ _staging_bytes = _proto("pkv_decode_step_staging_bytes", _sz, _i, _i, _i, _i, _i
 _decode_step_host = _proto("pkv_decode_step_host", _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp,
                            _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
                            _vp, _sz, _vp, _vp)
+_decode_order = _proto("pkv_decode_order", _i, _vp, _i, _vp)
+_paged_attn_decode_ordered = _proto("pkv_paged_attn_decode_ordered", _i, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz,
+                                    _vp, _vp)
+_paged_attn_decode_fp8_ordered = _proto("pkv_paged_attn_decode_fp8_ordered", _i, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                        _i, _i, _i, _i, _vp, _sz, _vp, _vp)
 _testing_decode_wait = _proto("pkv_testing_decode_wait", _i, ctypes.c_uint64, _i)
 _pipeline_staging_bytes = _proto("pkv_decode_pipeline_staging_bytes", _sz, _i, _i, _i, _i, _i, _i,
                                  _i)
@@ -202,10 +209,23 @@ def alloc_workspace(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
 
 
+def decode_order(context_lens):
+    """Longest-first sequence order (int32 host tensor) for a host tensor or
+    array of context lengths; see pkv_decode_order."""
+    lens = torch.as_tensor(context_lens, dtype=torch.int32).contiguous()
+    if lens.is_cuda:
+        raise ValueError("context_lens must be on the host")
+    order = torch.empty_like(lens)
+    _check(_decode_order(_ptr(lens), lens.numel(), _ptr(order)), "decode_order")
+    return order
+
+
 def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
                       block_size, max_context_len, partition_size=0, workspace=None,
-                      dev_err=None, stream=None):
-    """Paged decode attention; writes out [S, H, D].  See include/pagedkv.h."""
+                      dev_err=None, stream=None, seq_order=None):
+    """Paged decode attention; writes out [S, H, D].  With ``seq_order`` (a
+    device int32 permutation, e.g. decode_order's) the CTAs take the
+    sequences in that order.  See include/pagedkv.h."""
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     _dev(block_tables, "block_tables", torch.int32)
@@ -225,6 +245,18 @@ def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scal
             workspace.record_stream(stream)   # the temporary must outlive the launch
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if seq_order is not None:
+        _dev(seq_order, "seq_order", torch.int32)
+        if seq_order.shape != (s,):
+            raise ValueError("seq_order must be [S]")
+        _check(_paged_attn_decode_ordered(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(block_tables), _ptr(context_lens), _ptr(seq_order),
+                                          float(scale), s, h, hkv, d, bs, block_tables.shape[1],
+                                          max_context_len, num_blocks, _dtype_code(q),
+                                          partition_size, ws_ptr, ws_bytes, _ptr(dev_err),
+                                          _stream(stream)),
+               "paged_attn_decode_ordered")
+        return
     _check(_paged_attn_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                               _ptr(block_tables), _ptr(context_lens), float(scale), s, h, hkv, d,
                               bs, block_tables.shape[1], max_context_len, num_blocks,
@@ -322,9 +354,10 @@ def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scales, 
 
 def paged_attn_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scales,
                           v_scales, num_kv_heads, block_size, max_context_len, partition_size=0,
-                          workspace=None, dev_err=None, stream=None):
+                          workspace=None, dev_err=None, stream=None, seq_order=None):
     """Paged decode attention over E4M3 caches (values = code * scale of the
-    kv head); q and out are 16-bit.  See include/pagedkv.h."""
+    kv head); q and out are 16-bit.  ``seq_order`` as for paged_attn_decode.
+    See include/pagedkv.h."""
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     _dev(block_tables, "block_tables", torch.int32)
@@ -347,6 +380,19 @@ def paged_attn_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, 
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     ks, vs = _scales_for(k_scales, v_scales, hkv, q.device, stream)
+    if seq_order is not None:
+        _dev(seq_order, "seq_order", torch.int32)
+        if seq_order.shape != (s,):
+            raise ValueError("seq_order must be [S]")
+        _check(_paged_attn_decode_fp8_ordered(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                              _ptr(block_tables), _ptr(context_lens),
+                                              _ptr(seq_order), float(scale), _ptr(ks), _ptr(vs),
+                                              s, h, hkv, d, bs, block_tables.shape[1],
+                                              max_context_len, num_blocks, _dtype_code(q),
+                                              partition_size, ws_ptr, ws_bytes, _ptr(dev_err),
+                                              _stream(stream)),
+               "paged_attn_decode_fp8_ordered")
+        return
     _check(_paged_attn_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                   _ptr(block_tables), _ptr(context_lens), float(scale),
                                   _ptr(ks), _ptr(vs), s, h, hkv, d, bs,

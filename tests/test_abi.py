@@ -239,3 +239,19 @@ def test_testing_wait_hook_validates_on_the_host():
         with pytest.raises(pk.PagedKVError):
             pk.testing_decode_wait(bad, False)
     pk.testing_decode_wait(2_000_000_000, False)      # the default, accepted
+
+
+@pytest.mark.parametrize("seed,n", [(0, 0), (1, 1), (2, 64), (3, 257), (4, 1000)])
+def test_decode_order_is_longest_first_by_bucket(seed, n):
+    """pkv_decode_order: a permutation; buckets of 256 tokens in descending
+    order; index order inside a bucket (the definition, restated with a
+    stable lexicographic sort)."""
+    import numpy as np
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, 40000, size=n).astype(np.int32)
+    lens[: n // 3] = rng.integers(1000, 1300, size=n // 3)      # many ties in one bucket
+    order = pk.decode_order(lens).numpy()
+    assert sorted(order.tolist()) == list(range(n))
+    expect = np.lexsort((np.arange(n), -(lens // 256)))
+    assert np.array_equal(order, expect)

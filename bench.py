@@ -567,7 +567,7 @@ def bench_decode(run, workload, headline):
     }
     if sharing is not None:
         line["shared_blocks"] = sharing
-    if not headline:
+    if not headline or args.no_e2e:
         del ws
         return line
 
@@ -780,7 +780,7 @@ def bench_prefill(run, workload, headline):
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
-    if not headline:
+    if not headline or args.no_e2e:
         return line
 
     # end to end through the Python API: pinned host inputs in, output back
@@ -1217,6 +1217,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-other", action="store_true",
                     help="time the named workload only (the default run also times the other "
                          "configurations as nested objects of the headline line)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffer) loops, e.g. under a profiler")
     ap.add_argument("--kernel-seconds", type=float, default=1.0,
                     help="length of the loop that times the dominant kernel alone")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

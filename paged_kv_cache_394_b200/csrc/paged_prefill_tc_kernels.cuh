@@ -212,7 +212,13 @@ struct TcPrefillTraits {
   static constexpr bool kFp8 = FP8_;
   using DT = DT_;
   using T = typename DT::T;
-  static constexpr bool kBf16 = std::is_same<DT, Bf16>::value;
+  // Element type of the MMAs and of P.  Over E4M3 caches it is fp16 for bf16
+  // queries too: the codes widen exactly to fp16, the query tiles are rounded
+  // to fp16 in shared memory once per CTA (saturating at +-65504, as the E4M3
+  // decode does), and fp16 P needs no hi + lo split, so P.V runs once.
+  using MT = std::conditional_t<kFp8, Fp16, DT>;
+  static constexpr bool kBf16 = std::is_same<MT, Bf16>::value;
+  static constexpr bool kQToFp16 = kFp8 && std::is_same<DT, Bf16>::value;
   static constexpr int M = 128;                  // rows of one query tile (one TMEM lane each)
   static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
   static constexpr int NKEY = 64;                // keys per KV tile
@@ -237,8 +243,9 @@ struct TcPrefillTraits {
   static constexpr int OFF_BAR = OFF_STG + 2 * NSTG * STG_TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
   // per query tile s_full[2], p_full[2], o_done[2]; then (E4M3) the staging
-  // slots' stg_full[2][NSTG]; then the TMEM address slot
-  static constexpr int NBAR = 1 + 4 * NS + 6 * QT + 2 * NSTG;
+  // slots' stg_full[2][NSTG]; then q_ready (query tiles rounded to fp16);
+  // then the TMEM address slot
+  static constexpr int NBAR = 1 + 4 * NS + 6 * QT + 2 * NSTG + 1;
   // the softmax reference max moves only when a row max exceeds it by more
   // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
   static constexpr float kRescaleThreshold = 8.f;
@@ -278,6 +285,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   auto bar_stg = [&](int kind, int s) {
     return smem_addr(bars + 1 + 4 * NS + 6 * QT + kind * Tr::NSTG + s);
   };
+  const uint32_t bar_q_ready = smem_addr(bars + Tr::NBAR - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
 
   const int warp = threadIdx.x >> 5;
@@ -397,6 +405,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       mbar_init(bar_stg(0, s), 1);
       mbar_init(bar_stg(1, s), 1);
     }
+    mbar_init(bar_q_ready, 4 * QT);  // one arrival per softmax warp
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -521,8 +530,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           uint32_t h[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            h[2 * e] = tc::e4m3x2_to(w[e] & 0xffffu, DT());
-            h[2 * e + 1] = tc::e4m3x2_to(w[e] >> 16, DT());
+            h[2 * e] = tc::e4m3x2_to(w[e] & 0xffffu, typename Tr::MT());
+            h[2 * e + 1] = tc::e4m3x2_to(w[e] >> 16, typename Tr::MT());
           }
           const uint32_t row = dst + (c >> 2) * Tr::KV_HALF + r * 128;
           const int c0 = (c & 3) * 2;
@@ -608,7 +617,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   } else if (warp == 1 || warp == Tr::PV_WARP) {
     // ---- MMA issuers ----------------------------------------------------------------
     if (lane == 0) {
-      bool ok = warp != 1 || mbar_wait_bounded(bar_q, 0);  // only S reads Q
+      // only S reads Q (rounded to fp16 first when the MMAs run in fp16 for bf16 queries)
+      bool ok = warp != 1 || mbar_wait_bounded(Tr::kQToFp16 ? bar_q_ready : bar_q, 0);
       // Operand descriptors as a base plus a start-address step: the 14-bit
       // start field holds address / 16 and never carries, since shared memory
       // ends below 2^18 bytes.  This keeps the issuing thread's work per MMA to
@@ -711,9 +721,33 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           warp == 3 && lane == 0 && tile == 0)
         set_err(p.err, PKV_DEVERR_BAD_SCALE);
     }
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < my_tiles; ++t) {
+    if constexpr (Tr::kQToFp16) {
+      // round this query tile from bf16 to fp16 in place (the MMAs run in
+      // fp16 over E4M3 caches); every softmax warp arrives, whatever its rows
+      ok = __all_sync(kFullMask, mbar_wait_bounded(bar_q, 0));
+      if (ok) {
+        unsigned char* qt = smem + Tr::OFF_Q + qg * Tr::Q_TILE;
+        for (int idx = r; idx < Tr::Q_TILE / 16; idx += 128) {
+          uint4* at = reinterpret_cast<uint4*>(qt + idx * 16);
+          const uint4 u = *at;
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t h[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = fminf(fmaxf(__uint_as_float(w[e] << 16), -65504.f), 65504.f);
+            const float hi = fminf(fmaxf(__uint_as_float(w[e] & 0xffff0000u), -65504.f), 65504.f);
+            h[e] = pack2(lo, hi, Fp16());
+          }
+          *at = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+      }
+      fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_q_ready);
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int t = 0; ok && t < my_tiles; ++t) {
       const int kv0 = t * NKEY;
       ok = mbar_wait_bounded(bar_s_full(qg, t & 1), (t >> 1) & 1);
       if (!__all_sync(kFullMask, ok)) {
@@ -808,7 +842,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float a = s[32 * h + 2 * e], b = s[32 * h + 2 * e + 1];
-            w[e] = pack2(a, b, DT());
+            w[e] = pack2(a, b, typename Tr::MT());
             if constexpr (Tr::kBf16)
               wl[e] = pack2(a - __uint_as_float(w[e] << 16),
                             b - __uint_as_float(w[e] & 0xffff0000u), Bf16());

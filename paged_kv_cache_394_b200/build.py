@@ -1,12 +1,15 @@
 """Build ``libpagedkv.so`` in-tree with nvcc for sm_100a.
 
-    python -m paged_kv_cache_394_b200.build [--verbose-ptxas] [-j N]
+    python -m paged_kv_cache_394_b200.build [--verbose-ptxas] [-j N] [--force]
+                                            [--define NAME=VALUE ...]
 
 Each source under ``csrc/`` is compiled to an object in ``_build/`` (in
 parallel, skipped when up to date), then linked into
 ``paged_kv_cache_394_b200/libpagedkv.so`` with the CUDA runtime linked
 statically, so the library does not depend on which libcudart the host
-process has loaded.
+process has loaded.  ``--define`` passes a preprocessor definition to every
+source (the tuning and comparison switches the sources document); objects
+built with other definitions are rebuilt.
 """
 
 import argparse
@@ -45,13 +48,16 @@ def headers_mtime():
     return max(os.path.getmtime(p) for p in paths)
 
 
-def compile_one(src, verbose_ptxas, force):
+def compile_one(src, verbose_ptxas, force, defines=()):
     obj = os.path.join(BUILD, src + ".o")
     srcp = os.path.join(CSRC, src)
-    if (not force and os.path.exists(obj)
+    stamp = obj + ".defines"
+    tag = " ".join(defines)
+    same_defines = os.path.exists(stamp) and open(stamp).read() == tag
+    if (not force and same_defines and os.path.exists(obj)
             and os.path.getmtime(obj) >= max(os.path.getmtime(srcp), headers_mtime())):
         return obj, ""
-    cmd = [nvcc()] + ARCH + COMMON + ["-c", srcp, "-o", obj]
+    cmd = [nvcc()] + ARCH + COMMON + ["-D" + d for d in defines] + ["-c", srcp, "-o", obj]
     if verbose_ptxas and src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"]
     if src.endswith(".cpp"):
@@ -59,14 +65,17 @@ def compile_one(src, verbose_ptxas, force):
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, r.stdout, r.stderr))
+    with open(stamp, "w") as f:
+        f.write(tag)
     return obj, r.stderr
 
 
-def build(verbose_ptxas=False, jobs=None, force=False, quiet=True):
+def build(verbose_ptxas=False, jobs=None, force=False, quiet=True, defines=()):
     os.makedirs(BUILD, exist_ok=True)
     srcs = sources()
+    defines = tuple(sorted(defines))
     with ThreadPoolExecutor(max_workers=jobs or min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(lambda s: compile_one(s, verbose_ptxas, force), srcs))
+        results = list(ex.map(lambda s: compile_one(s, verbose_ptxas, force, defines), srcs))
     objs = [o for o, _ in results]
     if verbose_ptxas:
         for _, log in results:
@@ -91,8 +100,9 @@ def main():
     ap.add_argument("--verbose-ptxas", action="store_true")
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-j", type=int, default=None)
+    ap.add_argument("--define", action="append", default=[], metavar="NAME=VALUE")
     a = ap.parse_args()
-    build(a.verbose_ptxas, a.j, a.force, quiet=False)
+    build(a.verbose_ptxas, a.j, a.force, quiet=False, defines=a.define)
 
 
 if __name__ == "__main__":

@@ -56,10 +56,28 @@ KernelEntry make_entry() {
   return KernelEntry{paged_decode_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(0)};
 }
 
+// Built with PKV_DECODE_GQA_CUDA_CORES=1 (python -m paged_kv_cache_394_b200.build
+// --define PKV_DECODE_GQA_CUDA_CORES=1), 16-bit caches run every group size on
+// the CUDA-core kernel: the comparison that shows what the tensor cores buy
+// for grouped-query decode.  The default build uses them for G >= 2.
+#ifndef PKV_DECODE_GQA_CUDA_CORES
+#define PKV_DECODE_GQA_CUDA_CORES 0
+#endif
+
 template <int D, int BS, class DT>
 KernelEntry entry_for_group(int g) {
+#if PKV_DECODE_GQA_CUDA_CORES
+  switch (g) {
+    case 1: return make_entry<D, BS, 1, DT>();
+    case 2: return make_entry<D, BS, 2, DT>();
+    case 4: return make_entry<D, BS, 4, DT>();
+    case 8: return make_entry<D, BS, 8, DT>();
+    default: return KernelEntry{nullptr, 0, 0};
+  }
+#else
   // one query head per kv head: the CUDA-core kernel (G >= 2 uses the tensor cores)
   return g == 1 ? make_entry<D, BS, 1, DT>() : KernelEntry{nullptr, 0, 0};
+#endif
 }
 
 template <class DT>
@@ -368,7 +386,7 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
 
   // 16-bit: G >= 2 on the tensor cores, G = 1 on the CUDA cores;
   // E4M3: every G on the tensor cores at head_dim 128, on the CUDA cores at 64
-  const bool use_mma = fp8 ? head_dim == 128 : group >= 2;
+  const bool use_mma = fp8 ? head_dim == 128 : group >= 2 && !PKV_DECODE_GQA_CUDA_CORES;
   const KernelEntry ke = use_mma ? KernelEntry{nullptr, 0, 0}
                          : fp8   ? fp8_decode_entry(head_dim, block_size, group, dtype)
                                  : decode_entry(head_dim, block_size, group, dtype);

@@ -849,45 +849,8 @@ __global__ void __launch_bounds__(Tr::THREADS)
     return;
   }
 
-  // The context length, q, the E4M3 scales and (without cascade) the
-  // partition's table slice depend only on the sequence: their loads are
-  // issued together so that their latencies overlap (see paged_decode_kernel).
   const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
   int ctx = p.context_lens[seq];
-  // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) + {0,1,8,9}
-  // (E4M3 cache: dims 16ks + 4(lane%4) + {0,1,2,3}, the permuted k order of
-  // mma_sub_block_fp8, as fp16)
-  uint32_t qf[KS][2];
-  const int qn = lane >> 2;
-  {
-    const int c = lane & 3;
-    const T* qrow = static_cast<const T*>(p.q) +
-                    (static_cast<size_t>(seq) * p.num_heads + kvh * G + min(qn, G - 1)) * D;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      if constexpr (Tr::kFp8) {
-        const uint2 u =
-            qn < G ? *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c) : make_uint2(0, 0);
-        qf[ks][0] = u.x;
-        qf[ks][1] = u.y;
-      } else {
-        qf[ks][0] = qn < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
-        qf[ks][1] = qn < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
-      }
-    }
-  }
-  float k_scale = 1.f, v_scale = 1.f;
-  if constexpr (Tr::kFp8) {
-    k_scale = p.k_scales[kvh];
-    v_scale = p.v_scales[kvh];
-  }
-  const bool cascade = p.group_start != nullptr;
-  const int32_t* seq_row = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
-  if (!cascade) {
-    const int b0 = part * p.part_blocks;
-    const int n0 = min(p.part_blocks, p.max_blocks_per_seq - b0);
-    for (int i = threadIdx.x; i < n0; i += Tr::THREADS) tbl[i] = seq_row[b0 + i];
-  }
   if (ctx < 0 || ctx > ctx_cap) {
     if (threadIdx.x == 0 && part == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
     ctx = min(max(ctx, 0), ctx_cap);
@@ -896,6 +859,7 @@ __global__ void __launch_bounds__(Tr::THREADS)
   const int start_blk =
       cascade_start_block(p, seq, nblk, threadIdx.x == 0 && part == 0 && kvh == 0);
   const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
+  const bool cascade = p.group_start != nullptr;
   if (part >= (cascade ? nparts : max(nparts, 1))) return;
   const bool direct = !cascade && nparts <= 1;
   const int blk_begin = start_blk + part * p.part_blocks;
@@ -903,9 +867,9 @@ __global__ void __launch_bounds__(Tr::THREADS)
   const int sb_begin = blk_begin * SPB;
   const int nsb = max(0, min((ctx + Tr::SUB - 1) / Tr::SUB, (blk_begin + nb) * SPB) - sb_begin);
 
-  if (cascade) {
-    for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = seq_row[blk_begin + i];
-  }
+  const int32_t* trow =
+      p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq + blk_begin;
+  for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = trow[i];
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < NS; ++s) mbar_init(smem_addr(bars + warp * NS + s), 1);
@@ -913,25 +877,44 @@ __global__ void __launch_bounds__(Tr::THREADS)
   }
   __syncthreads();
 
+  // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) + {0,1,8,9}
+  // (E4M3 cache: dims 16ks + 4(lane%4) + {0,1,2,3}, the permuted k order of
+  // mma_sub_block_fp8, as fp16)
+  uint32_t qf[KS][2];
   float qscale = p.qscale;
-  if constexpr (Tr::kFp8) {
-    if constexpr (std::is_same<typename Tr::DT, Bf16>::value) {
-      // bf16 -> fp16 for the fp16 mma; magnitudes beyond fp16 saturate
-      auto cv = [](uint32_t w) {
-        const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.f), 65504.f);
-        const float hi = fminf(fmaxf(__uint_as_float(w & 0xffff0000u), -65504.f), 65504.f);
-        return pack2(lo, hi, Fp16());
-      };
+  {
+    const int n = lane >> 2;
+    const int c = lane & 3;
+    const T* qrow = static_cast<const T*>(p.q) +
+                    (static_cast<size_t>(seq) * p.num_heads + kvh * G + min(n, G - 1)) * D;
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        qf[ks][0] = cv(qf[ks][0]);
-        qf[ks][1] = cv(qf[ks][1]);
+    for (int ks = 0; ks < KS; ++ks) {
+      if constexpr (Tr::kFp8) {
+        uint2 u = n < G ? *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c) : make_uint2(0, 0);
+        if constexpr (std::is_same<typename Tr::DT, Bf16>::value) {
+          // bf16 -> fp16 for the fp16 mma; magnitudes beyond fp16 saturate
+          auto cv = [](uint32_t w) {
+            const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.f), 65504.f);
+            const float hi = fminf(fmaxf(__uint_as_float(w & 0xffff0000u), -65504.f), 65504.f);
+            return pack2(lo, hi, Fp16());
+          };
+          u = make_uint2(cv(u.x), cv(u.y));
+        }
+        qf[ks][0] = u.x;
+        qf[ks][1] = u.y;
+      } else {
+        qf[ks][0] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c) : 0u;
+        qf[ks][1] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c) : 0u;
       }
     }
-    if (!(k_scale > 0.f && k_scale < INFINITY && v_scale > 0.f && v_scale < INFINITY) &&
-        threadIdx.x == 0 && part == 0)
-      set_err(p.err, PKV_DEVERR_BAD_SCALE);
-    qscale *= k_scale;
+    if constexpr (Tr::kFp8) {
+      const float ks = p.k_scales[kvh];
+      const float vs = p.v_scales[kvh];
+      if (!(ks > 0.f && ks < INFINITY && vs > 0.f && vs < INFINITY) && threadIdx.x == 0 &&
+          part == 0)
+        set_err(p.err, PKV_DEVERR_BAD_SCALE);
+      qscale *= ks;
+    }
   }
   float acc[KS][4];
 #pragma unroll

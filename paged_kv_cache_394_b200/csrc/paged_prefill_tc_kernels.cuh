@@ -230,7 +230,10 @@ struct TcPrefillTraits {
   // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
   // P.V issuer
   static constexpr int PV_WARP = 3 + 4 * QT;
-  static constexpr int THREADS = (PV_WARP + 1) * 32;
+  // E4M3: two warps per kind widen each tile (the producer warp and a helper,
+  // warps PV_WARP + 1 for K and PV_WARP + 2 for V), 32 rows each
+  static constexpr int NWIDEN = kFp8 ? 2 : 1;
+  static constexpr int THREADS = (PV_WARP + 1 + (NWIDEN - 1) * 2) * 32;
   // shared-memory layout (all 1024-byte aligned)
   static constexpr int Q_HALF = M * 128;         // [128 rows][64 dims] = 16 KiB
   static constexpr int Q_TILE = 2 * Q_HALF;
@@ -244,8 +247,11 @@ struct TcPrefillTraits {
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
   // per query tile s_full[2], p_full[2], o_done[2]; then (E4M3) the staging
   // slots' stg_full[2][NSTG]; then q_ready (query tiles rounded to fp16);
-  // then the TMEM address slot
-  static constexpr int NBAR = 1 + 4 * NS + 6 * QT + 2 * NSTG + 1;
+  // then (E4M3) stg_read[2][NSTG] (both widening warps are done with a
+  // slot); then the TMEM address slot
+  static constexpr int BAR_Q_READY = 1 + 4 * NS + 6 * QT + 2 * NSTG;
+  static constexpr int BAR_STG_READ = BAR_Q_READY + 1;
+  static constexpr int NBAR = BAR_STG_READ + 2 * NSTG;
   // the softmax reference max moves only when a row max exceeds it by more
   // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
   static constexpr float kRescaleThreshold = 8.f;
@@ -285,7 +291,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   auto bar_stg = [&](int kind, int s) {
     return smem_addr(bars + 1 + 4 * NS + 6 * QT + kind * Tr::NSTG + s);
   };
-  const uint32_t bar_q_ready = smem_addr(bars + Tr::NBAR - 1);
+  const uint32_t bar_q_ready = smem_addr(bars + Tr::BAR_Q_READY);
+  auto bar_stg_read = [&](int kind, int s) {
+    return smem_addr(bars + Tr::BAR_STG_READ + kind * Tr::NSTG + s);
+  };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Tr::NBAR);
 
   const int warp = threadIdx.x >> 5;
@@ -389,9 +398,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     // one arrival per softmax warp of the query tile
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_k_full(s), Tr::NWIDEN);  // E4M3: each widening warp arrives
       mbar_init(bar_k_empty(s), 1);
-      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_v_full(s), Tr::NWIDEN);
       mbar_init(bar_v_empty(s), 1);
     }
     for (int q = 0; q < QT; ++q) {
@@ -404,6 +413,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     for (int s = 0; s < Tr::NSTG; ++s) {
       mbar_init(bar_stg(0, s), 1);
       mbar_init(bar_stg(1, s), 1);
+      mbar_init(bar_stg_read(0, s), Tr::NWIDEN);
+      mbar_init(bar_stg_read(1, s), Tr::NWIDEN);
     }
     mbar_init(bar_q_ready, 4 * QT);  // one arrival per softmax warp
     fence_mbar_init();
@@ -417,16 +428,18 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == 2) {
+  if (warp == 0 || warp == 2 || warp > Tr::PV_WARP) {
     // ---- producers: warp 0 loads Q and the K tiles, warp 2 the V tiles ---------------
     // K of a stage is released once S has read it, V once P.V has, so the K
-    // loads can run further ahead than the V loads.
-    const bool is_k = warp == 0;
+    // loads can run further ahead than the V loads.  E4M3: a helper warp per
+    // kind widens half of each tile.
+    const bool helper = warp > Tr::PV_WARP;
+    const bool is_k = warp == 0 || warp == Tr::PV_WARP + 1;
     // prefix mode: the group's first member holds the shared blocks' ids
     const int32_t* trow = p.block_tables +
                           static_cast<size_t>(Tr::kPrefix ? q0 : seq) * p.max_blocks_per_seq;
     const int nblk = (nkv + BS - 1) / BS;
-    if (is_k && lane == 0) {
+    if (warp == 0 && lane == 0) {
       mbar_arrive_expect_tx(bar_q, QT * Tr::Q_TILE);
 #pragma unroll
       for (int q = 0; q < QT; ++q) {
@@ -500,7 +513,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         __syncwarp();
       };
-      for (int t = 0; t < min(Tr::NSTG, ntiles); ++t) stage_codes(t);
+      if (!helper)
+        for (int t = 0; t < min(Tr::NSTG, ntiles); ++t) stage_codes(t);
       for (int t = 0; t < ntiles; ++t) {
         const int stage = t % NS;
         bool ok = true;
@@ -512,15 +526,17 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         ok = __shfl_sync(kFullMask, ok, 0);
         if (!ok) break;
-        // 64 rows x 8 chunks of 16 codes; lane takes chunks lane, lane + 32, ...
-        // Chunk c of row r (dims 16c .. 16c + 15) becomes 16-bit chunks 2(c % 4)
-        // and 2(c % 4) + 1 of row r in dim half c / 4; both layouts use the
-        // 128-byte swizzle (16-byte chunk index XOR row % 8).
+        // 64 rows x 8 chunks of 16 codes; this warp's half of the rows, lane
+        // takes chunks lane, lane + 32, ...  Chunk c of row r (dims 16c ..
+        // 16c + 15) becomes 16-bit chunks 2(c % 4) and 2(c % 4) + 1 of row r in
+        // dim half c / 4; both layouts use the 128-byte swizzle (16-byte chunk
+        // index XOR row % 8).
         const uint32_t src = stg0 + (t % Tr::NSTG) * Tr::STG_TILE;
         const uint32_t dst = sbase + Tr::OFF_KV + stage * Tr::STAGE + (is_k ? 0 : 2 * Tr::KV_HALF);
+        const int first = helper ? 256 : 0;
 #pragma unroll 4
-        for (int k = 0; k < 16; ++k) {
-          const int idx = lane + 32 * k;
+        for (int k = 0; k < 16 / Tr::NWIDEN; ++k) {
+          const int idx = first + lane + 32 * k;
           const int r = idx >> 3, c = idx & 7;
           uint32_t w[4];
           asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -543,12 +559,24 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
                        "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
                        : "memory");
         }
-        // the widened tile is for the MMAs (async proxy); the slot's codes are
-        // read, so TMA may refill it
+        // the widened rows are for the MMAs (async proxy); this warp is done
+        // with the slot's codes
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(is_k ? bar_k_full(stage) : bar_v_full(stage));
-        if (t + Tr::NSTG < ntiles) stage_codes(t + Tr::NSTG);
+        if (lane == 0) {
+          mbar_arrive(is_k ? bar_k_full(stage) : bar_v_full(stage));
+          mbar_arrive(bar_stg_read(kind, t % Tr::NSTG));
+        }
+        if (!helper && t + Tr::NSTG < ntiles) {
+          // TMA refills the slot once both widening warps have read it
+          bool read = true;
+          if (lane == 0) {
+            read = mbar_wait_bounded(bar_stg_read(kind, t % Tr::NSTG), (t / Tr::NSTG) & 1);
+            if (!read) set_err(p.err, PKV_DEVERR_TIMEOUT);
+          }
+          if (!__shfl_sync(kFullMask, read, 0)) break;
+          stage_codes(t + Tr::NSTG);
+        }
       }
     } else {
       for (int t = 0; t < ntiles; ++t) {

@@ -273,9 +273,11 @@ constexpr int kSlots = 2 * 148;            // resident decode CTAs: two per SM, 
 // Partition size in tokens.  With enough (sequence, kv head) units to fill the
 // GPU and contexts of at most 2048 tokens, one pass (no reduce) is fastest.
 // Otherwise contexts are cut so there are about four CTAs per resident slot,
-// in partitions of 256..1024 tokens: measured on B200, 512-token partitions
-// are 4-8 % slower than 1024 (a CTA's start-up is not amortised) and one
-// pass over 4096-token contexts leaves an 8 % tail.
+// in partitions of 256..2048 tokens.  Measured on B200 with the sequences
+// taken longest first (decode kernel GB/s, partition 512 / 1024 / 2048):
+// GQA chat 5972 / 6310 / 6447, its E4M3 form 4632 / 5209 / 5522 (a CTA's
+// start-up is not amortised over short partitions).  In index order the GQA
+// chat batch read 6374 at 1024 against 6225 at 2048.
 int choose_partition(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
                      int requested) {
   if (requested > 0) return requested;
@@ -286,7 +288,7 @@ int choose_partition(int num_seqs, int num_kv_heads, int block_size, int max_con
   const long long parts = std::max(1LL, (4LL * kSlots + units - 1) / units);
   const long long want = (max_context_len + parts - 1) / parts;
   int part = 256;
-  while (part < want && part < 1024) part <<= 1;
+  while (part < want && part < 2048) part <<= 1;
   return std::min(whole, part);
 }
 

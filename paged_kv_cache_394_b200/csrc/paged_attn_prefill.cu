@@ -69,8 +69,11 @@ struct TcEntry {
 // on 2048 cached 376 -> 482, 2048 on 8192 cached 419 -> 607, the LLaMA-7B
 // prefill batch 350 -> 411.  bf16 (P split into hi + lo halves) gained once P
 // moved to TMEM with two query tiles: the GQA prefill batch 388 -> 453.
+#ifndef PKV_PREFILL_QUERY_TILES
+#define PKV_PREFILL_QUERY_TILES 2
+#endif
 template <class DT>
-constexpr int kTcQueryTiles = 2;
+constexpr int kTcQueryTiles = PKV_PREFILL_QUERY_TILES;
 
 template <int BS, int G, class DT, bool FP8>
 TcEntry make_tc() {

@@ -40,6 +40,10 @@
 #ifndef PKV_PREFIX_STAGES
 #define PKV_PREFIX_STAGES 6
 #endif
+// K/V stages of a one-query-tile prefill CTA (PKV_PREFILL_QUERY_TILES=1)
+#ifndef PKV_QT1_STAGES
+#define PKV_QT1_STAGES 6
+#endif
 
 namespace pkv {
 namespace tc {
@@ -225,7 +229,7 @@ struct TcPrefillTraits {
   static constexpr int kSortUnits = 512;         // (sequence, tile) units ranked per CTA
   // KV stages: what fits beside QT query tiles (P lives in TMEM, over S); the
   // cascade prefix pass (one query tile) keeps PKV_PREFIX_STAGES
-  static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : PKV_PREFIX_STAGES;
+  static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : kPrefix ? PKV_PREFIX_STAGES : PKV_QT1_STAGES;
   static constexpr int NSTG = kFp8 ? 2 : 0;      // E4M3 staging slots per kind
   // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
   // P.V issuer

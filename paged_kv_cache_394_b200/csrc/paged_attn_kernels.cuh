@@ -604,6 +604,56 @@ __device__ __forceinline__ uint32_t swizzled(int t, int ch) {
   return static_cast<uint32_t>((ch >> 3) * 2048 + t * 128 + (((ch & 7) ^ (t & 7)) << 4));
 }
 
+// The reference max of the tensor-core kernels' online softmax moves only
+// when a logit exceeds it by more than this (base-2 units), so P stays at
+// most 2^8 (fp16 and bf16 hold it) and most sub-blocks skip the max and its
+// shuffles.
+constexpr float kLazyMax = 8.f;
+
+// Online softmax of one 16-token sub-block for the two heads a lane holds in
+// the S^T fragment (x0, x2: head 2(lane % 4) at tokens lane / 4 and
+// lane / 4 + 8; x1, x3: head 2(lane % 4) + 1).  m[] is the reference max, the
+// same in the 8 lanes that share lane % 4; it is recomputed (a max over those
+// lanes, the O accumulator and l rescaled) only when a logit passes
+// m + kLazyMax.  l[] holds this lane's own partial sums, reduced over the 8
+// lanes once at the end.  Returns p = 2^(x - m).
+template <int KS>
+__device__ __forceinline__ void mma_softmax(float x0, float x1, float x2, float x3,
+                                            float (&m)[2], float (&l)[2], float (&acc)[KS][4],
+                                            float& p0, float& p1, float& p2, float& p3) {
+  const bool up = x0 > m[0] + kLazyMax || x2 > m[0] + kLazyMax || x1 > m[1] + kLazyMax ||
+                  x3 > m[1] + kLazyMax;
+  if (__any_sync(kFullMask, up)) {
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
+    }
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float a0 = exp2_approx(m[0] - mn0), a1 = exp2_approx(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    l[0] *= a0;
+    l[1] *= a1;
+    if (__any_sync(kFullMask, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        acc[mt][0] *= a0;
+        acc[mt][1] *= a1;
+        acc[mt][2] *= a0;
+        acc[mt][3] *= a1;
+      }
+    }
+  }
+  p0 = exp2_approx(x0 - m[0]);
+  p1 = exp2_approx(x1 - m[1]);
+  p2 = exp2_approx(x2 - m[0]);
+  p3 = exp2_approx(x3 - m[1]);
+  l[0] += p0 + p2;
+  l[1] += p1 + p3;
+}
+
 template <class Tr>
 __device__ __forceinline__ void mma_sub_block(uint32_t kt, uint32_t vt, int valid,
                                               const uint32_t (&qf)[Tr::KSTEPS][2],
@@ -630,36 +680,9 @@ __device__ __forceinline__ void mma_sub_block(uint32_t kt, uint32_t vt, int vali
     if (t0 >= valid) x0 = x1 = -INFINITY;
     if (t0 + 8 >= valid) x2 = x3 = -INFINITY;
   }
-  // ---- online softmax per head: reduce over the 8 lanes sharing lane % 4 ------
-  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
-  }
-  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-  const float a0 = exp2_approx(m[0] - mn0), a1 = exp2_approx(m[1] - mn1);
-  const float p0 = exp2_approx(x0 - mn0), p1 = exp2_approx(x1 - mn1);
-  const float p2 = exp2_approx(x2 - mn0), p3 = exp2_approx(x3 - mn1);
-  float s0 = p0 + p2, s1 = p1 + p3;
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    s0 += __shfl_xor_sync(kFullMask, s0, o);
-    s1 += __shfl_xor_sync(kFullMask, s1, o);
-  }
-  l[0] = l[0] * a0 + s0;
-  l[1] = l[1] * a1 + s1;
-  m[0] = mn0;
-  m[1] = mn1;
-  if (__any_sync(kFullMask, a0 != 1.f || a1 != 1.f)) {
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      acc[mt][0] *= a0;
-      acc[mt][1] *= a1;
-      acc[mt][2] *= a0;
-      acc[mt][3] *= a1;
-    }
-  }
+  // ---- online softmax per head (see mma_softmax) ---------------------------------
+  float p0, p1, p2, p3;
+  mma_softmax<KS>(x0, x1, x2, x3, m, l, acc, p0, p1, p2, p3);
   // ---- P as the B operand: transpose the S^T fragments in registers -----------
   // bf16 keeps 8 mantissa bits, too few for p near 1 at the required accuracy,
   // so bf16 P is split as hi + lo (both bf16, |P - hi - lo| <= 2^-18 P) and
@@ -750,35 +773,8 @@ __device__ __forceinline__ void mma_sub_block_fp8(uint32_t kt, uint32_t vt, int 
     if (t0 >= valid) x0 = x1 = -INFINITY;
     if (t0 + 8 >= valid) x2 = x3 = -INFINITY;
   }
-  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, o));
-  }
-  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-  const float a0 = exp2_approx(m[0] - mn0), a1 = exp2_approx(m[1] - mn1);
-  const float p0 = exp2_approx(x0 - mn0), p1 = exp2_approx(x1 - mn1);
-  const float p2 = exp2_approx(x2 - mn0), p3 = exp2_approx(x3 - mn1);
-  float s0 = p0 + p2, s1 = p1 + p3;
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    s0 += __shfl_xor_sync(kFullMask, s0, o);
-    s1 += __shfl_xor_sync(kFullMask, s1, o);
-  }
-  l[0] = l[0] * a0 + s0;
-  l[1] = l[1] * a1 + s1;
-  m[0] = mn0;
-  m[1] = mn1;
-  if (__any_sync(kFullMask, a0 != 1.f || a1 != 1.f)) {
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      acc[mt][0] *= a0;
-      acc[mt][1] *= a1;
-      acc[mt][2] *= a0;
-      acc[mt][3] *= a1;
-    }
-  }
+  float p0, p1, p2, p3;
+  mma_softmax<KS>(x0, x1, x2, x3, m, l, acc, p0, p1, p2, p3);
   // P in (0, 1] as fp16 (11 significant bits), transposed into the B operand
   const uint32_t b0 = movmatrix_trans(pack2(p0, p1, Fp16()));
   const uint32_t b1 = movmatrix_trans(pack2(p2, p3, Fp16()));
@@ -984,6 +980,12 @@ __global__ void __launch_bounds__(Tr::THREADS)
   }
 
   // ---- merge the warps -------------------------------------------------------
+  // each lane summed its own p: the sums of a head pair over its 8 lanes
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l[0] += __shfl_xor_sync(kFullMask, l[0], o);
+    l[1] += __shfl_xor_sync(kFullMask, l[1], o);
+  }
   __syncthreads();
   float* cm = reinterpret_cast<float*>(smem);
   float* cl = cm + W * G;

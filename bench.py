@@ -245,6 +245,8 @@ def hbm_peak():
 DECODE_SOURCES = ("common.cuh", "paged_attn_kernels.cuh", "paged_attn_decode.cu")
 PREFILL_SOURCES = ("common.cuh", "paged_prefill_kernels.cuh", "paged_prefill_tc_kernels.cuh",
                    "paged_attn_prefill.cu")
+# cascade decode: the tcgen05 prefix pass, the suffix decode and the merge
+CASCADE_SOURCES = DECODE_SOURCES + PREFILL_SOURCES[1:]
 
 
 def kernel_source_hash(sources=DECODE_SOURCES):
@@ -262,9 +264,11 @@ def kernel_source_hash(sources=DECODE_SOURCES):
 
 
 def committed_traffic(workload, kind="decode"):
-    """DRAM bytes per launch of the workload's dominant kernel from profiles/,
-    if the counters were taken on the current device code."""
-    sources = PREFILL_SOURCES if kind == "prefill" else DECODE_SOURCES
+    """DRAM bytes per launch of the workload's dominant kernel (cascade decode:
+    of its three launches together) from profiles/, if the counters were taken
+    on the current device code."""
+    sources = (PREFILL_SOURCES if kind == "prefill" else
+               CASCADE_SOURCES if workload.endswith("_cascade") else DECODE_SOURCES)
     path = os.path.join(ROOT, "profiles", "paged_%s_%s_traffic.md" % (kind, workload))
     try:
         text = open(path).read()

@@ -245,8 +245,8 @@ def hbm_peak():
 DECODE_SOURCES = ("common.cuh", "paged_attn_kernels.cuh", "paged_attn_decode.cu")
 PREFILL_SOURCES = ("common.cuh", "paged_prefill_kernels.cuh", "paged_prefill_tc_kernels.cuh",
                    "paged_attn_prefill.cu")
-# cascade decode: the tcgen05 prefix pass, the suffix decode and the merge
-CASCADE_SOURCES = DECODE_SOURCES + PREFILL_SOURCES[1:]
+# cascade decode: the shared-prefix pass, the suffix decode and the merge
+CASCADE_SOURCES = DECODE_SOURCES + PREFILL_SOURCES[1:] + ("paged_attn_cascade.cu",)
 
 
 def kernel_source_hash(sources=DECODE_SOURCES):

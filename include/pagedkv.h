@@ -45,8 +45,8 @@
  *    word after the stream has synchronized; outputs are then unreliable.
  *  - Alignment: every tensor pointer (16-bit or E4M3) must be 16-byte aligned.
  *  - Supported shapes: head_dim in {64, 128}, block_size in {16, 32},
- *    num_heads / num_kv_heads in {1, 2, 4, 8}, q/out dtype fp16 or bf16
- *    (cascade decode and E4M3 prefill: head_dim 128 only).
+ *    num_heads / num_kv_heads in {1, 2, 4, 8}, q/out dtype fp16 or bf16,
+ *    for every entry point and cache type.
  */
 #ifndef PAGEDKV_H_
 #define PAGEDKV_H_
@@ -321,8 +321,9 @@ pkv_status pkv_paged_attn_decode_static_ws(void* out, const void* q, const void*
  * context is shorter than its group's shared tokens sets
  * PKV_DEVERR_BAD_CONTEXT, and so does a shared_blocks[g] above
  * max_shared_blocks: both passes then treat the group as sharing only
- * max_shared_blocks blocks.  head_dim 128 only (PKV_ERR_UNSUPPORTED otherwise);
- * 16-bit caches.  Other arguments and errors as in pkv_paged_attn_decode.
+ * max_shared_blocks blocks.  head_dim 64 or 128; 16-bit caches (E4M3:
+ * pkv_paged_attn_decode_cascade_fp8).  Other arguments and errors as in
+ * pkv_paged_attn_decode.
  */
 size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
                                               int head_dim, int block_size,
@@ -397,14 +398,14 @@ pkv_status pkv_paged_attn_decode_fp8(void* out, const void* q, const void* k_cac
  * pkv_paged_attn_prefill_fp8 — pkv_paged_attn_prefill over E4M3 caches:
  *     out[t, h, :] = softmax(scale * q[t, h, :] . K~[0..p]^T) . V~[0..p]
  * with K~ and V~ decoded as for pkv_paged_attn_decode_fp8 (codes times the kv
- * head's k_scales / v_scales entry).  head_dim 128 only (else
- * PKV_ERR_UNSUPPORTED): the tcgen05 kernel stages each tile's codes by TMA
- * and widens them exactly to the 16-bit type of q (`dtype`) before the tensor
- * cores read them; the K scale folds into the logit scale and the V scale
- * into the final normalisation.  Every other argument and the error
- * behaviour are those of pkv_paged_attn_prefill; null scale pointers give
- * PKV_ERR_INVALID_ARG and a scale that is not finite and > 0 sets
- * PKV_DEVERR_BAD_SCALE.
+ * head's k_scales / v_scales entry).  The kernel stages each tile's codes by
+ * TMA and widens them exactly to fp16 before the tensor cores read them
+ * (tcgen05 at head_dim 128, mma.sync at 64); bf16 queries are rounded to fp16
+ * there, magnitudes above 65504 saturating.  The K scale folds into the logit
+ * scale and the V scale into the final normalisation.  Every other argument
+ * and the error behaviour are those of pkv_paged_attn_prefill; null scale
+ * pointers give PKV_ERR_INVALID_ARG and a scale that is not finite and > 0
+ * sets PKV_DEVERR_BAD_SCALE.
  */
 pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, const void* k_cache,
                                       const void* v_cache, const int32_t* block_tables,
@@ -415,6 +416,27 @@ pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, const void* k_ca
                                       int max_blocks_per_seq, int max_context_len,
                                       int max_query_len, int num_blocks, pkv_dtype dtype,
                                       unsigned* dev_err, void* stream);
+
+/*
+ * pkv_paged_attn_decode_cascade_fp8 — pkv_paged_attn_decode_cascade over E4M3
+ * caches: the result is that of pkv_paged_attn_decode_fp8 on the same
+ * arguments (K~, V~ = codes times the kv head's k_scales / v_scales entry).
+ * The shared-prefix pass widens the codes to fp16 as
+ * pkv_paged_attn_prefill_fp8 does (bf16 queries rounded to fp16 there), the
+ * members' own blocks are read as pkv_paged_attn_decode_fp8 reads them.
+ * Groups, workspace (pkv_paged_attn_cascade_workspace_bytes), head_dim 64 or
+ * 128 and errors as in pkv_paged_attn_decode_cascade; null scale pointers give
+ * PKV_ERR_INVALID_ARG and a scale that is not finite and > 0 sets
+ * PKV_DEVERR_BAD_SCALE.
+ */
+pkv_status pkv_paged_attn_decode_cascade_fp8(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
+    const int32_t* shared_blocks, float scale, const float* k_scales, const float* v_scales,
+    int num_seqs, int num_groups, int max_group_size, int max_shared_blocks, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream);
 
 /*
  * pkv_decode_step_host — one whole decode step from HOST buffers: copies the

@@ -23,10 +23,18 @@ inline int cache_elem_bytes(int dt) { return dt == PKV_FP8_E4M3 ? 1 : 2; }
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-// 2-D TMA tensor map over a cache viewed as [num_blocks * hkv * bs, d] rows,
-// boxes of 16 rows x 64 elements with the 128-byte swizzle (cached per thread).
+// 2-D TMA tensor map over a cache viewed as [num_blocks * hkv * bs, d] rows
+// (cached per thread): boxes of 16 rows x 128 bytes (64 16-bit elements or 128
+// E4M3 codes) with the 128-byte swizzle; E4M3 rows of 64 codes come as boxes of
+// 16 whole rows, unswizzled.
 pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, int hkv, int bs,
                             int d, pkv_dtype dt);
+
+// 3-D TMA tensor map over q [T, H, 128] (16-bit): boxes of (128/group tokens)
+// x (group heads) x 64 dims, i.e. a 128-row query tile ordered (token, head),
+// with the 128-byte swizzle.
+pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num_heads, int group,
+                        pkv_dtype dt);
 
 // Groups of cascade decode (device arrays): group g is sequences
 // group_start[g] .. group_start[g+1]-1, sharing their first shared_blocks[g]
@@ -39,15 +47,19 @@ struct CascadeGroups {
   int max_shared_blocks;
 };
 
-// The shared-prefix pass of cascade decode (tcgen05 kernel, head_dim 128):
-// writes each member's prefix partial (m, l, unnormalised o) into slot 0 of
-// its rows of the split-K workspace (max_parts slots per (sequence, head)).
+// The shared-prefix pass of cascade decode: writes each member's prefix
+// partial (m, l, unnormalised o) into slot 0 of its rows of the split-K
+// workspace (max_parts slots per (sequence, head)).  head_dim 128 runs the
+// tcgen05 kernel, 64 the mma.sync kernel; fp8: the caches hold E4M3 codes with
+// per-kv-head scales k_scales / v_scales (the V scale goes into o).
 pkv_status launch_cascade_prefix(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* block_tables, const int32_t* context_lens,
                                  const CascadeGroups& groups, float scale, int num_seqs,
-                                 int num_heads, int num_kv_heads, int block_size,
+                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
                                  int max_blocks_per_seq, int max_context_len, int num_blocks,
-                                 pkv_dtype dtype, float* ws_out, float* ws_max, float* ws_sum,
-                                 int max_parts, unsigned* dev_err, cudaStream_t stream);
+                                 pkv_dtype dtype, bool fp8, const float* k_scales,
+                                 const float* v_scales, float* ws_out, float* ws_max,
+                                 float* ws_sum, int max_parts, unsigned* dev_err,
+                                 cudaStream_t stream);
 
 }  // namespace pkv

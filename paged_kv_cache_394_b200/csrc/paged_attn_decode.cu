@@ -203,9 +203,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map over a cache viewed as rows of head_dim elements
-// ([num_blocks * num_kv_heads * block_size, head_dim]); boxes of 16 rows x 64
-// elements (128 bytes) with the 128-byte swizzle.  Encoded maps are cached per
-// thread, keyed by everything they depend on.
+// ([num_blocks * num_kv_heads * block_size, head_dim]); boxes of 16 rows x 128
+// bytes with the 128-byte swizzle, or of 16 whole rows unswizzled for E4M3
+// rows of 64 codes.  Encoded maps are cached per thread, keyed by everything
+// they depend on.
 pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, int hkv, int bs,
                             int d, pkv_dtype dt) {
   struct Slot {
@@ -226,10 +227,12 @@ pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, 
   if (enc == nullptr) return cuda_status(cudaErrorNotSupported);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d),
                         static_cast<cuuint64_t>(num_blocks) * hkv * bs};
-  // 16 rows x 128 bytes: 64 16-bit elements or 128 E4M3 codes
+  // 16 rows x 128 bytes: 64 16-bit elements or 128 E4M3 codes; E4M3 rows
+  // of 64 codes: 16 whole rows, unswizzled
   const int eb = cache_elem_bytes(dt);
+  const bool narrow = d * eb < 128;
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * eb};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), 16};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(narrow ? d : 128 / eb), 16};
   cuuint32_t estr[2] = {1, 1};
   Slot& sl = slots[next];
   next = (next + 1) % 4;
@@ -239,8 +242,8 @@ pkv_status cache_tensor_map(CUtensorMap* out, const void* base, int num_blocks, 
           : dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                            : CU_TENSOR_MAP_DATA_TYPE_UINT8,
           2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+          narrow ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     sl.base = nullptr;
     return cuda_status(cudaErrorInvalidValue);
@@ -568,10 +571,11 @@ extern "C" pkv_status pkv_decode_order(const int32_t* context_lens, int num_seqs
 // common prompts point at the same pages).  Plain decode reads those blocks
 // once per sample; the samples of a prompt run at about the same time, so the
 // repeats come from L2, and L2 bandwidth then bounds the step.  Here the
-// shared blocks are read once per group: the tcgen05 kernel in prefix mode
-// attends every member's query rows to them together (slot 0 of the split-K
-// workspace), the decode kernel covers each member's own blocks (slots 1..),
-// and the reduce merges the partials.  The result is that of plain decode.
+// shared blocks are read once per group: a chunked-prefill kernel in prefix
+// mode (tcgen05 at head_dim 128, mma.sync at 64) attends every member's query
+// rows to them together (slot 0 of the split-K workspace), the decode kernel
+// covers each member's own blocks (slots 1..), and the reduce merges the
+// partials.  The result is that of plain decode, over 16-bit or E4M3 caches.
 // ---------------------------------------------------------------------------
 extern "C" size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_heads,
                                                          int num_kv_heads, int head_dim,
@@ -589,23 +593,28 @@ extern "C" size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_h
       .total;
 }
 
-extern "C" pkv_status pkv_paged_attn_decode_cascade(
-    void* out, const void* q, const void* k_cache, const void* v_cache,
-    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
-    const int32_t* shared_blocks, float scale, int num_seqs, int num_groups, int max_group_size,
-    int max_shared_blocks, int num_heads, int num_kv_heads, int head_dim, int block_size,
-    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
-    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err,
-    void* stream) {
-  using namespace pkv;
+namespace pkv {
+namespace {
+
+// Shared body of the 16-bit and the E4M3 cascade entry points.
+pkv_status cascade_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          const int32_t* group_start, const int32_t* shared_blocks, float scale,
+                          int num_seqs, int num_groups, int max_group_size, int max_shared_blocks,
+                          int num_heads, int num_kv_heads, int head_dim, int block_size,
+                          int max_blocks_per_seq, int max_context_len, int num_blocks,
+                          pkv_dtype dtype, int partition_size, void* workspace,
+                          size_t workspace_bytes, unsigned* dev_err, void* stream, bool fp8,
+                          const float* k_scales, const float* v_scales) {
   if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0 ||
       num_kv_heads <= 0 || block_size <= 0 ||
       static_cast<long long>(max_shared_blocks) * block_size > max_context_len ||
       (num_seqs > 0 && (num_groups == 0 || max_group_size == 0)))
     return PKV_ERR_INVALID_ARG;
-  if (head_dim != 128) return PKV_ERR_UNSUPPORTED;  // the prefix pass is the tcgen05 kernel
+  if (!head_dim_supported(head_dim)) return PKV_ERR_UNSUPPORTED;
   if (num_seqs == 0) return PKV_OK;
-  if (!group_start || !shared_blocks || !workspace) return PKV_ERR_INVALID_ARG;
+  if (!group_start || !shared_blocks || !workspace || (fp8 && (!k_scales || !v_scales)))
+    return PKV_ERR_INVALID_ARG;
   const CascadeGroups groups{group_start, shared_blocks, num_groups, max_group_size,
                              max_shared_blocks};
   // validate everything (and the workspace) before the first launch
@@ -634,15 +643,51 @@ extern "C" pkv_status pkv_paged_attn_decode_cascade(
   if (max_shared_blocks > 0) {
     const pkv_status st = launch_cascade_prefix(
         q, k_cache, v_cache, block_tables, context_lens, groups, scale, num_seqs, num_heads,
-        num_kv_heads, block_size, max_blocks_per_seq, max_context_len, num_blocks, dtype,
-        reinterpret_cast<float*>(ws + wl.out_off), reinterpret_cast<float*>(ws + wl.max_off),
-        reinterpret_cast<float*>(ws + wl.sum_off), max_parts, dev_err, as_stream(stream));
+        num_kv_heads, head_dim, block_size, max_blocks_per_seq, max_context_len, num_blocks,
+        dtype, fp8, k_scales, v_scales, reinterpret_cast<float*>(ws + wl.out_off),
+        reinterpret_cast<float*>(ws + wl.max_off), reinterpret_cast<float*>(ws + wl.sum_off),
+        max_parts, dev_err, as_stream(stream));
     if (st != PKV_OK) return st;
   }
   return decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
                        num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                        max_context_len, num_blocks, dtype, partition_size, workspace,
-                       workspace_bytes, dev_err, stream, false, nullptr, nullptr, &groups);
+                       workspace_bytes, dev_err, stream, fp8, k_scales, v_scales, &groups);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attn_decode_cascade(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
+    const int32_t* shared_blocks, float scale, int num_seqs, int num_groups, int max_group_size,
+    int max_shared_blocks, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err,
+    void* stream) {
+  return pkv::cascade_launch(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                             shared_blocks, scale, num_seqs, num_groups, max_group_size,
+                             max_shared_blocks, num_heads, num_kv_heads, head_dim, block_size,
+                             max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                             partition_size, workspace, workspace_bytes, dev_err, stream, false,
+                             nullptr, nullptr);
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_cascade_fp8(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
+    const int32_t* shared_blocks, float scale, const float* k_scales, const float* v_scales,
+    int num_seqs, int num_groups, int max_group_size, int max_shared_blocks, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream) {
+  return pkv::cascade_launch(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                             shared_blocks, scale, num_seqs, num_groups, max_group_size,
+                             max_shared_blocks, num_heads, num_kv_heads, head_dim, block_size,
+                             max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                             partition_size, workspace, workspace_bytes, dev_err, stream, true,
+                             k_scales, v_scales);
 }
 
 // ---------------------------------------------------------------------------

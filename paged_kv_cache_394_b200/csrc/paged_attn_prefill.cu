@@ -26,29 +26,33 @@ struct PrefillEntry {
 
 constexpr int kPrefillStages = 4;
 
-template <int D, int BS, int G, class DT>
+template <int D, int BS, int G, class DT, bool FP8>
 PrefillEntry make_prefill() {
-  using Tr = PrefillTraits<D, BS, G, DT, kPrefillStages>;
+  using Tr = PrefillTraits<D, BS, G, DT, kPrefillStages, false, FP8>;
   return PrefillEntry{paged_prefill_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(), Tr::ROWS};
 }
 
-template <int D, int BS, class DT>
+template <int D, int BS, class DT, bool FP8>
 PrefillEntry prefill_group(int g) {
   switch (g) {
-    case 1: return make_prefill<D, BS, 1, DT>();
-    case 2: return make_prefill<D, BS, 2, DT>();
-    case 4: return make_prefill<D, BS, 4, DT>();
-    case 8: return make_prefill<D, BS, 8, DT>();
+    case 1: return make_prefill<D, BS, 1, DT, FP8>();
+    case 2: return make_prefill<D, BS, 2, DT, FP8>();
+    case 4: return make_prefill<D, BS, 4, DT, FP8>();
+    case 8: return make_prefill<D, BS, 8, DT, FP8>();
     default: return PrefillEntry{nullptr, 0, 0, 0};
   }
 }
 
-template <class DT>
+// (head_dim, block size, group) -> mma.sync kernel; fp8: the cache holds E4M3
+// codes (head_dim 64)
+template <class DT, bool FP8 = false>
 PrefillEntry prefill_for(int d, int bs, int g) {
-  if (d == 128 && bs == 16) return prefill_group<128, 16, DT>(g);
-  if (d == 128 && bs == 32) return prefill_group<128, 32, DT>(g);
-  if (d == 64 && bs == 16) return prefill_group<64, 16, DT>(g);
-  if (d == 64 && bs == 32) return prefill_group<64, 32, DT>(g);
+  if constexpr (!FP8) {
+    if (d == 128 && bs == 16) return prefill_group<128, 16, DT, false>(g);
+    if (d == 128 && bs == 32) return prefill_group<128, 32, DT, false>(g);
+  }
+  if (d == 64 && bs == 16) return prefill_group<64, 16, DT, FP8>(g);
+  if (d == 64 && bs == 32) return prefill_group<64, 32, DT, FP8>(g);
   return PrefillEntry{nullptr, 0, 0, 0};
 }
 
@@ -100,34 +104,11 @@ TcEntry tc_for(int bs, int g) {
   return TcEntry{nullptr, 0, 0, 0};
 }
 
-// Prefix mode (the shared-prefix pass of cascade decode): one 128-row query
-// tile per CTA; a group's members and their heads are its rows.
-template <int BS, int G, class DT>
-TcEntry make_prefix_tc() {
-  using Tr = TcPrefillTraits<BS, G, DT, 1, true>;
-  return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(), Tr::ROWS};
-}
+}  // namespace
+}  // namespace pkv
 
-template <int BS, class DT>
-TcEntry prefix_group(int g) {
-  switch (g) {
-    case 1: return make_prefix_tc<BS, 1, DT>();
-    case 2: return make_prefix_tc<BS, 2, DT>();
-    case 4: return make_prefix_tc<BS, 4, DT>();
-    case 8: return make_prefix_tc<BS, 8, DT>();
-    default: return TcEntry{nullptr, 0, 0, 0};
-  }
-}
+namespace pkv {
 
-template <class DT>
-TcEntry prefix_for(int bs, int g) {
-  if (bs == 16) return prefix_group<16, DT>(g);
-  if (bs == 32) return prefix_group<32, DT>(g);
-  return TcEntry{nullptr, 0, 0, 0};
-}
-
-// 3-D tensor map over q [T, H, 128]: boxes of (128/G tokens) x (G heads) x 64 dims,
-// i.e. a tile's 128 rows ordered (token, head), 128-byte swizzle.
 pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num_heads, int group,
                         pkv_dtype dt) {
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
@@ -154,84 +135,13 @@ pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num
   return r == CUDA_SUCCESS ? PKV_OK : cuda_status(cudaErrorInvalidValue);
 }
 
-}  // namespace
-}  // namespace pkv
-
-namespace pkv {
-
-pkv_status launch_cascade_prefix(const void* q, const void* k_cache, const void* v_cache,
-                                 const int32_t* block_tables, const int32_t* context_lens,
-                                 const CascadeGroups& groups, float scale, int num_seqs,
-                                 int num_heads, int num_kv_heads, int block_size,
-                                 int max_blocks_per_seq, int max_context_len, int num_blocks,
-                                 pkv_dtype dtype, float* ws_out, float* ws_max, float* ws_sum,
-                                 int max_parts, unsigned* dev_err, cudaStream_t stream) {
-  const int group = num_heads / num_kv_heads;
-  const TcEntry te = dtype == PKV_FP16 ? prefix_for<Fp16>(block_size, group)
-                                       : prefix_for<Bf16>(block_size, group);
-  if (te.fn == nullptr) return PKV_ERR_UNSUPPORTED;
-  const long long rows = static_cast<long long>(groups.max_group_size) * group;
-  const int q_tiles = static_cast<int>((rows + te.rows - 1) / te.rows);
-  const long long grid = static_cast<long long>(groups.num_groups) * num_kv_heads * q_tiles;
-  if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
-  if (grid == 0) return PKV_OK;
-  CUtensorMap kmap, vmap, qmap;
-  pkv_status st =
-      cache_tensor_map(&kmap, k_cache, num_blocks, num_kv_heads, block_size, 128, dtype);
-  if (st != PKV_OK) return st;
-  st = cache_tensor_map(&vmap, v_cache, num_blocks, num_kv_heads, block_size, 128, dtype);
-  if (st != PKV_OK) return st;
-  st = q_tensor_map(&qmap, q, num_seqs, num_heads, group, dtype);  // the members' queries
-  if (st != PKV_OK) return st;
-  st = cuda_status(cudaFuncSetAttribute(reinterpret_cast<const void*>(te.fn),
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(te.smem)));
-  if (st != PKV_OK) return st;
-
-  PrefillParams p = {};
-  p.q = q;
-  p.k_cache = k_cache;
-  p.v_cache = v_cache;
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
-  p.qscale = scale * kLog2e;
-  p.num_seqs = groups.num_groups;
-  p.num_heads = num_heads;
-  p.num_kv_heads = num_kv_heads;
-  p.max_blocks_per_seq = max_blocks_per_seq;
-  p.max_context_len = max_context_len;
-  p.max_query_len = groups.max_group_size;
-  p.num_blocks = num_blocks;
-  p.q_tiles = q_tiles;
-  p.err = dev_err;
-  p.group_start = groups.group_start;
-  p.shared_blocks = groups.shared_blocks;
-  p.max_shared_blocks = groups.max_shared_blocks;
-  p.ws_out = ws_out;
-  p.ws_max = ws_max;
-  p.ws_sum = ws_sum;
-  p.max_parts = max_parts;
-
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(te.threads);
-  cfg.dynamicSmemBytes = te.smem;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, te.fn, p, qmap, kmap, vmap));
-}
-
 }  // namespace pkv
 
 namespace pkv {
 namespace {
 
-// Validates and launches prefill; fp8: the caches hold E4M3 codes (head_dim
-// 128, the tcgen05 kernel) with per-kv-head scales k_scales / v_scales.
+// Validates and launches prefill; fp8: the caches hold E4M3 codes with
+// per-kv-head scales k_scales / v_scales.
 pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
                           const int32_t* block_tables, const int32_t* context_lens,
                           const int32_t* query_start, float scale, int num_seqs, int num_tokens,
@@ -248,7 +158,6 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
     return PKV_ERR_UNSUPPORTED;
   const int group = num_heads / num_kv_heads;
   if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
-  if (fp8 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
   if (static_cast<long long>(max_context_len) >
       static_cast<long long>(max_blocks_per_seq) * block_size)
     return PKV_ERR_INVALID_ARG;
@@ -259,9 +168,12 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
   const bool use_tc = head_dim == 128;
-  const PrefillEntry pe = use_tc ? PrefillEntry{nullptr, 0, 0, 0}
-                          : dtype == PKV_FP16 ? prefill_for<Fp16>(head_dim, block_size, group)
-                                              : prefill_for<Bf16>(head_dim, block_size, group);
+  const PrefillEntry pe =
+      use_tc ? PrefillEntry{nullptr, 0, 0, 0}
+      : fp8  ? (dtype == PKV_FP16 ? prefill_for<Fp16, true>(head_dim, block_size, group)
+                                  : prefill_for<Bf16, true>(head_dim, block_size, group))
+      : dtype == PKV_FP16 ? prefill_for<Fp16>(head_dim, block_size, group)
+                          : prefill_for<Bf16>(head_dim, block_size, group);
   const TcEntry te = !use_tc ? TcEntry{nullptr, 0, 0, 0}
                      : fp8 ? (dtype == PKV_FP16 ? tc_for<Fp16, true>(block_size, group)
                                                 : tc_for<Bf16, true>(block_size, group))

@@ -188,21 +188,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Two E4M3 codes (low bytes first) -> two values packed as fp16x2 or bf16x2;
-// exact, since every E4M3 value is an fp16 and a bf16 value.
-__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t two, Fp16) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
-      : "=r"(r)
-      : "r"(two));
-  return r;
-}
-__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t two, Bf16) {
-  const uint32_t h = e4m3x2_to(two, Fp16());
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
-  return pack2(f.x, f.y, Bf16());
-}
-
 }  // namespace tc
 
 template <int BS_, int G_, class DT_, int QT_, bool PREFIX_ = false, bool FP8_ = false>
@@ -263,7 +248,6 @@ struct TcPrefillTraits {
   // per query tile q: S buffers at 256q and 256q + 64, O at 256q + 128
   static constexpr uint32_t TMEM_COLS = 256 * QT;
   static_assert(QT == 1 || QT == 2, "one or two query tiles per CTA");
-  static_assert(!(kFp8 && kPrefix), "the cascade prefix pass reads 16-bit caches");
   static_assert(1024 + SMEM <= 232448, "shared memory per CTA");
   static size_t smem_bytes() { return 1024 + static_cast<size_t>(SMEM); }
 };
@@ -550,8 +534,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           uint32_t h[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            h[2 * e] = tc::e4m3x2_to(w[e] & 0xffffu, typename Tr::MT());
-            h[2 * e + 1] = tc::e4m3x2_to(w[e] >> 16, typename Tr::MT());
+            h[2 * e] = e4m3x2_to(w[e] & 0xffffu, typename Tr::MT());
+            h[2 * e + 1] = e4m3x2_to(w[e] >> 16, typename Tr::MT());
           }
           const uint32_t row = dst + (c >> 2) * Tr::KV_HALF + r * 128;
           const int c0 = (c & 3) * 2;
@@ -929,9 +913,12 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         tc::tmem_ld16(lane_addr + 128 + c, v);
         tc::tmem_wait_ld();
         if (active) {
+          // E4M3: the V scale goes into o (m and l do not hold it)
           float4* o = reinterpret_cast<float4*>(p.ws_out + slot * Tr::D + c);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 4; ++i)
+            o[i] = make_float4(v[4 * i] * v_scale, v[4 * i + 1] * v_scale, v[4 * i + 2] * v_scale,
+                               v[4 * i + 3] * v_scale);
         }
       }
     } else if (ok && my_tiles > 0) {

@@ -54,6 +54,9 @@ _cascade_workspace_bytes = _proto("pkv_paged_attn_cascade_workspace_bytes", _sz,
 _paged_attn_decode_cascade = _proto("pkv_paged_attn_decode_cascade", _i, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _vp, _sz, _vp, _vp)
+_paged_attn_decode_cascade_fp8 = _proto("pkv_paged_attn_decode_cascade_fp8", _i, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i,
+                                        _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
 _reshape_and_cache_fp8 = _proto("pkv_reshape_and_cache_fp8", _i, _vp, _vp, _vp, _vp, _vp, _i, _i,
                                 _i, _i, _i, _i, _vp, _vp, _vp, _vp)
 _paged_attn_decode_fp8 = _proto("pkv_paged_attn_decode_fp8", _i, _vp, _vp, _vp, _vp, _vp, _vp, _f,
@@ -294,10 +297,12 @@ def cascade_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_s
 def paged_attn_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
                               shared_blocks, scale, num_kv_heads, block_size, max_context_len,
                               max_group_size, max_shared_blocks, partition_size=0,
-                              workspace=None, dev_err=None, stream=None):
+                              workspace=None, dev_err=None, stream=None, k_scales=None,
+                              v_scales=None):
     """Decode for groups of sequences sharing their first shared_blocks[g]
     blocks (members consecutive, group g = group_start[g] .. group_start[g+1]-1).
-    Same result as paged_attn_decode.  See include/pagedkv.h."""
+    Same result as paged_attn_decode; with E4M3 caches (uint8 codes and
+    k_scales / v_scales given) as paged_attn_decode_fp8.  See include/pagedkv.h."""
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     for n, t in (("block_tables", block_tables), ("context_lens", context_lens),
@@ -307,8 +312,12 @@ def paged_attn_decode_cascade(out, q, k_cache, v_cache, block_tables, context_le
     num_blocks, hkv, bs, dk = k_cache.shape
     if (hkv, bs, dk) != (num_kv_heads, block_size, d) or out.shape != q.shape:
         raise ValueError("shape mismatch")
-    if q.dtype != k_cache.dtype or out.dtype != q.dtype:
-        raise TypeError("q, out and caches must share a dtype")
+    fp8 = _cache_dtype_code(k_cache) == FP8_E4M3
+    if fp8 != (k_scales is not None) or (k_scales is None) != (v_scales is None):
+        raise TypeError("E4M3 caches take k_scales and v_scales; 16-bit caches take neither")
+    if (v_cache.dtype != k_cache.dtype or out.dtype != q.dtype
+            or (not fp8 and q.dtype != k_cache.dtype)):
+        raise TypeError("q, out and caches must share a dtype (E4M3 caches: uint8 codes)")
     g = shared_blocks.shape[0]
     if group_start.shape != (g + 1,):
         raise ValueError("group_start must be [num_groups + 1]")
@@ -318,6 +327,16 @@ def paged_attn_decode_cascade(out, q, k_cache, v_cache, block_tables, context_le
         if stream is not None:
             workspace.record_stream(stream)   # the temporary must outlive the launch
     ws_bytes = workspace.numel() * workspace.element_size()
+    if fp8:
+        ks, vs = _scales_for(k_scales, v_scales, hkv, q.device, stream)
+        _check(_paged_attn_decode_cascade_fp8(
+            _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            _ptr(context_lens), _ptr(group_start), _ptr(shared_blocks), float(scale), _ptr(ks),
+            _ptr(vs), s, g, max_group_size, max_shared_blocks, h, hkv, d, bs,
+            block_tables.shape[1], max_context_len, num_blocks, _dtype_code(q), partition_size,
+            _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream)),
+            "paged_attn_decode_cascade_fp8")
+        return
     _check(_paged_attn_decode_cascade(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                       _ptr(block_tables), _ptr(context_lens), _ptr(group_start),
                                       _ptr(shared_blocks), float(scale), s, g, max_group_size,

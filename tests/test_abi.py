@@ -156,7 +156,7 @@ def test_prefill_fp8_host_validation_without_gpu():
         # out q k v tables lens qstart scale ks vs S T H Hkv D bs maxblk maxctx maxq nblk dt
         return pk._paged_attn_prefill_fp8(ptr, ptr, ptr, ptr, ptr, ptr, ptr, 0.125, ks, vs, s, 8,
                                           h, 2, d, 16, 4, 64, 4, 8, dt, null, null)
-    assert pre8(d=64) == pk.ERR_UNSUPPORTED               # E4M3 prefill: head_dim 128 only
+    assert pre8(d=96) == pk.ERR_UNSUPPORTED               # head_dim 64 or 128
     assert pre8(h=6) == pk.ERR_UNSUPPORTED                # G = 3
     assert pre8(ks=null) == pk.ERR_INVALID_ARG
     assert pre8(vs=null) == pk.ERR_INVALID_ARG
@@ -193,13 +193,23 @@ def test_cascade_host_validation_without_gpu():
                                              mgs, msb, 8, 2, d, 16, 16, mc, 64, 0, part, good,
                                              wsb, null, null)
     assert cas(s=0) == pk.OK
-    assert cas(d=64) == pk.ERR_UNSUPPORTED                 # the prefix pass is head_dim 128
+    assert cas(d=96) == pk.ERR_UNSUPPORTED                 # head_dim 64 or 128
     assert cas(g=0) == pk.ERR_INVALID_ARG                  # sequences but no groups
     assert cas(msb=17) == pk.ERR_INVALID_ARG               # 17 * 16 > max_context_len
     assert cas(gptr=null) == pk.ERR_INVALID_ARG
     assert cas(wsb=ws - 16) == pk.ERR_WORKSPACE
     assert cas(ptr=bad) == pk.ERR_INVALID_ARG
     assert cas(part=24) == pk.ERR_INVALID_ARG              # not a multiple of block_size
+
+    def cas8(s=4, d=64, ks=good, vs=good, dt=pk.BF16):
+        return pk._paged_attn_decode_cascade_fp8(good, good, good, good, good, good, good, good,
+                                                 0.125, ks, vs, s, 2, 2, 4, 8, 2, d, 16, 16, 256,
+                                                 64, dt, 0, good, ws, null, null)
+    assert cas8(s=0) == pk.OK
+    assert cas8(d=96) == pk.ERR_UNSUPPORTED
+    assert cas8(ks=null) == pk.ERR_INVALID_ARG
+    assert cas8(vs=null) == pk.ERR_INVALID_ARG
+    assert cas8(dt=pk.FP8_E4M3) == pk.ERR_INVALID_ARG      # q/out must be 16-bit
 
 
 def test_pipeline_staging_and_host_validation_without_gpu():

@@ -56,6 +56,77 @@ def test_cascade_matches_oracle(pk, prompts, samples, plen, h, hkv, bs, dtype):
         assert_close(dev_to_bits(dw.out), ref, w)
 
 
+# head_dim 64: the prefix pass is the mma.sync kernel in prefix mode; G = 1
+# reads each member's own blocks on the CUDA cores, G >= 2 on the tensor cores
+CASES_D64 = [(3, 4, 37, 8, 2, 16, "bf16"), (2, 8, 64, 4, 4, 32, "fp16"),
+             (4, 2, 100, 16, 2, 16, "fp16"), (1, 16, 300, 8, 8, 32, "bf16")]
+
+
+@pytest.mark.parametrize("prompts,samples,plen,h,hkv,bs,dtype", CASES_D64)
+def test_cascade_head_dim_64_matches_oracle(pk, prompts, samples, plen, h, hkv, bs, dtype):
+    w = W.build_prefix_share_workload(prompts, samples, plen, 5, 40, h, hkv, 64, bs, dtype,
+                                      seed=plen + samples + 64, allocator=block_allocator)
+    dw = DeviceWorkload(w)
+    assert run_step(pk, dw, decode=False) == 0
+    group_start, shared = W.cascade_groups(w)
+    kc, vc = oracle_caches(w)
+    ref = oracle_decode(w, kc, vc)
+    for part in (0, bs):
+        dw.out.zero_()
+        assert run_cascade(pk, dw, group_start, shared, partition_size=part) == 0
+        assert_close(dev_to_bits(dw.out), ref, w)
+
+
+# E4M3 caches: (prompts, samples, prompt_len, heads, kv heads, head_dim, block, dtype)
+CASES_FP8 = [(3, 4, 37, 8, 2, 128, 16, "bf16"), (2, 8, 64, 8, 1, 128, 32, "fp16"),
+             (4, 2, 100, 4, 4, 128, 16, "fp16"), (3, 4, 37, 8, 2, 64, 16, "bf16"),
+             (2, 8, 64, 4, 4, 64, 32, "fp16"), (1, 16, 300, 8, 8, 64, 16, "bf16")]
+
+
+@pytest.mark.parametrize("prompts,samples,plen,h,hkv,d,bs,dtype", CASES_FP8)
+def test_cascade_fp8_matches_oracle(pk, prompts, samples, plen, h, hkv, d, bs, dtype):
+    """Cascade decode over E4M3 caches equals the oracle's decode over its own
+    quantised caches (the plain E4M3 decode's reference)."""
+    from test_gpu_fp8 import Fp8Device, oracle_codes, oracle_decode8
+    w = W.build_prefix_share_workload(prompts, samples, plen, 5, 40, h, hkv, d, bs, dtype,
+                                      seed=plen + samples + d, allocator=block_allocator)
+    dev = Fp8Device(pk, w)
+    assert dev.step(pk, decode=False) == 0
+    kq, vq = oracle_codes(w)
+    assert np.array_equal(dev.k8.cpu().numpy(), kq)
+    ref = oracle_decode8(w, kq, vq)
+    gs, shared = W.cascade_groups(w)
+    gs_t = torch.from_numpy(np.asarray(gs, np.int32)).cuda()
+    sb_t = torch.from_numpy(np.asarray(shared, np.int32)).cuda()
+    for part in (0, bs):
+        dev.out.zero_()
+        pk.paged_attn_decode_cascade(dev.out, dev.q, dev.k8, dev.v8, dev.tables, dev.lens, gs_t,
+                                     sb_t, w.scale, w.num_kv_heads, w.block_size,
+                                     w.max_context_len, int(np.diff(gs).max()),
+                                     int(np.max(shared)), partition_size=part, dev_err=dev.err,
+                                     k_scales=dev.ks, v_scales=dev.vs)
+        torch.cuda.synchronize()
+        assert int(dev.err.item()) == 0
+        assert_close(dev_to_bits(dev.out), ref, w)
+
+
+def test_cascade_fp8_reports_a_bad_scale(pk):
+    from test_gpu_fp8 import Fp8Device
+    w = W.build_prefix_share_workload(2, 4, 64, 5, 40, 4, 2, 128, 16, "fp16", seed=5,
+                                      allocator=block_allocator)
+    dev = Fp8Device(pk, w)
+    assert dev.step(pk, decode=False) == 0
+    gs, shared = W.cascade_groups(w)
+    bad_v = torch.tensor([0.01, float("inf")], dtype=torch.float32, device="cuda")
+    pk.paged_attn_decode_cascade(dev.out, dev.q, dev.k8, dev.v8, dev.tables, dev.lens,
+                                 torch.from_numpy(gs).cuda(), torch.from_numpy(shared).cuda(),
+                                 w.scale, w.num_kv_heads, w.block_size, w.max_context_len,
+                                 int(np.diff(gs).max()), int(np.max(shared)), dev_err=dev.err,
+                                 k_scales=dev.ks, v_scales=bad_v)
+    torch.cuda.synchronize()
+    assert int(dev.err.item()) & pk.DEVERR_BAD_SCALE
+
+
 def test_cascade_with_fewer_shared_blocks_and_singletons(pk):
     """Declaring less sharing than there is, or none, changes nothing."""
     w = W.build_prefix_share_workload(3, 4, 70, 5, 40, 8, 2, 128, 16, "fp16", seed=9,

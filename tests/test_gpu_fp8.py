@@ -300,6 +300,40 @@ def test_fp8_prefill_small(pk, bs, g, dtype):
     assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq), w)
 
 
+PREFILL_SHAPES_D64 = [(16, 1, "fp16"), (32, 2, "bf16"), (16, 4, "bf16"), (32, 8, "fp16"),
+                      (16, 8, "bf16"), (32, 1, "bf16")]
+
+
+@pytest.mark.parametrize("bs,g,dtype", PREFILL_SHAPES_D64)
+def test_fp8_prefill_head_dim_64(pk, bs, g, dtype):
+    """head_dim 64 runs the mma.sync kernel over codes widened to fp16 by its
+    producer warp: the same cases as the tcgen05 kernel's."""
+    w = W.build_prefill_workload(PREFILL_HIST, PREFILL_NEW, 2 * g, 2, 64, bs, dtype,
+                                 seed=41 + bs + g)
+    dev = Fp8Device(pk, w)
+    assert run_prefill8(pk, dev) == 0
+    kq, vq = oracle_codes(w)
+    assert np.array_equal(dev.k8.cpu().numpy(), kq)
+    assert np.array_equal(dev.v8.cpu().numpy(), vq)
+    assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq), w)
+
+
+def test_fp8_prefill_head_dim_64_long_history_and_bad_block(pk):
+    """A long history (many 16-key stages through the two widened stages) on
+    sampled rows; then a table entry out of range is reported, not read."""
+    w = W.build_prefill_workload([2000, 0, 333], [100, 150, 77], 8, 2, 64, 16, "bf16", seed=8)
+    dev = Fp8Device(pk, w)
+    assert run_prefill8(pk, dev) == 0
+    kq, vq = oracle_codes(w)
+    rows = [(0, 0), (50, 3), (99, 7), (100, 1), (249, 6), (250, 2), (326, 5)]
+    assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq, rows), w, pairs=rows)
+    tables = w.block_tables.copy()
+    tables[0, 3] = w.num_blocks + 5
+    dev.tables = torch.from_numpy(tables).cuda()
+    dev.err.zero_()
+    assert run_prefill8(pk, dev) & pk.DEVERR_BAD_BLOCK
+
+
 def test_fp8_prefill_long_history_sampled(pk):
     w = W.build_prefill_workload([3000, 0, 777], [200, 300, 129], 16, 4, 128, 16, "bf16", seed=6)
     dev = Fp8Device(pk, w)
@@ -312,8 +346,9 @@ def test_fp8_prefill_long_history_sampled(pk):
     assert_close(dev_to_bits(dev.out), oracle_prefill8(w, kq, vq, rows), w, pairs=rows)
 
 
-def test_fp8_prefill_of_one_token_matches_fp8_decode(pk):
-    w = W.build_decode_workload(RAGGED, 8, 2, 128, 16, "fp16", 23)
+@pytest.mark.parametrize("d", [128, 64])
+def test_fp8_prefill_of_one_token_matches_fp8_decode(pk, d):
+    w = W.build_decode_workload(RAGGED, 8, 2, d, 16, "fp16", 23)
     w.query_start = np.arange(w.num_seqs + 1, dtype=np.int32)
     dev = Fp8Device(pk, w)
     assert run_prefill8(pk, dev) == 0

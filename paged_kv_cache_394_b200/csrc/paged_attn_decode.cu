@@ -353,7 +353,7 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
                          size_t workspace_bytes, unsigned* dev_err, void* stream, bool fp8,
                          const float* k_scales, const float* v_scales,
                          const CascadeGroups* cascade = nullptr,
-                         const int32_t* seq_order = nullptr) {
+                         const int32_t* seq_order = nullptr, bool after_prefix = false) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0 || num_blocks <= 0 || partition_size < 0 || !dtype_valid(dtype) ||
       num_heads % num_kv_heads != 0 || !isfinite(scale))
@@ -439,6 +439,7 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   p.num_groups = cascade ? cascade->num_groups : 0;
   p.max_shared_blocks = cascade ? cascade->max_shared_blocks : 0;
   p.seq_order = cascade ? nullptr : seq_order;  // cascade groups stay together
+  p.independent_of_prior = after_prefix ? 1 : 0;
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   p.withhold_first_load = g_withhold_first_load.load(std::memory_order_relaxed);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -469,6 +470,9 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   rcfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4));
   rcfg.blockDim = dim3(128);
   rcfg.dynamicSmemBytes = 0;
+  // after a prefix pass the decode kernel did not wait for it, so the merge
+  // must wait for both in plain stream order
+  if (after_prefix) rcfg.numAttrs = 0;
   return cuda_status(cudaLaunchKernelEx(&rcfg, reduce_entry(head_dim, dtype), p));
 }
 
@@ -640,6 +644,12 @@ pkv_status cascade_launch(void* out, const void* q, const void* k_cache, const v
     return PKV_ERR_UNSUPPORTED;
   const WorkspaceLayout wl = workspace_layout(num_seqs, num_heads, head_dim, max_parts);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
+  // The prefix pass goes first; each of its CTAs waits for the cache writes
+  // before it lets the next grid start, so the suffix decode, which reads
+  // nothing the prefix pass writes, starts without waiting for it and fills
+  // the SMs the prefix pass frees; the merge waits for both in stream order.
+  // Measured on B200 (parallel-sampling batch, one cascade decode): 0.192 ms
+  // with the suffix waiting for the prefix pass, 0.178 ms without.
   if (max_shared_blocks > 0) {
     const pkv_status st = launch_cascade_prefix(
         q, k_cache, v_cache, block_tables, context_lens, groups, scale, num_seqs, num_heads,
@@ -652,7 +662,8 @@ pkv_status cascade_launch(void* out, const void* q, const void* k_cache, const v
   return decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_seqs,
                        num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                        max_context_len, num_blocks, dtype, partition_size, workspace,
-                       workspace_bytes, dev_err, stream, fp8, k_scales, v_scales, &groups);
+                       workspace_bytes, dev_err, stream, fp8, k_scales, v_scales, &groups,
+                       nullptr, max_shared_blocks > 0);
 }
 
 }  // namespace

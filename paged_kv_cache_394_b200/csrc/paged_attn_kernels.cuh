@@ -85,6 +85,10 @@ struct DecodeParams {
   // Optional order of the sequences over the grid (a permutation of
   // 0 .. num_seqs-1, longest first; see pkv_decode_order), else null.
   const int32_t* seq_order;
+  // 1: the preceding kernel in the stream writes nothing this one reads (the
+  // cascade suffix after its prefix pass, whose CTAs all waited for the cache
+  // writes before letting this grid start), so skip griddepcontrol.wait.
+  int independent_of_prior;
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
@@ -374,7 +378,7 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
 
   // Inputs may come from the previous kernel in the stream (e.g. the cache
   // write); wait for it before reading anything, then let the next one start.
-  grid_dependency_wait();
+  if (!p.independent_of_prior) grid_dependency_wait();
   trigger_dependents();
   // the sequence this CTA serves: in index order, or in the caller's order
   const int rank = unit / p.num_kv_heads;
@@ -835,7 +839,7 @@ __global__ void __launch_bounds__(Tr::THREADS)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  grid_dependency_wait();
+  if (!p.independent_of_prior) grid_dependency_wait();
   trigger_dependents();
   // the sequence this CTA serves: in index order, or in the caller's order
   const int rank = unit / p.num_kv_heads;

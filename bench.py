@@ -432,7 +432,8 @@ def bench_decode(run, workload, headline):
     out = torch.empty_like(q)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     part_req = w.partition_size if args.partition is None else args.partition
-    part = pk.partition_size(w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len, part_req)
+    part = (pk.partition_size_fp8 if fp8 else pk.partition_size)(
+        w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len, part_req)
     split = part < w.max_context_len
     if cascade:
         gs_np, sb_np = W.cascade_groups(w)

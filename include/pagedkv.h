@@ -131,16 +131,22 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_ma
  * sequence is cut into partitions of partition_size tokens; each partition
  * produces a (max logit, exp-sum, unnormalised output) triple in the
  * workspace and a second kernel merges them.  pkv_paged_attn_partition_size
- * returns the partition size `pkv_paged_attn_decode` will use:
+ * returns the partition size `pkv_paged_attn_decode` will use (16-bit caches),
+ * pkv_paged_attn_partition_size_fp8 the one `pkv_paged_attn_decode_fp8` will:
  *   requested > 0  -> requested (must be a multiple of block_size);
- *   requested == 0 -> chosen from the shape; a value >= max_context_len
- *                     means single pass (no workspace needed).
+ *   requested == 0 -> chosen from the shape, at most 4096 tokens (E4M3: 2048,
+ *                     since a 1-byte cache is read twice as fast and a long
+ *                     partition's CTA would outlast the launch); a value >=
+ *                     max_context_len means single pass (no workspace needed).
  */
 int pkv_paged_attn_partition_size(int num_seqs, int num_kv_heads, int block_size,
                                   int max_context_len, int requested);
+int pkv_paged_attn_partition_size_fp8(int num_seqs, int num_kv_heads, int block_size,
+                                      int max_context_len, int requested);
 
-/* Workspace bytes pkv_paged_attn_decode needs for these arguments (0 when it
- * runs single-pass).  Returns 0 too for invalid arguments. */
+/* Workspace bytes pkv_paged_attn_decode and pkv_paged_attn_decode_fp8 need
+ * for these arguments (the larger of the two; 0 when both run single-pass).
+ * Returns 0 too for invalid arguments. */
 size_t pkv_paged_attn_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
                                       int head_dim, int block_size, int max_context_len,
                                       int partition_size);

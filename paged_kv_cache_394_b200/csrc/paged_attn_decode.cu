@@ -273,25 +273,33 @@ std::atomic<int> g_withhold_first_load{0};
 constexpr int kMaxPartitionBlocks = 4096;  // block-table slice kept in shared memory
 constexpr int kSlots = 2 * 148;            // resident decode CTAs: two per SM, 148 SMs
 
-// Partition size in tokens.  With enough (sequence, kv head) units to fill the
-// GPU and contexts of at most 2048 tokens, one pass (no reduce) is fastest.
-// Otherwise contexts are cut so there are about four CTAs per resident slot,
-// in partitions of 256..2048 tokens.  Measured on B200 with the sequences
-// taken longest first (decode kernel GB/s, partition 512 / 1024 / 2048):
-// GQA chat 5972 / 6310 / 6447, its E4M3 form 4632 / 5209 / 5522 (a CTA's
-// start-up is not amortised over short partitions).  In index order the GQA
-// chat batch read 6374 at 1024 against 6225 at 2048.
+// Partition size in tokens, at most `cap` when chosen.  With enough
+// (sequence, kv head) units to fill the GPU and contexts of at most `cap`
+// tokens, one pass (no reduce) is fastest.  Otherwise contexts are cut so
+// there are about four CTAs per resident slot, in partitions of 256..cap
+// tokens.  Measured on B200 with the sequences taken longest first (decode
+// kernel GB/s, partition 512 / 1024 / 2048): GQA chat 5972 / 6310 / 6447, its
+// E4M3 form 4632 / 5209 / 5522 (a CTA's start-up is not amortised over short
+// partitions).  The cap is the most a partition may hold before its CTA, which
+// gets only its share of the bandwidth while the GPU is full, outlasts the
+// launch: 4096 tokens for 16-bit caches (GQA chat, contexts up to 4096: 6519
+// -> 6769 GB/s kernel, 6468 -> 6742 per step without the reduce) and 2048 for
+// E4M3 ones, which are read twice as fast (4096 there gained 5612 -> 5916 on
+// back-to-back launches, whose next launch hides the tail, but lost 5475 ->
+// 5071 per step, behind the cache write).
+constexpr int kAutoPartitionCap16 = 4096;
+constexpr int kAutoPartitionCap8 = 2048;
 int choose_partition(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
-                     int requested) {
+                     int requested, int cap) {
   if (requested > 0) return requested;
   const int whole =
       std::max(block_size, (max_context_len + block_size - 1) / block_size * block_size);
   const long long units = std::max(1LL, static_cast<long long>(num_seqs) * num_kv_heads);
-  if (units >= kSlots && max_context_len <= 2048) return whole;
+  if (units >= kSlots && max_context_len <= cap) return whole;
   const long long parts = std::max(1LL, (4LL * kSlots + units - 1) / units);
   const long long want = (max_context_len + parts - 1) / parts;
   int part = 256;
-  while (part < want && part < 2048) part <<= 1;
+  while (part < want && part < cap) part <<= 1;
   return std::min(whole, part);
 }
 
@@ -322,7 +330,15 @@ int parts_for(int max_context_len, int block_size, int partition) {
 extern "C" int pkv_paged_attn_partition_size(int num_seqs, int num_kv_heads, int block_size,
                                              int max_context_len, int requested) {
   if (block_size <= 0) return 0;
-  return pkv::choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, requested);
+  return pkv::choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, requested,
+                               pkv::kAutoPartitionCap16);
+}
+
+extern "C" int pkv_paged_attn_partition_size_fp8(int num_seqs, int num_kv_heads, int block_size,
+                                                 int max_context_len, int requested) {
+  if (block_size <= 0) return 0;
+  return pkv::choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, requested,
+                               pkv::kAutoPartitionCap8);
 }
 
 extern "C" size_t pkv_paged_attn_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
@@ -332,8 +348,9 @@ extern "C" size_t pkv_paged_attn_workspace_bytes(int num_seqs, int num_heads, in
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_context_len < 0 || partition_size < 0)
     return 0;
-  const int part =
-      choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
+  // the E4M3 rule's partitions are never longer, so its count covers both
+  const int part = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                    partition_size, kAutoPartitionCap8);
   if (part % block_size != 0) return 0;
   const int max_parts = parts_for(max_context_len, block_size, part);
   return workspace_layout(num_seqs, num_heads, head_dim, max_parts).total;
@@ -373,8 +390,9 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
 
-  const int part =
-      choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
+  const int part = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                    partition_size,
+                                    fp8 ? kAutoPartitionCap8 : kAutoPartitionCap16);
   const int part_blocks = part / block_size;
   if (part_blocks > kMaxPartitionBlocks) return PKV_ERR_UNSUPPORTED;
   // cascade decode: workspace slot 0 holds the prefix pass's partial and the
@@ -589,8 +607,8 @@ extern "C" size_t pkv_paged_attn_cascade_workspace_bytes(int num_seqs, int num_h
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_context_len < 0 || partition_size < 0)
     return 0;
-  const int part =
-      choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
+  const int part = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                    partition_size, kAutoPartitionCap8);
   if (part % block_size != 0) return 0;
   return workspace_layout(num_seqs, num_heads, head_dim,
                           1 + parts_for(max_context_len, block_size, part))
@@ -636,8 +654,9 @@ pkv_status cascade_launch(void* out, const void* q, const void* k_cache, const v
   const int group = num_heads / num_kv_heads;
   if (group != 1 && group != 2 && group != 4 && group != 8) return PKV_ERR_UNSUPPORTED;
   if (!block_size_supported(block_size)) return PKV_ERR_UNSUPPORTED;
-  const int part =
-      choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
+  const int part = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                    partition_size,
+                                    fp8 ? kAutoPartitionCap8 : kAutoPartitionCap16);
   if (part / block_size > kMaxPartitionBlocks) return PKV_ERR_UNSUPPORTED;
   const int max_parts = 1 + parts_for(max_context_len, block_size, part);
   if (static_cast<long long>(num_seqs) * num_kv_heads * max_parts > 0x7fffffffLL)

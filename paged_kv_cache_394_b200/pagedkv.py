@@ -42,6 +42,7 @@ _reshape_and_cache = _proto("pkv_reshape_and_cache", _i, _vp, _vp, _vp, _vp, _vp
                             _i, _i, _vp, _vp)
 _copy_blocks = _proto("pkv_copy_blocks", _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp)
 _partition_size = _proto("pkv_paged_attn_partition_size", _i, _i, _i, _i, _i, _i)
+_partition_size_fp8 = _proto("pkv_paged_attn_partition_size_fp8", _i, _i, _i, _i, _i, _i)
 _workspace_bytes = _proto("pkv_paged_attn_workspace_bytes", _sz, _i, _i, _i, _i, _i, _i, _i)
 _paged_attn_decode = _proto("pkv_paged_attn_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i,
                             _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
@@ -197,6 +198,11 @@ def copy_blocks(k_cache, v_cache, block_mapping, dev_err=None, stream=None):
 
 def partition_size(num_seqs, num_kv_heads, block_size, max_context_len, requested=0):
     return _partition_size(num_seqs, num_kv_heads, block_size, max_context_len, requested)
+
+
+def partition_size_fp8(num_seqs, num_kv_heads, block_size, max_context_len, requested=0):
+    """The partition paged_attn_decode_fp8 uses (E4M3 caches)."""
+    return _partition_size_fp8(num_seqs, num_kv_heads, block_size, max_context_len, requested)
 
 
 def workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,

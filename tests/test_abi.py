@@ -85,13 +85,17 @@ def test_partition_and_workspace_queries():
     # short contexts over many (sequence, kv head) units: single pass
     assert pk.partition_size(64, 32, 16, 2048) >= 2048
     assert pk.workspace_bytes(64, 32, 32, 128, 16, 2048) == 0
-    # long contexts over few units: 2048-token partitions
-    assert pk.partition_size(8, 40, 16, 32768) == 2048
+    # long contexts over few units: 4096-token partitions (E4M3: 2048)
+    assert pk.partition_size(8, 40, 16, 32768) == 4096
+    assert pk.partition_size_fp8(8, 40, 16, 32768) == 2048
     n = 8 * 40 * 16
     assert pk.workspace_bytes(8, 40, 40, 128, 16, 32768) >= n * (128 + 2) * 4
     # many units but long contexts: split too; a context that fits one
     # partition runs in one pass
-    assert pk.partition_size(256, 8, 32, 4096) == 2048
+    assert pk.partition_size(256, 8, 32, 4096) >= 4096     # enough units: one pass
+    assert pk.partition_size_fp8(256, 8, 32, 4096) == 2048
+    # the workspace covers the E4M3 rule's partitions too
+    assert pk.workspace_bytes(256, 32, 8, 128, 32, 4096) >= 256 * 32 * 2 * 130 * 4
     assert pk.partition_size(4, 4, 16, 100) >= 100
     # few units: small partitions for parallelism, never below 256 tokens
     assert pk.partition_size(1, 8, 16, 2000) == 256

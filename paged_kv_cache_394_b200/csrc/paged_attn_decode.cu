@@ -24,7 +24,10 @@ namespace pkv {
 // GB/s): with 2 stages (32 KiB of ring, about five CTAs per SM) it reads
 // LLaMA-7B shapes at 5667 (G = 1; the CUDA-core kernel: 5087), GQA chat at
 // 5135 (G = 4), long contexts at 6203; with 3 stages 5549 / 4964 / 6162;
-// with 6 stages 4396 / 3457 / 4207.
+// with 6 stages 4396 / 3457 / 4207.  Later, with sequences longest first and
+// the lazy reference max (LLaMA-7B / GQA chat / long contexts): 4 warps x 2
+// stages 6241 / 5585 / 6360; 4 x 3: 6013 / 5473 / 6314; 8 x 2: 5485 / 4528 /
+// 5208; 8 x 3: 5582 / 4492 / 5099; 2 x 4: 5905 / 5382 / 6228.
 constexpr int kFp8MmaStages = 2;
 
 // Warps per CTA and ring stages per warp for a (head_dim, block_size): about

@@ -268,7 +268,7 @@ def committed_traffic(workload, kind="decode"):
     of its three launches together) from profiles/, if the counters were taken
     on the current device code."""
     sources = (PREFILL_SOURCES if kind == "prefill" else
-               CASCADE_SOURCES if workload.endswith("_cascade") else DECODE_SOURCES)
+               CASCADE_SOURCES if "_cascade" in workload else DECODE_SOURCES)
     path = os.path.join(ROOT, "profiles", "paged_%s_%s_traffic.md" % (kind, workload))
     try:
         text = open(path).read()
@@ -289,7 +289,8 @@ def committed_traffic(workload, kind="decode"):
 # sampling with and without cascade), E4M3 caches and chunked prefill, each a
 # nested object of the headline line with its own value, roofline and clocks.
 OTHER_WORKLOADS = ("llama7b_fp8", "long_splitk", "long_splitk_fp8", "gqa_chat", "gqa_chat_fp8",
-                   "prefix_share", "prefix_share_cascade", "llama7b_prefill",
+                   "prefix_share", "prefix_share_cascade", "prefix_share_cascade_fp8",
+                   "llama7b_prefill",
                    "llama7b_prefill_fp8", "gqa_prefill", "gqa_prefill_fp8")
 
 
@@ -297,14 +298,12 @@ def split_name(workload):
     """(base workload, E4M3 cache?, cascade decode?) of a bench workload name."""
     from paged_kv_cache_394_b200 import workloads as W
     fp8 = workload.endswith("_fp8")
-    cascade = workload.endswith("_cascade")
+    cascade = workload.removesuffix("_fp8").endswith("_cascade")
     base = workload.removesuffix("_fp8").removesuffix("_cascade")
     if base not in W.NAMES + W.PREFILL_NAMES:
         raise ValueError("unknown workload %r" % workload)
     if cascade and base != "prefix_share":
         raise ValueError("cascade decode needs the prefix-sharing workload (prefix_share_cascade)")
-    if cascade and fp8:
-        raise ValueError("cascade decode reads 16-bit caches")
     return base, fp8, cascade
 
 
@@ -459,17 +458,19 @@ def bench_decode(run, workload, headline):
                   out=out, order=order)
 
     def decode(t=inputs):
-        if fp8:
-            pk.paged_attn_decode_fp8(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
-                                     scales[0], scales[1], w.num_kv_heads, w.block_size,
-                                     w.max_context_len, partition_size=part_req, workspace=ws,
-                                     dev_err=err, stream=stream, seq_order=t["order"])
-        elif cascade:
+        if cascade:
             pk.paged_attn_decode_cascade(t["out"], t["q"], kc, vc, t["tables"], t["lens"], gstart,
                                          gshared, w.scale, w.num_kv_heads, w.block_size,
                                          w.max_context_len, max_group, max_shared,
                                          partition_size=part_req, workspace=ws, dev_err=err,
-                                         stream=stream)
+                                         stream=stream,
+                                         k_scales=scales[0] if fp8 else None,
+                                         v_scales=scales[1] if fp8 else None)
+        elif fp8:
+            pk.paged_attn_decode_fp8(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
+                                     scales[0], scales[1], w.num_kv_heads, w.block_size,
+                                     w.max_context_len, partition_size=part_req, workspace=ws,
+                                     dev_err=err, stream=stream, seq_order=t["order"])
         else:
             pk.paged_attn_decode(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
                                  w.num_kv_heads, w.block_size, w.max_context_len,
@@ -678,7 +679,7 @@ def bench_decode(run, workload, headline):
                     stream.wait_event(ev_down[bb])
         e2e_api = ("Python binding (reshape_and_cache%s, paged_attn_decode%s) with "
                    "pinned-host copies on side streams, consecutive steps overlapped"
-                   % (("_fp8", "_fp8") if fp8 else ("", "_cascade")))
+                   % ("_fp8" if fp8 else "", "_cascade" if cascade else "_fp8" if fp8 else ""))
     for i in range(args.warmup):
         e2e_pipelined(i)
     torch.cuda.synchronize(dev)

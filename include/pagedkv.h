@@ -433,7 +433,9 @@ pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, const void* k_ca
  * Groups, workspace (pkv_paged_attn_cascade_workspace_bytes), head_dim 64 or
  * 128 and errors as in pkv_paged_attn_decode_cascade; null scale pointers give
  * PKV_ERR_INVALID_ARG and a scale that is not finite and > 0 sets
- * PKV_DEVERR_BAD_SCALE.
+ * PKV_DEVERR_BAD_SCALE.  The shared pass widens every shared tile through
+ * shared memory, so with 1-byte codes (whose repeats plain decode finds in
+ * L2) it can be slower than pkv_paged_attn_decode_fp8 on the same batch.
  */
 pkv_status pkv_paged_attn_decode_cascade_fp8(
     void* out, const void* q, const void* k_cache, const void* v_cache,

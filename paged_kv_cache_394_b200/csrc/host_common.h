@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "pagedkv.h"
 
 namespace pkv {
@@ -22,6 +24,25 @@ inline bool cache_dtype_valid(int dt) { return dtype_valid(dt) || dt == PKV_FP8_
 inline int cache_elem_bytes(int dt) { return dt == PKV_FP8_E4M3 ? 1 : 2; }
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Launches `kernel` with programmatic stream serialisation: its CTAs may be
+// scheduled while the previous kernel in the stream drains, so the kernel
+// must call griddepcontrol.wait before it touches memory that kernel uses.
+template <class... KArgs, class... Args>
+cudaError_t launch_after_previous(void (*kernel)(KArgs...), dim3 grid, dim3 block, void* stream,
+                                  Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = as_stream(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // 2-D TMA tensor map over a cache viewed as [num_blocks * hkv * bs, d] rows
 // (cached per thread): boxes of 16 rows x 128 bytes (64 16-bit elements or 128

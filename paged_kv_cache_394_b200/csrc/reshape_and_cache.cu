@@ -19,8 +19,11 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ k_cache,
     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_tokens,
     int num_kv_heads, int chunks_per_row, int block_size, int64_t num_slots, unsigned* err) {
-  // The decode kernel that usually follows may start its prologue now; it
+  // Launched with programmatic serialisation: wait for the previous kernel
+  // (the last step's decode reads the cache) before touching memory; the
+  // decode kernel that usually follows may then start its prologue, and it
   // still waits for this grid to finish before reading the cache.
+  grid_dependency_wait();
   trigger_dependents();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * chunks_per_row;
@@ -73,6 +76,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
     uint2* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_tokens,
     int num_kv_heads, int chunks_per_row, int block_size, int64_t num_slots,
     const float* __restrict__ k_scales, const float* __restrict__ v_scales, unsigned* err) {
+  grid_dependency_wait();
   trigger_dependents();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * chunks_per_row;
@@ -121,11 +125,11 @@ extern "C" pkv_status pkv_reshape_and_cache(const void* key, const void* value, 
   const int threads = 256;
   const int64_t grid = (total + threads - 1) / threads;
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
-  reshape_and_cache_kernel<<<static_cast<unsigned>(grid), threads, 0, as_stream(stream)>>>(
+  return cuda_status(launch_after_previous(
+      reshape_and_cache_kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), stream,
       static_cast<const uint4*>(key), static_cast<const uint4*>(value),
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, num_tokens,
-      num_kv_heads, chunks, block_size, static_cast<int64_t>(num_blocks) * block_size, dev_err);
-  return cuda_status(cudaGetLastError());
+      num_kv_heads, chunks, block_size, static_cast<int64_t>(num_blocks) * block_size, dev_err));
 }
 
 extern "C" pkv_status pkv_reshape_and_cache_fp8(const void* key, const void* value,
@@ -152,10 +156,10 @@ extern "C" pkv_status pkv_reshape_and_cache_fp8(const void* key, const void* val
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
   auto kernel = dtype == PKV_FP16 ? reshape_and_cache_fp8_kernel<Fp16>
                                   : reshape_and_cache_fp8_kernel<Bf16>;
-  kernel<<<static_cast<unsigned>(grid), threads, 0, as_stream(stream)>>>(
+  return cuda_status(launch_after_previous(
+      kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), stream,
       static_cast<const uint4*>(key), static_cast<const uint4*>(value),
       static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache), slot_mapping, num_tokens,
       num_kv_heads, chunks, block_size, static_cast<int64_t>(num_blocks) * block_size, k_scales,
-      v_scales, dev_err);
-  return cuda_status(cudaGetLastError());
+      v_scales, dev_err));
 }

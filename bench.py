@@ -357,19 +357,41 @@ def device_caches(pk, w, dev, fp8):
     return q, kc, vc, key, val, scales
 
 
-def time_steps(run, stream, step, n):
+TIMING_NOTE = {False: "the timed steps captured once in a CUDA graph, replayed between two "
+                      "events on the step's stream",
+               True: "the timed steps launched directly between two events on the step's stream"}
+
+
+def time_steps(run, stream, step, n, graph=False):
     """n back-to-back steps between two CUDA events on `stream`, bracketed by
     a barrier and a synchronize on both sides; the max over ranks, per step,
-    with the clocks sampled meanwhile."""
+    with the clocks sampled meanwhile.  With `graph` the n steps are captured
+    once into a CUDA graph (untimed) and the timed region replays it, so the
+    host's launch calls do not gap the device; the device work is the same
+    n steps."""
     import torch
+    g = None
+    if graph:
+        torch.cuda.synchronize(run.dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(i)
+        with torch.cuda.stream(stream):
+            g.replay()                     # untimed: the first launch uploads the graph
+        torch.cuda.synchronize(run.dev)
     clocks = ClockSampler(run.local)
     clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(run.dev)
     torch.cuda.synchronize(run.dev)
     t0.record(stream)
-    for i in range(n):
-        step(i)
+    if g is not None:
+        with torch.cuda.stream(stream):
+            g.replay()
+    else:
+        for i in range(n):
+            step(i)
     t1.record(stream)
     torch.cuda.synchronize(run.dev)
     barrier(run.dev)
@@ -496,7 +518,7 @@ def bench_decode(run, workload, headline):
         raise RuntimeError("%s: device error word %d during warm-up" % (workload, int(err.item())))
 
     # ---- timed region: K whole steps, nothing else on the stream -------------
-    ms_per_step, clk = time_steps(run, stream, step, args.steps)
+    ms_per_step, clk = time_steps(run, stream, step, args.steps, graph=not args.no_graph)
     sbytes = step_bytes(w, kv_elem)
     all_bytes = sum_over_ranks(sbytes, dev)
     value = all_bytes / (ms_per_step * 1e-3) / 1e9
@@ -550,6 +572,7 @@ def bench_decode(run, workload, headline):
                        partition_used=part, split_k=split,
                        seq_order="index order (cascade groups)" if cascade else
                        "longest first in 256-token buckets (pkv_decode_order on the host)",
+                       timing=TIMING_NOTE[bool(args.no_graph)],
                        l2=("no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
                            % (dbytes / 1e9)) if ubytes >= dbytes else
                           ("no flush between steps: %.2f GB of logical KV reads (%.2f GB of "
@@ -754,7 +777,7 @@ def bench_prefill(run, workload, headline):
     torch.cuda.synchronize(dev)
     if int(err.item()) != 0:
         raise RuntimeError("%s: device error word %d during warm-up" % (workload, int(err.item())))
-    ms_per_step, clk = time_steps(run, stream, step, args.steps)
+    ms_per_step, clk = time_steps(run, stream, step, args.steps, graph=not args.no_graph)
     kern_ms, kern_n, sus_ms, sus_n, sus_clk = time_kernel(run, stream, attend, ms_per_step)
     flops = prefill_flops(w)
     all_flops = sum_over_ranks(flops, dev)
@@ -768,6 +791,7 @@ def bench_prefill(run, workload, headline):
         "config": dict(W.describe(w), workload=workload,
                        kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
                        if fp8 else w.dtype,
+                       timing=TIMING_NOTE[bool(args.no_graph)],
                        l2="no flush: each step rewrites the new tokens' K/V"),
         "tokens_per_s": round(run.world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
@@ -1217,6 +1241,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama7b")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the steps as direct launches instead of one captured CUDA graph")
     ap.add_argument("--partition", type=int, default=None,
                     help="partition size in tokens (0 = let the library choose)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -79,9 +79,12 @@ struct TcEntry {
 template <class DT>
 constexpr int kTcQueryTiles = PKV_PREFILL_QUERY_TILES;
 
+#ifndef PKV_PREFILL_NKEY
+#define PKV_PREFILL_NKEY 64
+#endif
 template <int BS, int G, class DT, bool FP8>
 TcEntry make_tc() {
-  using Tr = TcPrefillTraits<BS, G, DT, kTcQueryTiles<DT>, false, FP8>;
+  using Tr = TcPrefillTraits<BS, G, DT, kTcQueryTiles<DT>, false, FP8, FP8 ? 64 : PKV_PREFILL_NKEY>;
   return TcEntry{paged_prefill_tc_kernel<Tr>, Tr::THREADS, Tr::smem_bytes(), Tr::ROWS};
 }
 

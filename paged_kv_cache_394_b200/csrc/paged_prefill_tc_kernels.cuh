@@ -190,7 +190,8 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 
 }  // namespace tc
 
-template <int BS_, int G_, class DT_, int QT_, bool PREFIX_ = false, bool FP8_ = false>
+template <int BS_, int G_, class DT_, int QT_, bool PREFIX_ = false, bool FP8_ = false,
+          int NKEY_ = 64>
 struct TcPrefillTraits {
   static constexpr int D = 128, BS = BS_, G = G_, QT = QT_;
   // prefix mode: the shared-prefix pass of cascade decode (no causal mask,
@@ -210,11 +211,21 @@ struct TcPrefillTraits {
   static constexpr bool kQToFp16 = kFp8 && std::is_same<DT, Bf16>::value;
   static constexpr int M = 128;                  // rows of one query tile (one TMEM lane each)
   static constexpr int ROWS = QT * M;            // query rows per CTA; they share every KV tile
-  static constexpr int NKEY = 64;                // keys per KV tile
+  // keys per KV tile: 64 with two S buffers per query tile, or 128 with one
+  // (two query tiles then fill TMEM with S 128 + O 128 each, and each S MMA
+  // reads Q once per 128 keys)
+  static constexpr int NKEY = NKEY_;
+  static constexpr int NSB = NKEY == 128 ? 1 : 2;   // S buffers per query tile
+  static constexpr int PIECES = NKEY / 16;          // 16-key TMA boxes per tile and kind
+  static constexpr int HALVES = NKEY / 64;          // 64-column passes of the softmax
+  // bf16 P as hi + lo: with 128-key tiles each 16-key group keeps its 8 hi
+  // columns and 8 lo columns together, so the P of one 64-key half lies
+  // within the S columns that half has already been read from
   static constexpr int kSortUnits = 512;         // (sequence, tile) units ranked per CTA
   // KV stages: what fits beside QT query tiles (P lives in TMEM, over S); the
   // cascade prefix pass (one query tile) keeps PKV_PREFIX_STAGES
-  static constexpr int NS = kFp8 ? 4 : QT == 2 ? 5 : kPrefix ? PKV_PREFIX_STAGES : PKV_QT1_STAGES;
+  static constexpr int NS = NKEY == 128 ? 2
+                            : kFp8 ? 4 : QT == 2 ? 5 : kPrefix ? PKV_PREFIX_STAGES : PKV_QT1_STAGES;
   static constexpr int NSTG = kFp8 ? 2 : 0;      // E4M3 staging slots per kind
   // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
   // P.V issuer
@@ -226,28 +237,33 @@ struct TcPrefillTraits {
   // shared-memory layout (all 1024-byte aligned)
   static constexpr int Q_HALF = M * 128;         // [128 rows][64 dims] = 16 KiB
   static constexpr int Q_TILE = 2 * Q_HALF;
-  static constexpr int KV_HALF = NKEY * 128;     // [64 keys][64 dims] = 8 KiB
+  static constexpr int KV_HALF = NKEY * 128;     // [NKEY keys][64 dims]
   static constexpr int STAGE = 4 * KV_HALF;      // K0 K1 V0 V1
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = QT * Q_TILE;
-  static constexpr int STG_TILE = NKEY * 128;   // [64 keys][128 codes], 128-byte swizzle
+  static constexpr int STG_TILE = NKEY * 128;   // [NKEY keys][128 codes], 128-byte swizzle
   static constexpr int OFF_STG = OFF_KV + NS * STAGE;            // K slots, then V slots
   static constexpr int OFF_BAR = OFF_STG + 2 * NSTG * STG_TILE;
   // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], then
-  // per query tile s_full[2], p_full[2], o_done[2]; then (E4M3) the staging
+  // per query tile s_full[NSB], p_full[NSB], o_done[NSB]; then (E4M3) the staging
   // slots' stg_full[2][NSTG]; then q_ready (query tiles rounded to fp16);
   // then (E4M3) stg_read[2][NSTG] (both widening warps are done with a
   // slot); then the TMEM address slot
-  static constexpr int BAR_Q_READY = 1 + 4 * NS + 6 * QT + 2 * NSTG;
+  static constexpr int BAR_Q_READY = 1 + 4 * NS + 3 * NSB * QT + 2 * NSTG;
   static constexpr int BAR_STG_READ = BAR_Q_READY + 1;
   static constexpr int NBAR = BAR_STG_READ + 2 * NSTG;
   // the softmax reference max moves only when a row max exceeds it by more
   // than this (base-2 units), so P stays below 2^8 and O is rarely rescaled
   static constexpr float kRescaleThreshold = 8.f;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
-  // per query tile q: S buffers at 256q and 256q + 64, O at 256q + 128
-  static constexpr uint32_t TMEM_COLS = 256 * QT;
+  // TMEM per query tile q, from q * QCOLS: NSB S buffers of NKEY columns (P
+  // over S), then O (128 columns)
+  static constexpr int O_COL = NSB * NKEY;
+  static constexpr int QCOLS = O_COL + 128;
+  static constexpr uint32_t TMEM_COLS = QT * QCOLS <= 256 ? 256 : 512;
   static_assert(QT == 1 || QT == 2, "one or two query tiles per CTA");
+  static_assert(NKEY == 64 || (NKEY == 128 && !kFp8), "128-key tiles: 16-bit caches");
+  static_assert(QT * QCOLS <= 512, "tensor memory");
   static_assert(1024 + SMEM <= 232448, "shared memory per CTA");
   static size_t smem_bytes() { return 1024 + static_cast<size_t>(SMEM); }
 };
@@ -262,6 +278,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   constexpr int G = Tr::G, BS = Tr::BS, M = Tr::M, NKEY = Tr::NKEY, NS = Tr::NS;
   constexpr int QT = Tr::QT, ROWS = Tr::ROWS;
   constexpr uint32_t IDESC_S = tc::idesc_f16(Tr::kBf16, M, NKEY, false);
+  constexpr int PIECES = Tr::PIECES, NSB = Tr::NSB;
+  // TMEM column (within a tile's S buffer) of 16-key group kk's P: hi, lo
+  auto p_col_hi = [](int kk) { return Tr::NKEY == 128 && Tr::kBf16 ? 16 * kk : 8 * kk; };
+  auto p_col_lo = [](int kk) { return Tr::NKEY == 128 ? 16 * kk + 8 : Tr::NKEY / 2 + 8 * kk; };
   constexpr uint32_t IDESC_O = tc::idesc_f16(Tr::kBf16, M, 128, true);
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -273,11 +293,17 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   auto bar_k_empty = [&](int s) { return smem_addr(bars + 1 + NS + s); };
   auto bar_v_full = [&](int s) { return smem_addr(bars + 1 + 2 * NS + s); };
   auto bar_v_empty = [&](int s) { return smem_addr(bars + 1 + 3 * NS + s); };
-  auto bar_s_full = [&](int q, int b) { return smem_addr(bars + 1 + 4 * NS + 6 * q + b); };
-  auto bar_p = [&](int q, int b) { return smem_addr(bars + 3 + 4 * NS + 6 * q + b); };
-  auto bar_o = [&](int q, int b) { return smem_addr(bars + 5 + 4 * NS + 6 * q + b); };
+  auto bar_s_full = [&](int q, int b) {
+    return smem_addr(bars + 1 + 4 * NS + 3 * Tr::NSB * q + b);
+  };
+  auto bar_p = [&](int q, int b) {
+    return smem_addr(bars + 1 + 4 * NS + 3 * Tr::NSB * q + Tr::NSB + b);
+  };
+  auto bar_o = [&](int q, int b) {
+    return smem_addr(bars + 1 + 4 * NS + 3 * Tr::NSB * q + 2 * Tr::NSB + b);
+  };
   auto bar_stg = [&](int kind, int s) {
-    return smem_addr(bars + 1 + 4 * NS + 6 * QT + kind * Tr::NSTG + s);
+    return smem_addr(bars + 1 + 4 * NS + 3 * Tr::NSB * QT + kind * Tr::NSTG + s);
   };
   const uint32_t bar_q_ready = smem_addr(bars + Tr::BAR_Q_READY);
   auto bar_stg_read = [&](int kind, int s) {
@@ -392,7 +418,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       mbar_init(bar_v_empty(s), 1);
     }
     for (int q = 0; q < QT; ++q) {
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < Tr::NSB; ++b) {
         mbar_init(bar_s_full(q, b), 1);
         mbar_init(bar_p(q, b), 4);
         mbar_init(bar_o(q, b), 1);
@@ -441,10 +467,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     // the 16-key pieces of tile t that hold keys this CTA needs (pb = -1 past
     // them); t must not decrease from call to call (the table is read in
     // 32-entry chunks)
-    auto lookup = [&](int t, int (&pb)[4]) {
+    auto lookup = [&](int t, int (&pb)[PIECES]) {
       int npieces = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < PIECES; ++i) {
         const int key0 = t * NKEY + i * 16;
         pb[i] = -1;
         if (key0 < nkv) {
@@ -471,11 +497,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       const int kind = is_k ? 0 : 1;
       const uint32_t stg0 = sbase + Tr::OFF_STG + kind * Tr::NSTG * Tr::STG_TILE;
       auto stage_codes = [&](int t) {  // all lanes (the table lookup is warp-wide)
-        int pb[4];
+        int pb[PIECES];
         const int npieces = lookup(t, pb);
         int bytes = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < PIECES; ++i)
           if (i < npieces && valid_block(pb[i])) bytes += 2048;
         const uint32_t bar = bar_stg(kind, t % Tr::NSTG);
         if (lane == 0) {
@@ -487,11 +513,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
             mbar_arrive(bar);
         }
         __syncwarp();
-        if (lane < 4) {
-          int pbi = pb[0];
-          if (lane == 1) pbi = pb[1];
-          if (lane == 2) pbi = pb[2];
-          if (lane == 3) pbi = pb[3];
+        if (lane < PIECES) {
+          int pbi = -1;
+#pragma unroll
+          for (int i = 0; i < PIECES; ++i)
+            if (i == lane) pbi = pb[i];
           if (lane < npieces && valid_block(pbi)) {
             const int key0 = t * NKEY + lane * 16;
             const int y = (pbi * p.num_kv_heads + kvh) * BS + (key0 % BS);
@@ -521,9 +547,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         // index XOR row % 8).
         const uint32_t src = stg0 + (t % Tr::NSTG) * Tr::STG_TILE;
         const uint32_t dst = sbase + Tr::OFF_KV + stage * Tr::STAGE + (is_k ? 0 : 2 * Tr::KV_HALF);
-        const int first = helper ? 256 : 0;
+        const int first = helper ? NKEY * 8 / 2 : 0;
 #pragma unroll 4
-        for (int k = 0; k < 16 / Tr::NWIDEN; ++k) {
+        for (int k = 0; k < NKEY * 8 / Tr::NWIDEN / 32; ++k) {
           const int idx = first + lane + 32 * k;
           const int r = idx >> 3, c = idx & 7;
           uint32_t w[4];
@@ -579,9 +605,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         if (!ok) break;
         // the 16-key pieces of this tile that hold keys this CTA needs
         int npieces = 0;
-        int pb[4];
+        int pb[PIECES];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < PIECES; ++i) {
           const int key0 = t * NKEY + i * 16;
           pb[i] = -1;
           if (key0 < nkv) {
@@ -597,7 +623,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         }
         int bytes = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < PIECES; ++i)
           if (i < npieces && static_cast<unsigned>(pb[i]) < static_cast<unsigned>(p.num_blocks))
             bytes += 2 * 2048;
         const uint32_t bar = is_k ? bar_k_full(stage) : bar_v_full(stage);
@@ -611,14 +637,15 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
             mbar_arrive(bar);
         }
         __syncwarp();
-        // lanes 0..7 issue the tile's 8 boxes of K (or V) at once: lane = piece * 2 +
-        // half; kind 0 / 1 = K low / high dims, 2 / 3 = V low / high dims
-        if (lane < 8) {
+        // lanes 0 .. 2 PIECES - 1 issue the tile's boxes of K (or V) at once:
+        // lane = piece * 2 + half; kind 0 / 1 = K low / high dims, 2 / 3 = V
+        // low / high dims
+        if (lane < 2 * PIECES) {
           const int i = lane >> 1, kind = (is_k ? 0 : 2) + (lane & 1);
-          int pbi = pb[0];
-          if (i == 1) pbi = pb[1];
-          if (i == 2) pbi = pb[2];
-          if (i == 3) pbi = pb[3];
+          int pbi = -1;
+#pragma unroll
+          for (int i2 = 0; i2 < PIECES; ++i2)
+            if (i2 == i) pbi = pb[i2];
           if (i < npieces && static_cast<unsigned>(pbi) < static_cast<unsigned>(p.num_blocks)) {
             const uint32_t st = sbase + Tr::OFF_KV + stage * Tr::STAGE;
             const int key0 = t * NKEY + i * 16;
@@ -645,17 +672,18 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       // O_q += P_q V for tile t
       auto issue_pv = [&](int q, int t) {
         const uint64_t v0 = d_v + static_cast<uint32_t>((t % NS) * (Tr::STAGE >> 4));
-        const uint32_t o_tmem = tmem + q * 256 + 128;
-        // P in TMEM: columns 0..31 of the tile's S buffer (bf16 lo halves in 32..63)
-        const uint32_t p_tmem = tmem + q * 256 + (t & 1) * 64;
+        const uint32_t o_tmem = tmem + q * Tr::QCOLS + Tr::O_COL;
+        // P in TMEM over the tile's S buffer (p_col_hi / p_col_lo)
+        const uint32_t p_tmem = tmem + q * Tr::QCOLS + (t % NSB) * NKEY;
 #pragma unroll
         for (int kk = 0; kk < NKEY / 16; ++kk) {
           const uint64_t bdesc = v0 + kk * (2048 >> 4);
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          tc::umma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, IDESC_O, acc);
-          if constexpr (Tr::kBf16) tc::umma_f16_ts(o_tmem, p_tmem + 32 + kk * 8, bdesc, IDESC_O, 1u);
+          tc::umma_f16_ts(o_tmem, p_tmem + p_col_hi(kk), bdesc, IDESC_O, acc);
+          if constexpr (Tr::kBf16)
+            tc::umma_f16_ts(o_tmem, p_tmem + p_col_lo(kk), bdesc, IDESC_O, 1u);
         }
-        tc::umma_commit(bar_o(q, t & 1));
+        tc::umma_commit(bar_o(q, t % NSB));
       };
       // S_q = Q_q K^T of tile t
       auto issue_s = [&](int q, int t) {
@@ -665,10 +693,10 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t step = (ks < 4 ? 0 : Tr::Q_HALF >> 4) + (ks & 3) * 2;
           const uint32_t kstep = (ks < 4 ? 0 : Tr::KV_HALF >> 4) + (ks & 3) * 2;
-          tc::umma_f16(tmem + q * 256 + (t & 1) * 64, q0d + step, k0 + kstep, IDESC_S,
+          tc::umma_f16(tmem + q * Tr::QCOLS + (t % NSB) * NKEY, q0d + step, k0 + kstep, IDESC_S,
                        ks > 0 ? 1u : 0u);
         }
-        tc::umma_commit(bar_s_full(q, t & 1));
+        tc::umma_commit(bar_s_full(q, t % NSB));
       };
       // Two issuing threads, each taking its MMAs in order with one wait at a
       // time: warp 1 issues S of tile u once its K has landed and P.V of tile
@@ -684,8 +712,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll
           for (int q = 0; q < QT; ++q) {
             if (!ok || u >= ntq[q]) continue;
-            // the S buffer of tile u - 2 holds that tile's P until P.V has read it
-            if (u >= 2) ok = mbar_wait_bounded(bar_o(q, u & 1), ((u - 2) >> 1) & 1);
+            // the S buffer of tile u - NSB holds that tile's P until P.V has read it
+            if (u >= NSB) ok = mbar_wait_bounded(bar_o(q, u % NSB), ((u - NSB) / NSB) & 1);
             if (!ok) break;
             tc::tc_fence_after();
             issue_s(q, u);
@@ -698,12 +726,12 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
           const bool last = t == ntiles - 1;
 #pragma unroll
           for (int q = 0; q < QT; ++q)
-            if (ok && last && t < ntq[q]) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+            if (ok && last && t < ntq[q]) ok = mbar_wait_bounded(bar_p(q, t % NSB), (t / NSB) & 1);
           if (ok) ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
 #pragma unroll
           for (int q = 0; q < QT; ++q) {
             if (!ok || t >= ntq[q]) continue;
-            if (!last) ok = mbar_wait_bounded(bar_p(q, t & 1), (t >> 1) & 1);
+            if (!last) ok = mbar_wait_bounded(bar_p(q, t % NSB), (t / NSB) & 1);
             if (!ok) break;
             tc::tc_fence_after();
             issue_pv(q, t);
@@ -720,7 +748,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const int qg = (warp - 3) >> 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
-    const uint32_t lane_addr = tmem + qg * 256 + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t lane_addr = tmem + qg * Tr::QCOLS + (static_cast<uint32_t>(quarter * 32) << 16);
     const int crow = qg * M + r;   // row within the CTA
     const bool active = crow < rows_total - tile * ROWS;
     const int j = tok0 + crow / G;
@@ -765,43 +793,58 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     float m = -INFINITY, l = 0.f;
     for (int t = 0; ok && t < my_tiles; ++t) {
       const int kv0 = t * NKEY;
-      ok = mbar_wait_bounded(bar_s_full(qg, t & 1), (t >> 1) & 1);
+      ok = mbar_wait_bounded(bar_s_full(qg, t % NSB), (t / NSB) & 1);
       if (!__all_sync(kFullMask, ok)) {
         ok = false;
         break;
       }
       tc::tc_fence_after();
-      float s[NKEY];
-#pragma unroll
-      for (int c = 0; c < NKEY; c += 16) {
-        float v[16];
-        tc::tmem_ld16(lane_addr + (t & 1) * 64 + c, v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) s[c + i] = v[i];
-      }
-      tc::tmem_wait_ld();
+      const uint32_t sbuf = lane_addr + (t % NSB) * NKEY;  // this tile's S (then P) columns
       // Scaled logits are x = s * qscale.  For qscale > 0 the row max of x is
       // (max s) * qscale exactly, so s is masked and reduced unscaled and the
       // scale folds into the exponent's FFMA: p = 2^(s * qscale - m).
-      float mult = p.qscale * k_scale;
-      const bool needs_mask = kv0 + NKEY - 1 > pos;  // this tile reaches past the row
-      if (mult > 0.f) {
-        if (needs_mask) {
+      const float mult0 = p.qscale * k_scale;
+      const float mult = mult0 > 0.f ? mult0 : 1.f;
+      // 64 columns of the row from TMEM (half hf of a 128-key tile), masked
+      // (and, for a scale <= 0, scaled before the max)
+      auto load_half = [&](int hf, float (&v64)[64]) {
 #pragma unroll
-          for (int c = 0; c < NKEY; ++c) s[c] = (kv0 + c <= pos) ? s[c] : -INFINITY;
+        for (int c = 0; c < 64; c += 16) {
+          float v[16];
+          tc::tmem_ld16(sbuf + hf * 64 + c, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v64[c + i] = v[i];
         }
-      } else {
+        tc::tmem_wait_ld();
+        const int k0 = kv0 + hf * 64;
+        if (mult0 > 0.f) {
+          if (k0 + 63 > pos) {  // these keys reach past the row
 #pragma unroll
-        for (int c = 0; c < NKEY; ++c) s[c] = (kv0 + c <= pos) ? s[c] * mult : -INFINITY;
-        mult = 1.f;
+            for (int c = 0; c < 64; ++c) v64[c] = (k0 + c <= pos) ? v64[c] : -INFINITY;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) v64[c] = (k0 + c <= pos) ? v64[c] * mult0 : -INFINITY;
+        }
+      };
+      auto max64 = [&](const float (&v64)[64]) {
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) mx4[u] = tc::max3(mx4[u], v64[c + u], v64[c + 4 + u]);
+        }
+        return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      };
+      float s[64];
+      float smax = -INFINITY;
+#pragma unroll
+      for (int hf = 0; hf < Tr::HALVES; ++hf) {
+        // the max pass (with 128-key tiles both halves are read again below)
+        load_half(hf, s);
+        smax = fmaxf(smax, max64(s));
       }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int c = 0; c < NKEY; c += 8) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) mx4[u] = tc::max3(mx4[u], s[c + u], s[c + 4 + u]);
-      }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * mult;
+      const float mx = smax * mult;
       // move the reference max only when this tile would push P above 2^8
       float alpha = 1.f;
       if (active && mx > m + Tr::kRescaleThreshold) {
@@ -814,16 +857,57 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       const uint64_t mult2 = tc::f2_pack(mult, mult), neg_m2 = tc::f2_pack(neg_m, neg_m);
       uint64_t sum2[2] = {tc::f2_pack(0.f, 0.f), tc::f2_pack(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < NKEY; c += 4) {
+      for (int hf = 0; hf < Tr::HALVES; ++hf) {
+        // a 64-key tile is still in registers; each half of a 128-key tile is
+        // read again, and its P goes over S columns already read (keys
+        // 64 hf .. 64 hf + 63 -> the P columns of groups 4 hf .. 4 hf + 3)
+        if (Tr::HALVES > 1) load_half(hf, s);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float x0, x1;
-          tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[c + 2 * h], s[c + 2 * h + 1]), mult2, neg_m2), x0, x1);
-          s[c + 2 * h] = exp2_approx(x0);
-          s[c + 2 * h + 1] = exp2_approx(x1);
-          sum2[h] = tc::f2_add(sum2[h], tc::f2_pack(s[c + 2 * h], s[c + 2 * h + 1]));
+        for (int c = 0; c < 64; c += 4) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float x0, x1;
+            tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[c + 2 * h], s[c + 2 * h + 1]), mult2, neg_m2),
+                          x0, x1);
+            s[c + 2 * h] = exp2_approx(x0);
+            s[c + 2 * h + 1] = exp2_approx(x1);
+            sum2[h] = tc::f2_add(sum2[h], tc::f2_pack(s[c + 2 * h], s[c + 2 * h + 1]));
+          }
+        }
+        // P (16-bit; bf16 as hi + lo) into TMEM over the S just read, 16 keys
+        // (8 columns of 2 values) per group kk
+#pragma unroll
+        for (int g4 = 0; g4 < 4; g4 += 2) {
+          const int kk = 4 * hf + g4;  // two groups: 16 columns per store
+          uint32_t w[16], wl[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = s[16 * g4 + 2 * e], b = s[16 * g4 + 2 * e + 1];
+            w[e] = pack2(a, b, typename Tr::MT());
+            if constexpr (Tr::kBf16)
+              wl[e] = pack2(a - __uint_as_float(w[e] << 16),
+                            b - __uint_as_float(w[e] & 0xffff0000u), Bf16());
+          }
+          if constexpr (NKEY == 128 && Tr::kBf16) {
+            // hi and lo of each group side by side: group kk -> columns
+            // 16 kk .. 16 kk + 7 (hi) and 16 kk + 8 .. 16 kk + 15 (lo)
+            uint32_t h0[16], h1[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              h0[e] = w[e];
+              h0[8 + e] = wl[e];
+              h1[e] = w[8 + e];
+              h1[8 + e] = wl[8 + e];
+            }
+            tc::tmem_st16u(sbuf + p_col_hi(kk), h0);
+            tc::tmem_st16u(sbuf + p_col_hi(kk + 1), h1);
+          } else {
+            tc::tmem_st16u(sbuf + p_col_hi(kk), w);
+            if constexpr (Tr::kBf16) tc::tmem_st16u(sbuf + p_col_lo(kk), wl);
+          }
         }
       }
+      tc::tmem_wait_st();
       float sum4[4];
       tc::f2_unpack(sum2[0], sum4[0], sum4[1]);
       tc::f2_unpack(sum2[1], sum4[2], sum4[3]);
@@ -831,7 +915,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       l = l * alpha + sum;
       if (t > 0 && __any_sync(kFullMask, alpha != 1.f)) {
         // O must hold every earlier tile before it is rescaled
-        ok = mbar_wait_bounded(bar_o(qg, (t - 1) & 1), ((t - 1) >> 1) & 1);
+        ok = mbar_wait_bounded(bar_o(qg, (t - 1) % NSB), ((t - 1) / NSB) & 1);
         if (!__all_sync(kFullMask, ok)) {
           ok = false;
           break;
@@ -840,38 +924,18 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll 1
         for (int c = 0; c < 128; c += 16) {
           float v[16];
-          tc::tmem_ld16(lane_addr + 128 + c, v);
+          tc::tmem_ld16(lane_addr + Tr::O_COL + c, v);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] *= alpha;
-          tc::tmem_st16(lane_addr + 128 + c, v);
-        }
-        tc::tmem_wait_st();
-      }
-      {
-        // P (16-bit; bf16 as hi + lo) into TMEM over the S just read:
-        // columns 0..31 of the tile's S buffer (bf16 lo halves in 32..63)
-        const uint32_t pt = lane_addr + (t & 1) * 64;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w[16], wl[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float a = s[32 * h + 2 * e], b = s[32 * h + 2 * e + 1];
-            w[e] = pack2(a, b, typename Tr::MT());
-            if constexpr (Tr::kBf16)
-              wl[e] = pack2(a - __uint_as_float(w[e] << 16),
-                            b - __uint_as_float(w[e] & 0xffff0000u), Bf16());
-          }
-          tc::tmem_st16u(pt + 16 * h, w);
-          if constexpr (Tr::kBf16) tc::tmem_st16u(pt + 32 + 16 * h, wl);
+          tc::tmem_st16(lane_addr + Tr::O_COL + c, v);
         }
         tc::tmem_wait_st();
       }
       // keys past the context, or not loaded, hold stale data: zero their V rows
       // (every query tile that uses the stage writes the same zeros)
       const int loaded_end = min(kv0 + NKEY, ((nkv + 15) / 16) * 16);
-      const int vz = min(ctx, loaded_end) - kv0;  // V rows [vz, 64) must be zero
+      const int vz = min(ctx, loaded_end) - kv0;  // V rows [vz, NKEY) must be zero
       if (vz < NKEY) {
         // V of this tile may still be in flight: let it land before zeroing rows
         ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
@@ -891,11 +955,11 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p(qg, t & 1));
+      if (lane == 0) mbar_arrive(bar_p(qg, t % NSB));
     }
     // ---- epilogue ------------------------------------------------------------------------
     if (ok && my_tiles > 0) {
-      ok = mbar_wait_bounded(bar_o(qg, (my_tiles - 1) & 1), ((my_tiles - 1) >> 1) & 1);
+      ok = mbar_wait_bounded(bar_o(qg, (my_tiles - 1) % NSB), ((my_tiles - 1) / NSB) & 1);
       ok = __all_sync(kFullMask, ok);
     }
     if (ok && my_tiles > 0 && Tr::kPrefix) {
@@ -910,7 +974,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < 128; c += 16) {
         float v[16];
-        tc::tmem_ld16(lane_addr + 128 + c, v);
+        tc::tmem_ld16(lane_addr + Tr::O_COL + c, v);
         tc::tmem_wait_ld();
         if (active) {
           // E4M3: the V scale goes into o (m and l do not hold it)
@@ -929,7 +993,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < 128; c += 16) {
         float v[16];
-        tc::tmem_ld16(lane_addr + 128 + c, v);
+        tc::tmem_ld16(lane_addr + Tr::O_COL + c, v);
         tc::tmem_wait_ld();
         if (active) {
           float a[8], b[8];

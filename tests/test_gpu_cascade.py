@@ -41,7 +41,8 @@ CASES = [(3, 4, 37, 8, 2, 16, "bf16"), (2, 8, 64, 8, 1, 16, "fp16"), (4, 2, 100,
          (2, 3, 96, 16, 2, 32, "bf16"), (5, 1, 50, 2, 1, 16, "fp16"), (1, 16, 300, 8, 8, 16, "bf16")]
 
 
-@pytest.mark.parametrize("prompts,samples,plen,h,hkv,bs,dtype", CASES)
+@pytest.mark.parametrize("prompts,samples,plen,h,hkv,bs,dtype",
+                         CASES + [(1, 40, 70, 8, 2, 16, "bf16")])  # 40 x G 4: two 128-row tiles
 def test_cascade_matches_oracle(pk, prompts, samples, plen, h, hkv, bs, dtype):
     w = W.build_prefix_share_workload(prompts, samples, plen, 5, 40, h, hkv, 128, bs, dtype,
                                       seed=plen + samples, allocator=block_allocator)
@@ -59,7 +60,8 @@ def test_cascade_matches_oracle(pk, prompts, samples, plen, h, hkv, bs, dtype):
 # head_dim 64: the prefix pass is the mma.sync kernel in prefix mode; G = 1
 # reads each member's own blocks on the CUDA cores, G >= 2 on the tensor cores
 CASES_D64 = [(3, 4, 37, 8, 2, 16, "bf16"), (2, 8, 64, 4, 4, 32, "fp16"),
-             (4, 2, 100, 16, 2, 16, "fp16"), (1, 16, 300, 8, 8, 32, "bf16")]
+             (4, 2, 100, 16, 2, 16, "fp16"), (1, 16, 300, 8, 8, 32, "bf16"),
+             (2, 16, 64, 16, 2, 16, "fp16")]   # 16 members x G 8: two 64-row tiles
 
 
 @pytest.mark.parametrize("prompts,samples,plen,h,hkv,bs,dtype", CASES_D64)
@@ -80,7 +82,9 @@ def test_cascade_head_dim_64_matches_oracle(pk, prompts, samples, plen, h, hkv, 
 # E4M3 caches: (prompts, samples, prompt_len, heads, kv heads, head_dim, block, dtype)
 CASES_FP8 = [(3, 4, 37, 8, 2, 128, 16, "bf16"), (2, 8, 64, 8, 1, 128, 32, "fp16"),
              (4, 2, 100, 4, 4, 128, 16, "fp16"), (3, 4, 37, 8, 2, 64, 16, "bf16"),
-             (2, 8, 64, 4, 4, 64, 32, "fp16"), (1, 16, 300, 8, 8, 64, 16, "bf16")]
+             (2, 8, 64, 4, 4, 64, 32, "fp16"), (1, 16, 300, 8, 8, 64, 16, "bf16"),
+             (1, 40, 70, 8, 2, 128, 16, "bf16"),   # two 128-row tiles
+             (2, 16, 64, 16, 2, 64, 16, "fp16")]   # two 64-row tiles
 
 
 @pytest.mark.parametrize("prompts,samples,plen,h,hkv,d,bs,dtype", CASES_FP8)

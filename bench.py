@@ -472,12 +472,21 @@ def bench_decode(run, workload, headline):
     # cache write (+ block copy) + decode (+ reduce); cascade: prefix pass + suffix + reduce
     launches_per_step = (1 + (1 if has_pairs else 0) +
                          (3 if cascade else 1 + (1 if split else 0)))
-    # the sequences longest first (pkv_decode_order, on the host from the
-    # step's lengths): long sequences do not start last; cascade keeps its groups
-    h_order = None if cascade else pk.decode_order(w.context_lens).pin_memory()
-    order = None if cascade else h_order.to(dev)
+    # CTA schedule, computed on the host from the step's lengths so that long
+    # sequences do not start last: by default one CTA per partition that
+    # exists, longest first (pkv_decode_plan); or the full grid with the
+    # sequences longest first (pkv_decode_order).  Cascade keeps its groups.
+    planned = args.schedule == "plan" and not cascade
+    sched_key = None if cascade else "work" if planned else "order"
+
+    def schedule(h_lens):
+        return (pk.decode_plan(h_lens, w.block_size, part) if planned
+                else pk.decode_order(h_lens))
+    h_sched = None if cascade else schedule(w.context_lens).pin_memory()
     inputs = dict(q=q, key=key, val=val, slots=slots, pairs=pairs, tables=tables, lens=lens,
-                  out=out, order=order)
+                  out=out, order=None, work=None)
+    if sched_key is not None:
+        inputs[sched_key] = h_sched.to(dev)
 
     def decode(t=inputs):
         if cascade:
@@ -491,13 +500,16 @@ def bench_decode(run, workload, headline):
         elif fp8:
             pk.paged_attn_decode_fp8(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
                                      scales[0], scales[1], w.num_kv_heads, w.block_size,
-                                     w.max_context_len, partition_size=part_req, workspace=ws,
-                                     dev_err=err, stream=stream, seq_order=t["order"])
+                                     w.max_context_len,
+                                     partition_size=part if planned else part_req, workspace=ws,
+                                     dev_err=err, stream=stream, seq_order=t["order"],
+                                     work=t["work"])
         else:
             pk.paged_attn_decode(t["out"], t["q"], kc, vc, t["tables"], t["lens"], w.scale,
                                  w.num_kv_heads, w.block_size, w.max_context_len,
-                                 partition_size=part_req, workspace=ws, dev_err=err,
-                                 stream=stream, seq_order=t["order"])
+                                 partition_size=part if planned else part_req, workspace=ws,
+                                 dev_err=err, stream=stream, seq_order=t["order"],
+                                 work=t["work"])
 
     def step(i=0, t=inputs):
         if has_pairs:
@@ -571,6 +583,8 @@ def bench_decode(run, workload, headline):
                        if fp8 else w.dtype,
                        partition_used=part, split_k=split,
                        seq_order="index order (cascade groups)" if cascade else
+                       ("work list of the existing partitions, longest first in 256-token "
+                        "buckets (pkv_decode_plan on the host)") if planned else
                        "longest first in 256-token buckets (pkv_decode_order on the host)",
                        timing=TIMING_NOTE[bool(args.no_graph)],
                        l2=("no flush: %.2f GB of KV read per step, larger than the 126 MB L2"
@@ -613,10 +627,11 @@ def bench_decode(run, workload, headline):
     staging = torch.empty(pk.staging_bytes(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim,
                                            w.max_blocks_per_seq, len(w.slot_mapping),
                                            len(w.cow_pairs)), dtype=torch.uint8, device=dev)
-    # the per-step order (computed on the host from the step's lengths) is uploaded too
+    # the per-step order or work list (computed on the host from the step's
+    # lengths) is uploaded too
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_val, h_slots, h_pairs,
                                                      h_tables, h_lens)
-              + ((h_order,) if h_order is not None else ()))
+              + ((h_sched,) if h_sched is not None else ()))
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step(i=0):
@@ -630,8 +645,8 @@ def bench_decode(run, workload, headline):
             srcs = [(q, h_q), (key, h_key), (val, h_val), (slots, h_slots), (tables, h_tables),
                     (lens, h_lens)]
             if not cascade:
-                h_order.copy_(pk.decode_order(h_lens))
-                srcs.append((order, h_order))
+                h_sched.copy_(schedule(h_lens))
+                srcs.append((inputs[sched_key], h_sched))
             for dst, src in srcs:
                 dst.copy_(src, non_blocking=True)
             if has_pairs:
@@ -674,16 +689,18 @@ def bench_decode(run, workload, headline):
         ev_comp = [torch.cuda.Event() for _ in range(2)]
         ev_down = [torch.cuda.Event() for _ in range(2)]
         h_src = dict(q=h_q, key=h_key, val=h_val, slots=h_slots, pairs=h_pairs, tables=h_tables,
-                     lens=h_lens, order=h_order)
-        h_orders = [h_order, None if cascade else h_order.clone().pin_memory()]
+                     lens=h_lens)
+        if not cascade:
+            h_src[sched_key] = h_sched
+        h_scheds = [h_sched, None if cascade else h_sched.clone().pin_memory()]
 
         def e2e_pipelined(i):
             b, t = i % 2, bufs[i % 2]
             up.wait_event(ev_comp[b])          # step i-2 has finished reading buffer b
             if not cascade:
-                ev_up[b].synchronize()         # step i-2's upload has read h_orders[b]
-                h_orders[b].copy_(pk.decode_order(h_lens))
-                h_src["order"] = h_orders[b]
+                ev_up[b].synchronize()         # step i-2's upload has read h_scheds[b]
+                h_scheds[b].copy_(schedule(h_lens))
+                h_src[sched_key] = h_scheds[b]
             with torch.cuda.stream(up):
                 for k, src in h_src.items():
                     if (k != "pairs" or has_pairs) and src is not None:
@@ -1243,6 +1260,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the steps as direct launches instead of one captured CUDA graph")
+    ap.add_argument("--schedule", choices=("order", "plan"), default="plan",
+                    help="decode CTAs: sequences longest first over the full grid (order), "
+                         "or one CTA per existing partition from pkv_decode_plan (plan)")
     ap.add_argument("--partition", type=int, default=None,
                     help="partition size in tokens (0 = let the library choose)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -79,7 +79,8 @@ typedef enum { PKV_FP16 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
                                      blocks than max_blocks_per_seq                        */
 #define PKV_DEVERR_TIMEOUT 16u    /* decode: a bounded wait for an async copy gave up      */
 #define PKV_DEVERR_BAD_SCALE 32u  /* *_fp8: a scale that is not finite and > 0            */
-#define PKV_DEVERR_BAD_ORDER 64u  /* *_ordered: an order entry outside [0, num_seqs)       */
+#define PKV_DEVERR_BAD_ORDER 64u  /* *_ordered, *_planned: an entry outside [0, num_seqs),
+                                     or a work item that disagrees with its context length */
 
 /* Library version string, e.g. "pagedkv 0.1.0 sm_100a". */
 const char* pkv_version(void);
@@ -246,6 +247,56 @@ pkv_status pkv_paged_attn_decode_ordered(void* out, const void* q, const void* k
 pkv_status pkv_paged_attn_decode_fp8_ordered(
     void* out, const void* q, const void* k_cache, const void* v_cache,
     const int32_t* block_tables, const int32_t* context_lens, const int32_t* seq_order,
+    float scale, const float* k_scales, const float* v_scales, int num_seqs, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream);
+
+/*
+ * Planned decode.  A split-K decode grid holds max-context / partition CTAs
+ * for every (sequence, kv head), and those past a shorter sequence's end
+ * find no tokens and exit.  When the caller knows the context lengths on the
+ * host (the scheduler that owns the block tables does), pkv_decode_plan lists
+ * only the (sequence, partition) items that exist, and the planned decode
+ * launches one CTA per item and kv head.  Results are identical to
+ * pkv_paged_attn_decode with the same partition_size.  Not in the pages: a
+ * scheduling choice for B200.
+ *
+ * pkv_decode_plan (host only): context_lens is a host int32 [num_seqs];
+ * partition_size > 0 and a multiple of block_size (e.g. what
+ * pkv_paged_attn_partition_size or _fp8 returns for the batch).  Writes the
+ * item count, sum over sequences of max(1, ceil(ceil(len / block_size) /
+ * (partition_size / block_size))), into *num_items and, when work is not
+ * NULL, the items into work (host int32 [capacity][2]; capacity below the
+ * count is PKV_ERR_INVALID_ARG): item i is (sequence, partition | count << 16)
+ * where count is the sequence's partition count.  Items come longest first
+ * by their own token count, in buckets of 256 tokens, in (sequence,
+ * partition) order within a bucket.  A sequence of more than 65535
+ * partitions is PKV_ERR_UNSUPPORTED.  With work == NULL it only counts.
+ *
+ * pkv_paged_attn_decode_planned / pkv_paged_attn_decode_fp8_planned take the
+ * arguments of pkv_paged_attn_decode / _fp8 and the plan's items: work is the
+ * device copy (8-byte aligned) of pkv_decode_plan's output for these
+ * context lengths, num_items its count (at least num_seqs), partition_size
+ * the one it was planned with (0 is PKV_ERR_INVALID_ARG).  Workspace as for
+ * pkv_paged_attn_decode with that partition_size.  An item whose sequence is
+ * outside [0, num_seqs), or whose partition count disagrees with the
+ * sequence's context length on the device, sets PKV_DEVERR_BAD_ORDER (the
+ * sequence's output is then not to be trusted: a list planned from other
+ * lengths may lack partitions); a list that leaves a sequence out leaves its
+ * output unwritten.
+ */
+pkv_status pkv_decode_plan(const int32_t* context_lens, int num_seqs, int block_size,
+                           int partition_size, int32_t* work, int capacity, int* num_items);
+pkv_status pkv_paged_attn_decode_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* work, int num_items,
+    float scale, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err, void* stream);
+pkv_status pkv_paged_attn_decode_fp8_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* work, int num_items,
     float scale, const float* k_scales, const float* v_scales, int num_seqs, int num_heads,
     int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
     int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
@@ -484,10 +535,15 @@ pkv_status pkv_decode_step_host(
  *   create   staging: device scratch of >= pkv_decode_pipeline_staging_bytes
  *            bytes (16-byte aligned): two areas, used by alternate steps, each
  *            sized for max_new_tokens new tokens and max_pairs copy pairs.
- *            The pipeline creates its two copy streams and six events (no
- *            device memory) and keeps `stream` as its compute stream.
+ *            The pipeline creates its two copy streams, six events and a
+ *            pinned host buffer for two work lists (no device memory) and
+ *            keeps `stream` as its compute stream.
  *   step     enqueues one step and returns; the cache work of consecutive
- *            steps stays in order on the compute stream.  num_new_tokens and
+ *            steps stays in order on the compute stream.  The decode is
+ *            planned on the host from the step's context lengths
+ *            (pkv_decode_plan, with the partition pkv_paged_attn_partition_size
+ *            gives for partition_size) and its work list is uploaded with the
+ *            inputs.  num_new_tokens and
  *            num_pairs may vary per step up to the maxima.  The step's host
  *            buffers (pinned memory keeps the copies asynchronous) must stay
  *            valid and unchanged, and *out_host unread, until the step has

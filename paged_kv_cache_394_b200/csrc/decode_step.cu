@@ -22,10 +22,14 @@ namespace pkv {
 namespace step {
 
 struct StagingLayout {
-  size_t q, key, value, slots, pairs, tables, lens, order, out, total;
+  size_t q, key, value, slots, pairs, tables, lens, work, out, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t work_items(int num_seqs, int max_blocks_per_seq) {
+  return static_cast<size_t>(num_seqs) * max_blocks_per_seq;
+}
 
 StagingLayout staging_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                              int max_blocks_per_seq, int num_new_tokens, int num_pairs) {
@@ -45,7 +49,9 @@ StagingLayout staging_layout(int num_seqs, int num_heads, int num_kv_heads, int 
   l.pairs = take(static_cast<size_t>(num_pairs) * 16);
   l.tables = take(static_cast<size_t>(num_seqs) * max_blocks_per_seq * 4);
   l.lens = take(static_cast<size_t>(num_seqs) * 4);
-  l.order = take(static_cast<size_t>(num_seqs) * 4);   // pipeline: the sequence order
+  // pipeline: the step's work list (pkv_decode_plan), at most one item per
+  // block of each sequence (an empty sequence has one item and no block)
+  l.work = take(work_items(num_seqs, max_blocks_per_seq) * 8);
   l.out = take(qo);
   l.total = off;
   return l;
@@ -141,7 +147,7 @@ struct pkv_decode_pipeline {
   pkv_dtype dtype;
   unsigned char* staging[2];  // two areas of `layout.total` bytes
   pkv::step::StagingLayout layout;  // offsets inside one area, sized for the maxima
-  int32_t* order_host;        // pinned [2][num_seqs]: each area's sequence order
+  int32_t* work_host;         // pinned [2][work_items][2]: each area's work list
   cudaStream_t compute, up, down;
   cudaEvent_t ev_up[2], ev_comp[2], ev_down[2];
   long long steps;
@@ -166,7 +172,7 @@ void pipeline_release(pkv_decode_pipeline* pl) {
   }
   if (pl->up) cudaStreamDestroy(pl->up);
   if (pl->down) cudaStreamDestroy(pl->down);
-  if (pl->order_host) cudaFreeHost(pl->order_host);
+  if (pl->work_host) cudaFreeHost(pl->work_host);
 }
 }  // namespace step
 }  // namespace pkv
@@ -216,10 +222,11 @@ extern "C" pkv_status pkv_decode_pipeline_create(
   pl->layout = staging_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                               max_new_tokens, max_pairs);
   pl->compute = as_stream(stream);
-  // pinned host memory for the per-step order (no device memory is allocated)
-  pkv_status st = cuda_status(cudaHostAlloc(reinterpret_cast<void**>(&pl->order_host),
-                                            2 * static_cast<size_t>(std::max(num_seqs, 1)) * 4,
-                                            cudaHostAllocDefault));
+  // pinned host memory for the per-step work list (no device memory is allocated)
+  pkv_status st = cuda_status(cudaHostAlloc(
+      reinterpret_cast<void**>(&pl->work_host),
+      2 * std::max<size_t>(work_items(num_seqs, max_blocks_per_seq), 1) * 8,
+      cudaHostAllocDefault));
   if (st == PKV_OK) st = cuda_status(cudaStreamCreateWithFlags(&pl->up, cudaStreamNonBlocking));
   if (st == PKV_OK) st = cuda_status(cudaStreamCreateWithFlags(&pl->down, cudaStreamNonBlocking));
   for (int b = 0; b < 2 && st == PKV_OK; ++b) {
@@ -259,13 +266,20 @@ extern "C" pkv_status pkv_decode_pipeline_step(
   const int b = static_cast<int>(pl->steps & 1);
   unsigned char* st = pl->staging[b];
   const StagingLayout& l = pl->layout;
-  // the sequence order, longest first, computed on the host from this step's
-  // lengths into the area's pinned buffer once step i-2 has uploaded it
-  int32_t* order_host = pl->order_host + static_cast<size_t>(b) * std::max(S, 1);
+  // the work list (the partitions that exist, longest first), planned on the
+  // host from this step's lengths into the area's pinned buffer once step
+  // i-2 has uploaded it
+  if (max_context_len < 0 || partition_size < 0) return PKV_ERR_INVALID_ARG;
+  const size_t cap = std::max<size_t>(work_items(S, pl->max_blocks_per_seq), 1);
+  int32_t* work_host = pl->work_host + static_cast<size_t>(b) * cap * 2;
+  const int part =
+      pkv_paged_attn_partition_size(S, HKV, pl->block_size, max_context_len, partition_size);
+  int items = 0;
   pkv_status r = cuda_status(cudaEventSynchronize(pl->ev_up[b]));
   if (r != PKV_OK) return r;
   if (S > 0) {
-    r = pkv_decode_order(context_lens_host, S, order_host);
+    r = pkv_decode_plan(context_lens_host, S, pl->block_size, part, work_host,
+                        static_cast<int>(std::min<size_t>(cap, 0x7fffffff)), &items);
     if (r != PKV_OK) return r;
   }
   const size_t qo = static_cast<size_t>(S) * H * D * 2;
@@ -282,7 +296,7 @@ extern "C" pkv_status pkv_decode_pipeline_step(
       {l.pairs, block_mapping_host, static_cast<size_t>(num_pairs) * 16},
       {l.tables, block_tables_host, static_cast<size_t>(S) * pl->max_blocks_per_seq * 4},
       {l.lens, context_lens_host, static_cast<size_t>(S) * 4},
-      {l.order, order_host, static_cast<size_t>(S) * 4},
+      {l.work, work_host, static_cast<size_t>(items) * 8},
   };
   // upload: once step i-2 has finished reading this area's inputs
   r = cuda_status(cudaStreamWaitEvent(pl->up, pl->ev_comp[b], 0));
@@ -304,13 +318,13 @@ extern "C" pkv_status pkv_decode_pipeline_step(
                               reinterpret_cast<const int64_t*>(st + l.slots), num_new_tokens, HKV,
                               D, pl->block_size, num_blocks, pl->dtype, dev_err, cs);
   if (r == PKV_OK)
-    r = pkv_paged_attn_decode_ordered(st + l.out, st + l.q, k_cache, v_cache,
+    r = pkv_paged_attn_decode_planned(st + l.out, st + l.q, k_cache, v_cache,
                                       reinterpret_cast<const int32_t*>(st + l.tables),
                                       reinterpret_cast<const int32_t*>(st + l.lens),
-                                      reinterpret_cast<const int32_t*>(st + l.order), scale, S,
-                                      H, HKV, D, pl->block_size, pl->max_blocks_per_seq,
-                                      max_context_len, num_blocks, pl->dtype, partition_size,
-                                      workspace, workspace_bytes, dev_err, cs);
+                                      reinterpret_cast<const int32_t*>(st + l.work), items,
+                                      scale, S, H, HKV, D, pl->block_size,
+                                      pl->max_blocks_per_seq, max_context_len, num_blocks,
+                                      pl->dtype, part, workspace, workspace_bytes, dev_err, cs);
   if (r == PKV_OK) r = cuda_status(cudaEventRecord(pl->ev_comp[b], pl->compute));
   // download: once this step's output is written
   if (r == PKV_OK) r = cuda_status(cudaStreamWaitEvent(pl->down, pl->ev_comp[b], 0));

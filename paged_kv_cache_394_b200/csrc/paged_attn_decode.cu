@@ -322,6 +322,10 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int 
   return w;
 }
 
+// A work item packs its partition and its sequence's partition count into
+// 16 bits each.
+constexpr int kMaxPlannedParts = 0xffff;
+
 int parts_for(int max_context_len, int block_size, int partition) {
   const int nblk = (max_context_len + block_size - 1) / block_size;
   const int pb = partition / block_size;
@@ -373,7 +377,8 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
                          size_t workspace_bytes, unsigned* dev_err, void* stream, bool fp8,
                          const float* k_scales, const float* v_scales,
                          const CascadeGroups* cascade = nullptr,
-                         const int32_t* seq_order = nullptr, bool after_prefix = false) {
+                         const int32_t* seq_order = nullptr, bool after_prefix = false,
+                         const int32_t* work = nullptr, int num_work = 0) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0 || num_blocks <= 0 || partition_size < 0 || !dtype_valid(dtype) ||
       num_heads % num_kv_heads != 0 || !isfinite(scale))
@@ -392,6 +397,11 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
     return PKV_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
+  // a work list holds at least one item per sequence, for the partition size
+  // it was planned with
+  if (work != nullptr && (partition_size == 0 || num_work < num_seqs ||
+                          (reinterpret_cast<uintptr_t>(work) & 7u) != 0))
+    return PKV_ERR_INVALID_ARG;
 
   const int part = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
                                     partition_size,
@@ -407,7 +417,9 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
     if (workspace == nullptr || workspace_bytes < wl.total) return PKV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return PKV_ERR_INVALID_ARG;
   }
-  const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * grid_parts;
+  if (work != nullptr && grid_parts > kMaxPlannedParts) return PKV_ERR_UNSUPPORTED;
+  const long long grid = static_cast<long long>(work ? num_work : num_seqs) * num_kv_heads *
+                         (work ? 1 : grid_parts);
   if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
 
   // 16-bit: G >= 2 on the tensor cores, G = 1 on the CUDA cores;
@@ -461,6 +473,7 @@ pkv_status decode_launch(void* out, const void* q, const void* k_cache, const vo
   p.max_shared_blocks = cascade ? cascade->max_shared_blocks : 0;
   p.seq_order = cascade ? nullptr : seq_order;  // cascade groups stay together
   p.independent_of_prior = after_prefix ? 1 : 0;
+  p.work = reinterpret_cast<const int2*>(work);
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   p.withhold_first_load = g_withhold_first_load.load(std::memory_order_relaxed);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -586,6 +599,84 @@ extern "C" pkv_status pkv_decode_order(const int32_t* context_lens, int num_seqs
   for (int k = 1; k <= top + 1; ++k) start[k] += start[k - 1];
   for (int i = 0; i < num_seqs; ++i) order[start[top - bucket(i)]++] = i;
   return PKV_OK;
+}
+
+// Work list of (sequence, partition) items, longest first in buckets of
+// kOrderBucket tokens of the item's own length (index order within a
+// bucket): a counting sort, as for pkv_decode_order.
+extern "C" pkv_status pkv_decode_plan(const int32_t* context_lens, int num_seqs, int block_size,
+                                      int partition_size, int32_t* work, int capacity,
+                                      int* num_items) {
+  constexpr int kOrderBucket = 256;
+  if (num_seqs < 0 || block_size <= 0 || partition_size <= 0 ||
+      partition_size % block_size != 0 || capacity < 0 || num_items == nullptr ||
+      (num_seqs > 0 && context_lens == nullptr))
+    return PKV_ERR_INVALID_ARG;
+  const int pb = partition_size / block_size;
+  auto parts = [&](int i) {
+    const long long nblk = (std::max(context_lens[i], 0) + 0LL + block_size - 1) / block_size;
+    return std::max(1LL, (nblk + pb - 1) / pb);
+  };
+  long long n = 0;
+  for (int i = 0; i < num_seqs; ++i) {
+    const long long np = parts(i);
+    if (np > pkv::kMaxPlannedParts) return PKV_ERR_UNSUPPORTED;
+    n += np;
+  }
+  if (n > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+  *num_items = static_cast<int>(n);
+  if (work == nullptr) return PKV_OK;  // size query
+  if (capacity < n) return PKV_ERR_INVALID_ARG;
+  // tokens of item (i, j): the partition's share of the context
+  auto bucket = [&](int i, int j) {
+    const long long len = std::max(context_lens[i], 0);
+    const long long rest = len - static_cast<long long>(j) * partition_size;
+    return static_cast<int>(std::min<long long>(rest, partition_size) / kOrderBucket);
+  };
+  const int top = partition_size / kOrderBucket;
+  std::vector<long long> start(static_cast<size_t>(top) + 2, 0);
+  for (int i = 0; i < num_seqs; ++i)
+    for (int j = 0, np = static_cast<int>(parts(i)); j < np; ++j) ++start[top - bucket(i, j) + 1];
+  for (int k = 1; k <= top + 1; ++k) start[k] += start[k - 1];
+  for (int i = 0; i < num_seqs; ++i) {
+    const int np = static_cast<int>(parts(i));
+    for (int j = 0; j < np; ++j) {
+      const long long at = start[top - bucket(i, j)]++;
+      work[2 * at] = i;
+      work[2 * at + 1] = j | (np << 16);
+    }
+  }
+  return PKV_OK;
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* work, int num_items,
+    float scale, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int num_blocks, pkv_dtype dtype,
+    int partition_size, void* workspace, size_t workspace_bytes, unsigned* dev_err,
+    void* stream) {
+  if (num_seqs > 0 && work == nullptr) return PKV_ERR_INVALID_ARG;
+  return pkv::decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                            partition_size, workspace, workspace_bytes, dev_err, stream, false,
+                            nullptr, nullptr, nullptr, nullptr, false, work, num_items);
+}
+
+extern "C" pkv_status pkv_paged_attn_decode_fp8_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* work, int num_items,
+    float scale, const float* k_scales, const float* v_scales, int num_seqs, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int num_blocks, pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream) {
+  if (num_seqs > 0 && work == nullptr) return PKV_ERR_INVALID_ARG;
+  return pkv::decode_launch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len, num_blocks, dtype,
+                            partition_size, workspace, workspace_bytes, dev_err, stream, true,
+                            k_scales, v_scales, nullptr, nullptr, false, work, num_items);
 }
 
 // ---------------------------------------------------------------------------

@@ -89,9 +89,47 @@ struct DecodeParams {
   // cascade suffix after its prefix pass, whose CTAs all waited for the cache
   // writes before letting this grid start), so skip griddepcontrol.wait.
   int independent_of_prior;
+  // Optional work list (see pkv_decode_plan), else null: CTA b serves item
+  // b / num_kv_heads for kv head b % num_kv_heads, and item i is the pair
+  // (sequence, partition | partitions the planner counted for it << 16).
+  // The grid then holds no CTA for a partition past a sequence's end.
+  const int2* work;
 };
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+// The (sequence, kv head, partition) a decode CTA serves: from the grid
+// (sequence-major, in index order or the caller's order, partitions
+// innermost) or from the work list.  `planned` is the work list's partition
+// count for the sequence (0 without one); seq is not yet range-checked.
+struct DecodeCta {
+  int seq, kvh, part, planned;
+};
+__device__ __forceinline__ DecodeCta decode_cta(const DecodeParams& p) {
+  DecodeCta c;
+  if (p.work != nullptr) {
+    const int2 w = p.work[blockIdx.x / p.num_kv_heads];
+    c.kvh = blockIdx.x % p.num_kv_heads;
+    c.seq = w.x;
+    c.part = w.y & 0xffff;
+    c.planned = static_cast<int>(static_cast<unsigned>(w.y) >> 16);
+  } else {
+    const int unit = blockIdx.x / p.grid_parts;
+    c.part = blockIdx.x % p.grid_parts;
+    c.kvh = unit % p.num_kv_heads;
+    const int rank = unit / p.num_kv_heads;
+    c.seq = p.seq_order != nullptr ? p.seq_order[rank] : rank;
+    c.planned = 0;
+  }
+  return c;
+}
+
+// Whether a work item disagrees with the context length the kernel read: a
+// list built from other lengths may miss partitions, so the call reports it.
+__device__ __forceinline__ bool plan_mismatch(const DecodeParams& p, const DecodeCta& c,
+                                              int nparts) {
+  return p.work != nullptr && (c.planned != (nparts > 1 ? nparts : 1) || c.part >= c.planned);
+}
+
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
@@ -370,9 +408,6 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   float* pbuf_all = reinterpret_cast<float*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
   int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES + Tr::PBUF_BYTES);
 
-  const int part = blockIdx.x % p.grid_parts;
-  const int unit = blockIdx.x / p.grid_parts;
-  const int kvh = unit % p.num_kv_heads;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -380,9 +415,8 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   // write); wait for it before reading anything, then let the next one start.
   if (!p.independent_of_prior) grid_dependency_wait();
   trigger_dependents();
-  // the sequence this CTA serves: in index order, or in the caller's order
-  const int rank = unit / p.num_kv_heads;
-  const int seq = p.seq_order != nullptr ? p.seq_order[rank] : rank;
+  const DecodeCta cta = decode_cta(p);
+  const int seq = cta.seq, kvh = cta.kvh, part = cta.part;
   if (static_cast<unsigned>(seq) >= static_cast<unsigned>(p.num_seqs)) {
     if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
     return;
@@ -419,6 +453,7 @@ __global__ void __launch_bounds__(Tr::THREADS) paged_decode_kernel(const DecodeP
   const int start_blk =
       cascade_start_block(p, seq, nblk, threadIdx.x == 0 && part == 0 && kvh == 0);
   const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
+  if (threadIdx.x == 0 && plan_mismatch(p, cta, nparts)) set_err(p.err, PKV_DEVERR_BAD_ORDER);
   if (part >= (cascade ? nparts : max(nparts, 1))) return;
   const bool direct = !cascade && nparts <= 1;
   const int blk_begin = start_blk + part * p.part_blocks;
@@ -833,17 +868,13 @@ __global__ void __launch_bounds__(Tr::THREADS)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::RING_BYTES);
   int* tbl = reinterpret_cast<int*>(smem + Tr::RING_BYTES + Tr::BAR_BYTES);
 
-  const int part = blockIdx.x % p.grid_parts;
-  const int unit = blockIdx.x / p.grid_parts;
-  const int kvh = unit % p.num_kv_heads;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (!p.independent_of_prior) grid_dependency_wait();
   trigger_dependents();
-  // the sequence this CTA serves: in index order, or in the caller's order
-  const int rank = unit / p.num_kv_heads;
-  const int seq = p.seq_order != nullptr ? p.seq_order[rank] : rank;
+  const DecodeCta cta = decode_cta(p);
+  const int seq = cta.seq, kvh = cta.kvh, part = cta.part;
   if (static_cast<unsigned>(seq) >= static_cast<unsigned>(p.num_seqs)) {
     if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
     return;
@@ -860,6 +891,7 @@ __global__ void __launch_bounds__(Tr::THREADS)
       cascade_start_block(p, seq, nblk, threadIdx.x == 0 && part == 0 && kvh == 0);
   const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
   const bool cascade = p.group_start != nullptr;
+  if (threadIdx.x == 0 && plan_mismatch(p, cta, nparts)) set_err(p.err, PKV_DEVERR_BAD_ORDER);
   if (part >= (cascade ? nparts : max(nparts, 1))) return;
   const bool direct = !cascade && nparts <= 1;
   const int blk_begin = start_blk + part * p.part_blocks;

@@ -20,7 +20,8 @@ and copy them on write ([cortexgrid] FAQ on parallel sampling).
 3. on the GPU: ``copy_blocks`` for the pairs, ``reshape_and_cache`` for every
    new token (whole prompts of admitted requests, one token per running
    sequence), ``paged_attn_prefill`` for the admitted prompts and
-   ``paged_attn_decode`` for the running sequences;
+   ``paged_attn_decode`` for the running sequences (with a work list that
+   ``decode_plan`` makes from the host's context lengths);
 4. fork the samples of a request whose prompt was just prefilled, retire
    sequences that reached their output length, free their pages.
 
@@ -167,6 +168,9 @@ class ContinuousBatcher:
                                     dtype=torch.int32, device=self.device)
             ctx_list = alloc.context_lens(decoded)
             d_ctx = torch.tensor(ctx_list, dtype=torch.int32, device=self.device)
+            # one CTA per partition that exists, planned from the host's lengths
+            d_part = pk.partition_size(n_dec, self.hkv, self.bs, max(ctx_list))
+            d_work = pk.decode_plan(ctx_list, self.bs, d_part).to(self.device)
             d_q = self.values("q_decode", (n_dec, self.h, self.d))
             d_out = torch.empty_like(d_q)
         pair_t = torch.tensor(pairs, dtype=torch.int64, device=self.device) if pairs else None
@@ -185,7 +189,8 @@ class ContinuousBatcher:
             self.last_outputs["prefill"] = (ids, p_q, p_out, p_tables, p_ctx, p_qs)
         if decoded:
             pk.paged_attn_decode(d_out, d_q, self.k_cache, self.v_cache, d_tables, d_ctx,
-                                 self.scale, self.hkv, self.bs, max(ctx_list), dev_err=self.err)
+                                 self.scale, self.hkv, self.bs, max(ctx_list),
+                                 partition_size=d_part, dev_err=self.err, work=d_work)
             self.last_outputs["decode"] = (decoded, d_q, d_out, d_tables, d_ctx)
         if n_pre + n_dec:
             self.last_outputs["write"] = (key, val)

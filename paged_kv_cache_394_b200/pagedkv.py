@@ -79,6 +79,13 @@ _paged_attn_decode_ordered = _proto("pkv_paged_attn_decode_ordered", _i, _vp, _v
 _paged_attn_decode_fp8_ordered = _proto("pkv_paged_attn_decode_fp8_ordered", _i, _vp, _vp, _vp,
                                         _vp, _vp, _vp, _vp, _f, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                         _i, _i, _i, _i, _vp, _sz, _vp, _vp)
+_decode_plan = _proto("pkv_decode_plan", _i, _vp, _i, _i, _i, _vp, _i, _vp)
+_paged_attn_decode_planned = _proto("pkv_paged_attn_decode_planned", _i, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, _i, _f, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                    _sz, _vp, _vp)
+_paged_attn_decode_fp8_planned = _proto("pkv_paged_attn_decode_fp8_planned", _i, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _i, _i, _i, _i, _i,
+                                        _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
 _testing_decode_wait = _proto("pkv_testing_decode_wait", _i, ctypes.c_uint64, _i)
 _pipeline_staging_bytes = _proto("pkv_decode_pipeline_staging_bytes", _sz, _i, _i, _i, _i, _i, _i,
                                  _i)
@@ -229,12 +236,41 @@ def decode_order(context_lens):
     return order
 
 
+def decode_plan(context_lens, block_size, partition_size):
+    """Work list (int32 host tensor [items, 2]) of the (sequence, partition)
+    items a decode with this partition size has, longest first, for a host
+    tensor or array of context lengths; see pkv_decode_plan."""
+    lens = torch.as_tensor(context_lens, dtype=torch.int32).contiguous()
+    if lens.is_cuda:
+        raise ValueError("context_lens must be on the host")
+    n = ctypes.c_int(0)
+    _check(_decode_plan(_ptr(lens), lens.numel(), block_size, partition_size, None, 0,
+                        ctypes.byref(n)), "decode_plan")
+    work = torch.empty((n.value, 2), dtype=torch.int32)
+    _check(_decode_plan(_ptr(lens), lens.numel(), block_size, partition_size, _ptr(work),
+                        n.value, ctypes.byref(n)), "decode_plan")
+    return work
+
+
+def _work_arg(work, partition_size):
+    _dev(work, "work", torch.int32)
+    if work.dim() != 2 or work.shape[1] != 2 or not work.is_contiguous():
+        raise ValueError("work must be a contiguous [items, 2] list from decode_plan")
+    if partition_size <= 0:
+        raise ValueError("a planned decode takes the partition size it was planned with")
+    return work.shape[0]
+
+
 def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
                       block_size, max_context_len, partition_size=0, workspace=None,
-                      dev_err=None, stream=None, seq_order=None):
+                      dev_err=None, stream=None, seq_order=None, work=None):
     """Paged decode attention; writes out [S, H, D].  With ``seq_order`` (a
     device int32 permutation, e.g. decode_order's) the CTAs take the
-    sequences in that order.  See include/pagedkv.h."""
+    sequences in that order; with ``work`` (the device copy of decode_plan's
+    list for ``partition_size``) one CTA per item and kv head.  See
+    include/pagedkv.h."""
+    if work is not None and seq_order is not None:
+        raise ValueError("give seq_order or work, not both")
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     _dev(block_tables, "block_tables", torch.int32)
@@ -254,6 +290,16 @@ def paged_attn_decode(out, q, k_cache, v_cache, block_tables, context_lens, scal
             workspace.record_stream(stream)   # the temporary must outlive the launch
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if work is not None:
+        n = _work_arg(work, partition_size)
+        _check(_paged_attn_decode_planned(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(block_tables), _ptr(context_lens), _ptr(work), n,
+                                          float(scale), s, h, hkv, d, bs, block_tables.shape[1],
+                                          max_context_len, num_blocks, _dtype_code(q),
+                                          partition_size, ws_ptr, ws_bytes, _ptr(dev_err),
+                                          _stream(stream)),
+               "paged_attn_decode_planned")
+        return
     if seq_order is not None:
         _dev(seq_order, "seq_order", torch.int32)
         if seq_order.shape != (s,):
@@ -379,10 +425,12 @@ def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scales, 
 
 def paged_attn_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scales,
                           v_scales, num_kv_heads, block_size, max_context_len, partition_size=0,
-                          workspace=None, dev_err=None, stream=None, seq_order=None):
+                          workspace=None, dev_err=None, stream=None, seq_order=None, work=None):
     """Paged decode attention over E4M3 caches (values = code * scale of the
-    kv head); q and out are 16-bit.  ``seq_order`` as for paged_attn_decode.
-    See include/pagedkv.h."""
+    kv head); q and out are 16-bit.  ``seq_order`` and ``work`` as for
+    paged_attn_decode.  See include/pagedkv.h."""
+    if work is not None and seq_order is not None:
+        raise ValueError("give seq_order or work, not both")
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     _dev(block_tables, "block_tables", torch.int32)
@@ -405,6 +453,16 @@ def paged_attn_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, 
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     ks, vs = _scales_for(k_scales, v_scales, hkv, q.device, stream)
+    if work is not None:
+        n = _work_arg(work, partition_size)
+        _check(_paged_attn_decode_fp8_planned(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                              _ptr(block_tables), _ptr(context_lens), _ptr(work),
+                                              n, float(scale), _ptr(ks), _ptr(vs), s, h, hkv, d,
+                                              bs, block_tables.shape[1], max_context_len,
+                                              num_blocks, _dtype_code(q), partition_size, ws_ptr,
+                                              ws_bytes, _ptr(dev_err), _stream(stream)),
+               "paged_attn_decode_fp8_planned")
+        return
     if seq_order is not None:
         _dev(seq_order, "seq_order", torch.int32)
         if seq_order.shape != (s,):

@@ -269,3 +269,66 @@ def test_decode_order_is_longest_first_by_bucket(seed, n):
     assert sorted(order.tolist()) == list(range(n))
     expect = np.lexsort((np.arange(n), -(lens // 256)))
     assert np.array_equal(order, expect)
+
+
+@pytest.mark.parametrize("seed,n,bs,part", [(0, 0, 16, 256), (1, 1, 16, 512), (2, 64, 32, 2048),
+                                            (3, 257, 16, 1024), (4, 1000, 16, 4096),
+                                            (5, 50, 16, 16)])
+def test_decode_plan_lists_every_partition_longest_first(seed, n, bs, part):
+    """pkv_decode_plan: exactly the (sequence, partition) items that exist,
+    each once, with its sequence's partition count; descending in buckets
+    of 256 tokens of the item's own length, (sequence, partition) order
+    within a bucket (restated with a stable lexicographic sort)."""
+    import numpy as np
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, 9000, size=n).astype(np.int32)
+    lens[: n // 4] = 0                                          # empty sequences: one item
+    lens[n // 4: n // 2] = part * rng.integers(1, 4, size=n // 2 - n // 4)   # exact multiples
+    work = pk.decode_plan(lens, bs, part).numpy()
+    seqs, parts, counts, sizes = [], [], [], []
+    for i, L in enumerate(lens.tolist()):
+        nblk = -(-L // bs)
+        np_ = max(1, -(-nblk // (part // bs)))
+        for j in range(np_):
+            seqs.append(i); parts.append(j); counts.append(np_)
+            sizes.append(max(0, min(part, L - j * part)))
+    seqs, parts, counts, sizes = map(np.asarray, (seqs, parts, counts, sizes))
+    key = np.lexsort((parts, seqs, -(sizes // 256)))
+    assert work.shape == (len(seqs), 2)
+    assert np.array_equal(work[:, 0], seqs[key])
+    assert np.array_equal(work[:, 1] & 0xFFFF, parts[key])
+    assert np.array_equal(work[:, 1] >> 16, counts[key])
+
+
+def test_decode_plan_and_planned_decode_validate_on_the_host():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    null = None
+    good = ctypes.c_void_p(0x1000)
+    n = ctypes.c_int(-1)
+    lens = (ctypes.c_int32 * 3)(100, 5000, 0)
+    work = (ctypes.c_int32 * 8)()
+    assert pk._decode_plan(lens, 3, 16, 2048, null, 0, ctypes.byref(n)) == pk.OK and n.value == 5
+    assert pk._decode_plan(lens, 3, 16, 2048, work, 4, ctypes.byref(n)) == pk.ERR_INVALID_ARG
+    assert pk._decode_plan(lens, 3, 16, 2048, work, 4, null) == pk.ERR_INVALID_ARG
+    assert pk._decode_plan(lens, 3, 16, 24, work, 4, ctypes.byref(n)) == pk.ERR_INVALID_ARG
+    assert pk._decode_plan(lens, 3, 16, 0, work, 4, ctypes.byref(n)) == pk.ERR_INVALID_ARG
+    assert pk._decode_plan(null, 3, 16, 2048, work, 4, ctypes.byref(n)) == pk.ERR_INVALID_ARG
+    assert pk._decode_plan(null, 0, 16, 2048, null, 0, ctypes.byref(n)) == pk.OK and n.value == 0
+    long = (ctypes.c_int32 * 1)(16 * 65536)                    # 65536 partitions of one block
+    assert pk._decode_plan(long, 1, 16, 16, null, 0, ctypes.byref(n)) == pk.ERR_UNSUPPORTED
+
+    def dec(part, items=4, w=good, fp8=False):
+        if fp8:
+            return pk._paged_attn_decode_fp8_planned(good, good, good, good, good, good, w, items,
+                                                     0.125, good, good, 2, 8, 2, 128, 16, 256,
+                                                     4096, 512, 0, part, good, 1 << 30, null, null)
+        return pk._paged_attn_decode_planned(good, good, good, good, good, good, w, items, 0.125,
+                                             2, 8, 2, 128, 16, 256, 4096, 512, 0, part, good,
+                                             1 << 30, null, null)
+    for fp8 in (False, True):
+        assert dec(0, fp8=fp8) == pk.ERR_INVALID_ARG                 # no partition size
+        assert dec(2048, items=1, fp8=fp8) == pk.ERR_INVALID_ARG     # fewer items than sequences
+        assert dec(2048, w=null, fp8=fp8) == pk.ERR_INVALID_ARG
+        assert dec(2048, w=ctypes.c_void_p(0x1004), fp8=fp8) == pk.ERR_INVALID_ARG  # alignment
+        assert dec(24, fp8=fp8) == pk.ERR_INVALID_ARG                # not a multiple of 16

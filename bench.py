@@ -766,6 +766,17 @@ def bench_prefill(run, workload, headline):
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     max_q = int(np.diff(w.query_start).max())
     stream = torch.cuda.Stream(device=dev)
+    # the units of the longest histories cut into key pieces, planned on the
+    # host from the step's lengths (pkv_prefill_plan; head_dim 128)
+    planned = args.schedule == "plan" and w.head_dim == 128
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def make_plan(qs_host, lens_host):
+        return pk.prefill_plan(qs_host, lens_host, w.num_heads, w.num_kv_heads, w.head_dim, sms)
+    h_plan = make_plan(w.query_start, w.context_lens) if planned else None
+    plan = h_plan.to(dev) if planned else None
+    plan_ws = (torch.empty(max(16, h_plan.workspace_bytes), dtype=torch.uint8, device=dev)
+               if planned else None)
 
     def write(k, v, s):
         if fp8:
@@ -774,15 +785,15 @@ def bench_prefill(run, workload, headline):
         else:
             pk.reshape_and_cache(k, v, kc, vc, s, dev_err=err, stream=stream)
 
-    def attend(o=out, qq=q, t=tables, l_=lens, qs=qstart):
+    def attend(o=out, qq=q, t=tables, l_=lens, qs=qstart, pl=plan):
         if fp8:
             pk.paged_attn_prefill_fp8(o, qq, kc, vc, t, l_, qs, w.scale, scales[0], scales[1],
                                       w.num_kv_heads, w.block_size, w.max_context_len, max_q,
-                                      dev_err=err, stream=stream)
+                                      dev_err=err, stream=stream, plan=pl, workspace=plan_ws)
         else:
             pk.paged_attn_prefill(o, qq, kc, vc, t, l_, qs, w.scale, w.num_kv_heads,
                                   w.block_size, w.max_context_len, max_q, dev_err=err,
-                                  stream=stream)
+                                  stream=stream, plan=pl, workspace=plan_ws)
 
     def step(i=0):
         write(key, val, slots)
@@ -809,6 +820,10 @@ def bench_prefill(run, workload, headline):
                        kv_cache="e4m3, per-kv-head scales (all %g here)" % FP8_K_SCALE
                        if fp8 else w.dtype,
                        timing=TIMING_NOTE[bool(args.no_graph)],
+                       schedule=("planned (pkv_prefill_plan on the host, %d SMs): %d CTAs per kv "
+                                 "head, %d units cut into key pieces and merged"
+                                 % (sms, len(h_plan.work), len(h_plan.merges))) if planned else
+                                "one CTA per (sequence, query tile, kv head), longest first",
                        l2="no flush: each step rewrites the new tokens' K/V"),
         "tokens_per_s": round(run.world * int(w.query_start[-1]) / (ms_per_step * 1e-3), 1),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
@@ -824,9 +839,11 @@ def bench_prefill(run, workload, headline):
                                    "clocks": sus_clk},
                      "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same "
                                     "dense rate)" % peak_kind},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (2 + (1 if planned and len(h_plan.merges) else 0)) * args.steps,
         "clocks": clk,
     }
+    if planned and len(h_plan.merges):
+        line["roofline"]["kernel"] += " + paged_prefill_merge_kernel"
     if not headline or args.no_e2e:
         return line
 
@@ -840,12 +857,18 @@ def bench_prefill(run, workload, headline):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(key), torch.empty_like(val)
     ds, dt_, dl, dqs = (torch.empty_like(slots), torch.empty_like(tables), torch.empty_like(lens),
                         torch.empty_like(qstart))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, ht, hl, hqs))
+    # the plan (made on the host from the batch's lengths, which stay the same
+    # from step to step here) is uploaded with each step's inputs
+    h_pw = h_pm = None
+    if planned:
+        h_pw, h_pm = h_plan.work.pin_memory(), h_plan.merges.pin_memory()
+    extra_h = (h_pw, h_pm) if planned else ()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, ht, hl, hqs) + extra_h)
     d2h = hout.numel() * hout.element_size()
 
-    host_in = (hq, hk, hv, hs, ht, hl, hqs)
-    dev_in = [(dq, dk, dv, ds, dt_, dl, dqs),
-              tuple(torch.empty_like(t) for t in (dq, dk, dv, ds, dt_, dl, dqs))]
+    host_in = (hq, hk, hv, hs, ht, hl, hqs) + extra_h
+    dev0 = (dq, dk, dv, ds, dt_, dl, dqs) + tuple(t.to(dev) for t in extra_h)
+    dev_in = [dev0, tuple(torch.empty_like(t) for t in dev0)]
     douts = [out, torch.empty_like(out)]
     houts = [hout, torch.empty_like(hout).pin_memory()]
 
@@ -856,9 +879,10 @@ def bench_prefill(run, workload, headline):
                     h, non_blocking=True)
 
     def compute(bufs, o):
-        bq, bk, bv, bs, bt, bl, bqs = bufs
+        bq, bk, bv, bs, bt, bl, bqs = bufs[:7]
+        pl = pk.PrefillPlan(bufs[7], bufs[8], h_plan.workspace_bytes) if planned else None
         write(bk, bv, bs)
-        attend(o, bq, bt, bl, bqs)
+        attend(o, bq, bt, bl, bqs, pl)
 
     def e2e_step(i=0):  # serial: copies in, compute, copy out, all on one stream
         upload(dev_in[0], stream)

@@ -80,7 +80,7 @@ typedef enum { PKV_FP16 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
 #define PKV_DEVERR_TIMEOUT 16u    /* decode: a bounded wait for an async copy gave up      */
 #define PKV_DEVERR_BAD_SCALE 32u  /* *_fp8: a scale that is not finite and > 0            */
 #define PKV_DEVERR_BAD_ORDER 64u  /* *_ordered, *_planned: an entry outside [0, num_seqs),
-                                     or a work item that disagrees with its context length */
+                                     or a work item that disagrees with the lengths */
 
 /* Library version string, e.g. "pagedkv 0.1.0 sm_100a". */
 const char* pkv_version(void);
@@ -473,6 +473,61 @@ pkv_status pkv_paged_attn_prefill_fp8(void* out, const void* q, const void* k_ca
                                       int max_blocks_per_seq, int max_context_len,
                                       int max_query_len, int num_blocks, pkv_dtype dtype,
                                       unsigned* dev_err, void* stream);
+
+/*
+ * Planned prefill (head_dim 128).  The tcgen05 prefill gives each (sequence,
+ * query tile of 256 rows) unit one CTA per kv head, which reads every key its
+ * rows see; in a batch of few sequences of very different histories the
+ * units of the longest one outlast the rest and the launch ends on them.
+ * pkv_prefill_plan (host only) cuts each unit whose CTA would cost more than
+ * 1.5 SM shares of the batch into up to 4 pieces of about one share: whole
+ * 64-key tiles of history, which every row of the unit sees, then the rest
+ * of its keys with the causal edge.  The planned prefill runs one CTA per
+ * item (a whole unit or a piece, most expensive first); the pieces of a
+ * unit write partials (m, l,
+ * unnormalised o in fp32) to the workspace and a merge kernel combines them
+ * as the split-K decode reduce does.  The result is that of
+ * pkv_paged_attn_prefill up to the rounding of that merge.  Not in the
+ * pages: a scheduling choice for B200.
+ *
+ * pkv_prefill_plan: query_start (host int32 [num_seqs + 1]) and context_lens
+ * (host int32 [num_seqs]) as the prefill will see them; num_sms the SMs the
+ * launch spreads over (148 on B200; <= 0 is PKV_ERR_INVALID_ARG).  Writes
+ * the item count to *num_items, the merge-entry count to *num_merges and,
+ * if workspace_bytes is not NULL, the workspace the planned prefill needs.
+ * work (host int32 [work_capacity][8]) and merges (host int32
+ * [merge_capacity][4]) may be NULL to count only; a capacity below the count
+ * is PKV_ERR_INVALID_ARG.  head_dim other than 128 is PKV_ERR_UNSUPPORTED.
+ *
+ * pkv_paged_attn_prefill_planned / pkv_paged_attn_prefill_fp8_planned take
+ * the arguments of pkv_paged_attn_prefill / _fp8, the device copies of the
+ * plan's work (num_items items) and merges (num_merges entries), and a
+ * workspace (16-byte aligned) of at least the plan's size (needed only when
+ * num_merges > 0, else PKV_ERR_WORKSPACE).  An item or merge entry that
+ * names no sequence, or whose key range does not fit the sequence's lengths
+ * on the device, sets PKV_DEVERR_BAD_ORDER and that unit's rows are not to
+ * be trusted; a plan that leaves a unit out leaves its rows unwritten.
+ */
+pkv_status pkv_prefill_plan(const int32_t* query_start, const int32_t* context_lens,
+                            int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                            int num_sms, int32_t* work, int work_capacity, int* num_items,
+                            int32_t* merges, int merge_capacity, int* num_merges,
+                            size_t* workspace_bytes);
+pkv_status pkv_paged_attn_prefill_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+    const int32_t* work, int num_items, const int32_t* merges, int num_merges, float scale,
+    int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int max_query_len, int num_blocks,
+    pkv_dtype dtype, void* workspace, size_t workspace_bytes, unsigned* dev_err, void* stream);
+pkv_status pkv_paged_attn_prefill_fp8_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+    const int32_t* work, int num_items, const int32_t* merges, int num_merges, float scale,
+    const float* k_scales, const float* v_scales, int num_seqs, int num_tokens, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int max_query_len, int num_blocks, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream);
 
 /*
  * pkv_paged_attn_decode_cascade_fp8 — pkv_paged_attn_decode_cascade over E4M3

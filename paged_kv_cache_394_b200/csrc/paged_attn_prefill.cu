@@ -4,9 +4,10 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <algorithm>
 #include <mutex>
-
 #include <type_traits>
+#include <vector>
 
 #include "host_common.h"
 #include "paged_prefill_kernels.cuh"
@@ -143,6 +144,36 @@ pkv_status q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num
 namespace pkv {
 namespace {
 
+// Planned prefill: the work items and merge entries of pkv_prefill_plan on
+// the device, and the workspace for the pieces' partials.
+struct PrefillPlanArgs {
+  const int32_t* work;
+  int num_items;
+  const int32_t* merges;
+  int num_merges;
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+// Rows of a planned unit: the tcgen05 kernel's query rows per CTA.
+constexpr int kPlanRows = PKV_PREFILL_QUERY_TILES * 128;
+
+struct PlanWorkspace {
+  size_t out_off, max_off, sum_off, total;
+};
+
+// [num_merges][H_kv][kPlanRows][kMaxPieces] partial rows: o (128 floats), m, l
+PlanWorkspace plan_workspace(int num_merges, int num_kv_heads) {
+  const size_t n = static_cast<size_t>(num_merges) * num_kv_heads * kPlanRows * kMaxPieces;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  PlanWorkspace w;
+  w.out_off = 0;
+  w.max_off = up(n * 128 * sizeof(float));
+  w.sum_off = w.max_off + up(n * sizeof(float));
+  w.total = w.sum_off + up(n * sizeof(float));
+  return w;
+}
+
 // Validates and launches prefill; fp8: the caches hold E4M3 codes with
 // per-kv-head scales k_scales / v_scales.
 pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -151,7 +182,8 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
                           int num_heads, int num_kv_heads, int head_dim, int block_size,
                           int max_blocks_per_seq, int max_context_len, int max_query_len,
                           int num_blocks, pkv_dtype dtype, bool fp8, const float* k_scales,
-                          const float* v_scales, unsigned* dev_err, void* stream) {
+                          const float* v_scales, unsigned* dev_err, void* stream,
+                          const PrefillPlanArgs* plan = nullptr) {
   if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
       max_blocks_per_seq <= 0 ||
       max_context_len < 0 || max_query_len < 0 || num_blocks <= 0 || !dtype_valid(dtype) ||
@@ -171,6 +203,20 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
   const bool use_tc = head_dim == 128;
+  if (plan != nullptr) {
+    // the plan's units are the tcgen05 kernel's (head_dim 128); its pieces
+    // write partials into the workspace that the merge kernel combines
+    if (!use_tc) return PKV_ERR_UNSUPPORTED;
+    if (plan->work == nullptr || plan->num_items < 0 || plan->num_merges < 0 ||
+        (plan->num_merges > 0 && plan->merges == nullptr))
+      return PKV_ERR_INVALID_ARG;
+    if (plan->num_merges > 0) {
+      const PlanWorkspace pw = plan_workspace(plan->num_merges, num_kv_heads);
+      if (plan->workspace == nullptr || plan->workspace_bytes < pw.total)
+        return PKV_ERR_WORKSPACE;
+      if (!aligned16(plan->workspace)) return PKV_ERR_INVALID_ARG;
+    }
+  }
   const PrefillEntry pe =
       use_tc ? PrefillEntry{nullptr, 0, 0, 0}
       : fp8  ? (dtype == PKV_FP16 ? prefill_for<Fp16, true>(head_dim, block_size, group)
@@ -186,8 +232,15 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
   const int tile_rows = use_tc ? te.rows : pe.rows;
   const long long rows = static_cast<long long>(max_query_len) * group;
   const int q_tiles = static_cast<int>((rows + tile_rows - 1) / tile_rows);
-  const long long grid = static_cast<long long>(num_seqs) * num_kv_heads * q_tiles;
-  if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+  const long long grid =
+      static_cast<long long>(plan ? plan->num_items : num_seqs * static_cast<long long>(q_tiles)) *
+      num_kv_heads;
+  if (grid > 0x7fffffffLL ||
+      (plan && static_cast<long long>(plan->num_merges) * num_kv_heads * (kPlanRows / 8) >
+                   0x7fffffffLL))
+    return PKV_ERR_UNSUPPORTED;
+  if (plan && tile_rows != kPlanRows) return PKV_ERR_UNSUPPORTED;
+  if (grid == 0) return PKV_OK;
 
   CUtensorMap kmap, vmap, qmap;
   const pkv_dtype cdt = fp8 ? PKV_FP8_E4M3 : dtype;  // element type of the caches
@@ -227,6 +280,19 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
   p.err = dev_err;
   p.k_scales = k_scales;
   p.v_scales = v_scales;
+  if (plan != nullptr) {
+    p.work = plan->work;
+    p.merges = plan->merges;
+    p.num_merges = plan->num_merges;
+    p.unit_rows = kPlanRows;
+    if (plan->num_merges > 0) {
+      const PlanWorkspace pw = plan_workspace(plan->num_merges, num_kv_heads);
+      unsigned char* ws = static_cast<unsigned char*>(plan->workspace);
+      p.ws_out = reinterpret_cast<float*>(ws + pw.out_off);
+      p.ws_max = reinterpret_cast<float*>(ws + pw.max_off);
+      p.ws_sum = reinterpret_cast<float*>(ws + pw.sum_off);
+    }
+  }
 
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -238,8 +304,16 @@ pkv_status prefill_launch(void* out, const void* q, const void* k_cache, const v
   cfg.stream = as_stream(stream);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (use_tc) return cuda_status(cudaLaunchKernelEx(&cfg, te.fn, p, qmap, kmap, vmap));
-  return cuda_status(cudaLaunchKernelEx(&cfg, pe.fn, p, kmap, vmap));
+  if (!use_tc) return cuda_status(cudaLaunchKernelEx(&cfg, pe.fn, p, kmap, vmap));
+  st = cuda_status(cudaLaunchKernelEx(&cfg, te.fn, p, qmap, kmap, vmap));
+  if (st != PKV_OK || plan == nullptr || plan->num_merges == 0) return st;
+  cudaLaunchConfig_t mcfg = cfg;
+  mcfg.gridDim = dim3(static_cast<unsigned>(plan->num_merges * num_kv_heads * (kPlanRows / 8)));
+  mcfg.blockDim = dim3(256);
+  mcfg.dynamicSmemBytes = 0;
+  return cuda_status(dtype == PKV_FP16
+                         ? cudaLaunchKernelEx(&mcfg, paged_prefill_merge_kernel<Fp16>, p)
+                         : cudaLaunchKernelEx(&mcfg, paged_prefill_merge_kernel<Bf16>, p));
 }
 
 }  // namespace
@@ -268,4 +342,175 @@ extern "C" pkv_status pkv_paged_attn_prefill_fp8(
                              scale, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
                              block_size, max_blocks_per_seq, max_context_len, max_query_len,
                              num_blocks, dtype, true, k_scales, v_scales, dev_err, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Planned prefill.  A (sequence, query tile) unit of the tcgen05 kernel reads
+// every key its rows see; in a batch of few sequences the units of the
+// longest history outlast the rest and the launch ends on them.  The planner
+// cuts such units' keys into pieces (history tiles that every row sees, then
+// the rest with the causal edge), one CTA each, and a merge kernel combines
+// the pieces' partials as split-K decode does.  Not in the pages: a
+// scheduling choice for B200.
+// ---------------------------------------------------------------------------
+namespace pkv {
+namespace {
+
+// Per-CTA fixed cost (Q load, pipeline fill, epilogue) in query-tile x
+// 64-key tiles, the unit of the cost model.
+constexpr int kPlanCtaOverhead = 4;
+// A unit is cut only when its CTA would cost more than this many SM shares
+// of the batch.  Measured on B200 (kernel TFLOP/s, whole launch, unit cut at
+// 1x the share -> uncut): the LLaMA-7B prefill batch (longest unit 1.1x its
+// share) 572 -> 661, the GQA batch (1.3x) 570 -> 650; where the longest
+// units are 2-5x their share, cutting them paid (uncut -> cut): one sequence
+// of 256 new tokens on 4000 cached 216 -> 430, histories of 8192, 100, 50
+// and 0 tokens (2.0x) 510 -> 750.
+constexpr double kPlanCutShares = 1.5;
+
+struct PlanUnit {
+  int seq, tile, nq, cost, hist_tiles;
+};
+
+struct PlanPiece {
+  int seq, tile, kb, ke, piece, merge, pieces, cost;
+};
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_prefill_plan(const int32_t* query_start, const int32_t* context_lens,
+                                       int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int num_sms, int32_t* work,
+                                       int work_capacity, int* num_items, int32_t* merges,
+                                       int merge_capacity, int* num_merges,
+                                       size_t* workspace_bytes) {
+  using namespace pkv;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      num_sms <= 0 || work_capacity < 0 || merge_capacity < 0 || num_items == nullptr ||
+      num_merges == nullptr || (num_seqs > 0 && (query_start == nullptr || context_lens == nullptr)))
+    return PKV_ERR_INVALID_ARG;
+  if (head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  const int group = num_heads / num_kv_heads;
+  constexpr int NKEY = 64, M = 128, QT = kPlanRows / M;
+  // ---- units and their cost: key tiles summed over the unit's query tiles
+  std::vector<PlanUnit> units;
+  long long total = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const long long ql = static_cast<long long>(query_start[s + 1]) - query_start[s];
+    if (ql <= 0) continue;
+    const long long hist = std::max<long long>(0, static_cast<long long>(context_lens[s]) - ql);
+    const long long rows = ql * group;
+    for (long long t = 0; t * kPlanRows < rows; ++t) {
+      long long cost = 0;
+      int nq = 0;
+      for (int q = 0; q < QT; ++q) {
+        const long long r0 = t * kPlanRows + q * M;
+        if (r0 >= rows) break;
+        const long long last = (std::min(rows, r0 + M) - 1) / group;
+        cost += (hist + last + 1 + NKEY - 1) / NKEY;
+        ++nq;
+      }
+      if (cost > 0x3fffffff || t > 0x7fffffff) return PKV_ERR_UNSUPPORTED;
+      units.push_back(PlanUnit{s, static_cast<int>(t), nq, static_cast<int>(cost),
+                               static_cast<int>(std::min<long long>(hist / NKEY, 0x3fffffff))});
+      total += (cost + kPlanCtaOverhead) * num_kv_heads;
+    }
+  }
+  // ---- cut every unit whose CTA would cost more than kPlanCutShares SM
+  // shares of the batch into pieces of about one share (at most kMaxPieces,
+  // each history piece at least one key tile)
+  const double share = static_cast<double>(total) / num_sms;
+  std::vector<PlanPiece> pieces;
+  int n_merge = 0;
+  for (const PlanUnit& u : units) {
+    const double c = u.cost + kPlanCtaOverhead;
+    int n = 1;
+    if (c > kPlanCutShares * share)
+      n = std::min<int>(kMaxPieces, static_cast<int>(std::ceil(c / share)));
+    // history tiles for the first n - 1 pieces: balance them with the last
+    long long k = 0;
+    if (n > 1) {
+      k = std::min<long long>(u.hist_tiles,
+                              static_cast<long long>(static_cast<double>(u.cost) * (n - 1) /
+                                                     (static_cast<double>(n) * u.nq)));
+      if (k < n - 1) n = static_cast<int>(k) + 1;
+      if (n > 1) k = std::min<long long>(k, u.hist_tiles);
+    }
+    if (n <= 1) {
+      pieces.push_back(PlanPiece{u.seq, u.tile, 0, -1, 0, 0, 1, u.cost + kPlanCtaOverhead});
+      continue;
+    }
+    const int merge = n_merge++;
+    long long kb = 0;
+    for (int i = 0; i < n - 1; ++i) {
+      const long long tiles = k / (n - 1) + (i < k % (n - 1) ? 1 : 0);
+      pieces.push_back(PlanPiece{u.seq, u.tile, static_cast<int>(kb * NKEY),
+                                 static_cast<int>((kb + tiles) * NKEY), i, merge, n,
+                                 static_cast<int>(tiles * u.nq + kPlanCtaOverhead)});
+      kb += tiles;
+    }
+    pieces.push_back(PlanPiece{u.seq, u.tile, static_cast<int>(kb * NKEY), -1, n - 1, merge, n,
+                               static_cast<int>(u.cost - kb * u.nq + kPlanCtaOverhead)});
+  }
+  if (pieces.size() > 0x7fffffffULL) return PKV_ERR_UNSUPPORTED;
+  // ---- longest first; ties in (sequence, tile, piece) order
+  std::stable_sort(pieces.begin(), pieces.end(),
+                   [](const PlanPiece& a, const PlanPiece& b) { return a.cost > b.cost; });
+  *num_items = static_cast<int>(pieces.size());
+  *num_merges = n_merge;
+  if (workspace_bytes != nullptr)
+    *workspace_bytes = n_merge > 0 ? plan_workspace(n_merge, num_kv_heads).total : 0;
+  if (work != nullptr) {
+    if (work_capacity < static_cast<long long>(pieces.size())) return PKV_ERR_INVALID_ARG;
+    for (size_t i = 0; i < pieces.size(); ++i) {
+      const PlanPiece& q = pieces[i];
+      int32_t* it = work + i * kPlanItemInts;
+      const int32_t v[kPlanItemInts] = {q.seq, q.tile, q.kb, q.ke, q.piece, q.merge, q.pieces, 0};
+      std::copy(v, v + kPlanItemInts, it);
+    }
+  }
+  if (merges != nullptr) {
+    if (merge_capacity < n_merge) return PKV_ERR_INVALID_ARG;
+    for (const PlanPiece& q : pieces)
+      if (q.pieces > 1 && q.piece == 0) {
+        int32_t* m = merges + 4 * static_cast<size_t>(q.merge);
+        m[0] = q.seq;
+        m[1] = q.tile;
+        m[2] = q.pieces;
+        m[3] = 0;
+      }
+  }
+  return PKV_OK;
+}
+
+extern "C" pkv_status pkv_paged_attn_prefill_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+    const int32_t* work, int num_items, const int32_t* merges, int num_merges, float scale,
+    int num_seqs, int num_tokens, int num_heads, int num_kv_heads, int head_dim, int block_size,
+    int max_blocks_per_seq, int max_context_len, int max_query_len, int num_blocks,
+    pkv_dtype dtype, void* workspace, size_t workspace_bytes, unsigned* dev_err, void* stream) {
+  const pkv::PrefillPlanArgs plan{work, num_items, merges, num_merges, workspace,
+                                  workspace_bytes};
+  return pkv::prefill_launch(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                             scale, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, max_context_len, max_query_len,
+                             num_blocks, dtype, false, nullptr, nullptr, dev_err, stream, &plan);
+}
+
+extern "C" pkv_status pkv_paged_attn_prefill_fp8_planned(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+    const int32_t* work, int num_items, const int32_t* merges, int num_merges, float scale,
+    const float* k_scales, const float* v_scales, int num_seqs, int num_tokens, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int max_context_len,
+    int max_query_len, int num_blocks, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+    unsigned* dev_err, void* stream) {
+  const pkv::PrefillPlanArgs plan{work, num_items, merges, num_merges, workspace,
+                                  workspace_bytes};
+  return pkv::prefill_launch(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                             scale, num_seqs, num_tokens, num_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, max_context_len, max_query_len,
+                             num_blocks, dtype, true, k_scales, v_scales, dev_err, stream, &plan);
 }

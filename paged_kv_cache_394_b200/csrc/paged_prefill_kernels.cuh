@@ -62,7 +62,24 @@ struct PrefillParams {
   float* ws_max;                 // [S, H, max_parts]
   float* ws_sum;                 // [S, H, max_parts]
   int max_parts;
+  // Planned prefill (tcgen05 kernel, else null): CTA b serves work item
+  // b / num_kv_heads for kv head b % num_kv_heads.  An item is kPlanItemInts
+  // ints {sequence, query tile, first key, end key (-1: the tile's causal
+  // end), piece, merge, pieces, 0}: a (sequence, query tile) unit whole
+  // (pieces = 1), or one of the pieces its keys are cut into, whose partials
+  // (m, l, unnormalised o) go to the workspace rows of merge entry `merge`
+  // (ws_out / ws_max / ws_sum as [num_merges][H_kv][ROWS][kMaxPieces] (x D))
+  // for the merge kernel.
+  const int32_t* work;
+  int num_merges;
+  // the merge entries {sequence, query tile, pieces, 0} and the query rows
+  // of a unit (the tcgen05 kernel's rows per CTA)
+  const int32_t* merges;
+  int unit_rows;
 };
+
+constexpr int kPlanItemInts = 8;
+constexpr int kMaxPieces = 4;
 
 // Two E4M3 codes (the low 16 bits of `two`, low byte first) -> two values
 // packed as fp16x2 or bf16x2; exact, since every E4M3 value is an fp16 and a

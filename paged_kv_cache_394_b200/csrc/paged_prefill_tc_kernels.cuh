@@ -328,8 +328,24 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
   const int rank = static_cast<int>(blockIdx.x / p.num_kv_heads);
   int seq = rank / p.q_tiles;
   int tile = p.q_tiles - 1 - rank % p.q_tiles;
+  // a planned item: keys [kb, ke) of the unit (ke = -1: to its causal end),
+  // piece `piece` of `pieces`, partials to merge entry `merge`
+  int kb = 0, ke = -1, piece = 0, pieces = 1, merge = 0;
   if constexpr (!Tr::kPrefix) {
-    if (p.num_seqs * p.q_tiles <= Tr::kSortUnits) {
+    if (p.work != nullptr) {
+      const int32_t* it = p.work + static_cast<size_t>(rank) * kPlanItemInts;
+      seq = it[0];
+      tile = it[1];
+      kb = it[2];
+      ke = it[3];
+      piece = it[4];
+      merge = it[5];
+      pieces = it[6];
+      if (static_cast<unsigned>(seq) >= static_cast<unsigned>(p.num_seqs)) {
+        if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
+        return;
+      }
+    } else if (p.num_seqs * p.q_tiles <= Tr::kSortUnits) {
       int* keys_of = reinterpret_cast<int*>(smem + Tr::OFF_KV);  // [num_seqs] first key, tiles
       int* chosen = keys_of + 2 * p.num_seqs;
       const int cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
@@ -392,6 +408,22 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     return;
   }
   const int rows_total = q_len * G;
+  if (p.work != nullptr) {
+    // a piece before the last covers whole tiles of history keys, which every
+    // row sees; the last starts within the history and runs to the causal end
+    const int hist = ctx - q_len;
+    const bool last = piece == pieces - 1;
+    const bool bad =
+        tile < 0 || tile * ROWS >= rows_total || pieces < 1 || pieces > kMaxPieces ||
+        piece < 0 || piece >= pieces || kb < 0 || kb % NKEY != 0 ||
+        (pieces > 1 && static_cast<unsigned>(merge) >= static_cast<unsigned>(p.num_merges)) ||
+        (last ? (ke != -1 || kb > hist || (pieces == 1 && kb != 0))
+              : (ke % NKEY != 0 || ke <= kb || ke > hist));
+    if (bad) {
+      if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
+      return;
+    }
+  }
   if (tile * ROWS >= rows_total || (Tr::kPrefix && ctx == 0)) return;
   const int tok0 = tile * (ROWS / G);  // first query token of this CTA
   // KV tiles each query tile needs (later rows see more keys; 0 = no rows)
@@ -401,11 +433,16 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const int r0 = tile * ROWS + q * M;
     const int last = (min(rows_total, r0 + M) - 1) / G;
     const int keys = Tr::kPrefix ? ctx : ctx - q_len + last + 1;
-    ntq[q] = r0 < rows_total ? (keys + NKEY - 1) / NKEY : 0;
+    const int kq = ke >= 0 ? min(keys, ke) : keys;
+    ntq[q] = r0 < rows_total ? (kq - kb + NKEY - 1) / NKEY : 0;
   }
   const int last_tok = (min(rows_total, (tile + 1) * ROWS) - 1) / G;
-  const int nkv = Tr::kPrefix ? ctx : ctx - q_len + last_tok + 1;  // keys the CTA reads
-  const int ntiles = (nkv + NKEY - 1) / NKEY;
+  const int nkv_all = Tr::kPrefix ? ctx : ctx - q_len + last_tok + 1;
+  const int nkv = ke >= 0 ? min(nkv_all, ke) : nkv_all;  // end of the keys the CTA reads
+  const int ntiles = (nkv - kb + NKEY - 1) / NKEY;
+  // From here on key indices count from kb (a whole number of blocks): the
+  // table row starts at block kb / BS, and positions and ends are shifted.
+  const int nkv_r = nkv - kb;
 
   if (threadIdx.x == 0) {
     // one arrival each (an expect_tx arrive or a tcgen05.commit), except p_full:
@@ -451,8 +488,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const bool is_k = warp == 0 || warp == Tr::PV_WARP + 1;
     // prefix mode: the group's first member holds the shared blocks' ids
     const int32_t* trow = p.block_tables +
-                          static_cast<size_t>(Tr::kPrefix ? q0 : seq) * p.max_blocks_per_seq;
-    const int nblk = (nkv + BS - 1) / BS;
+                          static_cast<size_t>(Tr::kPrefix ? q0 : seq) * p.max_blocks_per_seq +
+                          kb / BS;
+    const int nblk = (nkv_r + BS - 1) / BS;
     if (warp == 0 && lane == 0) {
       mbar_arrive_expect_tx(bar_q, QT * Tr::Q_TILE);
 #pragma unroll
@@ -473,7 +511,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       for (int i = 0; i < PIECES; ++i) {
         const int key0 = t * NKEY + i * 16;
         pb[i] = -1;
-        if (key0 < nkv) {
+        if (key0 < nkv_r) {
           const int blk = key0 / BS;
           if ((blk >> 5) != chunk) {
             chunk = blk >> 5;
@@ -610,7 +648,7 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
         for (int i = 0; i < PIECES; ++i) {
           const int key0 = t * NKEY + i * 16;
           pb[i] = -1;
-          if (key0 < nkv) {
+          if (key0 < nkv_r) {
             const int blk = key0 / BS;
             if ((blk >> 5) != chunk) {
               chunk = blk >> 5;
@@ -753,7 +791,9 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     const bool active = crow < rows_total - tile * ROWS;
     const int j = tok0 + crow / G;
     const int g = crow % G;
-    const int pos = !active ? -1 : Tr::kPrefix ? ctx - 1 : ctx - q_len + j;
+    // the last key the row sees, counted from kb
+    const int pos = (!active ? -1 : Tr::kPrefix ? ctx - 1 : ctx - q_len + j) - kb;
+    const int ctx_r = ctx - kb;
     const int my_tiles = qg == 0 ? ntq[0] : ntq[QT - 1];
     // E4M3: a cached value is code x scale; the K scale folds into the logit
     // scale and the V scale into the final normalisation
@@ -934,8 +974,8 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
       }
       // keys past the context, or not loaded, hold stale data: zero their V rows
       // (every query tile that uses the stage writes the same zeros)
-      const int loaded_end = min(kv0 + NKEY, ((nkv + 15) / 16) * 16);
-      const int vz = min(ctx, loaded_end) - kv0;  // V rows [vz, NKEY) must be zero
+      const int loaded_end = min(kv0 + NKEY, ((nkv_r + 15) / 16) * 16);
+      const int vz = min(ctx_r, loaded_end) - kv0;  // V rows [vz, NKEY) must be zero
       if (vz < NKEY) {
         // V of this tile may still be in flight: let it land before zeroing rows
         ok = mbar_wait_bounded(bar_v_full(t % NS), (t / NS) & 1);
@@ -985,6 +1025,31 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
                                v[4 * i + 3] * v_scale);
         }
       }
+    } else if (ok && my_tiles > 0 && !Tr::kPrefix && p.work != nullptr &&
+               p.work[static_cast<size_t>(rank) * kPlanItemInts + 6] > 1) {
+      // a piece of a planned unit: its partial for the merge kernel (the
+      // item is read again here rather than held in registers all along)
+      const int32_t* it = p.work + static_cast<size_t>(rank) * kPlanItemInts;
+      const size_t slot =
+          ((static_cast<size_t>(it[5]) * p.num_kv_heads + kvh) * ROWS + crow) * kMaxPieces + it[4];
+      if (active) {
+        p.ws_max[slot] = m;
+        p.ws_sum[slot] = l;
+      }
+      float4* dst = reinterpret_cast<float4*>(p.ws_out + slot * Tr::D);
+      tc::tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 16) {
+        float v[16];
+        tc::tmem_ld16(lane_addr + Tr::O_COL + c, v);
+        tc::tmem_wait_ld();
+        if (active) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[c / 4 + i] = make_float4(v[4 * i] * v_scale, v[4 * i + 1] * v_scale,
+                                         v[4 * i + 2] * v_scale, v[4 * i + 3] * v_scale);
+        }
+      }
     } else if (ok && my_tiles > 0) {
       tc::tc_fence_after();
       const float inv = l > 0.f ? v_scale / l : 0.f;
@@ -1017,6 +1082,80 @@ __global__ void __launch_bounds__(Tr::THREADS, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, Tr::TMEM_COLS);
   }
+}
+
+// Merge of a planned unit's pieces (the same combination the decode reduce
+// makes of split-K partitions): for each (token, head) row of the unit,
+//   out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,   M = max_s m_s.
+// A warp per row, each lane 4 of the 128 dims; CTA b serves rows
+// 8 (b % R8) .. 8 (b % R8) + 7 of entry (b / R8) / H_kv for kv head
+// (b / R8) % H_kv, R8 = unit_rows / 8, so every row's loads are in flight at
+// once.  Launched after the planned prefill kernel, whose partials it waits
+// for in griddepcontrol.wait.
+template <class DT>
+__global__ void __launch_bounds__(256) paged_prefill_merge_kernel(const PrefillParams p) {
+  using T = typename DT::T;
+  constexpr int D = 128;
+  grid_dependency_wait();
+  trigger_dependents();
+  const int r8 = p.unit_rows / 8;
+  const int unit = static_cast<int>(blockIdx.x) / r8;
+  const int e = unit / p.num_kv_heads;
+  const int kvh = unit % p.num_kv_heads;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = (static_cast<int>(blockIdx.x) % r8) * 8 + warp;
+  const int32_t* me = p.merges + 4 * static_cast<size_t>(e);
+  const int seq = me[0], tile = me[1], pieces = me[2];
+  if (static_cast<unsigned>(seq) >= static_cast<unsigned>(p.num_seqs) || pieces < 2 ||
+      pieces > kMaxPieces || tile < 0) {
+    if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
+    return;
+  }
+  const int group = p.num_heads / p.num_kv_heads;
+  const int q0 = p.query_start[seq];
+  const int q_len = p.query_start[seq + 1] - q0;
+  const int nrows = min(p.unit_rows, q_len * group - tile * p.unit_rows);
+  if (q_len <= 0 || q_len > p.max_query_len || nrows <= 0) {
+    if (threadIdx.x == 0) set_err(p.err, PKV_DEVERR_BAD_ORDER);
+    return;
+  }
+  if (r >= nrows) return;
+  const size_t base =
+      ((static_cast<size_t>(e) * p.num_kv_heads + kvh) * p.unit_rows + r) * kMaxPieces;
+  float ms[kMaxPieces], ls[kMaxPieces];
+  float4 os[kMaxPieces];
+#pragma unroll
+  for (int s = 0; s < kMaxPieces; ++s) {
+    if (s < pieces) {
+      ms[s] = p.ws_max[base + s];
+      ls[s] = p.ws_sum[base + s];
+      os[s] = *reinterpret_cast<const float4*>(p.ws_out + (base + s) * D + lane * 4);
+    }
+  }
+  float big_m = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < kMaxPieces; ++s)
+    if (s < pieces) big_m = fmaxf(big_m, ms[s]);
+  float num[4] = {0.f, 0.f, 0.f, 0.f};
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxPieces; ++s) {
+    if (s < pieces) {
+      const float f = ms[s] == -INFINITY ? 0.f : exp2_approx(ms[s] - big_m);
+      den = fmaf(f, ls[s], den);
+      num[0] = fmaf(f, os[s].x, num[0]);
+      num[1] = fmaf(f, os[s].y, num[1]);
+      num[2] = fmaf(f, os[s].z, num[2]);
+      num[3] = fmaf(f, os[s].w, num[3]);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const int row = tile * p.unit_rows + r;
+  T* out = static_cast<T*>(p.out) +
+           (static_cast<size_t>(q0 + row / group) * p.num_heads + kvh * group + row % group) * D +
+           lane * 4;
+  *reinterpret_cast<uint2*>(out) =
+      make_uint2(pack2(num[0] * inv, num[1] * inv, DT()), pack2(num[2] * inv, num[3] * inv, DT()));
 }
 
 }  // namespace pkv

@@ -86,6 +86,15 @@ _paged_attn_decode_planned = _proto("pkv_paged_attn_decode_planned", _i, _vp, _v
 _paged_attn_decode_fp8_planned = _proto("pkv_paged_attn_decode_fp8_planned", _i, _vp, _vp, _vp,
                                         _vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _i, _i, _i, _i, _i,
                                         _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
+_prefill_plan = _proto("pkv_prefill_plan", _i, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
+                       _i, _vp, _vp)
+_paged_attn_prefill_planned = _proto("pkv_paged_attn_prefill_planned", _i, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _vp, _i, _vp, _i, _f, _i, _i, _i, _i, _i, _i,
+                                     _i, _i, _i, _i, _i, _vp, _sz, _vp, _vp)
+_paged_attn_prefill_fp8_planned = _proto("pkv_paged_attn_prefill_fp8_planned", _i, _vp, _vp, _vp,
+                                         _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _f, _vp, _vp, _i,
+                                         _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp,
+                                         _vp)
 _testing_decode_wait = _proto("pkv_testing_decode_wait", _i, ctypes.c_uint64, _i)
 _pipeline_staging_bytes = _proto("pkv_decode_pipeline_staging_bytes", _sz, _i, _i, _i, _i, _i, _i,
                                  _i)
@@ -509,11 +518,57 @@ def paged_attn_decode_static_ws(out, q, k_cache, v_cache, block_tables, context_
            "paged_attn_decode_static_ws")
 
 
+class PrefillPlan:
+    """A planned prefill's work list (pkv_prefill_plan): ``work`` [items, 8] and
+    ``merges`` [entries, 4] int32 host tensors, ``workspace_bytes``."""
+
+    def __init__(self, work, merges, workspace_bytes):
+        self.work, self.merges, self.workspace_bytes = work, merges, workspace_bytes
+
+    def to(self, device):
+        """The lists on the device, for paged_attn_prefill(plan=...)."""
+        return PrefillPlan(self.work.to(device), self.merges.to(device), self.workspace_bytes)
+
+
+def prefill_plan(query_start, context_lens, num_heads, num_kv_heads, head_dim=128, num_sms=148):
+    """Plan a prefill from host lengths (query_start [S+1], context_lens [S]);
+    see pkv_prefill_plan."""
+    qs = torch.as_tensor(query_start, dtype=torch.int32).contiguous()
+    lens = torch.as_tensor(context_lens, dtype=torch.int32).contiguous()
+    if qs.is_cuda or lens.is_cuda:
+        raise ValueError("query_start and context_lens must be on the host")
+    s = lens.numel()
+    if qs.numel() != s + 1:
+        raise ValueError("query_start must be [S+1]")
+    n, m, wb = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_size_t(0)
+    args = (_ptr(qs), _ptr(lens), s, num_heads, num_kv_heads, head_dim, num_sms)
+    _check(_prefill_plan(*args, None, 0, ctypes.byref(n), None, 0, ctypes.byref(m),
+                         ctypes.byref(wb)), "prefill_plan")
+    work = torch.zeros((n.value, 8), dtype=torch.int32)
+    merges = torch.zeros((m.value, 4), dtype=torch.int32)
+    _check(_prefill_plan(*args, _ptr(work), n.value, ctypes.byref(n), _ptr(merges), m.value,
+                         ctypes.byref(m), ctypes.byref(wb)), "prefill_plan")
+    return PrefillPlan(work, merges, wb.value)
+
+
+def _plan_args(plan, workspace, device, stream):
+    _dev(plan.work, "plan.work", torch.int32)
+    _dev(plan.merges, "plan.merges", torch.int32)
+    if workspace is None and plan.workspace_bytes:
+        workspace = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=device)
+        if stream is not None:
+            workspace.record_stream(stream)   # the temporary must outlive the launch
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return (_ptr(plan.work), plan.work.shape[0], _ptr(plan.merges) if plan.merges.numel() else None,
+            plan.merges.shape[0]), (_ptr(workspace), nbytes, workspace)
+
+
 def paged_attn_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start, scale,
                        num_kv_heads, block_size, max_context_len, max_query_len, dev_err=None,
-                       stream=None):
-    """Chunked-prefill attention; q/out are [T, H, D], query_start [S+1].  See
-    include/pagedkv.h."""
+                       stream=None, plan=None, workspace=None):
+    """Chunked-prefill attention; q/out are [T, H, D], query_start [S+1].  With
+    ``plan`` (prefill_plan(...).to(device)) the planned prefill, with its
+    partials in ``workspace`` (allocated if None).  See include/pagedkv.h."""
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     _dev(block_tables, "block_tables", torch.int32)
@@ -528,6 +583,16 @@ def paged_attn_prefill(out, q, k_cache, v_cache, block_tables, context_lens, que
         raise ValueError("query_start must be [S+1], block_tables [S, max_blocks]")
     if q.dtype != k_cache.dtype or out.dtype != q.dtype:
         raise TypeError("q, out and caches must share a dtype")
+    if plan is not None:
+        pa, (ws_ptr, ws_bytes, _ws) = _plan_args(plan, workspace, q.device, stream)
+        _check(_paged_attn_prefill_planned(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                           _ptr(block_tables), _ptr(context_lens),
+                                           _ptr(query_start), *pa, float(scale), s, t, h, hkv, d,
+                                           bs, block_tables.shape[1], max_context_len,
+                                           max_query_len, num_blocks, _dtype_code(q), ws_ptr,
+                                           ws_bytes, _ptr(dev_err), _stream(stream)),
+               "paged_attn_prefill_planned")
+        return
     _check(_paged_attn_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
                                float(scale), s, t, h, hkv, d, bs, block_tables.shape[1],
@@ -538,9 +603,10 @@ def paged_attn_prefill(out, q, k_cache, v_cache, block_tables, context_lens, que
 
 def paged_attn_prefill_fp8(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
                            scale, k_scales, v_scales, num_kv_heads, block_size, max_context_len,
-                           max_query_len, dev_err=None, stream=None):
+                           max_query_len, dev_err=None, stream=None, plan=None, workspace=None):
     """Chunked-prefill attention over E4M3 caches (values = code * scale of the
-    kv head); q and out are 16-bit, head_dim 128.  See include/pagedkv.h."""
+    kv head); q and out are 16-bit.  ``plan`` and ``workspace`` as for
+    paged_attn_prefill.  See include/pagedkv.h."""
     for n, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _dev(t, n)
     _dev(block_tables, "block_tables", torch.int32)
@@ -558,6 +624,17 @@ def paged_attn_prefill_fp8(out, q, k_cache, v_cache, block_tables, context_lens,
     if out.dtype != q.dtype:
         raise TypeError("q and out must share a dtype")
     ks, vs = _scales_for(k_scales, v_scales, hkv, q.device, stream)
+    if plan is not None:
+        pa, (ws_ptr, ws_bytes, _ws) = _plan_args(plan, workspace, q.device, stream)
+        _check(_paged_attn_prefill_fp8_planned(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                               _ptr(block_tables), _ptr(context_lens),
+                                               _ptr(query_start), *pa, float(scale), _ptr(ks),
+                                               _ptr(vs), s, t, h, hkv, d, bs,
+                                               block_tables.shape[1], max_context_len,
+                                               max_query_len, num_blocks, _dtype_code(q), ws_ptr,
+                                               ws_bytes, _ptr(dev_err), _stream(stream)),
+               "paged_attn_prefill_fp8_planned")
+        return
     _check(_paged_attn_prefill_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                    _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
                                    float(scale), _ptr(ks), _ptr(vs), s, t, h, hkv, d, bs,

@@ -332,3 +332,96 @@ def test_decode_plan_and_planned_decode_validate_on_the_host():
         assert dec(2048, w=null, fp8=fp8) == pk.ERR_INVALID_ARG
         assert dec(2048, w=ctypes.c_void_p(0x1004), fp8=fp8) == pk.ERR_INVALID_ARG  # alignment
         assert dec(24, fp8=fp8) == pk.ERR_INVALID_ARG                # not a multiple of 16
+
+
+@pytest.mark.parametrize("seed,n,h,hkv,sms", [(0, 4, 32, 32, 148), (1, 4, 32, 8, 148),
+                                              (2, 1, 8, 8, 148), (3, 9, 16, 2, 20),
+                                              (4, 30, 32, 8, 148), (5, 3, 8, 1, 4)])
+def test_prefill_plan_covers_every_key_once(seed, n, h, hkv, sms):
+    """pkv_prefill_plan: every (sequence, 256-row tile) unit with rows appears
+    whole or as 2-4 pieces whose key ranges tile [0, causal end) in order:
+    pieces before the last are whole 64-key tiles of history (every row sees
+    them), the last starts inside the history; merge entries name exactly the
+    cut units; items come longest first by the planner's cost."""
+    import numpy as np
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    rng = np.random.default_rng(seed)
+    ql = rng.integers(0, 700, size=n)
+    ql[0] = 512
+    hist = rng.integers(0, 9000, size=n)
+    qs = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
+    lens = (hist + ql).astype(np.int32)
+    plan = pk.prefill_plan(qs, lens, h, hkv, 128, sms)
+    work, merges = plan.work.numpy(), plan.merges.numpy()
+    g = h // hkv
+    units = {(s, t) for s in range(n) for t in range(-(-int(ql[s]) * g // 256))}
+    seen = {}
+    for it in work:
+        seen.setdefault((int(it[0]), int(it[1])), []).append(it)
+    assert set(seen) == units
+    cut = set()
+    for (s, t), its in seen.items():
+        its = sorted(its, key=lambda it: it[4])
+        pieces = int(its[0][6])
+        assert [int(it[4]) for it in its] == list(range(pieces)) and 1 <= pieces <= 4
+        assert all(int(it[6]) == pieces for it in its)
+        if pieces == 1:
+            assert (its[0][2], its[0][3]) == (0, -1)
+            continue
+        cut.add((s, t))
+        assert len({int(it[5]) for it in its}) == 1
+        kb = 0
+        for it in its[:-1]:
+            assert it[2] == kb and it[3] > kb and it[3] % 64 == 0 and it[3] <= hist[s]
+            kb = int(it[3])
+        assert its[-1][2] == kb and its[-1][3] == -1 and kb <= hist[s]
+        m = int(its[0][5])
+        assert tuple(merges[m][:3]) == (s, t, pieces)
+    assert len(merges) == len(cut)
+    if len(merges) == 0:
+        assert plan.workspace_bytes == 0
+    else:   # [merges][kv heads][256 rows][4 pieces] x (o, m, l) in fp32
+        assert plan.workspace_bytes >= len(merges) * hkv * 256 * 4 * 130 * 4
+
+
+def test_prefill_plan_splits_the_longest_unit():
+    """Four sequences, one with a long history: only its units are cut, and
+    its last query tile (the most keys) is among them."""
+    import numpy as np
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    ql = np.array([512, 512, 512, 512])
+    hist = np.array([3000, 300, 100, 50])
+    qs = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
+    plan = pk.prefill_plan(qs, (hist + ql).astype(np.int32), 32, 8, 128, 148)
+    work = plan.work.numpy()
+    assert len(plan.merges) > 0 and set(plan.merges.numpy()[:, 0]) == {0}
+    assert any(it[0] == 0 and it[1] == 7 and it[6] > 1 for it in work)
+
+
+def test_planned_prefill_validates_on_the_host():
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    null = None
+    good = ctypes.c_void_p(0x1000)
+    n, m, wb = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    qs = (ctypes.c_int32 * 3)(0, 512, 1024)
+    lens = (ctypes.c_int32 * 2)(4000, 600)
+    assert pk._prefill_plan(qs, lens, 2, 8, 2, 64, 148, null, 0, ctypes.byref(n), null, 0,
+                            ctypes.byref(m), null) == pk.ERR_UNSUPPORTED          # head_dim 64
+    assert pk._prefill_plan(qs, lens, 2, 8, 2, 128, 0, null, 0, ctypes.byref(n), null, 0,
+                            ctypes.byref(m), null) == pk.ERR_INVALID_ARG          # no SMs
+    assert pk._prefill_plan(qs, lens, 2, 8, 2, 128, 148, null, 0, ctypes.byref(n), null, 0,
+                            ctypes.byref(m), ctypes.byref(wb)) == pk.OK
+    assert n.value >= 2 and m.value >= 1 and wb.value > 0
+    work = (ctypes.c_int32 * (8 * n.value))()
+    assert pk._prefill_plan(qs, lens, 2, 8, 2, 128, 148, work, n.value - 1, ctypes.byref(n),
+                            null, 0, ctypes.byref(m), null) == pk.ERR_INVALID_ARG  # capacity
+
+    def pre(d=128, ws=good, wsb=1 << 30, nm=1, merges=good):
+        return pk._paged_attn_prefill_planned(good, good, good, good, good, good, good, good, 4,
+                                              merges, nm, 0.125, 2, 1024, 8, 2, d, 16, 256, 4096,
+                                              512, 512, 0, ws, wsb, null, null)
+    assert pre(d=64) == pk.ERR_UNSUPPORTED
+    assert pre(ws=null, wsb=0) == pk.ERR_WORKSPACE
+    assert pre(wsb=1024) == pk.ERR_WORKSPACE
+    assert pre(merges=null) == pk.ERR_INVALID_ARG
+    assert pre(ws=ctypes.c_void_p(0x1008)) == pk.ERR_INVALID_ARG

@@ -37,8 +37,16 @@
 #include "common.cuh"
 #include "paged_prefill_kernels.cuh"
 
+// The cascade prefix pass (one query tile, 256 TMEM columns): two K/V stages
+// and at most 128 registers a thread, so that two CTAs share an SM and one's
+// start and end overlap the other's tiles.  Measured on B200 (prefix-sharing
+// batch, one cascade decode): 6 stages, one CTA per SM 0.1778 ms; 4 stages
+// 0.1781; 3 stages 0.1799; 2 stages, two CTAs per SM 0.1616.
 #ifndef PKV_PREFIX_STAGES
-#define PKV_PREFIX_STAGES 6
+#define PKV_PREFIX_STAGES 2
+#endif
+#ifndef PKV_PREFIX_MIN_BLOCKS
+#define PKV_PREFIX_MIN_BLOCKS 2
 #endif
 // K/V stages of a one-query-tile prefill CTA (PKV_PREFILL_QUERY_TILES=1)
 #ifndef PKV_QT1_STAGES
@@ -227,6 +235,7 @@ struct TcPrefillTraits {
   static constexpr int NS = NKEY == 128 ? 2
                             : kFp8 ? 4 : QT == 2 ? 5 : kPrefix ? PKV_PREFIX_STAGES : PKV_QT1_STAGES;
   static constexpr int NSTG = kFp8 ? 2 : 0;      // E4M3 staging slots per kind
+  static constexpr int MIN_BLOCKS = kPrefix && !kFp8 ? PKV_PREFIX_MIN_BLOCKS : 1;  // CTAs per SM
   // warps: K producer, S issuer, V producer, 4 softmax warps per query tile,
   // P.V issuer
   static constexpr int PV_WARP = 3 + 4 * QT;
@@ -269,7 +278,7 @@ struct TcPrefillTraits {
 };
 
 template <class Tr>
-__global__ void __launch_bounds__(Tr::THREADS, 1)
+__global__ void __launch_bounds__(Tr::THREADS, Tr::MIN_BLOCKS)
     paged_prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap qmap,
                             const __grid_constant__ CUtensorMap kmap,
                             const __grid_constant__ CUtensorMap vmap) {

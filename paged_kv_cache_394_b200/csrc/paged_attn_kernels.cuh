@@ -880,8 +880,23 @@ __global__ void __launch_bounds__(Tr::THREADS)
     return;
   }
 
+  // Over E4M3 the context length and (without cascade) the partition's
+  // table slice, which starts at part * part_blocks whatever the length, are
+  // loaded together so that their latencies overlap; entries past the
+  // context are never used.  Otherwise (16-bit caches, where staging whole
+  // one-pass slices measured slower, or under cascade, where the slice
+  // starts after the group's shared blocks) the slice is staged once the
+  // length is known.
   const int ctx_cap = min(p.max_context_len, p.max_blocks_per_seq * BS);
   int ctx = p.context_lens[seq];
+  const bool cascade = p.group_start != nullptr;
+  const bool early_table = Tr::kFp8 && !cascade;
+  const int32_t* seq_row = p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq;
+  if (early_table) {
+    const int b0 = part * p.part_blocks;
+    const int n0 = min(p.part_blocks, p.max_blocks_per_seq - b0);
+    for (int i = threadIdx.x; i < n0; i += Tr::THREADS) tbl[i] = seq_row[b0 + i];
+  }
   if (ctx < 0 || ctx > ctx_cap) {
     if (threadIdx.x == 0 && part == 0 && kvh == 0) set_err(p.err, PKV_DEVERR_BAD_CONTEXT);
     ctx = min(max(ctx, 0), ctx_cap);
@@ -890,7 +905,6 @@ __global__ void __launch_bounds__(Tr::THREADS)
   const int start_blk =
       cascade_start_block(p, seq, nblk, threadIdx.x == 0 && part == 0 && kvh == 0);
   const int nparts = (nblk - start_blk + p.part_blocks - 1) / p.part_blocks;
-  const bool cascade = p.group_start != nullptr;
   if (threadIdx.x == 0 && plan_mismatch(p, cta, nparts)) set_err(p.err, PKV_DEVERR_BAD_ORDER);
   if (part >= (cascade ? nparts : max(nparts, 1))) return;
   const bool direct = !cascade && nparts <= 1;
@@ -899,22 +913,17 @@ __global__ void __launch_bounds__(Tr::THREADS)
   const int sb_begin = blk_begin * SPB;
   const int nsb = max(0, min((ctx + Tr::SUB - 1) / Tr::SUB, (blk_begin + nb) * SPB) - sb_begin);
 
-  const int32_t* trow =
-      p.block_tables + static_cast<size_t>(seq) * p.max_blocks_per_seq + blk_begin;
-  for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = trow[i];
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < NS; ++s) mbar_init(smem_addr(bars + warp * NS + s), 1);
-    fence_mbar_init();
+  if (!early_table) {
+    for (int i = threadIdx.x; i < nb; i += Tr::THREADS) tbl[i] = seq_row[blk_begin + i];
   }
-  __syncthreads();
-
-  // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) + {0,1,8,9}
-  // (E4M3 cache: dims 16ks + 4(lane%4) + {0,1,2,3}, the permuted k order of
-  // mma_sub_block_fp8, as fp16)
+  // q as mma B fragments: lane holds head lane/4, dims 16ks + 2(lane%4) +
+  // {0,1,8,9} (E4M3 cache: dims 16ks + 4(lane%4) + {0,1,2,3}, the permuted k
+  // order of mma_sub_block_fp8, as fp16).  Over 16-bit caches they load
+  // after the barrier; over E4M3 after the first K/V loads are issued, since
+  // the bf16 -> fp16 conversion and the scale check wait for them.
   uint32_t qf[KS][2];
   float qscale = p.qscale;
-  {
+  auto load_q = [&]() {
     const int n = lane >> 2;
     const int c = lane & 3;
     const T* qrow = static_cast<const T*>(p.q) +
@@ -947,7 +956,15 @@ __global__ void __launch_bounds__(Tr::THREADS)
         set_err(p.err, PKV_DEVERR_BAD_SCALE);
       qscale *= ks;
     }
+  };
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) mbar_init(smem_addr(bars + warp * NS + s), 1);
+    fence_mbar_init();
   }
+  __syncthreads();
+  if constexpr (!Tr::kFp8) load_q();
+
   float acc[KS][4];
 #pragma unroll
   for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
@@ -986,6 +1003,7 @@ __global__ void __launch_bounds__(Tr::THREADS)
   if (lane == 0) {
     for (int k = 0; k < min(NS, nbw); ++k) issue(k);
   }
+  if constexpr (Tr::kFp8) load_q();
   for (int k = 0; k < nbw; ++k) {
     const int stage = k % NS;
     const bool ok = mbar_wait_bounded(bar0 + stage * 8, (k / NS) & 1, p.wait_ns);

@@ -291,7 +291,7 @@ def committed_traffic(workload, kind="decode"):
 OTHER_WORKLOADS = ("llama7b_fp8", "long_splitk", "long_splitk_fp8", "gqa_chat", "gqa_chat_fp8",
                    "prefix_share", "prefix_share_cascade", "prefix_share_cascade_fp8",
                    "llama7b_prefill",
-                   "llama7b_prefill_fp8", "gqa_prefill", "gqa_prefill_fp8")
+                   "llama7b_prefill_fp8", "gqa_prefill", "gqa_prefill_fp8", "skew_prefill")
 
 
 def split_name(workload):

@@ -38,7 +38,7 @@ import numpy as np
 NAN_BITS = {"fp16": np.uint16(0x7E00), "bf16": np.uint16(0x7FC0)}
 SEED_BASE = 394
 NAMES = ("tiny", "llama7b", "gqa_chat", "long_splitk", "prefix_share")
-PREFILL_NAMES = ("llama7b_prefill", "gqa_prefill")
+PREFILL_NAMES = ("llama7b_prefill", "gqa_prefill", "skew_prefill")
 
 
 @dataclass
@@ -356,6 +356,11 @@ def make(name, seed=None, allocator=None):
     if name == "gqa_prefill":
         return build_prefill_workload(rng.integers(0, 3072 + 1, size=4), [512] * 4, 32, 8, 128,
                                       32, "bf16", seed, name=name)
+    if name == "skew_prefill":
+        # the same budget with one long cached history among short ones (a
+        # chunk of a long prompt, or a long shared prefix, beside new prompts)
+        return build_prefill_workload([8192, 100, 50, 0], [512] * 4, 32, 32, 128, 16, "fp16",
+                                      seed, name=name)
     if name == "tiny":
         return build_decode_workload([5, 17, 32, 100], 4, 4, 64, 16, "fp16", seed,
                                      num_blocks=64, name=name)

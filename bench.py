@@ -1285,8 +1285,11 @@ def parse_args(argv=None):
     ap.add_argument("--no-graph", action="store_true",
                     help="time the steps as direct launches instead of one captured CUDA graph")
     ap.add_argument("--schedule", choices=("order", "plan"), default="plan",
-                    help="decode CTAs: sequences longest first over the full grid (order), "
-                         "or one CTA per existing partition from pkv_decode_plan (plan)")
+                    help="CTA schedule made on the host from the step's lengths: decode "
+                         "sequences longest first over the full grid and the prefill's own "
+                         "in-kernel ranking (order), or the work lists of pkv_decode_plan "
+                         "(one CTA per existing partition) and pkv_prefill_plan (units by "
+                         "cost, the longest cut into key pieces) (plan)")
     ap.add_argument("--partition", type=int, default=None,
                     help="partition size in tokens (0 = let the library choose)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

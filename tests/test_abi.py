@@ -425,3 +425,31 @@ def test_planned_prefill_validates_on_the_host():
     assert pre(wsb=1024) == pk.ERR_WORKSPACE
     assert pre(merges=null) == pk.ERR_INVALID_ARG
     assert pre(ws=ctypes.c_void_p(0x1008)) == pk.ERR_INVALID_ARG
+
+
+def test_planners_edge_cases():
+    """Empty batches, empty queries, histories too short to cut, and one
+    huge history (at most four pieces, each history piece whole key tiles)."""
+    import numpy as np
+    from paged_kv_cache_394_b200 import pagedkv as pk
+    # no sequences
+    p = pk.prefill_plan(np.zeros(1, np.int32), np.zeros(0, np.int32), 8, 2)
+    assert p.work.shape == (0, 8) and p.merges.shape == (0, 4) and p.workspace_bytes == 0
+    assert pk.decode_plan(np.zeros(0, np.int32), 16, 256).shape == (0, 2)
+    # sequences without new tokens have no units
+    p = pk.prefill_plan(np.array([0, 0, 5, 5], np.int32), np.array([9, 20, 7], np.int32), 8, 2)
+    assert sorted(set(p.work[:, 0].tolist())) == [1]
+    # a history shorter than one key tile is never cut, however many SMs
+    p = pk.prefill_plan(np.array([0, 300], np.int32), np.array([363], np.int32), 8, 2, 128, 10**6)
+    assert len(p.merges) == 0
+    # one huge history: cut, at most four pieces, history pieces whole tiles
+    p = pk.prefill_plan(np.array([0, 64], np.int32), np.array([1_000_064], np.int32), 8, 8, 128, 148)
+    w = p.work.numpy()
+    assert len(p.merges) == 1 and (w[:, 6] <= 4).all() and (w[:, 6] >= 2).all()
+    hist = w[w[:, 3] >= 0]
+    assert (hist[:, 2] % 64 == 0).all() and (hist[:, 3] % 64 == 0).all()
+    assert (hist[:, 3] <= 1_000_000).all()
+    # decode: empty contexts still get one item each
+    d = pk.decode_plan(np.array([0, 0, 40], np.int32), 16, 32).numpy()
+    assert sorted(d[:, 0].tolist()) == [0, 1, 2, 2]
+    assert (d[d[:, 0] < 2, 1] == (0 | (1 << 16))).all()
